@@ -1,0 +1,166 @@
+"""Oracle pins for attention over the dequantised cache: brute force on tiny
+inputs in plain Python, closed-form special cases, and the GQA / causal
+structure."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import (attention_decode, attention_prefill, attention_decode_batch, lse_merge,
+                    quantize_kv, dequantize_kv)
+
+
+def _brute(q, k, v, scale):
+    """Plain-Python softmax attention for one query vector over rows of k, v."""
+    T = len(k)
+    s = [scale * sum(q[j] * k[t][j] for j in range(len(q))) for t in range(T)]
+    mx = max(s)
+    e = [math.exp(x - mx) for x in s]
+    z = sum(e)
+    return [sum(e[t] * v[t][j] for t in range(T)) / z for j in range(len(v[0]))]
+
+
+@pytest.mark.parametrize("T,Hq,Hkv,D", [(1, 2, 1, 32), (5, 4, 2, 32), (8, 8, 2, 32), (7, 3, 3, 32)])
+def test_decode_matches_brute_force(T, Hq, Hkv, D):
+    rng = np.random.default_rng(T * 100 + Hq)
+    q = rng.standard_normal((Hq, D))
+    k = rng.standard_normal((T, Hkv, D)) * 2
+    v = rng.standard_normal((T, Hkv, D))
+    scale = 1 / math.sqrt(D)
+    got = attention_decode(q, k, v)
+    G = Hq // Hkv
+    for h in range(Hq):
+        g = h // G
+        want = _brute(q[h].tolist(), k[:, g].tolist(), v[:, g].tolist(), scale)
+        assert np.allclose(got[h], want, rtol=1e-12, atol=1e-13)
+
+
+def test_gqa_mapping_is_consecutive_groups():
+    # KV head 0 holds V = 0, head 1 holds V = 1: q heads 0..G-1 read head 0
+    T, Hq, Hkv, D = 4, 8, 2, 32
+    rng = np.random.default_rng(1)
+    k = rng.standard_normal((T, Hkv, D))
+    v = np.zeros((T, Hkv, D))
+    v[:, 1] = 1.0
+    o = attention_decode(rng.standard_normal((Hq, D)), k, v)
+    assert np.allclose(o[:4], 0) and np.allclose(o[4:], 1)
+
+
+def test_constant_keys_give_the_mean_of_values():
+    T, D = 9, 64
+    rng = np.random.default_rng(2)
+    k = np.tile(rng.standard_normal((1, 1, D)), (T, 1, 1))
+    v = rng.standard_normal((T, 1, D))
+    o = attention_decode(rng.standard_normal((4, D)), k, v)
+    assert np.allclose(o, v[:, 0].mean(axis=0), rtol=1e-12, atol=1e-14)
+
+
+def test_dominant_logit_selects_its_value():
+    T, D = 6, 32
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((1, D))
+    k = rng.standard_normal((T, 1, D)) * 0.01
+    k[4, 0] = q[0] * 50                                  # logit ~ 50 |q|^2 / sqrt(D)
+    v = rng.standard_normal((T, 1, D))
+    o = attention_decode(q, k, v)
+    assert np.allclose(o[0], v[4, 0], atol=1e-12)
+
+
+def test_softmax_scale_argument():
+    T, D = 5, 32
+    rng = np.random.default_rng(4)
+    k = rng.standard_normal((T, 1, D))
+    v = rng.standard_normal((T, 1, D))
+    o = attention_decode(rng.standard_normal((1, D)), k, v, scale=0.0)
+    assert np.allclose(o[0], v[:, 0].mean(axis=0))
+    q = rng.standard_normal((1, D))
+    a = attention_decode(q, k, v, scale=0.3)
+    b = attention_decode(q * 0.3 * math.sqrt(D), k, v)
+    assert np.allclose(a, b, rtol=1e-12)
+
+
+def test_prefill_causal_structure():
+    # equal keys, one-hot values: row i averages tokens 0..n+i uniformly
+    n, C, D = 3, 5, 32
+    T = n + C
+    k = np.ones((T, 1, D))
+    v = np.zeros((T, 1, D))
+    for t in range(T):
+        v[t, 0, t] = 1.0
+    q = np.ones((C, 2, D))
+    o = attention_prefill(q, k, v, n)
+    for i in range(C):
+        want = np.zeros(D)
+        want[: n + i + 1] = 1.0 / (n + i + 1)
+        assert np.allclose(o[i, 0], want) and np.allclose(o[i, 1], want)
+
+
+def test_prefill_row_zero_of_an_empty_cache_is_its_own_value():
+    rng = np.random.default_rng(5)
+    C, D = 4, 64
+    k = rng.standard_normal((C, 2, D))
+    v = rng.standard_normal((C, 2, D))
+    o = attention_prefill(rng.standard_normal((C, 4, D)), k, v, 0)
+    assert np.allclose(o[0, :2], v[0, 0]) and np.allclose(o[0, 2:], v[0, 1])
+
+
+def test_prefill_rows_equal_decode_at_each_position():
+    rng = np.random.default_rng(6)
+    n, C, D = 10, 6, 32
+    k = rng.standard_normal((n + C, 2, D))
+    v = rng.standard_normal((n + C, 2, D))
+    q = rng.standard_normal((C, 4, D))
+    o = attention_prefill(q, k, v, n, rows=[5, 0, 3])
+    for r, i in enumerate([5, 0, 3]):
+        assert np.allclose(o[r], attention_decode(q[i], k[: n + i + 1], v[: n + i + 1]))
+
+
+def test_split_invariance_through_lse_merge():
+    rng = np.random.default_rng(7)
+    T, D = 50, 32
+    q = rng.standard_normal(D)
+    k = rng.standard_normal((T, 1, D)) * 3
+    v = rng.standard_normal((T, 1, D))
+    full = attention_decode(q[None], k, v)[0]
+    parts = []
+    for lo, hi in [(0, 7), (7, 31), (31, 50)]:
+        s = (k[lo:hi, 0] @ q) / math.sqrt(D)
+        m = s.max()
+        e = np.exp(s - m)
+        parts.append((e @ v[lo:hi, 0], m, e.sum()))
+    assert np.allclose(lse_merge(parts), full, rtol=1e-12)
+
+
+def test_batch_is_per_sequence():
+    rng = np.random.default_rng(8)
+    caches = [(rng.standard_normal((t, 2, 32)), rng.standard_normal((t, 2, 32))) for t in (3, 9)]
+    q = rng.standard_normal((2, 4, 32))
+    o = attention_decode_batch(q, caches)
+    assert np.allclose(o[1], attention_decode(q[1], *caches[1]))
+
+
+def test_empty_cache_rejected():
+    with pytest.raises(ValueError):
+        attention_decode(np.zeros((2, 32)), np.zeros((0, 1, 32)), np.zeros((0, 1, 32)))
+
+
+def test_keys_are_the_sensitive_half():
+    """The page's qualitative claim (section "Assimetria entre key e value"):
+    at equal bits, 4-bit keys with 8-bit values hurt attention more than
+    8-bit keys with 4-bit values, on keys with outlier channels."""
+    rng = np.random.default_rng(9)
+    T, Hq, Hkv, D = 512, 8, 2, 64
+    k = rng.standard_normal((T, Hkv, D))
+    k[:, :, [3, 17, 40]] *= 10
+    k = k.astype(np.float16)
+    v = rng.standard_normal((T, Hkv, D)).astype(np.float16)
+    q = rng.standard_normal((Hq, D)).astype(np.float16)
+    ref = attention_decode(q, k.astype(np.float64), v.astype(np.float64))
+
+    def err(kb, vb):
+        kh = dequantize_kv(*quantize_kv(k, kb), kb)
+        vh = dequantize_kv(*quantize_kv(v, vb), vb)
+        return np.abs(attention_decode(q, kh, vh) - ref).mean()
+
+    assert err(4, 8) > 2 * err(8, 4)
+    assert err(8, 8) < err(8, 4) < err(4, 4)
