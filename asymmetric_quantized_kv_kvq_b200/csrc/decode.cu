@@ -1,0 +1,89 @@
+// Split-KV decode: dispatch over cache formats, and the log-sum-exp combine
+// of partial results (O_s, m_s, l_s) written by the split kernel:
+//   o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  M = max_s m_s
+// (m in the log2 domain of the scaled scores).
+#include <cuda_fp16.h>
+
+#include "kvq_internal.cuh"
+
+namespace kvq {
+
+template <int KB, int VB>
+cudaError_t launch_decode_kv(const Layout&, int, const Batch&, const DecodePlan&, int, const void*, void*, float,
+                             void*, cudaStream_t);
+template <int KB, int VB>
+int decode_chunk_tokens_kv(int D);
+
+namespace {
+
+__global__ void lse_combine_kernel(const __grid_constant__ Batch b, int H, int G, int D, int n_q_heads, int64_t cpc,
+                                   const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
+                                   __half* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t wid = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (wid >= int64_t(b.n) * H * G) return;
+  const int item = int(wid / G), g = int(wid % G);
+  const int bi = item / H, h = item % H;
+  const int nch = b.s[bi].c;
+  const int64_t off = int64_t(b.s[bi].b) + int64_t(h) * nch;
+  const int64_t c0 = off / cpc, c1 = (off + nch - 1) / cpc;
+  if (c0 == c1) return;   // written directly by the split kernel
+  float M = -INFINITY;
+  for (int64_t c = c0; c <= c1; ++c) M = fmaxf(M, ws_ml[((c + item) * G + g) * 2]);
+  float L = 0.f;
+  for (int64_t c = c0; c <= c1; ++c) {
+    const float* ml = ws_ml + ((c + item) * G + g) * 2;
+    L += exp2f(ml[0] - M) * ml[1];
+  }
+  const float inv = 1.f / L;
+  for (int d = lane; d < D; d += 32) {
+    float acc = 0.f;
+    for (int64_t c = c0; c <= c1; ++c)
+      acc += exp2f(ws_ml[((c + item) * G + g) * 2] - M) * ws_o[((c + item) * G + g) * D + d];
+    out[(int64_t(bi) * n_q_heads + h * G + g) * D + d] = __float2half_rn(acc * inv);
+  }
+}
+
+}  // namespace
+
+int decode_max_ctas(int num_sms) { return num_sms; }
+
+size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D) {
+  const size_t slots = size_t(max_ctas) + size_t(n_items);
+  return slots * G * (D + 2) * sizeof(float);
+}
+
+int decode_chunk_tokens(const Layout& L) {
+  const int kb = L.k_bits, vb = L.v_bits, D = L.head_dim;
+  if (kb == 16) return decode_chunk_tokens_kv<16, 16>(D);
+  if (kb == 8 && vb == 8) return decode_chunk_tokens_kv<8, 8>(D);
+  if (kb == 8 && vb == 4) return decode_chunk_tokens_kv<8, 4>(D);
+  if (kb == 4 && vb == 4) return decode_chunk_tokens_kv<4, 4>(D);
+  return decode_chunk_tokens_kv<4, 8>(D);
+}
+
+cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const DecodePlan& plan, int n_q_heads,
+                          const void* q, void* out, float scale_log2, void* ws, cudaStream_t s) {
+  const int kb = L.k_bits, vb = L.v_bits;
+  cudaError_t e;
+  if (kb == 16) e = launch_decode_kv<16, 16>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  else if (kb == 8 && vb == 8) e = launch_decode_kv<8, 8>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  else if (kb == 8 && vb == 4) e = launch_decode_kv<8, 4>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  else if (kb == 4 && vb == 4) e = launch_decode_kv<4, 4>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  else e = launch_decode_kv<4, 8>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  if (e != cudaSuccess) return e;
+  // combine only when some item spans several CTAs
+  if (plan.n_cta > 1 || plan.n_items > 1) {
+    const int H = L.n_kv_heads, G = n_q_heads / H, D = L.head_dim;
+    const int64_t slots = int64_t(plan.max_ctas) + plan.n_items;
+    const float* ws_o = static_cast<const float*>(ws);
+    const float* ws_ml = ws_o + slots * G * D;
+    const int64_t warps = int64_t(plan.n_items) * G;
+    lse_combine_kernel<<<unsigned((warps + 7) / 8), 256, 0, s>>>(b, H, G, D, n_q_heads, plan.chunks_per_cta, ws_o,
+                                                                 ws_ml, static_cast<__half*>(out));
+    e = cudaGetLastError();
+  }
+  return e;
+}
+
+}  // namespace kvq

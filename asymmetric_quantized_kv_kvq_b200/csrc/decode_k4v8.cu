@@ -1,0 +1,8 @@
+// Split-KV decode kernels for K4V8 caches.
+#include "decode_launch.cuh"
+
+namespace kvq {
+template cudaError_t launch_decode_kv<4, 8>(const Layout&, int, const Batch&, const DecodePlan&, int, const void*,
+                                              void*, float, void*, cudaStream_t);
+template int decode_chunk_tokens_kv<4, 8>(int);
+}  // namespace kvq

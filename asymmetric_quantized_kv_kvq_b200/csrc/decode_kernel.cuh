@@ -1,0 +1,525 @@
+// Split-KV flash-decoding over the quantized paged cache (sm_100a, CUDA cores).
+//
+// Computes, for each sequence b, KV head h and query head g of its GQA group,
+//   o = sum_t p_t v^_t / sum_t p_t,  p_t = 2^(s_t - m),  s_t = (sigma log2 e) q . k^_t
+// over cache positions t < len (exact softmax attention read "through the
+// flash-attention path", KVSplit page, section "Exemplos de uso e opcoes de
+// CLI"), with k^ = d_k * c_k and v^ = d_v * c_v dequantised in registers from
+// the stored 8-bit / 4-bit codes (or read as fp16).
+//
+// Work decomposition ("stream-K" over the flat list of (sequence, KV head,
+// chunk) units): CTA c owns chunks [c * cpc, (c+1) * cpc) of that list, so
+// every SM streams the same number of bytes whatever the length mix.  A CTA
+// writes one partial (O, m, l) per item it touches; an item covered by one CTA
+// is normalised and written to `out` directly, the others are merged by the
+// log-sum-exp combine kernel.
+//
+// CTA = 1 producer warp + NW consumer warps, one CTA per SM (persistent):
+//  - producer: lane 0 streams each chunk's K codes, K scales, V codes and V
+//    scales (four contiguous ranges of one page's head block) into a ring of S
+//    shared-memory stages with 1-D TMA bulk copies (cp.async.bulk, L2
+//    evict-first) completing on the stage's "full" mbarrier;
+//  - consumers: warp w takes tokens [w*W, w*W + W) of each stage.
+//      QK: J = 16 head_dim elements per lane (LPT lanes per token), q held in
+//      registers (pre-scaled by sigma log2 e), codes converted exactly to fp32
+//      (byte permute into the mantissa of 2^23, one f32x2 subtract), f32x2
+//      FMAs, one multiply by the block scale, then a reduce-scatter across the
+//      token's lanes leaves each lane the full score of its own head(s).
+//      Softmax: online, per warp, with lazy rescaling (the running max is only
+//      moved when a score exceeds it by more than 2^8).
+//      PV: 8 head_dim elements per lane; p' = p * d_v is precomputed per
+//      (token, block, head) into a warp-private buffer as a duplicated pair,
+//      so the inner loop is one f32x2 FMA per two elements and head.
+//  - every wait is bounded (2 s); on expiry the kernel records an error code,
+//    raises a CTA-wide abort flag, drains its own copies and returns.
+#pragma once
+
+#include <cuda_fp16.h>
+
+#include "kvq_internal.cuh"
+#include "sm100_util.cuh"
+
+namespace kvq {
+
+template <int KB, int VB, int D, int G>
+struct DecodeTraits {
+  static constexpr int NW = G == 8 ? 4 : 8;              // consumer warps
+  static constexpr int NT = (NW + 1) * 32;
+  static constexpr int NB = D / 32;
+  static constexpr int K_ROW = KB == 16 ? 2 * D : KB == 8 ? D : D / 2;
+  static constexpr int V_ROW = VB == 16 ? 2 * D : VB == 8 ? D : D / 2;
+  static constexpr int KS_ROW = KB == 16 ? 0 : NB * 2;
+  static constexpr int VS_ROW = VB == 16 ? 0 : NB * 2;
+  static constexpr int TOK_BYTES = K_ROW + KS_ROW + V_ROW + VS_ROW;
+  static constexpr int C = TOK_BYTES <= 128 ? 256 : TOK_BYTES <= 320 ? 128 : 64;
+  static constexpr int W = C / NW;
+  static constexpr int J = 16;
+  static constexpr int LPT = D / J;
+  static constexpr int TPS = 32 / LPT;
+  static constexpr int NJ = W / TPS;
+  static constexpr int GPL = G > LPT ? G / LPT : 1;
+  static constexpr int REP = G < LPT ? LPT / G : 1;
+  static constexpr int LPV = D / 8;
+  static constexpr int TPV = 32 / LPV;
+  static constexpr int NPV = W / TPV;
+  static constexpr int NBP = VB == 16 ? 1 : NB;
+  static constexpr int OFF_KS = C * K_ROW;
+  static constexpr int OFF_VC = OFF_KS + C * KS_ROW;
+  static constexpr int OFF_VS = OFF_VC + C * V_ROW;
+  static constexpr int STAGE_BYTES = OFF_VS + C * VS_ROW;
+  static constexpr int PBUF_BYTES = NW * W * NBP * G * 8;
+  static constexpr int MRG_O_BYTES = NW * G * D * 4;
+  static constexpr int MRG_ML_BYTES = NW * G * 2 * 4;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int FIXED = PBUF_BYTES + MRG_O_BYTES + MRG_ML_BYTES + BAR_BYTES;
+  static constexpr int SMEM_LIMIT = 227 * 1024;
+  static constexpr int S_FIT = (SMEM_LIMIT - FIXED) / STAGE_BYTES;
+  static constexpr int S = S_FIT > 6 ? 6 : S_FIT;
+  static constexpr int SMEM = S * STAGE_BYTES + FIXED;
+  static_assert(S >= 2, "stage ring does not fit in shared memory");
+  static_assert(W % TPS == 0 && W % TPV == 0 && NJ >= 1, "warp tile");
+  static_assert(2 * S + 4 <= BAR_BYTES / 8, "barrier area");
+  static_assert(STAGE_BYTES % 16 == 0 && OFF_KS % 16 == 0 && OFF_VC % 16 == 0 && OFF_VS % 16 == 0, "alignment");
+};
+
+struct DecodeArgs {
+  Layout L;
+  int layer;
+  int n_q_heads;
+  const __half* q;
+  __half* out;
+  float* ws_o;        // [slots][G][D]
+  float* ws_ml;       // [slots][G][2]
+  float scale_log2;   // sigma * log2(e)
+  int64_t total_chunks;
+  int64_t cpc;        // chunks per CTA
+};
+
+struct DecodeSeg {
+  int bi, h, k0, n;
+};
+
+// Segment of the flat chunk list starting at x: (sequence, head, first chunk, count).
+__device__ __forceinline__ DecodeSeg decode_find_seg(const Batch& b, int64_t x, int64_t x1) {
+  int lo = 0, hi = b.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (b.s[mid].b <= x) lo = mid; else hi = mid - 1;
+  }
+  const int nch = b.s[lo].c;
+  const int64_t rel = x - b.s[lo].b;
+  const int h = int(rel / nch);
+  const int k0 = int(rel - int64_t(h) * nch);
+  const int64_t item_end = b.s[lo].b + int64_t(h + 1) * nch;
+  return {lo, h, k0, int((x1 < item_end ? x1 : item_end) - x)};
+}
+
+// ---- per-format element maps ----------------------------------------------------
+// QK lane `slice` owns 16 elements of the row; element index of its i-th value.
+template <int KB, int D>
+__device__ __forceinline__ int k_elem(int slice, int i) {
+  if (KB == 8) return 16 * slice + i;
+  if (KB == 4) return 32 * (slice >> 1) + 8 * (slice & 1) + (i < 8 ? i : i + 8);
+  return i < 8 ? 8 * slice + i : D / 2 + 8 * slice + (i - 8);
+}
+
+// Load and convert the lane's 16 K values of one row (exact integers or fp16 values).
+template <int KB, int D>
+__device__ __forceinline__ void load_k16(const uint8_t* row, int slice, float2 (&kf)[8]) {
+  if (KB == 8) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * slice);
+    cvt_s8x4(w.x, kf[0], kf[1]);
+    cvt_s8x4(w.y, kf[2], kf[3]);
+    cvt_s8x4(w.z, kf[4], kf[5]);
+    cvt_s8x4(w.w, kf[6], kf[7]);
+  } else if (KB == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * slice);
+    cvt_u4x4(w.x & 0x0F0F0F0Fu, kf[0], kf[1]);
+    cvt_u4x4(w.y & 0x0F0F0F0Fu, kf[2], kf[3]);
+    cvt_u4x4((w.x >> 4) & 0x0F0F0F0Fu, kf[4], kf[5]);
+    cvt_u4x4((w.y >> 4) & 0x0F0F0F0Fu, kf[6], kf[7]);
+  } else {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + 16 * slice);
+    const uint4 c = *reinterpret_cast<const uint4*>(row + D + 16 * slice);
+    kf[0] = h2_to_f2(a.x); kf[1] = h2_to_f2(a.y); kf[2] = h2_to_f2(a.z); kf[3] = h2_to_f2(a.w);
+    kf[4] = h2_to_f2(c.x); kf[5] = h2_to_f2(c.y); kf[6] = h2_to_f2(c.z); kf[7] = h2_to_f2(c.w);
+  }
+}
+
+// PV lane `vs` owns 8 elements of the row: element index of value i (0..7).
+template <int VB>
+__device__ __forceinline__ int v_elem(int vs, int i) {
+  if (VB == 4) return 32 * (vs >> 2) + 4 * (vs & 3) + (i < 4 ? i : i + 12);
+  return 8 * vs + i;
+}
+template <int VB>
+__device__ __forceinline__ int v_block(int vs) {
+  return VB == 16 ? 0 : (vs >> 2);
+}
+
+template <int VB>
+__device__ __forceinline__ void load_v8(const uint8_t* row, int vs, float2 (&vf)[4]) {
+  if (VB == 4) {
+    const uint32_t w = *reinterpret_cast<const uint32_t*>(row + 4 * vs);
+    cvt_u4x4(w & 0x0F0F0F0Fu, vf[0], vf[1]);
+    cvt_u4x4((w >> 4) & 0x0F0F0F0Fu, vf[2], vf[3]);
+  } else if (VB == 8) {
+    const uint2 w = *reinterpret_cast<const uint2*>(row + 8 * vs);
+    cvt_s8x4(w.x, vf[0], vf[1]);
+    cvt_s8x4(w.y, vf[2], vf[3]);
+  } else {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * vs);
+    vf[0] = h2_to_f2(w.x); vf[1] = h2_to_f2(w.y); vf[2] = h2_to_f2(w.z); vf[3] = h2_to_f2(w.w);
+  }
+}
+
+// Reduce-scatter of G partial sums over the LPT lanes of one token (lanes
+// differing in bits below LPT): afterwards this lane holds the full sums of
+// heads g0 .. g0 + GPL - 1 in v[0 .. GPL-1].
+template <int G, int LPT>
+__device__ __forceinline__ void reduce_scatter(float (&v)[G], int lane) {
+  int n = G;
+#pragma unroll
+  for (int o = LPT / 2; o >= 1; o >>= 1) {
+    if (n > 1) {
+      const bool upper = (lane & o) != 0;
+#pragma unroll
+      for (int i = 0; i < G / 2; ++i) {
+        if (i < n / 2) {
+          const float send = upper ? v[i] : v[i + n / 2];
+          const float keep = upper ? v[i + n / 2] : v[i];
+          v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      }
+      n >>= 1;
+    } else {
+      v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+    }
+  }
+}
+
+template <int KB, int VB, int D, int G>
+__global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
+    decode_split_kernel(const DecodeArgs a, const __grid_constant__ Batch b) {
+  using T = DecodeTraits<KB, VB, D, G>;
+  constexpr int S = T::S, C = T::C, W = T::W, NW = T::NW;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint8_t* stages = smem;
+  float2* pbuf = reinterpret_cast<float2*>(smem + S * T::STAGE_BYTES);
+  float* mrg_o = reinterpret_cast<float*>(smem + S * T::STAGE_BYTES + T::PBUF_BYTES);
+  float* mrg_ml = mrg_o + NW * G * D;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * T::STAGE_BYTES + T::PBUF_BYTES + T::MRG_O_BYTES +
+                                               T::MRG_ML_BYTES);
+  // bars[0..S) full, [S..2S) empty, [2S] merge-full, [2S+1] merge-free, then the abort flag
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 2 * S + 2);
+  const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + S);
+  const uint32_t mfull = smem_u32(bars + 2 * S), mfree = smem_u32(bars + 2 * S + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int H = a.L.n_kv_heads;
+  const int64_t x0 = int64_t(blockIdx.x) * a.cpc;
+  const int64_t x1 = min(a.total_chunks, x0 + a.cpc);
+
+  // stage ring starts zeroed so rows never written by a copy stay finite
+  for (int i = threadIdx.x; i < S * T::STAGE_BYTES / 16; i += T::NT)
+    reinterpret_cast<uint4*>(stages)[i] = make_uint4(0, 0, 0, 0);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, NW);
+    }
+    mbar_init(mfull, NW);
+    mbar_init(mfree, NW);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  __syncthreads();
+
+  // ------------------------------------------------------------------ producer
+  if (warp == NW) {
+    if (lane != 0) return;
+    const uint64_t pol = l2_evict_first_policy();
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t x = x0; x < x1 && ok;) {
+      const DecodeSeg sg = decode_find_seg(b, x, x1);
+      const SeqDesc sd = b.s[sg.bi];
+      for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
+        const int s = it % S;
+        if (!mbar_wait(empty0 + 8 * s, ((it / S) & 1) ^ 1, abort_flag)) {
+          record_error(a.L.err, kErrWaitTimeout | 1);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const int tok0 = k * C;
+        const int ntok = min(C, sd.a - tok0);
+        const int ncopy = min(C, (ntok + 15) & ~15);
+        const int page = a.L.page_table[int64_t(sd.seq_id) * a.L.max_pages_per_seq + tok0 / a.L.page_tokens];
+        if (page < 0 || page >= a.L.n_pages) {
+          record_error(a.L.err, kErrBadPage);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        const int r = tok0 % a.L.page_tokens;
+        const uint8_t* hb = a.L.head_ptr(a.layer, page, sg.h);
+        const uint32_t bar = full0 + 8 * s;
+        const uint32_t dst = smem_u32(stages + s * T::STAGE_BYTES);
+        mbar_arrive_expect_tx(bar, uint32_t(ncopy * T::TOK_BYTES));
+        bulk_g2s(dst, hb + int64_t(r) * T::K_ROW, ncopy * T::K_ROW, bar, pol);
+        if (T::KS_ROW) bulk_g2s(dst + T::OFF_KS, hb + a.L.k_scales_off + int64_t(r) * T::KS_ROW, ncopy * T::KS_ROW, bar, pol);
+        bulk_g2s(dst + T::OFF_VC, hb + a.L.v_codes_off + int64_t(r) * T::V_ROW, ncopy * T::V_ROW, bar, pol);
+        if (T::VS_ROW) bulk_g2s(dst + T::OFF_VS, hb + a.L.v_scales_off + int64_t(r) * T::VS_ROW, ncopy * T::VS_ROW, bar, pol);
+        ++it;
+      }
+      x += sg.n;
+    }
+    // no copy may outlive the CTA: wait (bounded) for the last fills to land
+    for (uint32_t j = it > uint32_t(S) ? it - S : 0; j < it; ++j) mbar_wait(full0 + 8 * (j % S), (j / S) & 1, nullptr);
+    return;
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int slice = lane % T::LPT, tis = lane / T::LPT;
+  const int vsl = lane % T::LPV, tslot = lane / T::LPV;
+  const int g0 = (slice / T::REP) * T::GPL;
+  const int rep = slice % T::REP;
+  const int ct = warp * 32 + lane;
+  uint32_t it = 0, itm = 0;
+
+  for (int64_t x = x0; x < x1;) {
+    const DecodeSeg sg = decode_find_seg(b, x, x1);
+    const SeqDesc sd = b.s[sg.bi];
+    const int item = sg.bi * H + sg.h;
+
+    // q slice in registers, pre-scaled by sigma * log2(e)
+    float2 qp[G][8];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const __half* qrow = a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + g) * D;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float e0 = __half2float(qrow[k_elem<KB, D>(slice, 2 * i)]);
+        const float e1 = __half2float(qrow[k_elem<KB, D>(slice, 2 * i + 1)]);
+        qp[g][i] = make_float2(e0 * a.scale_log2, e1 * a.scale_log2);
+      }
+    }
+    float2 O[G][4];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) O[g][k] = make_float2(0.f, 0.f);
+    float m_own[T::GPL], l_own[T::GPL];
+#pragma unroll
+    for (int gi = 0; gi < T::GPL; ++gi) {
+      m_own[gi] = -INFINITY;
+      l_own[gi] = 0.f;
+    }
+
+    for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
+      const int s = it % S;
+      if (!mbar_wait(full0 + 8 * s, (it / S) & 1, abort_flag)) {
+        if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 2);
+        *abort_flag = 1;
+        return;
+      }
+      ++it;
+      const int nvalid = min(C, sd.a - k * C);
+      const int nv_w = min(W, max(0, nvalid - warp * W));
+      if (nv_w > 0) {
+        const uint8_t* st = stages + s * T::STAGE_BYTES;
+        const int row0 = warp * W;
+        // ---- scores
+        float sc[T::NJ][T::GPL];
+#pragma unroll
+        for (int j = 0; j < T::NJ; ++j) {
+          const int t = j * T::TPS + tis;
+          const int row = row0 + t;
+          float2 kf[8];
+          load_k16<KB, D>(st + row * T::K_ROW, slice, kf);
+          float part[G];
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc = ffma2(qp[g][i], kf[i], acc);
+            part[g] = acc.x + acc.y;
+          }
+          if (KB != 16) {
+            const float dk =
+                __half2float(reinterpret_cast<const __half*>(st + T::OFF_KS + row * T::KS_ROW)[slice >> 1]);
+#pragma unroll
+            for (int g = 0; g < G; ++g) part[g] *= dk;
+          }
+          reduce_scatter<G, T::LPT>(part, lane);
+#pragma unroll
+          for (int gi = 0; gi < T::GPL; ++gi) sc[j][gi] = t < nv_w ? part[gi] : -INFINITY;
+        }
+        // ---- online softmax (max moved lazily)
+        float tmax[T::GPL];
+        bool need = false;
+#pragma unroll
+        for (int gi = 0; gi < T::GPL; ++gi) {
+          float mx = sc[0][gi];
+#pragma unroll
+          for (int j = 1; j < T::NJ; ++j) mx = fmaxf(mx, sc[j][gi]);
+#pragma unroll
+          for (int o = T::LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          tmax[gi] = mx;
+          need |= mx > m_own[gi] + 8.f;
+        }
+        if (__any_sync(0xffffffffu, need)) {
+          float alpha[T::GPL];
+#pragma unroll
+          for (int gi = 0; gi < T::GPL; ++gi) {
+            const float mn = fmaxf(m_own[gi], tmax[gi]);
+            alpha[gi] = exp2f(m_own[gi] - mn);
+            m_own[gi] = mn;
+            l_own[gi] *= alpha[gi];
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float al = __shfl_sync(0xffffffffu, alpha[g % T::GPL], (g / T::GPL) * T::REP);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) O[g][k] = fmul2(O[g][k], make_float2(al, al));
+          }
+        }
+        // ---- p and p' = p * d_v (duplicated pairs) into the warp's buffer
+        float2* pw = pbuf + size_t(warp) * W * T::NBP * G;
+#pragma unroll
+        for (int j = 0; j < T::NJ; ++j) {
+          const int t = j * T::TPS + tis;
+          const int row = row0 + t;
+#pragma unroll
+          for (int gi = 0; gi < T::GPL; ++gi) {
+            const float p = exp2f(sc[j][gi] - m_own[gi]);
+            l_own[gi] += p;
+            if (VB == 16) {
+              if (rep == 0) pw[t * G + g0 + gi] = make_float2(p, p);
+            } else {
+#pragma unroll
+              for (int bb = 0; bb < T::NBP; bb += T::REP) {
+                const int blk = bb + rep;
+                if (blk < T::NBP) {
+                  const float dv =
+                      __half2float(reinterpret_cast<const __half*>(st + T::OFF_VS + row * T::VS_ROW)[blk]);
+                  const float pv = t < nv_w ? p * dv : 0.f;
+                  pw[(t * T::NBP + blk) * G + g0 + gi] = make_float2(pv, pv);
+                }
+              }
+            }
+          }
+        }
+        __syncwarp();
+        // ---- O += p' v
+#pragma unroll 2
+        for (int j2 = 0; j2 < T::NPV; ++j2) {
+          const int t = j2 * T::TPV + tslot;
+          if (t < nv_w) {
+            float2 vf[4];
+            load_v8<VB>(st + T::OFF_VC + (row0 + t) * T::V_ROW, vsl, vf);
+            const float2* pp = pw + (t * T::NBP + v_block<VB>(vsl)) * G;
+#pragma unroll
+            for (int g = 0; g < G; g += 2) {
+              float2 p0, p1;
+              (void)p1;
+              if constexpr (G >= 2) {
+                const float4 pq = *reinterpret_cast<const float4*>(pp + g);
+                p0 = make_float2(pq.x, pq.y);
+                p1 = make_float2(pq.z, pq.w);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) O[g][kk] = ffma2(p0, vf[kk], O[g][kk]);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) O[g + 1][kk] = ffma2(p1, vf[kk], O[g + 1][kk]);
+              } else {
+                p0 = pp[g];
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk) O[g][kk] = ffma2(p0, vf[kk], O[g][kk]);
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * s);
+    }
+
+    // ---- merge token slots inside the warp, then the warps of the CTA
+#pragma unroll
+    for (int o = T::LPV; o < 32; o <<= 1)
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          O[g][k].x += __shfl_xor_sync(0xffffffffu, O[g][k].x, o);
+          O[g][k].y += __shfl_xor_sync(0xffffffffu, O[g][k].y, o);
+        }
+#pragma unroll
+    for (int gi = 0; gi < T::GPL; ++gi)
+#pragma unroll
+      for (int o = T::LPT; o < 32; o <<= 1) l_own[gi] += __shfl_xor_sync(0xffffffffu, l_own[gi], o);
+
+    if (!mbar_wait(mfree, (itm & 1) ^ 1, abort_flag)) {
+      if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 3);
+      *abort_flag = 1;
+      return;
+    }
+    if (tslot == 0) {
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          mrg_o[(warp * G + g) * D + v_elem<VB>(vsl, 2 * k)] = O[g][k].x;
+          mrg_o[(warp * G + g) * D + v_elem<VB>(vsl, 2 * k + 1)] = O[g][k].y;
+        }
+    }
+    if (tis == 0 && rep == 0) {
+#pragma unroll
+      for (int gi = 0; gi < T::GPL; ++gi) {
+        mrg_ml[(warp * G + g0 + gi) * 2] = m_own[gi];
+        mrg_ml[(warp * G + g0 + gi) * 2 + 1] = l_own[gi];
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(mfull);
+    if (!mbar_wait(mfull, itm & 1, abort_flag)) {
+      if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 4);
+      *abort_flag = 1;
+      return;
+    }
+    const int nch = sd.c;
+    const int64_t off = int64_t(sd.b) + int64_t(sg.h) * nch;
+    const bool single = (off / a.cpc) == ((off + nch - 1) / a.cpc);
+    for (int e = ct; e < G * D; e += NW * 32) {
+      const int g = e / D, d = e % D;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_ml[(w * G + g) * 2]);
+      float acc = 0.f, L = 0.f;
+#pragma unroll
+      for (int w = 0; w < NW; ++w) {
+        const float f = exp2f(mrg_ml[(w * G + g) * 2] - M);
+        acc += f * mrg_o[(w * G + g) * D + d];
+        L += f * mrg_ml[(w * G + g) * 2 + 1];
+      }
+      if (single) {
+        a.out[(int64_t(sg.bi) * a.n_q_heads + sg.h * G + g) * D + d] = __float2half_rn(acc / L);
+      } else {
+        const int64_t slot = int64_t(blockIdx.x) + item;
+        a.ws_o[(slot * G + g) * D + d] = acc;
+        if (d == 0) {
+          a.ws_ml[(slot * G + g) * 2] = M;
+          a.ws_ml[(slot * G + g) * 2 + 1] = L;
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(mfree);
+    ++itm;
+    x += sg.n;
+  }
+}
+
+}  // namespace kvq

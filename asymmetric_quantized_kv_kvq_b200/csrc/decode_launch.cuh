@@ -1,0 +1,53 @@
+// Host-side launch of the split-KV decode kernel for one (K bits, V bits)
+// pair; instantiated in one translation unit per pair.
+#pragma once
+
+#include "decode_kernel.cuh"
+
+namespace kvq {
+
+template <int KB, int VB, int D, int G>
+cudaError_t launch_decode_one(const Layout& L, int layer, const Batch& b, const DecodePlan& plan, int n_q_heads,
+                              const void* q, void* out, float scale_log2, void* ws, cudaStream_t s) {
+  using T = DecodeTraits<KB, VB, D, G>;
+  static bool configured = false;   // per instantiation; set once per process
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<KB, VB, D, G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  DecodeArgs a;
+  a.L = L;
+  a.layer = layer;
+  a.n_q_heads = n_q_heads;
+  a.q = static_cast<const __half*>(q);
+  a.out = static_cast<__half*>(out);
+  const int64_t slots = int64_t(plan.max_ctas) + plan.n_items;
+  a.ws_o = static_cast<float*>(ws);
+  a.ws_ml = a.ws_o + slots * G * D;
+  a.scale_log2 = scale_log2;
+  a.total_chunks = plan.total_chunks;
+  a.cpc = plan.chunks_per_cta;
+  decode_split_kernel<KB, VB, D, G><<<plan.n_cta, T::NT, T::SMEM, s>>>(a, b);
+  return cudaGetLastError();
+}
+
+template <int KB, int VB>
+cudaError_t launch_decode_kv(const Layout& L, int layer, const Batch& b, const DecodePlan& plan, int n_q_heads,
+                             const void* q, void* out, float scale_log2, void* ws, cudaStream_t s) {
+  const int G = n_q_heads / L.n_kv_heads;
+#define KVQ_DEC(D_, G_) \
+  if (L.head_dim == D_ && G == G_) return launch_decode_one<KB, VB, D_, G_>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  KVQ_DEC(128, 1) KVQ_DEC(128, 2) KVQ_DEC(128, 4) KVQ_DEC(128, 8)
+  KVQ_DEC(64, 1) KVQ_DEC(64, 2) KVQ_DEC(64, 4) KVQ_DEC(64, 8)
+#undef KVQ_DEC
+  return cudaErrorInvalidValue;
+}
+
+template <int KB, int VB>
+int decode_chunk_tokens_kv(int D) {
+  return D == 128 ? DecodeTraits<KB, VB, 128, 4>::C : DecodeTraits<KB, VB, 64, 4>::C;
+}
+
+}  // namespace kvq

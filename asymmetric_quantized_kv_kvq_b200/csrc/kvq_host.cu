@@ -1,0 +1,500 @@
+// Host side of the C ABI declared in include/kvq.h: argument validation, the
+// page allocator, page-table maintenance and kernel dispatch.  Every check
+// runs before anything is enqueued; a failed check leaves the cache unchanged.
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "kvq_internal.cuh"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kvq_status fail(kvq_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+kvq_status cuda_fail(cudaError_t e, const char* what) {
+  g_last_error = std::string(what) + ": " + cudaGetErrorString(e);
+  return e == cudaErrorMemoryAllocation ? KVQ_ERR_OUT_OF_MEMORY : KVQ_ERR_CUDA;
+}
+
+#define KVQ_CUDA(call, what)                    \
+  do {                                          \
+    cudaError_t e_ = (call);                    \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+bool bits_ok(int b) { return b == 4 || b == 8 || b == 16; }
+
+// Supported (k_bits, v_bits) pairs: both fp16, or both quantised.
+bool pair_supported(int kb, int vb) {
+  if (kb == 16 || vb == 16) return kb == vb;
+  return true;
+}
+
+int64_t bytes_per_token_head(int bits, int D) {
+  if (bits == 16) return 2LL * D;
+  if (bits == 8) return int64_t(D / 32) * 34;
+  return int64_t(D / 32) * 18;
+}
+
+kvq_status check_config(const kvq_cache_config* c) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "config is NULL");
+  if (c->n_layers < 1 || c->n_kv_heads < 1) return fail(KVQ_ERR_INVALID_ARG, "n_layers and n_kv_heads must be >= 1");
+  if (c->head_dim <= 0 || c->head_dim % 32) return fail(KVQ_ERR_INVALID_ARG, "head_dim must be a positive multiple of 32");
+  if (!bits_ok(c->k_bits) || !bits_ok(c->v_bits)) return fail(KVQ_ERR_INVALID_ARG, "k_bits and v_bits must be 16, 8 or 4");
+  if (c->head_dim != 64 && c->head_dim != 128) return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d not built (64, 128)", c->head_dim);
+  if (!pair_supported(c->k_bits, c->v_bits)) return fail(KVQ_ERR_UNSUPPORTED, "K%dV%d not built", c->k_bits, c->v_bits);
+  int P = c->page_tokens ? c->page_tokens : 256;
+  if (P < 64 || P > 4096 || P % 64) return fail(KVQ_ERR_INVALID_ARG, "page_tokens must be a multiple of 64 in [64, 4096]");
+  if (c->max_seqs < 1 || c->max_seqs > (1 << 22)) return fail(KVQ_ERR_INVALID_ARG, "max_seqs out of range");
+  if (c->max_tokens < 1) return fail(KVQ_ERR_INVALID_ARG, "max_tokens must be >= 1");
+  int64_t mst = c->max_seq_tokens ? c->max_seq_tokens : c->max_tokens;
+  if (mst < 1 || mst > (int64_t(1) << 30)) return fail(KVQ_ERR_INVALID_ARG, "max_seq_tokens out of range (<= 2^30)");
+  if (c->flags & ~KVQ_CACHE_HOST_ONLY) return fail(KVQ_ERR_INVALID_ARG, "unknown flags");
+  int64_t pages = (c->max_tokens + P - 1) / P;
+  if (pages > (int64_t(1) << 30)) return fail(KVQ_ERR_INVALID_ARG, "max_tokens too large");
+  int64_t mpps = (mst + P - 1) / P;
+  if (int64_t(c->max_seqs) * mpps > (int64_t(1) << 31) - 1) return fail(KVQ_ERR_INVALID_ARG, "page table too large");
+  return KVQ_OK;
+}
+
+}  // namespace
+
+struct kvq_cache {
+  kvq_cache_config cfg{};
+  bool host_only = false;
+  int device = 0;
+  int num_sms = 148;
+  kvq::Layout L{};
+  int64_t pool_bytes = 0;
+  int64_t bytes_per_token_layer = 0;
+  int32_t* d_page_table = nullptr;
+  uint32_t* d_err = nullptr;
+  std::vector<int32_t> table;        // host mirror of the page table
+  std::vector<int64_t> len;          // tokens per sequence
+  std::vector<int32_t> mapped;       // pages mapped per sequence
+  std::vector<int32_t> free_pages;   // stack; back() is handed out next
+  int64_t mapped_pages = 0;
+};
+
+namespace {
+
+kvq_status check_cache(const kvq_cache* c) {
+  if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
+  return KVQ_OK;
+}
+
+kvq_status check_seq(const kvq_cache* c, int32_t id) {
+  if (id < 0 || id >= c->cfg.max_seqs) return fail(KVQ_ERR_INVALID_ARG, "sequence id %d out of range", id);
+  return KVQ_OK;
+}
+
+kvq_status check_ids(const kvq_cache* c, int32_t n, const int32_t* ids) {
+  if (n < 1 || n > kvq::kMaxBatch) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [1, %d]", kvq::kMaxBatch);
+  if (!ids) return fail(KVQ_ERR_INVALID_ARG, "seq_ids is NULL");
+  std::vector<int32_t> sorted(ids, ids + n);
+  for (int i = 0; i < n; ++i)
+    if (kvq_status s = check_seq(c, ids[i])) return s;
+  std::sort(sorted.begin(), sorted.end());
+  for (int i = 1; i < n; ++i)
+    if (sorted[i] == sorted[i - 1]) return fail(KVQ_ERR_INVALID_ARG, "sequence id %d repeated", sorted[i]);
+  return KVQ_OK;
+}
+
+kvq_status check_layer(const kvq_cache* c, int32_t layer) {
+  if (layer < 0 || layer >= c->cfg.n_layers) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
+  return KVQ_OK;
+}
+
+kvq_status need_device(const kvq_cache* c) {
+  if (c->host_only) return fail(KVQ_ERR_UNSUPPORTED, "cache was created host-only");
+  return KVQ_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+kvq_status launched(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported";
+    case KVQ_ERR_OUT_OF_MEMORY: return "out of memory";
+    case KVQ_ERR_CAPACITY: return "page capacity exhausted";
+    case KVQ_ERR_CUDA: return "CUDA error";
+    case KVQ_ERR_DEVICE_CHECK: return "device-side check failed";
+    case KVQ_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+const char* kvq_last_error(void) { return g_last_error.c_str(); }
+
+kvq_status kvq_footprint_bytes(const kvq_cache_config* cfg, int64_t n_tokens, int64_t* allocated, int64_t* used) {
+  if (kvq_status s = check_config(cfg)) return s;
+  if (n_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "n_tokens must be >= 0");
+  int P = cfg->page_tokens ? cfg->page_tokens : 256;
+  int64_t per = int64_t(cfg->n_kv_heads) *
+                (bytes_per_token_head(cfg->k_bits, cfg->head_dim) + bytes_per_token_head(cfg->v_bits, cfg->head_dim));
+  int64_t pages = (n_tokens + P - 1) / P;
+  if (allocated) *allocated = int64_t(cfg->n_layers) * pages * P * per;
+  if (used) *used = int64_t(cfg->n_layers) * n_tokens * per;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
+  if (!out) return fail(KVQ_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  if (kvq_status s = check_config(cfg)) return s;
+  kvq_cache* c = new (std::nothrow) kvq_cache();
+  if (!c) return fail(KVQ_ERR_OUT_OF_MEMORY, "host allocation failed");
+  c->cfg = *cfg;
+  if (!c->cfg.page_tokens) c->cfg.page_tokens = 256;
+  if (!c->cfg.max_seq_tokens) c->cfg.max_seq_tokens = c->cfg.max_tokens;
+  c->host_only = (cfg->flags & KVQ_CACHE_HOST_ONLY) != 0;
+
+  const int P = c->cfg.page_tokens, D = c->cfg.head_dim, H = c->cfg.n_kv_heads;
+  kvq::Layout& L = c->L;
+  L.n_kv_heads = H;
+  L.page_tokens = P;
+  L.head_dim = D;
+  L.k_bits = c->cfg.k_bits;
+  L.v_bits = c->cfg.v_bits;
+  L.k_row = kvq::code_row_bytes(L.k_bits, D);
+  L.v_row = kvq::code_row_bytes(L.v_bits, D);
+  L.s_row = (D / kvq::QK) * 2;
+  const int ks = L.k_bits == 16 ? 0 : L.s_row, vs = L.v_bits == 16 ? 0 : L.s_row;
+  L.k_scales_off = P * L.k_row;
+  L.v_codes_off = L.k_scales_off + P * ks;
+  L.v_scales_off = L.v_codes_off + P * L.v_row;
+  L.head_block = int64_t(L.v_scales_off) + int64_t(P) * vs;
+  L.n_pages = int32_t((c->cfg.max_tokens + P - 1) / P);
+  L.max_pages_per_seq = int32_t((c->cfg.max_seq_tokens + P - 1) / P);
+  c->bytes_per_token_layer = int64_t(H) * (L.k_row + ks + L.v_row + vs);
+  c->pool_bytes = int64_t(c->cfg.n_layers) * L.n_pages * H * L.head_block;
+
+  try {
+    c->table.assign(size_t(c->cfg.max_seqs) * L.max_pages_per_seq, -1);
+    c->len.assign(c->cfg.max_seqs, 0);
+    c->mapped.assign(c->cfg.max_seqs, 0);
+    c->free_pages.resize(L.n_pages);
+  } catch (...) {
+    delete c;
+    return fail(KVQ_ERR_OUT_OF_MEMORY, "host bookkeeping allocation failed");
+  }
+  for (int32_t i = 0; i < L.n_pages; ++i) c->free_pages[i] = L.n_pages - 1 - i;  // page 0 first
+
+  if (!c->host_only) {
+    cudaError_t e;
+    if ((e = cudaGetDevice(&c->device)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device)) != cudaSuccess) {
+      delete c;
+      return cuda_fail(e, "cudaGetDevice");
+    }
+    auto cleanup = [&](cudaError_t err, const char* what) {
+      if (L.pool) cudaFree(L.pool);
+      if (c->d_page_table) cudaFree(c->d_page_table);
+      if (c->d_err) cudaFree(c->d_err);
+      delete c;
+      return cuda_fail(err, what);
+    };
+    if ((e = cudaMalloc(&L.pool, size_t(c->pool_bytes))) != cudaSuccess) return cleanup(e, "cudaMalloc(page pool)");
+    if ((e = cudaMalloc(&c->d_page_table, c->table.size() * sizeof(int32_t))) != cudaSuccess)
+      return cleanup(e, "cudaMalloc(page table)");
+    if ((e = cudaMalloc(&c->d_err, sizeof(uint32_t))) != cudaSuccess) return cleanup(e, "cudaMalloc(error word)");
+    if ((e = cudaMemset(L.pool, 0, size_t(c->pool_bytes))) != cudaSuccess) return cleanup(e, "cudaMemset(pool)");
+    if ((e = cudaMemset(c->d_page_table, 0xFF, c->table.size() * sizeof(int32_t))) != cudaSuccess)
+      return cleanup(e, "cudaMemset(page table)");
+    if ((e = cudaMemset(c->d_err, 0, sizeof(uint32_t))) != cudaSuccess) return cleanup(e, "cudaMemset(err)");
+    if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cleanup(e, "cudaDeviceSynchronize");
+    L.page_table = c->d_page_table;
+    L.err = c->d_err;
+  }
+  *out = c;
+  return KVQ_OK;
+}
+
+kvq_status kvq_cache_destroy(kvq_cache* c) {
+  if (!c) return KVQ_OK;
+  kvq_status st = KVQ_OK;
+  if (!c->host_only) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) st = cuda_fail(e, "cudaDeviceSynchronize");
+    cudaFree(c->L.pool);
+    cudaFree(c->d_page_table);
+    cudaFree(c->d_err);
+  }
+  delete c;
+  return st;
+}
+
+kvq_status kvq_cache_footprint(const kvq_cache* c, int64_t* pool, int64_t* mapped, int64_t* used) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (pool) *pool = c->pool_bytes;
+  if (mapped)
+    *mapped = c->mapped_pages * int64_t(c->cfg.n_layers) * c->L.n_kv_heads * c->L.head_block;
+  if (used) {
+    int64_t t = 0;
+    for (int64_t x : c->len) t += x;
+    *used = t * c->bytes_per_token_layer * c->cfg.n_layers;
+  }
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_length(const kvq_cache* c, int32_t id, int64_t* len) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_seq(c, id)) return s;
+  if (!len) return fail(KVQ_ERR_INVALID_ARG, "len is NULL");
+  *len = c->len[id];
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_page(const kvq_cache* c, int32_t id, int32_t page, int32_t* phys) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_seq(c, id)) return s;
+  if (!phys) return fail(KVQ_ERR_INVALID_ARG, "phys is NULL");
+  if (page < 0 || page >= c->L.max_pages_per_seq) return fail(KVQ_ERR_INVALID_ARG, "page index out of range");
+  *phys = c->table[size_t(id) * c->L.max_pages_per_seq + page];
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int32_t* n_new, kvq_stream_t stream) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_ids(c, n, ids)) return s;
+  if (!n_new) return fail(KVQ_ERR_INVALID_ARG, "n_new is NULL");
+  const int P = c->L.page_tokens;
+  int64_t need = 0;
+  for (int i = 0; i < n; ++i) {
+    if (n_new[i] < 0) return fail(KVQ_ERR_INVALID_ARG, "n_new[%d] < 0", i);
+    int64_t nl = c->len[ids[i]] + n_new[i];
+    if (nl > c->cfg.max_seq_tokens)
+      return fail(KVQ_ERR_CAPACITY, "sequence %d would hold %lld tokens > max_seq_tokens", ids[i], (long long)nl);
+    need += (nl + P - 1) / P - c->mapped[ids[i]];
+  }
+  if (need > int64_t(c->free_pages.size()))
+    return fail(KVQ_ERR_CAPACITY, "need %lld pages, %zu free", (long long)need, c->free_pages.size());
+
+  kvq::PtUpdate upd;
+  upd.n = 0;
+  auto flush = [&]() -> kvq_status {
+    if (upd.n == 0 || c->host_only) { upd.n = 0; return KVQ_OK; }
+    cudaError_t e = kvq::launch_pt_update(c->d_page_table, upd, (cudaStream_t)stream);
+    upd.n = 0;
+    return launched(e, "page-table update");
+  };
+  for (int i = 0; i < n; ++i) {
+    const int32_t id = ids[i];
+    const int64_t nl = c->len[id] + n_new[i];
+    const int32_t want = int32_t((nl + P - 1) / P);
+    while (c->mapped[id] < want) {
+      const int32_t page = c->free_pages.back();
+      c->free_pages.pop_back();
+      const int32_t slot = id * c->L.max_pages_per_seq + c->mapped[id];
+      c->table[slot] = page;
+      c->mapped[id]++;
+      c->mapped_pages++;
+      upd.idx[upd.n] = slot;
+      upd.val[upd.n] = page;
+      if (++upd.n == kvq::kMaxPtUpdates)
+        if (kvq_status s = flush()) return s;
+    }
+    c->len[id] = nl;
+  }
+  return flush();
+}
+
+kvq_status kvq_seq_release(kvq_cache* c, int32_t id) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_seq(c, id)) return s;
+  for (int32_t p = c->mapped[id] - 1; p >= 0; --p) {
+    int32_t& slot = c->table[size_t(id) * c->L.max_pages_per_seq + p];
+    c->free_pages.push_back(slot);
+    slot = -1;
+  }
+  c->mapped_pages -= c->mapped[id];
+  c->mapped[id] = 0;
+  c->len[id] = 0;
+  return KVQ_OK;
+}
+
+kvq_status kvq_append(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, const int32_t* n_new,
+                      const void* k, const void* v, kvq_stream_t stream) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (kvq_status s = check_ids(c, n, ids)) return s;
+  if (!n_new) return fail(KVQ_ERR_INVALID_ARG, "n_new is NULL");
+  kvq::Batch b;
+  b.n = n;
+  int64_t total = 0;
+  for (int i = 0; i < n; ++i) {
+    if (n_new[i] < 0 || n_new[i] > c->len[ids[i]])
+      return fail(KVQ_ERR_INVALID_ARG, "n_new[%d] = %d outside [0, len = %lld]", i, n_new[i], (long long)c->len[ids[i]]);
+    b.s[i] = {ids[i], int32_t(c->len[ids[i]] - n_new[i]), n_new[i], int32_t(total)};
+    total += n_new[i];
+    if (total > (int64_t(1) << 30)) return fail(KVQ_ERR_INVALID_ARG, "too many tokens in one append");
+  }
+  if (total == 0) return KVQ_OK;
+  if (!k || !v) return fail(KVQ_ERR_INVALID_ARG, "k or v is NULL");
+  if (!aligned16(k) || !aligned16(v)) return fail(KVQ_ERR_INVALID_ARG, "k and v must be 16-byte aligned");
+  if (kvq_status s = need_device(c)) return s;
+  return launched(kvq::launch_append(c->L, layer, b, int(total), k, v, (cudaStream_t)stream), "append");
+}
+
+kvq_status kvq_decode_workspace_size(const kvq_cache* c, int32_t n, int32_t n_q_heads, size_t* bytes) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (!bytes) return fail(KVQ_ERR_INVALID_ARG, "bytes is NULL");
+  if (n < 1 || n > kvq::kMaxBatch) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [1, %d]", kvq::kMaxBatch);
+  if (n_q_heads < 1 || n_q_heads % c->L.n_kv_heads) return fail(KVQ_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+  const int G = n_q_heads / c->L.n_kv_heads;
+  *bytes = kvq::decode_workspace_bytes(n * c->L.n_kv_heads, kvq::decode_max_ctas(c->num_sms), G, c->L.head_dim);
+  return KVQ_OK;
+}
+
+kvq_status kvq_decode_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, int32_t n_q_heads,
+                           const void* q, void* out, float softmax_scale, void* ws, size_t ws_bytes,
+                           kvq_stream_t stream) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (kvq_status s = check_ids(c, n, ids)) return s;
+  if (n_q_heads < 1 || n_q_heads % c->L.n_kv_heads) return fail(KVQ_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+  const int G = n_q_heads / c->L.n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KVQ_ERR_UNSUPPORTED, "GQA group %d not built (1, 2, 4, 8)", G);
+  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q or out is NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  if (ws && !aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return fail(KVQ_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  size_t need = 0;
+  if (kvq_status s = kvq_decode_workspace_size(c, n, n_q_heads, &need)) return s;
+  if (!ws || ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
+  if (kvq_status s = need_device(c)) return s;
+
+  kvq::DecodePlan plan;
+  plan.chunk_tokens = kvq::decode_chunk_tokens(c->L);
+  const int C = plan.chunk_tokens, H = c->L.n_kv_heads;
+  kvq::Batch b;
+  b.n = n;
+  int64_t flat = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t len = c->len[ids[i]];
+    if (len < 1) return fail(KVQ_ERR_INVALID_ARG, "sequence %d is empty", ids[i]);
+    const int32_t nch = int32_t((len + C - 1) / C);
+    b.s[i] = {ids[i], int32_t(len), int32_t(flat), nch};
+    flat += int64_t(H) * nch;
+  }
+  plan.n_items = n * H;
+  plan.total_chunks = flat;
+  const int max_ctas = kvq::decode_max_ctas(c->num_sms);
+  plan.max_ctas = max_ctas;
+  plan.chunks_per_cta = (flat + max_ctas - 1) / max_ctas;
+  plan.n_cta = int((flat + plan.chunks_per_cta - 1) / plan.chunks_per_cta);
+  if (flat >= (int64_t(1) << 31)) return fail(KVQ_ERR_INVALID_ARG, "batch too large");
+  const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(c->L.head_dim));
+  const float scale_log2 = sigma * 1.4426950408889634f;
+  return launched(kvq::launch_decode(c->L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, (cudaStream_t)stream),
+                  "decode");
+}
+
+kvq_status kvq_prefill_workspace_size(const kvq_cache* c, int32_t n, const int32_t* ids, const int32_t* q_lens,
+                                      int32_t n_q_heads, size_t* bytes) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_ids(c, n, ids)) return s;
+  if (!q_lens || !bytes) return fail(KVQ_ERR_INVALID_ARG, "q_lens or bytes is NULL");
+  if (n_q_heads < 1 || n_q_heads % c->L.n_kv_heads) return fail(KVQ_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+  kvq::Batch b;
+  b.n = n;
+  int64_t total = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t len = c->len[ids[i]];
+    if (q_lens[i] < 1 || q_lens[i] > len) return fail(KVQ_ERR_INVALID_ARG, "q_lens[%d] outside [1, len]", i);
+    b.s[i] = {ids[i], int32_t(len), q_lens[i], int32_t(total)};
+    total += q_lens[i];
+  }
+  *bytes = kvq::prefill_workspace_bytes(c->L, b);
+  return KVQ_OK;
+}
+
+kvq_status kvq_prefill_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, const int32_t* q_lens,
+                            int32_t n_q_heads, const void* q, void* out, float softmax_scale, void* ws,
+                            size_t ws_bytes, kvq_stream_t stream) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (kvq_status s = check_ids(c, n, ids)) return s;
+  if (!q_lens) return fail(KVQ_ERR_INVALID_ARG, "q_lens is NULL");
+  if (n_q_heads < 1 || n_q_heads % c->L.n_kv_heads) return fail(KVQ_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+  const int G = n_q_heads / c->L.n_kv_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KVQ_ERR_UNSUPPORTED, "GQA group %d not built (1, 2, 4, 8)", G);
+  if (c->L.head_dim != 128 && c->L.head_dim != 64) return fail(KVQ_ERR_UNSUPPORTED, "head_dim not built for prefill");
+  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q or out is NULL");
+  if (!aligned16(q) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  if (ws && !aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return fail(KVQ_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  kvq::Batch b;
+  b.n = n;
+  int64_t total = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t len = c->len[ids[i]];
+    if (q_lens[i] < 1 || q_lens[i] > len) return fail(KVQ_ERR_INVALID_ARG, "q_lens[%d] outside [1, len]", i);
+    b.s[i] = {ids[i], int32_t(len), q_lens[i], int32_t(total)};
+    total += q_lens[i];
+    if (total > (int64_t(1) << 30)) return fail(KVQ_ERR_INVALID_ARG, "too many query rows");
+  }
+  const size_t need = kvq::prefill_workspace_bytes(c->L, b);
+  if (need && (!ws || ws_bytes < need))
+    return fail(KVQ_ERR_WORKSPACE, "prefill needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
+  if (kvq_status s = need_device(c)) return s;
+  const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(c->L.head_dim));
+  return launched(kvq::launch_prefill(c->L, layer, b, int(total), n_q_heads, q, out, sigma, ws, ws_bytes,
+                                      c->num_sms, (cudaStream_t)stream),
+                  "prefill");
+}
+
+kvq_status kvq_export(const kvq_cache* c, int32_t layer, int32_t id, int64_t tok0, int64_t n_tok, void* kc,
+                      void* ks, void* vc, void* vs, kvq_stream_t stream) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_layer(c, layer)) return s;
+  if (kvq_status s = check_seq(c, id)) return s;
+  if (tok0 < 0 || n_tok < 0 || tok0 + n_tok > c->len[id]) return fail(KVQ_ERR_INVALID_ARG, "token range outside the sequence");
+  if (n_tok == 0) return KVQ_OK;
+  if (kvq_status s = need_device(c)) return s;
+  return launched(kvq::launch_export(c->L, layer, id, tok0, n_tok, kc, ks, vc, vs, (cudaStream_t)stream), "export");
+}
+
+kvq_status kvq_cache_check(kvq_cache* c, kvq_stream_t stream, uint32_t* detail) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (detail) *detail = 0;
+  if (c->host_only) return KVQ_OK;
+  KVQ_CUDA(cudaStreamSynchronize((cudaStream_t)stream), "cudaStreamSynchronize");
+  KVQ_CUDA(cudaGetLastError(), "earlier launch");
+  uint32_t code = 0;
+  KVQ_CUDA(cudaMemcpy(&code, c->d_err, sizeof code, cudaMemcpyDeviceToHost), "read device error word");
+  if (code) {
+    if (detail) *detail = code;
+    KVQ_CUDA(cudaMemset(c->d_err, 0, sizeof code), "clear device error word");
+    return fail(KVQ_ERR_DEVICE_CHECK, "device check failed, code 0x%x", code);
+  }
+  return KVQ_OK;
+}
+
+}  // extern "C"

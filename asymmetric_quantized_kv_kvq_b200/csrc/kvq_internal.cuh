@@ -1,0 +1,117 @@
+// Internal definitions shared by the host library and the sm_100a kernels.
+//
+// HBM layout of the page pool (one cudaMalloc per cache):
+//   pool[layer][page][kv_head] -> one "head block" of page_tokens tokens:
+//     K codes  [P][k_row]   int8 (8-bit) | packed nibbles (4-bit, D/2 B) | fp16 (16-bit)
+//     K scales [P][D/32]    fp16                     (absent for 16-bit)
+//     V codes  [P][v_row]
+//     V scales [P][D/32]    fp16                     (absent for 16-bit)
+//   Every sub-array is a multiple of 16 B (page_tokens is a multiple of 64), so
+//   a token range of one sub-array is one 16-B aligned bulk copy, and the head
+//   block holds exactly page_tokens * (K + V bytes per token): the footprint is
+//   the closed form of the KVSplit page's memory table with no padding.
+//   Rows are token-major and in canonical block order, so exporting a token
+//   range is a plain gather by page.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int QK = 32;                 // elements per quantisation block
+constexpr int kMaxBatch = KVQ_MAX_BATCH;
+
+// Device error codes (first one recorded wins; read by kvq_cache_check).
+enum : uint32_t {
+  kErrNone = 0,
+  kErrWaitTimeout = 0x100,             // | barrier id: an mbarrier wait exceeded its limit
+  kErrBadPage = 0x200,                 // a page-table entry was unmapped or out of range
+  kErrBadIndex = 0x300,
+};
+
+struct Layout {
+  uint8_t* pool;
+  const int32_t* page_table;           // [max_seqs][max_pages_per_seq], -1 = unmapped
+  uint32_t* err;                       // device error word
+  int64_t head_block;                  // bytes per (layer, page, head)
+  int32_t n_pages;                     // pages in the pool
+  int32_t max_pages_per_seq;
+  int32_t n_kv_heads;
+  int32_t page_tokens;
+  int32_t head_dim;
+  int32_t k_bits, v_bits;
+  int32_t k_row, v_row;                // code bytes per token
+  int32_t s_row;                       // scale bytes per token (D/32 * 2), 0 for 16-bit
+  int32_t k_scales_off, v_codes_off, v_scales_off;   // byte offsets inside a head block
+
+  __host__ __device__ __forceinline__ uint8_t* head_ptr(int layer, int page, int head) const {
+    return pool + ((int64_t(layer) * n_pages + page) * n_kv_heads + head) * head_block;
+  }
+};
+
+inline int code_row_bytes(int bits, int D) { return bits == 16 ? 2 * D : bits == 8 ? D : D / 2; }
+
+// One sequence of a batched call.  Field meaning depends on the operation:
+//   append : a = first position written (len - n_new), b = n_new, c = row offset in k/v
+//   decode : a = len, b = flat chunk offset of the sequence's first item, c = chunks per item
+//   prefill: a = len, b = q_len, c = row offset in q/out
+struct SeqDesc {
+  int32_t seq_id;
+  int32_t a, b, c;
+};
+
+struct Batch {
+  int32_t n;
+  SeqDesc s[kMaxBatch];
+};
+
+// Page-table update: entries (index into the table, value), applied in order.
+constexpr int kMaxPtUpdates = 1024;
+struct PtUpdate {
+  int32_t n;
+  int32_t idx[kMaxPtUpdates];
+  int32_t val[kMaxPtUpdates];
+};
+
+__device__ __forceinline__ void record_error(uint32_t* err, uint32_t code) {
+  atomicCAS(err, 0u, code);
+}
+
+// ---------------------------------------------------------------------------
+// launchers (defined in the kernel translation units)
+// ---------------------------------------------------------------------------
+cudaError_t launch_pt_update(int32_t* table, const PtUpdate& u, cudaStream_t s);
+
+cudaError_t launch_append(const Layout& L, int layer, const Batch& b, int total_tokens,
+                          const void* k, const void* v, cudaStream_t s);
+
+cudaError_t launch_export(const Layout& L, int layer, int seq_id, int64_t tok0, int64_t n_tok,
+                          void* k_codes, void* k_scales, void* v_codes, void* v_scales,
+                          cudaStream_t s);
+
+struct DecodePlan {
+  int chunk_tokens;      // tokens per stage / work unit
+  int n_items;           // n_seqs * n_kv_heads
+  int64_t total_chunks;
+  int64_t chunks_per_cta;
+  int n_cta;             // CTAs launched (<= max_ctas)
+  int max_ctas;          // CTA cap the workspace was sized for
+};
+
+// decode: workspace = partial slots [(max_ctas + n_items)][G][D + 2] fp32
+size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D);
+int decode_max_ctas(int num_sms);
+int decode_chunk_tokens(const Layout& L);
+cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const DecodePlan& plan,
+                          int n_q_heads, const void* q, void* out, float scale_log2,
+                          void* workspace, cudaStream_t s);
+
+size_t prefill_workspace_bytes(const Layout& L, const Batch& b);
+cudaError_t launch_prefill(const Layout& L, int layer, const Batch& b, int total_q, int n_q_heads,
+                           const void* q, void* out, float scale, void* workspace, size_t ws_bytes,
+                           int num_sms, cudaStream_t s);
+
+}  // namespace kvq

@@ -1,0 +1,134 @@
+// Small sm_100a helpers: mbarriers with bounded waits, 1-D TMA bulk copies,
+// packed f32x2 arithmetic and exact int -> fp32 conversions of stored codes.
+#pragma once
+
+#include <cstdint>
+#include <cuda_fp16.h>
+
+namespace kvq {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Every wait gives up after this long (or as soon as *abort is set), so a
+// lost arrival can never hang the GPU: the caller records an error and leaves.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 31) == 0) {
+      if (abort && *abort) return false;
+      if (global_ns() - t0 > kWaitLimitNs) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
+// 1-D bulk copy global -> shared (this CTA), completing on `bar` with tx bytes.
+// dst, src 16-B aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar,
+                                         uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// ---- packed fp32 pairs (sm_100 f32x2) ----
+__device__ __forceinline__ unsigned long long f2_bits(float2 a) {
+  return (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
+}
+__device__ __forceinline__ float2 bits_f2(unsigned long long b) {
+  return make_float2(__uint_as_float(uint32_t(b)), __uint_as_float(uint32_t(b >> 32)));
+}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)), "l"(f2_bits(c)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_bits(a)), "l"(f2_bits(b)));
+  return bits_f2(d);
+}
+
+// ---- exact conversions of stored integer codes to fp32 ----
+// A byte u placed in the low mantissa bits of the float 2^23 reads as
+// 2^23 + u exactly; subtracting (2^23 + bias) leaves u - bias exactly.
+constexpr float kTwo23 = 8388608.0f;
+
+__device__ __forceinline__ float2 bytes01_f(uint32_t w) {
+  return make_float2(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7540)),
+                     __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7541)));
+}
+__device__ __forceinline__ float2 bytes23_f(uint32_t w) {
+  return make_float2(__uint_as_float(__byte_perm(w, 0x4B000000u, 0x7542)),
+                     __uint_as_float(__byte_perm(w, 0x4B000000u, 0x7543)));
+}
+
+// four signed int8 codes (bytes 0..3 of w) -> (c0, c1), (c2, c3)
+__device__ __forceinline__ void cvt_s8x4(uint32_t w, float2& a, float2& b) {
+  const uint32_t u = w ^ 0x80808080u;
+  const float2 off = make_float2(-(kTwo23 + 128.f), -(kTwo23 + 128.f));
+  a = fadd2(bytes01_f(u), off);
+  b = fadd2(bytes23_f(u), off);
+}
+
+// four nibbles, one in the low 4 bits of each byte of w (others zero) -> (u - 8) pairs
+__device__ __forceinline__ void cvt_u4x4(uint32_t w, float2& a, float2& b) {
+  const float2 off = make_float2(-(kTwo23 + 8.f), -(kTwo23 + 8.f));
+  a = fadd2(bytes01_f(w), off);
+  b = fadd2(bytes23_f(w), off);
+}
+
+__device__ __forceinline__ float2 h2_to_f2(uint32_t w) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&w));
+}
+
+}  // namespace kvq

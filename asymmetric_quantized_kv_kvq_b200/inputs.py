@@ -20,6 +20,7 @@ regenerated on its own.
 from __future__ import annotations
 
 import dataclasses
+import functools
 from typing import Optional, Sequence
 
 import torch
@@ -96,6 +97,7 @@ def _randn(shape, seed: int, device) -> torch.Tensor:
     return torch.randn(shape, generator=g, device=device, dtype=torch.float32)
 
 
+@functools.lru_cache(maxsize=512)
 def outlier_channels(wl: Workload, layer: int) -> torch.Tensor:
     """Boolean mask [Hkv, D] of key channels scaled by OUTLIER_SCALE in `layer`."""
     H, D = wl.n_kv_heads, wl.head_dim
@@ -113,11 +115,16 @@ def outlier_channels(wl: Workload, layer: int) -> torch.Tensor:
     return mask
 
 
+@functools.lru_cache(maxsize=512)
+def _outlier_mask_on(wl: Workload, layer: int, device: str) -> torch.Tensor:
+    return outlier_channels(wl, layer).to(device)
+
+
 def _chunk(wl: Workload, kind: str, layer: int, seq: int, c: int, device) -> torch.Tensor:
     x = _randn((GEN_CHUNK, wl.n_kv_heads, wl.head_dim),
                seed_for(_wl_id(wl), _KINDS[kind], layer, seq, c), device)
     if kind == "k":
-        mask = outlier_channels(wl, layer).to(device)
+        mask = _outlier_mask_on(wl, layer, str(device))
         x = torch.where(mask, x * OUTLIER_SCALE, x)
     return x.to(torch.float16)
 

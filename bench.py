@@ -1,0 +1,485 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized-KV decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--precision K8V4]
+    python bench.py --impl reference ...      # the CPU oracle on host cores
+
+One step = one decode step of the workload: every sequence gains one token;
+for each layer the new token's K / V are quantised into the paged cache
+(kvq_append) and the query attends to the whole cache (kvq_decode_attn:
+split-KV kernel + log-sum-exp combine).  Metric: algorithmic KV bytes moved
+per second (cache codes + scales read by decode, fp16 q / out, the appended
+token's fp16 read and quantised write), and decode tokens/s = batch / step.
+
+Multi-GPU (torchrun): every rank holds an independent replica of the workload
+(sequences are independent, so the batch shards with no collective); value =
+bytes of all ranks / the slowest rank's time ("weak" scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "K8V4 decode-attention KV GB/s (fraction of HBM peak) and decode tokens/s"
+DEFAULT_WORKLOAD = "llama3-8b-b32-32k"
+L2_BYTES = 126 * 1024 * 1024
+PROFILE_DIR = os.path.join(ROOT, "profiles")
+
+
+# --------------------------------------------------------------------------- helpers
+def tok_bytes(bits: int, D: int) -> int:
+    """Stored bytes of one token's K or V row of one head (codes + scales)."""
+    return 2 * D if bits == 16 else (D // 32) * (34 if bits == 8 else 18)
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_sha() -> str:
+    """Hash of the decode kernel sources: ncu traffic figures are valid only for this hash."""
+    h = hashlib.sha256()
+    for name in ("decode_kernel.cuh", "decode_launch.cuh", "decode.cu", "sm100_util.cuh"):
+        with open(os.path.join(ROOT, "asymmetric_quantized_kv_kvq_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str, precision: str):
+    """DRAM bytes per launch of the decode kernel from the committed ncu summary
+    of this workload, if it was captured on the current kernel source."""
+    path = os.path.join(PROFILE_DIR, f"decode_split_{precision.lower()}_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append(parts)
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
+        mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
+        reasons = sorted({self.NAMES[i] for s in self.samples for i in range(4) if s[3 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------- decode workload
+class DecodeRun:
+    """A resident cache of the workload plus one decode step's inputs."""
+
+    def __init__(self, wl, kb: int, vb: int, capacity_extra: int, device):
+        import torch
+        from asymmetric_quantized_kv_kvq_b200 import kvq
+        from asymmetric_quantized_kv_kvq_b200.inputs import gen_kv, gen_q, GEN_CHUNK
+        self.wl, self.kb, self.vb, self.dev = wl, kb, vb, device
+        L, B, H, D, T = wl.n_layers, wl.batch, wl.n_kv_heads, wl.head_dim, wl.cached
+        P = 256
+        cap = T + capacity_extra
+        self.cache = kvq.Cache(L, H, D, kb, vb, max_seqs=B, max_tokens=B * (-(-cap // P)) * P, max_seq_tokens=cap)
+        self.ids = list(range(B))
+        # fill: chunk by chunk, every layer (the order a model's prefill writes the cache)
+        for c in range(-(-T // GEN_CHUNK)):
+            n = min(GEN_CHUNK, T - c * GEN_CHUNK)
+            self.cache.extend(self.ids, [n] * B)
+            for layer in range(L):
+                ks, vs = [], []
+                for b in self.ids:
+                    k, v = gen_kv(wl, layer, b, c * GEN_CHUNK, n, device=device)
+                    ks.append(k)
+                    vs.append(v)
+                self.cache.append(layer, self.ids, [n] * B, torch.cat(ks), torch.cat(vs))
+                del ks, vs
+        torch.cuda.synchronize()
+        # one decode step's inputs (same values every step)
+        self.k_new, self.v_new, self.q, self.out = [], [], [], []
+        for layer in range(L):
+            ks, vs = zip(*[gen_kv(wl, layer, b, T, 1, device=device) for b in self.ids])
+            self.k_new.append(torch.cat(ks).contiguous())
+            self.v_new.append(torch.cat(vs).contiguous())
+            self.q.append(gen_q(wl, layer, 0, device=device))
+            self.out.append(torch.empty_like(self.q[-1]))
+        self.ws = torch.empty(self.cache.decode_workspace_size(B, wl.n_q_heads), dtype=torch.uint8, device=device)
+        self.ones = [1] * B
+        self.ev = None
+
+    def lengths(self):
+        return [self.cache.length(b) for b in self.ids]
+
+    def step_bytes(self, lens) -> tuple:
+        """(decode bytes, append bytes) of one step whose sequences end at `lens`."""
+        wl = self.wl
+        H, D, L, Hq = wl.n_kv_heads, wl.head_dim, wl.n_layers, wl.n_q_heads
+        per_tok = H * (tok_bytes(self.kb, D) + tok_bytes(self.vb, D))
+        dec = sum(lens) * per_tok + 2 * len(lens) * Hq * D * 2
+        app = len(lens) * (H * D * 2 * 2 + per_tok)
+        return L * dec, L * app
+
+    def launches_per_step(self, lens_before) -> int:
+        pt = 1 if any(n % 256 == 0 for n in lens_before) else 0
+        return pt + self.wl.n_layers * 3   # append, decode split, combine
+
+    def step(self, record=None):
+        self.cache.extend(self.ids, self.ones)
+        for layer in range(self.wl.n_layers):
+            self.cache.append(layer, self.ids, self.ones, self.k_new[layer], self.v_new[layer])
+            if record is not None:
+                record[layer][0].record()
+            self.cache.decode(layer, self.ids, self.q[layer], out=self.out[layer], workspace=self.ws)
+            if record is not None:
+                record[layer][1].record()
+
+
+def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    extra = args.warmup + 2 * args.steps + 8
+    t0 = time.time()
+    run = DecodeRun(wl, kb, vb, extra, dev)
+    setup_s = time.time() - t0
+    L = wl.n_layers
+    lens0 = run.lengths()
+    total_kv = sum(lens0) * wl.n_kv_heads * (tok_bytes(kb, wl.head_dim) + tok_bytes(vb, wl.head_dim)) * L
+    flush = total_kv < 2 * L2_BYTES
+    scratch = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
+
+    for _ in range(args.warmup):
+        run.step()
+    run.cache.check()
+    barrier(world)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, CUDA events on the launching stream
+    ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
+    dec_ms, step_ms, dec_bytes, app_bytes, launches = [], [], 0, 0, 0
+    gpu_id = gpu_uuid(dev)
+    with ClockSampler(gpu_id) as clk:
+        for _ in range(args.steps):
+            if flush:
+                scratch.zero_()
+            lens_before = run.lengths()
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            run.step(record=ev)
+            s1.record()
+            torch.cuda.synchronize()
+            step_ms.append(s0.elapsed_time(s1))
+            dec_ms.extend(e0.elapsed_time(e1) for e0, e1 in ev)
+            d, a = run.step_bytes([n + 1 for n in lens_before])
+            dec_bytes += d
+            app_bytes += a
+            launches += run.launches_per_step(lens_before)
+    barrier(world)
+    torch.cuda.synchronize()
+    run.cache.check()
+
+    local_ms = sum(step_ms)
+    max_ms = all_reduce_max(local_ms, world, dev)
+    tot_bytes = all_reduce_sum(float(dec_bytes + app_bytes), world, dev)
+    tot_tokens = all_reduce_sum(float(wl.batch * args.steps), world, dev)
+    res = {
+        "ms_per_step": max_ms / args.steps,
+        "value": tot_bytes / (max_ms * 1e-3) / 1e9,
+        "decode_tokens_per_s": tot_tokens / (max_ms * 1e-3),
+        "dec_bytes_per_launch": dec_bytes / (args.steps * L),
+        "dec_ms_per_launch": statistics.mean(dec_ms),
+        "launches": launches,
+        "clocks": clk.summary(),
+        "flush": flush,
+        "setup_s": setup_s,
+    }
+
+    # ---- end to end through the public API with host buffers
+    if not args.no_e2e:
+        res["e2e"] = run_e2e(run, args, world, dev)
+    run.cache.close()
+    return res
+
+
+def run_e2e(run, args, world, dev) -> dict:
+    """Same step, but every step copies its inputs (q, new K / V for all layers)
+    from pinned host memory and reads all outputs back to pinned host memory."""
+    import torch
+    L = run.wl.n_layers
+    hq = [t.cpu().pin_memory() for t in run.q]
+    hk = [t.cpu().pin_memory() for t in run.k_new]
+    hv = [t.cpu().pin_memory() for t in run.v_new]
+    ho = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in run.out]
+    h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv)
+    d2h = sum(t.numel() * t.element_size() for t in ho)
+    for _ in range(2):
+        run.step()
+    barrier(world)
+    torch.cuda.synchronize()
+    nbytes, ms = 0, 0.0
+    for _ in range(args.steps):
+        lens_before = run.lengths()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for layer in range(L):
+            run.q[layer].copy_(hq[layer], non_blocking=True)
+            run.k_new[layer].copy_(hk[layer], non_blocking=True)
+            run.v_new[layer].copy_(hv[layer], non_blocking=True)
+        run.step()
+        for layer in range(L):
+            ho[layer].copy_(run.out[layer], non_blocking=True)
+        s1.record()
+        torch.cuda.synchronize()
+        ms += s0.elapsed_time(s1)
+        d, a = run.step_bytes([n + 1 for n in lens_before])
+        nbytes += d + a
+    barrier(world)
+    max_ms = all_reduce_max(ms, world, dev)
+    tot = all_reduce_sum(float(nbytes), world, dev)
+    return {"value": tot / (max_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h}
+
+
+# --------------------------------------------------------------------------- distributed plumbing
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _all_reduce(x: float, world: int, dev, op):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=op)
+    return float(t.item())
+
+
+def all_reduce_max(x, world, dev):
+    import torch.distributed as dist
+    return _all_reduce(x, world, dev, dist.ReduceOp.MAX) if world > 1 else x
+
+
+def all_reduce_sum(x, world, dev):
+    import torch.distributed as dist
+    return _all_reduce(x, world, dev, dist.ReduceOp.SUM) if world > 1 else x
+
+
+def gpu_uuid(dev) -> str:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return "0"
+
+
+# --------------------------------------------------------------------------- CPU oracle leg
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return 1
+
+
+def prepare_oracle_slice(wl, kb, vb, layer=0, seq=0):
+    """Stored form of one (layer, sequence) slice of the decode workload and its
+    query, prepared (untimed) by the oracle's own quantiser."""
+    import oracle
+    from asymmetric_quantized_kv_kvq_b200.inputs import gen_kv, gen_q
+    k, v = gen_kv(wl, layer, seq, 0, wl.cached)
+    kc, ks = oracle.quantize_kv(k.numpy(), kb)
+    vc, vs = oracle.quantize_kv(v.numpy(), vb)
+    return kc, ks, vc, vs, gen_q(wl, layer, 0)[seq].numpy()
+
+
+def time_oracle_slice(sl, kb, vb) -> float:
+    """One decode step of the oracle on a slice: read the stored cache
+    (dequantise codes + scales to float64) and attend with every query head."""
+    import oracle
+    kc, ks, vc, vs, q = sl
+    t0 = time.perf_counter()
+    kh = oracle.dequantize_kv(kc, ks, kb)
+    vh = oracle.dequantize_kv(vc, vs, vb)
+    oracle.attention_decode(q, kh, vh)
+    return time.perf_counter() - t0
+
+
+def slice_bytes(wl, kb, vb) -> int:
+    D = wl.head_dim
+    return wl.cached * wl.n_kv_heads * (tok_bytes(kb, D) + tok_bytes(vb, D)) + 2 * wl.n_q_heads * D * 2
+
+
+def oracle_decode_slices(wl, kb, vb, budget_s: float) -> dict:
+    """CPU baseline: the oracle timed on repeated decode steps of one
+    (layer, sequence) slice until `budget_s` seconds of work are done."""
+    sl = prepare_oracle_slice(wl, kb, vb)
+    done, secs = 0, 0.0
+    while secs < budget_s or done == 0:
+        secs += time_oracle_slice(sl, kb, vb)
+        done += 1
+    return {"value": done * slice_bytes(wl, kb, vb) / secs / 1e9, "unit": "GB/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{done} decode steps of one (layer, sequence) slice: {wl.cached} tokens x "
+                      f"{wl.n_kv_heads} KV heads x {wl.group} q heads, dequantise + attention in float64 "
+                      f"NumPy ({secs:.1f} s)"}
+
+
+# --------------------------------------------------------------------------- main
+def parse():
+    from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=[w for w in WORKLOADS if WORKLOADS[w].cached], default=DEFAULT_WORKLOAD)
+    ap.add_argument("--precision", default=None, help="K8V4, K8V8, K4V4, K4V8 or FP16 (default: first of the workload)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    a = ap.parse_args()
+    if a.warmup < 3 and a.impl == "ours":
+        ap.error("--warmup must be >= 3")
+    return a
+
+
+def config_of(wl, precision, world, flush) -> dict:
+    return {"workload": wl.name, "precision": precision, "layers": wl.n_layers, "q_heads": wl.n_q_heads,
+            "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "batch": wl.batch, "cached_tokens": wl.cached,
+            "page_tokens": 256, "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed between steps (2x L2 write)" if flush else "inputs larger than L2 (no flush)"}
+
+
+def main():
+    args = parse()
+    from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS, parse_precision
+    wl = WORKLOADS[args.workload]
+    precision = (args.precision or wl.precisions[0]).upper()
+    kb, vb = parse_precision(precision)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        sl = prepare_oracle_slice(wl, kb, vb)
+        times = [time_oracle_slice(sl, kb, vb) for _ in range(args.warmup + args.steps)][args.warmup:]
+        secs = sum(times)
+        val = args.steps * slice_bytes(wl, kb, vb) / secs / 1e9
+        line = {"metric": METRIC, "value": val, "unit": "GB/s", "impl": "reference", "n_gpus": 0,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "config": config_of(wl, precision, 1, False),
+                "cpu_baseline": {"value": val, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                                 "sample": f"each step: one (layer, sequence) slice of {wl.cached} tokens, "
+                                           f"dequantise + attention in float64 NumPy"},
+                "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from asymmetric_quantized_kv_kvq_b200 import build as kbuild
+    if rank == 0:
+        kbuild.build()
+    barrier(world)
+
+    res = run_decode_bench(args, wl, kb, vb, rank, world)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_decode_slices(wl, kb, vb, args.cpu_seconds)
+    if rank == 0:
+        peaks = measured_peaks()
+        achieved = res["dec_bytes_per_launch"] / (res["dec_ms_per_launch"] * 1e-3) / 1e9
+        traffic = ncu_traffic(wl.name, precision)
+        line = {
+            "metric": METRIC, "value": res["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_of(wl, precision, world, res["flush"]),
+            "decode_tokens_per_s": res["decode_tokens_per_s"],
+            "roofline": {"bound": "hbm", "kernel": "decode_split_kernel + lse_combine_kernel",
+                         "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                         "frac_of_8tbs_nominal": achieved / 8000.0,
+                         "bytes_per_launch": res["dec_bytes_per_launch"], "traffic": traffic},
+            "cpu_baseline": None if cpu is None else {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
+            "e2e": res.get("e2e"),
+            "clocks": res["clocks"],
+            "gpu_launches": res["launches"],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

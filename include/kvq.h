@@ -1,0 +1,213 @@
+/*
+ * kvq.h - C ABI of an asymmetric-precision quantized KV cache for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (source pages cited by title and section):
+ *
+ *  - "KVSplit - contexto 2 a 3 vezes mais longo em Apple Silicon"
+ *    (pt.news.hada.io/topic?id=20969), sections "Problema que o KVSplit tenta
+ *    resolver" and "Exemplos de uso e opcoes de CLI": keys and values of the
+ *    attention KV cache are stored at independently chosen bit widths
+ *    (--kvq-key / --kvq-val: 16, 8 or 4), e.g. K8V4 = 8-bit keys, 4-bit values.
+ *  - Same page, "Uso de memoria conforme o comprimento da sequencia": the KV
+ *    memory table is exact for 32-element blocks carrying one fp16 scale each
+ *    (34 B per 8-bit block, 18 B per 4-bit block) with 256-token page
+ *    capacity; kvq_cache_footprint / kvq_footprint_bytes reproduce it.
+ *  - Same page, Hacker News reply on .gguf compatibility: the cache is quantised
+ *    at run time as tokens are processed, independently of the weights
+ *    (kvq_append).
+ *  - Same page, "Exemplos de uso e opcoes de CLI" (--flash-attn): attention is
+ *    read through the flash-attention path (kvq_decode_attn: split-KV
+ *    flash-decoding; kvq_prefill_attn: causal chunk attention).
+ *  - "Reutilizacao de Cache KV para Conversas Longas no Apple Silicon"
+ *    (openclawradar.com), "Principais Descobertas e Benchmarks": keep the cache
+ *    resident and process only the new tokens (append a chunk, then
+ *    kvq_prefill_attn over cache + chunk).
+ *
+ * Storage format of one 32-element block along head_dim (the pages fix the
+ * byte counts; the rounding rules are this library's reading, stated exactly):
+ *    8-bit: d = fp16(fp32(amax / 127)); c_j = clamp(roundf(x_j / d), -127, 127)
+ *           (fp32 division, ties away from zero; d == 0 gives c = 0); x^ = d * c.
+ *    4-bit: m = element of largest |x| (lowest index on ties); d = fp16(m / -8);
+ *           c_j = clamp(roundf(x_j / d), -8, 7); nibble u_j = c_j + 8;
+ *           byte i (0..15) = u_i | u_{i+16} << 4; x^ = d * (u - 8).
+ *   16-bit: fp16 copy.
+ *
+ * Conventions for every call:
+ *  - Returns a kvq_status; never aborts or throws across the ABI.  Arguments
+ *    are validated on the host before anything is launched; on a validation
+ *    error nothing is modified.  Errors of earlier asynchronous work are
+ *    reported by kvq_cache_check.
+ *  - "device" pointers are CUDA global-memory addresses on the cache's device;
+ *    "host" pointers are ordinary CPU memory read during the call only.  The
+ *    caller owns every pointer it passes; the library owns the page pool,
+ *    the page table and its host bookkeeping.
+ *  - fp16 tensors are IEEE binary16, contiguous, row-major in the shapes given.
+ *  - Work is enqueued on `stream` (NULL = legacy default stream).  Calls on one
+ *    cache must be serialised by the caller (one host thread at a time, and
+ *    device work ordered on one stream or by the caller's events).
+ *  - Query head h reads KV head h / (n_q_heads / n_kv_heads).
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define KVQ_API __attribute__((visibility("default")))
+#else
+#define KVQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t (a CUDA runtime / driver stream handle). */
+typedef struct CUstream_st* kvq_stream_t;
+
+typedef enum {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,    /* bad pointer, size, id, layer or shape          */
+  KVQ_ERR_UNSUPPORTED = 2,    /* valid but not built (bit width, head_dim, ...) */
+  KVQ_ERR_OUT_OF_MEMORY = 3,  /* device or host allocation failed               */
+  KVQ_ERR_CAPACITY = 4,       /* page pool or per-sequence page table exhausted */
+  KVQ_ERR_CUDA = 5,           /* a CUDA runtime call failed                     */
+  KVQ_ERR_DEVICE_CHECK = 6,   /* a kernel gave up a bounded wait or found a bad index */
+  KVQ_ERR_WORKSPACE = 7       /* workspace missing or smaller than required     */
+} kvq_status;
+
+/* Cache geometry.  k_bits / v_bits in {16, 8, 4}; head_dim in {64, 128};
+ * page_tokens a multiple of 64 in [64, 4096] (0 selects 256); sequences are
+ * named by ids 0 .. max_seqs-1; max_tokens is the pool capacity in tokens over
+ * all sequences (rounded up to whole pages); max_seq_tokens (0 = max_tokens)
+ * bounds one sequence's length and sizes its page-table row. */
+typedef struct {
+  int32_t n_layers;
+  int32_t n_kv_heads;
+  int32_t head_dim;
+  int32_t k_bits;
+  int32_t v_bits;
+  int32_t page_tokens;
+  int32_t max_seqs;
+  int32_t flags;            /* KVQ_CACHE_* bits */
+  int64_t max_tokens;
+  int64_t max_seq_tokens;
+} kvq_cache_config;
+
+/* flags: KVQ_CACHE_HOST_ONLY creates the page bookkeeping without touching a
+ * GPU (no device memory); calls that would launch work then return
+ * KVQ_ERR_UNSUPPORTED.  Used to test the host logic on machines without a GPU. */
+#define KVQ_CACHE_HOST_ONLY 1
+
+/* Most sequences one append / decode / prefill call may name. */
+#define KVQ_MAX_BATCH 256
+
+typedef struct kvq_cache kvq_cache;
+
+/* Closed-form KV bytes of n_tokens of one sequence under cfg, over all layers:
+ * *allocated_bytes counts whole pages (the pages' table), *used_bytes counts
+ * the tokens only.  Pure host arithmetic; either output may be NULL. */
+KVQ_API kvq_status kvq_footprint_bytes(const kvq_cache_config* cfg, int64_t n_tokens,
+                               int64_t* allocated_bytes, int64_t* used_bytes);
+
+/* Create a cache on the current CUDA device: one device allocation holding
+ * every layer's pages (zero-filled), a device page table, and host
+ * bookkeeping.  *out receives the handle (NULL on error). */
+KVQ_API kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out);
+
+/* Free everything the cache owns.  Synchronises the device first.  NULL is a no-op. */
+KVQ_API kvq_status kvq_cache_destroy(kvq_cache* cache);
+
+/* Bytes of the whole pool, of the pages currently mapped to sequences, and of
+ * the tokens held (all layers).  Any output may be NULL. */
+KVQ_API kvq_status kvq_cache_footprint(const kvq_cache* cache, int64_t* pool_bytes,
+                               int64_t* mapped_bytes, int64_t* used_bytes);
+
+/* Grow sequences: for i < n_seqs, sequence seq_ids[i] gains n_new[i] >= 0
+ * token positions at its end, mapping free pages as needed (host arrays).
+ * Page-table updates are enqueued on `stream`.  The new positions hold no data
+ * until kvq_append writes them, layer by layer.  All-or-nothing: on
+ * KVQ_ERR_CAPACITY no sequence changes.  A sequence id may appear once. */
+KVQ_API kvq_status kvq_seq_extend(kvq_cache* cache, int32_t n_seqs, const int32_t* seq_ids,
+                          const int32_t* n_new, kvq_stream_t stream);
+
+/* Drop a sequence: its pages return to the pool and its length becomes 0. */
+KVQ_API kvq_status kvq_seq_release(kvq_cache* cache, int32_t seq_id);
+
+/* Current length (token positions) of a sequence. */
+KVQ_API kvq_status kvq_seq_length(const kvq_cache* cache, int32_t seq_id, int64_t* len);
+
+/* Physical page index of logical page `page` of a sequence (host bookkeeping;
+ * -1 if unmapped).  For tests of the allocator. */
+KVQ_API kvq_status kvq_seq_page(const kvq_cache* cache, int32_t seq_id, int32_t page, int32_t* phys);
+
+/* Quantise-on-append.  For i < n_seqs (host arrays seq_ids, n_new), writes the
+ * K and V of the LAST n_new[i] positions of sequence seq_ids[i] in `layer`,
+ * i.e. positions [len - n_new[i], len).  k, v: device fp16
+ * [sum_i n_new[i], n_kv_heads, head_dim], sequences' rows in call order.
+ * Quantises every 32-element block along head_dim to the cache's K / V bit
+ * widths (format above) and stores codes and scales into the sequence's pages. */
+KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                      const int32_t* n_new, const void* k, const void* v, kvq_stream_t stream);
+
+/* Workspace bytes kvq_decode_attn needs for a batch of n_seqs sequences with
+ * n_q_heads query heads (independent of lengths).  Pure host arithmetic. */
+KVQ_API kvq_status kvq_decode_workspace_size(const kvq_cache* cache, int32_t n_seqs, int32_t n_q_heads,
+                                     size_t* bytes);
+
+/* Decode attention, one query position per sequence: for i < n_seqs the query
+ * q[i] (position len-1 of sequence seq_ids[i]) attends to cache positions
+ * 0 .. len-1 of `layer`:  o = softmax(sigma * q K^T) V over the dequantised
+ * K, V, sigma = softmax_scale (0 selects 1/sqrt(head_dim)).
+ * q, out: device fp16 [n_seqs, n_q_heads, head_dim].  Split-KV flash-decoding:
+ * partial (O, max, sum) per slice of the cache in `workspace` (device,
+ * ws_bytes >= kvq_decode_workspace_size), merged by a log-sum-exp combine.
+ * Every named sequence must have len >= 1. */
+KVQ_API kvq_status kvq_decode_attn(kvq_cache* cache, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                           int32_t n_q_heads, const void* q, void* out, float softmax_scale,
+                           void* workspace, size_t ws_bytes, kvq_stream_t stream);
+
+/* Workspace bytes kvq_prefill_attn needs for these sequences (host arrays;
+ * uses their current lengths). */
+KVQ_API kvq_status kvq_prefill_workspace_size(const kvq_cache* cache, int32_t n_seqs, const int32_t* seq_ids,
+                                      const int32_t* q_lens, int32_t n_q_heads, size_t* bytes);
+
+/* Chunked prefill attention.  For i < n_seqs, sequence seq_ids[i] has a chunk
+ * of q_lens[i] >= 1 query rows at positions [len - q_lens[i], len) (already
+ * appended to the cache); row r attends causally to positions
+ * 0 .. len - q_lens[i] + r, i.e. the cached tokens and the chunk up to itself,
+ * all dequantised.  q, out: device fp16 [sum_i q_lens[i], n_q_heads, head_dim].
+ * Tensor cores (tcgen05) compute Q K^T and P V in fp16 with fp32 accumulation;
+ * the dequantised K / V are rounded to fp16 first. */
+KVQ_API kvq_status kvq_prefill_attn(kvq_cache* cache, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
+                            const int32_t* q_lens, int32_t n_q_heads, const void* q, void* out,
+                            float softmax_scale, void* workspace, size_t ws_bytes,
+                            kvq_stream_t stream);
+
+/* Copy tokens [tok0, tok0 + n_tok) of a sequence in `layer` out in canonical
+ * form (device destinations, any may be NULL to skip):
+ *   k_codes  int8 [n_tok, Hkv, D] (8-bit) | uint8 [n_tok, Hkv, D/2] (4-bit, packed
+ *            as above) | fp16 [n_tok, Hkv, D] (16-bit); v_codes likewise;
+ *   k_scales, v_scales fp16 [n_tok, Hkv, D/32] (ignored for 16-bit). */
+KVQ_API kvq_status kvq_export(const kvq_cache* cache, int32_t layer, int32_t seq_id, int64_t tok0,
+                      int64_t n_tok, void* k_codes, void* k_scales, void* v_codes, void* v_scales,
+                      kvq_stream_t stream);
+
+/* Synchronise `stream` and report errors of earlier work: KVQ_ERR_CUDA for a
+ * failed launch or runtime error, KVQ_ERR_DEVICE_CHECK if a kernel recorded a
+ * bounded-wait timeout or an out-of-range index (then *detail, if not NULL,
+ * receives the recorded code).  Clears the recorded device code. */
+KVQ_API kvq_status kvq_cache_check(kvq_cache* cache, kvq_stream_t stream, uint32_t* detail);
+
+/* Static description of a status code. */
+KVQ_API const char* kvq_status_string(kvq_status status);
+
+/* Text of the last error on this thread (a CUDA error string or a validation
+ * message); never NULL. */
+KVQ_API const char* kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVQ_H */

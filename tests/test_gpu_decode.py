@@ -1,0 +1,116 @@
+"""GPU parity: split-KV decode attention against the oracle's float64 softmax
+attention over its own dequantisation of the same fp16 inputs."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from asymmetric_quantized_kv_kvq_b200.inputs import random_fp16
+from gpu_common import kvq, decode_kv, oracle_dequant, assert_close_attention
+
+FORMATS = [(8, 4), (8, 8), (4, 4), (4, 8), (16, 16)]
+
+
+def _build(m, kb, vb, D, H, lens, layers=1, seed=0, page_tokens=256):
+    cache = m.Cache(n_layers=layers, n_kv_heads=H, head_dim=D, k_bits=kb, v_bits=vb, max_seqs=len(lens) + 1,
+                    max_tokens=sum(lens) + 256 * (len(lens) + 1), page_tokens=page_tokens)
+    ids = list(range(len(lens)))
+    cache.extend(ids, lens)
+    hat = {}
+    for layer in range(layers):
+        ks = [decode_kv(L, H, D, seed + 100 * s + layer) for s, L in enumerate(lens)]
+        vs = [random_fp16((L, H, D), seed + 7 + 100 * s + layer) for s, L in enumerate(lens)]
+        cache.append(layer, ids, lens, torch.cat(ks).cuda(), torch.cat(vs).cuda())
+        for s in ids:
+            hat[(layer, s)] = (oracle_dequant(ks[s], kb), oracle_dequant(vs[s], vb))
+    return cache, ids, hat
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("kb,vb", FORMATS)
+@pytest.mark.parametrize("D,H,G", [(64, 4, 8), (128, 8, 4), (128, 2, 2), (64, 2, 1), (128, 1, 8)])
+def test_decode_matches_oracle(kb, vb, D, H, G):
+    m = kvq()
+    lens = [1, 5, 32, 129, 300, 1000]
+    cache, ids, hat = _build(m, kb, vb, D, H, lens, layers=2)
+    for layer in range(2):
+        q = random_fp16((len(lens), H * G, D), 77 + layer)
+        out = cache.decode(layer, ids, q.cuda())
+        cache.check()
+        ref = oracle.attention_decode_batch(q.numpy(), [hat[(layer, s)] for s in ids])
+        assert_close_attention(out, ref, f"K{kb}V{vb} D{D} H{H} G{G} layer {layer}")
+    cache.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("kb,vb", [(8, 4), (16, 16)])
+def test_decode_long_sequence_spans_many_ctas(kb, vb):
+    """One long sequence: every item is split over many CTAs and merged by the combine kernel."""
+    m = kvq()
+    D, H, G = 128, 8, 4
+    lens = [20011]
+    cache, ids, hat = _build(m, kb, vb, D, H, lens)
+    q = random_fp16((1, H * G, D), 5)
+    out = cache.decode(0, ids, q.cuda())
+    cache.check()
+    ref = oracle.attention_decode_batch(q.numpy(), [hat[(0, 0)]])
+    assert_close_attention(out, ref, "long")
+    cache.close()
+
+
+@pytest.mark.gpu
+def test_decode_is_independent_of_batch_composition():
+    m = kvq()
+    D, H, G = 128, 8, 4
+    lens = [700, 3000, 45, 1]
+    cache, ids, hat = _build(m, 8, 4, D, H, lens)
+    q = random_fp16((len(lens), H * G, D), 9).cuda()
+    full = cache.decode(0, ids, q)
+    for i in ids:
+        one = cache.decode(0, [i], q[i:i + 1].contiguous())
+        assert torch.allclose(one.float(), full[i:i + 1].float(), atol=2e-3, rtol=1e-2)
+    rev = cache.decode(0, ids[::-1], q.flip(0).contiguous())
+    assert torch.allclose(rev.flip(0).float(), full.float(), atol=2e-3, rtol=1e-2)
+    cache.check()
+    cache.close()
+
+
+@pytest.mark.gpu
+def test_decode_softmax_scale_and_small_pages():
+    m = kvq()
+    D, H, G = 64, 2, 4
+    lens = [65, 200, 1]
+    cache, ids, hat = _build(m, 8, 4, D, H, lens, page_tokens=64)
+    q = random_fp16((len(lens), H * G, D), 11)
+    out = cache.decode(0, ids, q.cuda(), softmax_scale=0.05)
+    cache.check()
+    ref = oracle.attention_decode_batch(q.numpy(), [hat[(0, s)] for s in ids], scale=0.05)
+    assert_close_attention(out, ref, "scale 0.05")
+    cache.close()
+
+
+@pytest.mark.gpu
+def test_decode_after_incremental_appends():
+    """Decode step by step while tokens are appended one at a time (the serving loop)."""
+    m = kvq()
+    D, H, G = 128, 2, 4
+    cache = m.Cache(1, H, D, 8, 4, max_seqs=2, max_tokens=4096)
+    ks, vs = [], []
+    for step in range(300):
+        cache.extend([0], [1])
+        k = decode_kv(1, H, D, 300 + step)
+        v = random_fp16((1, H, D), 900 + step)
+        cache.append(0, [0], [1], k.cuda(), v.cuda())
+        ks.append(k)
+        vs.append(v)
+        if step in (0, 1, 31, 32, 255, 256, 299):
+            q = random_fp16((1, H * G, D), step)
+            out = cache.decode(0, [0], q.cuda())
+            kh = oracle_dequant(torch.cat(ks), 8)
+            vh = oracle_dequant(torch.cat(vs), 4)
+            ref = oracle.attention_decode(q[0].numpy(), kh, vh)[None]
+            assert_close_attention(out, ref, f"step {step}")
+    cache.check()
+    cache.close()

@@ -1,0 +1,176 @@
+"""Host-side tests of the C-ABI library (no GPU needed): exported symbols, the
+library's footprint closed form against the KVSplit page's table, the page
+allocator and argument validation on a host-only cache."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from asymmetric_quantized_kv_kvq_b200 import build as kbuild
+from oracle import footprint_bytes as oracle_footprint
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    kbuild.build()
+    from asymmetric_quantized_kv_kvq_b200 import kvq as m
+    m.load_library()
+    return m
+
+
+def _declared_symbols():
+    with open(os.path.join(ROOT, "include", "kvq.h")) as f:
+        text = f.read()
+    return set(re.findall(r"KVQ_API\s+[\w\s\*]+?\b(kvq_\w+)\s*\(", text))
+
+
+def test_header_symbols_are_exported(kvq):
+    declared = _declared_symbols()
+    assert len(declared) >= 17
+    lib = ctypes.CDLL(kvq.LIB_PATH)
+    for name in declared:
+        assert hasattr(lib, name), name
+    # the binding marshals exactly the declared calls
+    assert declared == set(kvq.SIGNATURES)
+
+
+def test_status_strings(kvq):
+    lib = kvq.load_library()
+    for code in range(8):
+        assert lib.kvq_status_string(code)
+    assert lib.kvq_status_string(0) == b"ok"
+
+
+BITS = {"FP16": (16, 16), "K8V8": (8, 8), "K8V4": (8, 4), "K4V8": (4, 8), "K4V4": (4, 4)}
+
+
+@pytest.mark.parametrize("cfg", list(BITS))
+@pytest.mark.parametrize("tokens", [1, 128, 255, 256, 257, 4096, 8192, 100000])
+def test_library_footprint_matches_oracle(kvq, cfg, tokens):
+    kb, vb = BITS[cfg]
+    alloc, used = kvq.footprint_bytes(22, 4, 64, kb, vb, tokens)
+    assert alloc == oracle_footprint(22, 4, 64, kb, vb, tokens)
+    assert used == 22 * tokens * (alloc // (22 * (-(-tokens // 256)) * 256))
+
+
+def test_library_footprint_reproduces_the_printed_table(kvq):
+    mib = 1 << 20
+    want = {("FP16", 8192): 176.00, ("K8V8", 8192): 93.50, ("K8V4", 8192): 71.50, ("K4V4", 8192): 49.50,
+            ("FP16", 4096): 88.00, ("K8V4", 4096): 35.75, ("K4V4", 4096): 24.75,
+            ("FP16", 128): 5.50, ("K8V4", 128): 2.23, ("K4V4", 128): 1.55}
+    for (cfg, tokens), v in want.items():
+        kb, vb = BITS[cfg]
+        assert round(kvq.footprint_bytes(22, 4, 64, kb, vb, tokens)[0] / mib, 2) == v
+
+
+def _host_cache(kvq, **kw):
+    args = dict(n_layers=2, n_kv_heads=2, head_dim=64, k_bits=8, v_bits=4, max_seqs=4, max_tokens=1024,
+                page_tokens=256, host_only=True)
+    args.update(kw)
+    return kvq.Cache(**args)
+
+
+def test_host_only_allocator(kvq):
+    c = _host_cache(kvq)
+    pool, mapped, used = c.footprint()
+    per_tok = 2 * 2 * (64 + 4 + 32 + 4)          # layers * heads * (K8 + V4 bytes)
+    assert pool == 4 * 256 * per_tok and mapped == 0 and used == 0
+    c.extend([0, 1], [1, 300])
+    assert c.length(0) == 1 and c.length(1) == 300
+    assert c.page(0, 0) == 0 and c.page(1, 0) == 1 and c.page(1, 1) == 2 and c.page(1, 2) == -1
+    assert c.footprint()[1] == 3 * 256 * per_tok
+    assert c.footprint()[2] == 301 * per_tok
+    c.extend([0], [255])                           # fills page 0 exactly
+    assert c.page(0, 1) == -1 and c.length(0) == 256
+    c.extend([0], [1])
+    assert c.page(0, 1) == 3
+    # pool exhausted: all-or-nothing
+    with pytest.raises(kvq.KvqError) as e:
+        c.extend([2, 3], [1, 1])
+    assert e.value.name == "KVQ_ERR_CAPACITY"
+    assert c.length(2) == 0 and c.length(3) == 0
+    c.release(1)
+    assert c.length(1) == 0 and c.page(1, 0) == -1
+    c.extend([2], [512])                            # reuses the two released pages
+    assert sorted([c.page(2, 0), c.page(2, 1)]) == [1, 2]
+    c.close()
+
+
+def test_max_seq_tokens_bound(kvq):
+    c = _host_cache(kvq, max_seq_tokens=300)
+    c.extend([0], [300])
+    with pytest.raises(kvq.KvqError) as e:
+        c.extend([0], [1])
+    assert e.value.name == "KVQ_ERR_CAPACITY"
+    c.close()
+
+
+@pytest.mark.parametrize("kw,name", [
+    (dict(k_bits=3), "KVQ_ERR_INVALID_ARG"),
+    (dict(head_dim=48), "KVQ_ERR_INVALID_ARG"),
+    (dict(head_dim=96), "KVQ_ERR_UNSUPPORTED"),
+    (dict(k_bits=16, v_bits=4), "KVQ_ERR_UNSUPPORTED"),
+    (dict(page_tokens=100), "KVQ_ERR_INVALID_ARG"),
+    (dict(max_seqs=0), "KVQ_ERR_INVALID_ARG"),
+    (dict(max_tokens=0), "KVQ_ERR_INVALID_ARG"),
+    (dict(n_layers=0), "KVQ_ERR_INVALID_ARG"),
+])
+def test_bad_configs(kvq, kw, name):
+    with pytest.raises(kvq.KvqError) as e:
+        _host_cache(kvq, **kw)
+    assert e.value.name == name
+
+
+def test_bad_calls_leave_the_cache_unchanged(kvq):
+    c = _host_cache(kvq)
+    c.extend([0], [10])
+    lib = kvq.load_library()
+    ids = (ctypes.c_int32 * 2)(0, 0)
+    n = (ctypes.c_int32 * 2)(1, 1)
+    assert lib.kvq_seq_extend(c._h, 2, ids, n, None) == 1          # repeated id
+    ids1 = (ctypes.c_int32 * 1)(9)
+    assert lib.kvq_seq_extend(c._h, 1, ids1, n, None) == 1         # unknown id
+    assert lib.kvq_seq_extend(c._h, 0, ids1, n, None) == 1         # empty batch
+    neg = (ctypes.c_int32 * 1)(-1)
+    ids0 = (ctypes.c_int32 * 1)(0)
+    assert lib.kvq_seq_extend(c._h, 1, ids0, neg, None) == 1       # negative count
+    assert c.length(0) == 10
+    # append: layer out of range, more new tokens than the length, NULL data
+    n11 = (ctypes.c_int32 * 1)(11)
+    one = (ctypes.c_int32 * 1)(1)
+    assert lib.kvq_append(c._h, 2, 1, ids0, one, 1, 1, None) == 1
+    assert lib.kvq_append(c._h, 0, 1, ids0, n11, 1, 1, None) == 1
+    assert lib.kvq_append(c._h, 0, 1, ids0, one, None, None, None) == 1
+    # decode: bad head grouping, GQA group not built, missing workspace, host-only
+    assert lib.kvq_decode_attn(c._h, 0, 1, ids0, 3, 16, 16, 0.0, 16, 1 << 20, None) == 1
+    assert lib.kvq_decode_attn(c._h, 0, 1, ids0, 6, 16, 16, 0.0, 16, 1 << 20, None) == 2
+    assert lib.kvq_decode_attn(c._h, 0, 1, ids0, 4, 16, 16, 0.0, None, 0, None) == 7
+    assert lib.kvq_decode_attn(c._h, 0, 1, ids0, 4, 16, 16, -1.0, 16, 1 << 20, None) == 1
+    assert lib.kvq_decode_attn(c._h, 0, 1, ids0, 4, 16, 16, 0.0, 16, 1 << 20, None) == 2
+    assert lib.kvq_decode_attn(c._h, 0, 1, ids0, 4, 8, 16, 0.0, 16, 1 << 20, None) == 1
+    # export beyond the length
+    assert lib.kvq_export(c._h, 0, 0, 5, 6, 1, 1, 1, 1, None) == 1
+    # prefill: chunk longer than the sequence
+    assert lib.kvq_prefill_attn(c._h, 0, 1, ids0, n11, 4, 1, 1, 0.0, None, 0, None) == 1
+    assert c.length(0) == 10
+    assert b"out of range" in lib.kvq_last_error() or lib.kvq_last_error()
+    c.close()
+
+
+def test_decode_workspace_is_length_independent(kvq):
+    c = _host_cache(kvq)
+    a = c.decode_workspace_size(1, 4)
+    b = c.decode_workspace_size(2, 4)
+    assert 0 < a < b
+    with pytest.raises(kvq.KvqError):
+        c.decode_workspace_size(0, 4)
+    with pytest.raises(kvq.KvqError):
+        c.decode_workspace_size(300, 4)
+    c.close()
+
+
+def test_destroy_null_is_noop(kvq):
+    assert kvq.load_library().kvq_cache_destroy(None) == 0
