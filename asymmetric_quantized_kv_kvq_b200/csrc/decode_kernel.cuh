@@ -93,6 +93,7 @@ struct DecodeArgs {
   float scale_log2;   // sigma * log2(e)
   int64_t total_chunks;
   int64_t cpc;        // chunks per CTA
+  int chunk;          // tokens per work chunk: gcd(C, page_tokens) <= C, so a chunk never crosses a page
 };
 
 struct DecodeSeg {
@@ -253,9 +254,9 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
           ok = false;
           break;
         }
-        const int tok0 = k * C;
-        const int ntok = min(C, sd.a - tok0);
-        const int ncopy = min(C, (ntok + 15) & ~15);
+        const int tok0 = k * a.chunk;
+        const int ntok = min(a.chunk, sd.a - tok0);
+        const int ncopy = min(a.chunk, (ntok + 15) & ~15);
         const int page = a.L.page_table[int64_t(sd.seq_id) * a.L.max_pages_per_seq + tok0 / a.L.page_tokens];
         if (page < 0 || page >= a.L.n_pages) {
           record_error(a.L.err, kErrBadPage);
@@ -326,7 +327,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         return;
       }
       ++it;
-      const int nvalid = min(C, sd.a - k * C);
+      const int nvalid = min(a.chunk, sd.a - k * a.chunk);
       const int nv_w = min(W, max(0, nvalid - warp * W));
       if (nv_w > 0) {
         const uint8_t* st = stages + s * T::STAGE_BYTES;

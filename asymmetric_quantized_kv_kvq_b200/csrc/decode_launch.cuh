@@ -29,6 +29,7 @@ cudaError_t launch_decode_one(const Layout& L, int layer, const Batch& b, const 
   a.scale_log2 = scale_log2;
   a.total_chunks = plan.total_chunks;
   a.cpc = plan.chunks_per_cta;
+  a.chunk = plan.chunk_tokens;
   decode_split_kernel<KB, VB, D, G><<<plan.n_cta, T::NT, T::SMEM, s>>>(a, b);
   return cudaGetLastError();
 }

@@ -78,11 +78,13 @@ def test_decode_is_independent_of_batch_composition():
 
 
 @pytest.mark.gpu
-def test_decode_softmax_scale_and_small_pages():
+@pytest.mark.parametrize("page_tokens,D", [(64, 64), (192, 64), (64, 128), (320, 128)])
+def test_decode_softmax_scale_and_small_pages(page_tokens, D):
+    """Pages smaller than (or not a multiple of) the kernel's stage: work chunks must stay inside a page."""
     m = kvq()
-    D, H, G = 64, 2, 4
-    lens = [65, 200, 1]
-    cache, ids, hat = _build(m, 8, 4, D, H, lens, page_tokens=64)
+    H, G = 2, 4
+    lens = [65, 200, 1, 700]
+    cache, ids, hat = _build(m, 8, 4, D, H, lens, page_tokens=page_tokens)
     q = random_fp16((len(lens), H * G, D), 11)
     out = cache.decode(0, ids, q.cuda(), softmax_scale=0.05)
     cache.check()
