@@ -396,6 +396,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=[w for w in WORKLOADS if WORKLOADS[w].cached], default=DEFAULT_WORKLOAD)
     ap.add_argument("--precision", default=None, help="K8V4, K8V8, K4V4, K4V8 or FP16 (default: first of the workload)")
+    ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling)")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
+    ap.add_argument("--cached", type=int, default=0, help="override the cached tokens per sequence (profiling)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -416,6 +419,10 @@ def main():
     args = parse()
     from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS, parse_precision
     wl = WORKLOADS[args.workload]
+    if args.layers or args.batch or args.cached:
+        import dataclasses
+        wl = dataclasses.replace(wl, n_layers=args.layers or wl.n_layers, batch=args.batch or wl.batch,
+                                 cached=args.cached or wl.cached)
     precision = (args.precision or wl.precisions[0]).upper()
     kb, vb = parse_precision(precision)
     rank = int(os.environ.get("RANK", 0))
