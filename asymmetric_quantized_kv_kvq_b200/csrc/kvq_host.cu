@@ -74,6 +74,11 @@ kvq_status check_config(const kvq_cache_config* c) {
 
 }  // namespace
 
+kvq_status kvq::set_last_error(kvq_status s, const char* msg) {
+  g_last_error = msg;
+  return s;
+}
+
 struct kvq_cache {
   kvq_cache_config cfg{};
   bool host_only = false;

@@ -80,6 +80,9 @@ __device__ __forceinline__ void record_error(uint32_t* err, uint32_t code) {
   atomicCAS(err, 0u, code);
 }
 
+// Sets the text kvq_last_error() returns on this thread; returns `s`.
+kvq_status set_last_error(kvq_status s, const char* msg);
+
 // ---------------------------------------------------------------------------
 // launchers (defined in the kernel translation units)
 // ---------------------------------------------------------------------------

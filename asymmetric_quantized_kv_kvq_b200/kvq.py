@@ -20,6 +20,7 @@ STATUS_NAMES = {
 }
 KVQ_CACHE_HOST_ONLY = 1
 KVQ_MAX_BATCH = 256
+KVQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class KvqError(RuntimeError):
@@ -56,6 +57,7 @@ SIGNATURES = {
     "kvq_append": (_i32, [_p, _i32, _i32, _pi32, _pi32, _p, _p, _p]),
     "kvq_decode_workspace_size": (_i32, [_p, _i32, _i32, _psz]),
     "kvq_decode_attn": (_i32, [_p, _i32, _i32, _pi32, _i32, _p, _p, _f32, _p, _sz, _p]),
+    "kvq_decode_attn_noalloc": (_i32, [_p, _i32, _i32, _pi32, _i32, _p, _p, _f32, _p]),
     "kvq_prefill_workspace_size": (_i32, [_p, _i32, _pi32, _pi32, _i32, _psz]),
     "kvq_prefill_attn": (_i32, [_p, _i32, _i32, _pi32, _pi32, _i32, _p, _p, _f32, _p, _sz, _p]),
     "kvq_export": (_i32, [_p, _i32, _i32, _i64, _i64, _p, _p, _p, _p, _p]),
@@ -223,6 +225,21 @@ class Cache:
         _check(self._lib.kvq_decode_attn(self._h, layer, B, _i32_array(seq_ids), Hq, q.data_ptr(),
                                          out.data_ptr(), softmax_scale, ws.data_ptr(),
                                          ws.numel() * ws.element_size(), _stream(stream)))
+        return out
+
+    def decode_noalloc(self, layer: int, seq_ids: Sequence[int], q, out=None, softmax_scale: float = 0.0,
+                       stream=None):
+        """kvq_decode_attn_noalloc: same result as decode(), scratch in the library's fixed array."""
+        import torch
+        B = len(seq_ids)
+        if q.dim() != 3 or q.shape[0] != B or q.shape[2] != self.head_dim:
+            raise KvqError(1, f"q has shape {tuple(q.shape)}, expected [{B}, Hq, {self.head_dim}]")
+        _dev_fp16(q, "q")
+        if out is None:
+            out = torch.empty_like(q)
+        _dev_fp16(out, "out", tuple(q.shape))
+        _check(self._lib.kvq_decode_attn_noalloc(self._h, layer, B, _i32_array(seq_ids), q.shape[1],
+                                                 q.data_ptr(), out.data_ptr(), softmax_scale, _stream(stream)))
         return out
 
     def prefill_workspace_size(self, seq_ids: Sequence[int], q_lens: Sequence[int], n_q_heads: int) -> int:

@@ -168,6 +168,28 @@ KVQ_API kvq_status kvq_decode_attn(kvq_cache* cache, int32_t layer, int32_t n_se
                            int32_t n_q_heads, const void* q, void* out, float softmax_scale,
                            void* workspace, size_t ws_bytes, kvq_stream_t stream);
 
+/* Size of the scratch array compiled into the library for
+ * kvq_decode_attn_noalloc (8 MiB per GPU that loads the library). */
+#define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* kvq_decode_attn without a workspace argument: for callers that cannot
+ * allocate device memory (a plugin inside a host application that owns all
+ * GPU memory and passes only inputs and outputs, an engine whose allocator has
+ * reserved the whole device, a serving loop that must never call cudaMalloc /
+ * cudaFree because they can synchronise the device).  The source pages have no
+ * counterpart of this call; it computes exactly what kvq_decode_attn computes.
+ * The split-KV partials go to a fixed device array of KVQ_NOALLOC_SCRATCH_BYTES
+ * inside the library instead of a caller buffer; the call allocates nothing.
+ * The first call on each device looks up that array's device address
+ * (cudaGetSymbolAddress, with the device current), so make it before any stream
+ * capture.  All calls share the array and it keeps the last call's contents:
+ * calls that overlap on the GPU race and must be ordered by the caller.
+ * Returns KVQ_ERR_WORKSPACE when kvq_decode_workspace_size for this batch
+ * exceeds KVQ_NOALLOC_SCRATCH_BYTES (nothing is launched then). */
+KVQ_API kvq_status kvq_decode_attn_noalloc(kvq_cache* cache, int32_t layer, int32_t n_seqs,
+                                           const int32_t* seq_ids, int32_t n_q_heads, const void* q,
+                                           void* out, float softmax_scale, kvq_stream_t stream);
+
 /* Workspace bytes kvq_prefill_attn needs for these sequences (host arrays;
  * uses their current lengths). */
 KVQ_API kvq_status kvq_prefill_workspace_size(const kvq_cache* cache, int32_t n_seqs, const int32_t* seq_ids,
