@@ -344,6 +344,24 @@ kvq_status kvq_seq_release(kvq_cache* c, int32_t id) {
   return KVQ_OK;
 }
 
+kvq_status kvq_seq_truncate(kvq_cache* c, int32_t id, int64_t new_len) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_seq(c, id)) return s;
+  if (new_len < 0 || new_len > c->len[id])
+    return fail(KVQ_ERR_INVALID_ARG, "new_len %lld outside [0, len = %lld]", (long long)new_len, (long long)c->len[id]);
+  const int P = c->L.page_tokens;
+  const int32_t keep = int32_t((new_len + P - 1) / P);
+  for (int32_t p = c->mapped[id] - 1; p >= keep; --p) {
+    int32_t& slot = c->table[size_t(id) * c->L.max_pages_per_seq + p];
+    c->free_pages.push_back(slot);
+    slot = -1;
+  }
+  c->mapped_pages -= c->mapped[id] - keep;
+  c->mapped[id] = keep;
+  c->len[id] = new_len;
+  return KVQ_OK;
+}
+
 kvq_status kvq_append(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, const int32_t* n_new,
                       const void* k, const void* v, kvq_stream_t stream) {
   if (kvq_status s = check_cache(c)) return s;

@@ -52,6 +52,7 @@ SIGNATURES = {
     "kvq_cache_footprint": (_i32, [_p, _pi64, _pi64, _pi64]),
     "kvq_seq_extend": (_i32, [_p, _i32, _pi32, _pi32, _p]),
     "kvq_seq_release": (_i32, [_p, _i32]),
+    "kvq_seq_truncate": (_i32, [_p, _i32, _i64]),
     "kvq_seq_length": (_i32, [_p, _i32, _pi64]),
     "kvq_seq_page": (_i32, [_p, _i32, _i32, _pi32]),
     "kvq_append": (_i32, [_p, _i32, _i32, _pi32, _pi32, _p, _p, _p]),
@@ -177,6 +178,9 @@ class Cache:
 
     def release(self, seq_id: int) -> None:
         _check(self._lib.kvq_seq_release(self._h, seq_id))
+
+    def truncate(self, seq_id: int, new_len: int) -> None:
+        _check(self._lib.kvq_seq_truncate(self._h, seq_id, new_len))
 
     def length(self, seq_id: int) -> int:
         n = ctypes.c_int64()

@@ -298,6 +298,158 @@ def run_e2e(run, args, world, dev) -> dict:
             "d2h_bytes_per_step": d2h}
 
 
+PREFILL_METRIC = "K8V4 chunked-prefill TFLOP/s (causal FLOPs) and quantise-on-append GB/s"
+
+
+class PrefillRun:
+    """Ragged sequences with cached prefixes; one step appends a chunk to every
+    sequence (quantise-on-append) and runs causal prefill of the chunk over
+    cache + chunk, then rewinds the sequences to their prefixes."""
+
+    def __init__(self, wl, kb: int, vb: int, device):
+        import torch
+        from asymmetric_quantized_kv_kvq_b200 import kvq
+        from asymmetric_quantized_kv_kvq_b200.inputs import gen_kv, gen_q_chunk, cached_lengths, GEN_CHUNK
+        self.wl, self.kb, self.vb, self.dev = wl, kb, vb, device
+        H, D, C = wl.n_kv_heads, wl.head_dim, wl.chunk
+        self.T = cached_lengths(wl)
+        n = len(self.T)
+        self.ids = list(range(n))
+        P = 256
+        cap = sum(-(-(t + C) // P) * P for t in self.T)
+        self.cache = kvq.Cache(wl.n_layers, H, D, kb, vb, max_seqs=n, max_tokens=cap, max_seq_tokens=max(self.T) + C)
+        for b, t in enumerate(self.T):
+            for c in range(-(-t // GEN_CHUNK)):
+                m = min(GEN_CHUNK, t - c * GEN_CHUNK)
+                self.cache.extend([b], [m])
+                for layer in range(wl.n_layers):
+                    k, v = gen_kv(wl, layer, b, c * GEN_CHUNK, m, device=device)
+                    self.cache.append(layer, [b], [m], k, v)
+        kv = [gen_kv(wl, 0, b, t, C, device=device) for b, t in enumerate(self.T)]
+        self.k_new = torch.cat([k for k, _ in kv]).contiguous()
+        self.v_new = torch.cat([v for _, v in kv]).contiguous()
+        self.q = torch.cat([gen_q_chunk(wl, 0, b, C, device=device) for b in self.ids]).contiguous()
+        self.out = torch.empty_like(self.q)
+        self.chunks = [C] * n
+        self.cache.extend(self.ids, self.chunks)
+        self.ws = torch.empty(self.cache.prefill_workspace_size(self.ids, self.chunks, wl.n_q_heads),
+                              dtype=torch.uint8, device=device)
+        for b, t in enumerate(self.T):
+            self.cache.truncate(b, t)
+        torch.cuda.synchronize()
+
+    def flops(self) -> float:
+        wl, C = self.wl, self.wl.chunk
+        return 4.0 * wl.n_q_heads * wl.head_dim * sum(C * t + C * (C + 1) / 2 for t in self.T)
+
+    def append_bytes(self) -> int:
+        wl = self.wl
+        D = wl.head_dim
+        per_tok = wl.n_kv_heads * (2 * D * 2 + tok_bytes(self.kb, D) + tok_bytes(self.vb, D))
+        return len(self.T) * wl.chunk * per_tok
+
+    def step(self, ev=None):
+        self.cache.extend(self.ids, self.chunks)
+        if ev is not None:
+            ev[0].record()
+        self.cache.append(0, self.ids, self.chunks, self.k_new, self.v_new)
+        if ev is not None:
+            ev[1].record()
+        self.cache.prefill(0, self.ids, self.chunks, self.q, out=self.out, workspace=self.ws)
+        if ev is not None:
+            ev[2].record()
+        for b, t in enumerate(self.T):
+            self.cache.truncate(b, t)
+
+
+def run_prefill_bench(args, wl, kb, vb, rank, world) -> dict:
+    import torch
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    t0 = time.time()
+    run = PrefillRun(wl, kb, vb, dev)
+    setup_s = time.time() - t0
+    for _ in range(args.warmup):
+        run.step()
+    run.cache.check()
+    barrier(world)
+    torch.cuda.synchronize()
+    app_ms, pre_ms, step_ms = [], [], []
+    with ClockSampler(gpu_uuid(dev)) as clk:
+        for _ in range(args.steps):
+            ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            run.step(ev)
+            torch.cuda.synchronize()
+            app_ms.append(ev[0].elapsed_time(ev[1]))
+            pre_ms.append(ev[1].elapsed_time(ev[2]))
+            step_ms.append(ev[0].elapsed_time(ev[2]))
+    barrier(world)
+    torch.cuda.synchronize()
+    run.cache.check()
+    local = sum(step_ms)
+    max_ms = all_reduce_max(local, world, dev)
+    flops = all_reduce_sum(run.flops() * args.steps, world, dev)
+    res = {"ms_per_step": max_ms / args.steps, "value": flops / (max_ms * 1e-3) / 1e12,
+           "prefill_ms": statistics.mean(pre_ms), "append_ms": statistics.mean(app_ms),
+           "prefill_tflops": run.flops() / (statistics.mean(pre_ms) * 1e-3) / 1e12,
+           "append_gbs": run.append_bytes() / (statistics.mean(app_ms) * 1e-3) / 1e9,
+           "clocks": clk.summary(), "setup_s": setup_s, "launches": args.steps * 4,
+           "cached": run.T, "flops_per_step": run.flops()}
+    if not args.no_e2e:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (run.q, run.k_new, run.v_new))
+        ho = torch.empty(run.out.shape, dtype=run.out.dtype, pin_memory=True)
+        barrier(world)
+        torch.cuda.synchronize()
+        ms = 0.0
+        for _ in range(args.steps):
+            s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s0.record()
+            run.q.copy_(hq, non_blocking=True)
+            run.k_new.copy_(hk, non_blocking=True)
+            run.v_new.copy_(hv, non_blocking=True)
+            run.step()
+            ho.copy_(run.out, non_blocking=True)
+            s1.record()
+            torch.cuda.synchronize()
+            ms += s0.elapsed_time(s1)
+        max_e = all_reduce_max(ms, world, dev)
+        res["e2e"] = {"value": flops / (max_e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in (hq, hk, hv)),
+                      "d2h_bytes_per_step": ho.numel() * ho.element_size()}
+    run.cache.close()
+    return res
+
+
+def oracle_prefill_rows(wl, kb, vb, budget_s: float) -> dict:
+    """CPU baseline for prefill: the oracle's causal attention for chunk rows of
+    one (sequence, KV head) slice (dequantise + attention in float64), timed
+    over as many rows as fit in the budget; scaled to FLOP/s."""
+    import numpy as np
+    import oracle
+    from asymmetric_quantized_kv_kvq_b200.inputs import gen_kv, gen_q_chunk, cached_lengths
+    T = cached_lengths(wl)[0]
+    C = wl.chunk
+    k, v = gen_kv(wl, 0, 0, 0, T + C)
+    kc, ks = oracle.quantize_kv(k.numpy(), kb)
+    vc, vs = oracle.quantize_kv(v.numpy(), vb)
+    q = gen_q_chunk(wl, 0, 0, C).numpy()
+    rows, secs, flops = 0, 0.0, 0.0
+    t0 = time.perf_counter()
+    kh = oracle.dequantize_kv(kc, ks, kb)
+    vh = oracle.dequantize_kv(vc, vs, vb)
+    secs += time.perf_counter() - t0
+    while secs < budget_s or rows == 0:
+        r = (rows * 997) % C
+        t0 = time.perf_counter()
+        oracle.attention_prefill(q, kh, vh, T, rows=[r])
+        secs += time.perf_counter() - t0
+        flops += 4.0 * wl.n_q_heads * wl.head_dim * (T + r + 1)
+        rows += 1
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} chunk rows (all {wl.n_q_heads} q heads) of sequence 0 (cached {T}, chunk {C}): "
+                      f"dequantise + causal attention in float64 NumPy, {secs:.1f} s"}
+
+
 # --------------------------------------------------------------------------- distributed plumbing
 def barrier(world):
     if world > 1:
@@ -394,7 +546,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=[w for w in WORKLOADS if WORKLOADS[w].cached], default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=list(WORKLOADS), default=DEFAULT_WORKLOAD)
     ap.add_argument("--precision", default=None, help="K8V4, K8V8, K4V4, K4V8 or FP16 (default: first of the workload)")
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
@@ -431,6 +583,19 @@ def main():
     if args.impl == "reference":
         if rank != 0:
             return
+        if wl.chunk:
+            r = oracle_prefill_rows(wl, kb, vb, budget_s=0.0)
+            vals = [oracle_prefill_rows(wl, kb, vb, budget_s=1.0) for _ in range(args.steps)]
+            val = statistics.mean(v["value"] for v in vals)
+            line = {"metric": PREFILL_METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference", "n_gpus": 0,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
+                    "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                    "config": {"workload": wl.name, "precision": precision},
+                    "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                                     "sample": r["sample"]},
+                    "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            print(json.dumps(line), flush=True)
+            return
         sl = prepare_oracle_slice(wl, kb, vb)
         times = [time_oracle_slice(sl, kb, vb) for _ in range(args.warmup + args.steps)][args.warmup:]
         secs = sum(times)
@@ -457,6 +622,12 @@ def main():
         kbuild.build()
     barrier(world)
 
+    if wl.chunk:
+        prefill_main(args, wl, precision, kb, vb, rank, world)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
     res = run_decode_bench(args, wl, kb, vb, rank, world)
 
     cpu = None
@@ -486,6 +657,46 @@ def main():
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def prefill_main(args, wl, precision, kb, vb, rank, world):
+    res = run_prefill_bench(args, wl, kb, vb, rank, world)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_prefill_rows(wl, kb, vb, args.cpu_seconds)
+    if rank != 0:
+        return
+    peak = measured_tensor_peak()
+    line = {
+        "metric": PREFILL_METRIC, "value": res["value"], "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f16 MMA, f32 accumulate", "data": "synthetic",
+        "config": {"workload": wl.name, "precision": precision, "layers": wl.n_layers, "q_heads": wl.n_q_heads,
+                   "kv_heads": wl.n_kv_heads, "head_dim": wl.head_dim, "sequences": wl.batch, "chunk": wl.chunk,
+                   "cached_tokens": res["cached"], "page_tokens": 256,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2 (no flush)"},
+        "prefill_tflops": res["prefill_tflops"], "append_gbs": res["append_gbs"],
+        "prefill_ms": res["prefill_ms"], "append_ms": res["append_ms"],
+        "roofline": {"bound": "tensor", "kernel": "dequant_tiles_kernel + prefill_attn_kernel",
+                     "achieved": res["prefill_tflops"], "peak": peak["value"], "unit": "TFLOP/s",
+                     "frac": res["prefill_tflops"] / peak["value"], "peak_source": peak["source"],
+                     "flops_per_launch": res["flops_per_step"], "traffic": None},
+        "cpu_baseline": cpu, "e2e": res.get("e2e"), "clocks": res["clocks"], "gpu_launches": res["launches"],
+    }
+    print(json.dumps(line), flush=True)
+
+
+def measured_tensor_peak() -> dict:
+    """Dense fp16 / bf16 tensor peak (same rate on B200): the sustained figure,
+    since one prefill launch runs tens of milliseconds of tensor work."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"value": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured bf16 dense, sustained (fp16 runs at the same rate)"}
+    return {"value": 1400.0, "source": "fallback sustained"}
 
 
 if __name__ == "__main__":

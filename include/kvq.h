@@ -135,6 +135,14 @@ KVQ_API kvq_status kvq_seq_extend(kvq_cache* cache, int32_t n_seqs, const int32_
 /* Drop a sequence: its pages return to the pool and its length becomes 0. */
 KVQ_API kvq_status kvq_seq_release(kvq_cache* cache, int32_t seq_id);
 
+/* Shorten a sequence to new_len <= its length (rewind a chunk, or keep a
+ * session's prefix and drop its last turn, as in reusing a conversation's
+ * cache and processing only the new tokens: "Reutilizacao de Cache KV para
+ * Conversas Longas no Apple Silicon", "Principais Descobertas e Benchmarks").
+ * Whole pages past new_len return to the pool.  Host bookkeeping only: the
+ * caller orders it after device work that still reads the dropped positions. */
+KVQ_API kvq_status kvq_seq_truncate(kvq_cache* cache, int32_t seq_id, int64_t new_len);
+
 /* Current length (token positions) of a sequence. */
 KVQ_API kvq_status kvq_seq_length(const kvq_cache* cache, int32_t seq_id, int64_t* len);
 

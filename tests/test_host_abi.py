@@ -99,6 +99,23 @@ def test_host_only_allocator(kvq):
     c.close()
 
 
+def test_truncate_returns_whole_pages(kvq):
+    c = _host_cache(kvq)
+    c.extend([0], [600])                         # pages 0, 1, 2
+    assert [c.page(0, i) for i in range(3)] == [0, 1, 2]
+    c.truncate(0, 300)                           # keeps 2 pages
+    assert c.length(0) == 300 and c.page(0, 2) == -1
+    c.truncate(0, 256)                           # exactly one page
+    assert c.page(0, 1) == -1 and c.page(0, 0) == 0
+    with pytest.raises(kvq.KvqError):
+        c.truncate(0, 257)                       # cannot grow
+    c.extend([0], [1])                           # the next page is the last one freed
+    assert c.page(0, 1) == 1
+    c.truncate(0, 0)
+    assert c.footprint()[1] == 0 and c.length(0) == 0
+    c.close()
+
+
 def test_max_seq_tokens_bound(kvq):
     c = _host_cache(kvq, max_seq_tokens=300)
     c.extend([0], [300])
