@@ -12,7 +12,7 @@ template <int KB, int VB>
 cudaError_t launch_decode_kv(const Layout&, int, const Batch&, const DecodePlan&, int, const void*, void*, float,
                              void*, cudaStream_t);
 template <int KB, int VB>
-int decode_chunk_tokens_kv(int D);
+int decode_chunk_tokens_kv(int D, int G);
 
 namespace {
 
@@ -53,25 +53,25 @@ size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D) {
   return slots * G * (D + 2) * sizeof(float);
 }
 
-static int stage_tokens(const Layout& L) {
+static int stage_tokens(const Layout& L, int G) {
   const int kb = L.k_bits, vb = L.v_bits, D = L.head_dim;
-  if (kb == 16) return decode_chunk_tokens_kv<16, 16>(D);
-  if (kb == 8 && vb == 8) return decode_chunk_tokens_kv<8, 8>(D);
-  if (kb == 8 && vb == 4) return decode_chunk_tokens_kv<8, 4>(D);
-  if (kb == 4 && vb == 4) return decode_chunk_tokens_kv<4, 4>(D);
-  return decode_chunk_tokens_kv<4, 8>(D);
+  if (kb == 16) return decode_chunk_tokens_kv<16, 16>(D, G);
+  if (kb == 8 && vb == 8) return decode_chunk_tokens_kv<8, 8>(D, G);
+  if (kb == 8 && vb == 4) return decode_chunk_tokens_kv<8, 4>(D, G);
+  if (kb == 4 && vb == 4) return decode_chunk_tokens_kv<4, 4>(D, G);
+  return decode_chunk_tokens_kv<4, 8>(D, G);
 }
 
 // Work chunk = gcd(stage capacity, page_tokens): both are multiples of 64, the
 // chunk divides the page, so one chunk is one contiguous range of one page.
-int decode_chunk_tokens(const Layout& L) {
-  int a = stage_tokens(L), b = L.page_tokens;
-  while (b) {
-    const int t = a % b;
-    a = b;
-    b = t;
+int decode_chunk_tokens(const Layout& L, int G) {
+  int x = stage_tokens(L, G), y = L.page_tokens;
+  while (y) {
+    const int t = x % y;
+    x = y;
+    y = t;
   }
-  return a;
+  return x;
 }
 
 cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const DecodePlan& plan, int n_q_heads,

@@ -4,5 +4,5 @@
 namespace kvq {
 template cudaError_t launch_decode_kv<4, 8>(const Layout&, int, const Batch&, const DecodePlan&, int, const void*,
                                               void*, float, void*, cudaStream_t);
-template int decode_chunk_tokens_kv<4, 8>(int);
+template int decode_chunk_tokens_kv<4, 8>(int, int);
 }  // namespace kvq

@@ -20,11 +20,19 @@
 //    shared-memory stages with 1-D TMA bulk copies (cp.async.bulk, L2
 //    evict-first) completing on the stage's "full" mbarrier;
 //  - consumers: warp w takes tokens [w*W, w*W + W) of each stage.
-//      QK: J = 16 head_dim elements per lane (LPT lanes per token), q held in
-//      registers (pre-scaled by sigma log2 e), codes converted exactly to fp32
-//      (byte permute into the mantissa of 2^23, one f32x2 subtract), f32x2
-//      FMAs, one multiply by the block scale, then a reduce-scatter across the
-//      token's lanes leaves each lane the full score of its own head(s).
+//      QK on quantized keys: integer dot products.  Each lane owns J head_dim
+//      elements (a whole 32-element block when G <= 4) of every query head of
+//      the group.  The query, pre-scaled by sigma log2 e, is held as two int8
+//      digits per element against one fp32 scale per (head, lane slice):
+//      q ~= s * (256 hi + lo), |q - s (256 hi + lo)| <= s / 2 with
+//      s = max|q| / 32512, i.e. 15-bit precision.  dp4a multiplies the stored
+//      int8 codes (4-bit codes unpacked to bytes, offset -8 folded into a
+//      per-head correction) by both digit words with exact int32
+//      accumulation; the block's scales (s * d_k) are applied once per
+//      (token, head, slice).  No code is converted to floating point.
+//      QK on fp16 keys: f32x2 FMAs on converted halves.
+//      A reduce-scatter across the token's lanes then leaves each lane the
+//      full score of its own head(s).
 //      Softmax: online, per warp, with lazy rescaling (the running max is only
 //      moved when a score exceeds it by more than 2^8).
 //      PV: 8 head_dim elements per lane; p' = p * d_v is precomputed per
@@ -43,7 +51,8 @@ namespace kvq {
 
 template <int KB, int VB, int D, int G>
 struct DecodeTraits {
-  static constexpr int NW = G == 8 ? 4 : 8;              // consumer warps
+  static constexpr bool INT_QK = KB != 16;              // dp4a path for quantized keys
+  static constexpr int NW = G == 8 ? 4 : 8;              // consumer warps (8 heads of state need the registers)
   static constexpr int NT = (NW + 1) * 32;
   static constexpr int NB = D / 32;
   static constexpr int K_ROW = KB == 16 ? 2 * D : KB == 8 ? D : D / 2;
@@ -53,7 +62,7 @@ struct DecodeTraits {
   static constexpr int TOK_BYTES = K_ROW + KS_ROW + V_ROW + VS_ROW;
   static constexpr int C = TOK_BYTES <= 128 ? 256 : TOK_BYTES <= 320 ? 128 : 64;
   static constexpr int W = C / NW;
-  static constexpr int J = 16;
+  static constexpr int J = (INT_QK && G <= 4) ? 32 : 16;   // head_dim elements per lane in QK
   static constexpr int LPT = D / J;
   static constexpr int TPS = 32 / LPT;
   static constexpr int NJ = W / TPS;
@@ -122,6 +131,36 @@ __device__ __forceinline__ int k_elem(int slice, int i) {
   if (KB == 8) return 16 * slice + i;
   if (KB == 4) return 32 * (slice >> 1) + 8 * (slice & 1) + (i < 8 ? i : i + 8);
   return i < 8 ? 8 * slice + i : D / 2 + 8 * slice + (i - 8);
+}
+
+// Integer QK path: element index of digit i (0 .. J-1) of lane `slice`, and the
+// lane's code words in the same order (4-bit codes unpacked to one byte each,
+// values 0..15, read as non-negative int8 by dp4a).
+template <int KB, int J>
+__device__ __forceinline__ int kq_elem(int slice, int i) {
+  if (KB == 8) return J * slice + i;
+  if (J == 32) return 32 * slice + i;          // whole block: low nibbles 0..15, high nibbles 16..31
+  return 32 * (slice >> 1) + 8 * (slice & 1) + (i < 8 ? i : i + 8);
+}
+template <int KB, int J>
+__device__ __forceinline__ void load_kcodes(const uint8_t* row, int slice, uint32_t (&cw)[J / 4]) {
+  if (KB == 8) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + J * slice);
+    cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
+    if constexpr (J == 32) {
+      const uint4 c = *reinterpret_cast<const uint4*>(row + J * slice + 16);
+      cw[4] = c.x; cw[5] = c.y; cw[6] = c.z; cw[7] = c.w;
+    }
+  } else if constexpr (J == 32) {
+    const uint4 a = *reinterpret_cast<const uint4*>(row + 16 * slice);
+    cw[0] = a.x & 0x0F0F0F0Fu; cw[1] = a.y & 0x0F0F0F0Fu; cw[2] = a.z & 0x0F0F0F0Fu; cw[3] = a.w & 0x0F0F0F0Fu;
+    cw[4] = (a.x >> 4) & 0x0F0F0F0Fu; cw[5] = (a.y >> 4) & 0x0F0F0F0Fu;
+    cw[6] = (a.z >> 4) & 0x0F0F0F0Fu; cw[7] = (a.w >> 4) & 0x0F0F0F0Fu;
+  } else {
+    const uint2 a = *reinterpret_cast<const uint2*>(row + 16 * (slice >> 1) + 8 * (slice & 1));
+    cw[0] = a.x & 0x0F0F0F0Fu; cw[1] = a.y & 0x0F0F0F0Fu;
+    cw[2] = (a.x >> 4) & 0x0F0F0F0Fu; cw[3] = (a.y >> 4) & 0x0F0F0F0Fu;
+  }
 }
 
 // Load and convert the lane's 16 K values of one row (exact integers or fp16 values).
@@ -203,7 +242,7 @@ template <int KB, int VB, int D, int G>
 __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
     decode_split_kernel(const DecodeArgs a, const __grid_constant__ Batch b) {
   using T = DecodeTraits<KB, VB, D, G>;
-  constexpr int S = T::S, C = T::C, W = T::W, NW = T::NW;
+  constexpr int S = T::S, W = T::W, NW = T::NW;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
   float2* pbuf = reinterpret_cast<float2*>(smem + S * T::STAGE_BYTES);
@@ -296,15 +335,50 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
     const int item = sg.bi * H + sg.h;
 
     // q slice in registers, pre-scaled by sigma * log2(e)
-    float2 qp[G][8];
+    float2 qp[T::INT_QK ? 1 : G][8];          // fp16-key path: fp32 pairs
+    uint32_t qh[T::INT_QK ? G : 1][T::J / 4], ql[T::INT_QK ? G : 1][T::J / 4];   // integer path: digit words
+    float qsc[G];
+    int qcorr[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       const __half* qrow = a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + g) * D;
+      if constexpr (T::INT_QK) {
+        float qv[T::J];
+        float amax = 0.f;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float e0 = __half2float(qrow[k_elem<KB, D>(slice, 2 * i)]);
-        const float e1 = __half2float(qrow[k_elem<KB, D>(slice, 2 * i + 1)]);
-        qp[g][i] = make_float2(e0 * a.scale_log2, e1 * a.scale_log2);
+        for (int i = 0; i < T::J; ++i) {
+          qv[i] = __half2float(qrow[kq_elem<KB, T::J>(slice, i)]) * a.scale_log2;
+          amax = fmaxf(amax, fabsf(qv[i]));
+        }
+        const float inv = amax > 0.f ? 32512.f / amax : 0.f;
+        qsc[g] = amax * (1.f / 32512.f);
+        int corr = 0;
+#pragma unroll
+        for (int k = 0; k < T::J / 4; ++k) {
+          uint32_t hw = 0, lw = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            int n = __float2int_rn(qv[4 * k + e] * inv);
+            n = max(-32512, min(32512, n));
+            const int lo = ((n + 128) & 255) - 128;
+            const int hi = (n - lo) >> 8;
+            hw |= uint32_t(hi & 255) << (8 * e);
+            lw |= uint32_t(lo & 255) << (8 * e);
+            corr += n;
+          }
+          qh[g][k] = hw;
+          ql[g][k] = lw;
+        }
+        qcorr[g] = KB == 4 ? 8 * corr : 0;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float e0 = __half2float(qrow[k_elem<KB, D>(slice, 2 * i)]);
+          const float e1 = __half2float(qrow[k_elem<KB, D>(slice, 2 * i + 1)]);
+          qp[g][i] = make_float2(e0 * a.scale_log2, e1 * a.scale_log2);
+        }
+        qsc[g] = 1.f;
+        qcorr[g] = 0;
       }
     }
     float2 O[G][4];
@@ -338,44 +412,58 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         for (int j = 0; j < T::NJ; ++j) {
           const int t = j * T::TPS + tis;
           const int row = row0 + t;
-          float2 kf[8];
-          load_k16<KB, D>(st + row * T::K_ROW, slice, kf);
           float part[G];
+          if constexpr (T::INT_QK) {
+            uint32_t cw[T::J / 4];
+            load_kcodes<KB, T::J>(st + row * T::K_ROW, slice, cw);
+            const float dk = __half2float(
+                reinterpret_cast<const __half*>(st + T::OFF_KS + row * T::KS_ROW)[(slice * T::J) >> 5]);
+            int hs[G], ls[G];
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
-            float2 acc = make_float2(0.f, 0.f);
+            for (int g = 0; g < G; ++g) hs[g] = ls[g] = 0;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) acc = ffma2(qp[g][i], kf[i], acc);
-            part[g] = acc.x + acc.y;
-          }
-          if (KB != 16) {
-            const float dk =
-                __half2float(reinterpret_cast<const __half*>(st + T::OFF_KS + row * T::KS_ROW)[slice >> 1]);
+            for (int q = 0; q < T::J / 4; ++q) {        // 2G independent dp4a chains, interleaved
 #pragma unroll
-            for (int g = 0; g < G; ++g) part[g] *= dk;
+              for (int g = 0; g < G; ++g) {
+                hs[g] = __dp4a(int(cw[q]), int(qh[g][q]), hs[g]);
+                ls[g] = __dp4a(int(cw[q]), int(ql[g][q]), ls[g]);
+              }
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) part[g] = __int2float_rn(hs[g] * 256 + ls[g] - qcorr[g]) * (qsc[g] * dk);
+          } else {
+            float2 kf[8];
+            load_k16<KB, D>(st + row * T::K_ROW, slice, kf);
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+              float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) acc = ffma2(qp[g][i], kf[i], acc);
+              part[g] = acc.x + acc.y;
+            }
           }
           reduce_scatter<G, T::LPT>(part, lane);
 #pragma unroll
           for (int gi = 0; gi < T::GPL; ++gi) sc[j][gi] = t < nv_w ? part[gi] : -INFINITY;
         }
-        // ---- online softmax (max moved lazily)
-        float tmax[T::GPL];
+        // ---- online softmax, max moved lazily: a vote decides whether any score
+        //      exceeds the running max by more than 2^8; only then is the exact
+        //      tile max reduced across lanes and O, l rescaled
         bool need = false;
 #pragma unroll
-        for (int gi = 0; gi < T::GPL; ++gi) {
-          float mx = sc[0][gi];
+        for (int gi = 0; gi < T::GPL; ++gi)
 #pragma unroll
-          for (int j = 1; j < T::NJ; ++j) mx = fmaxf(mx, sc[j][gi]);
-#pragma unroll
-          for (int o = T::LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-          tmax[gi] = mx;
-          need |= mx > m_own[gi] + 8.f;
-        }
+          for (int j = 0; j < T::NJ; ++j) need |= sc[j][gi] > m_own[gi] + 8.f;
         if (__any_sync(0xffffffffu, need)) {
           float alpha[T::GPL];
 #pragma unroll
           for (int gi = 0; gi < T::GPL; ++gi) {
-            const float mn = fmaxf(m_own[gi], tmax[gi]);
+            float mx = sc[0][gi];
+#pragma unroll
+            for (int j = 1; j < T::NJ; ++j) mx = fmaxf(mx, sc[j][gi]);
+#pragma unroll
+            for (int o = T::LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            const float mn = fmaxf(m_own[gi], mx);
             alpha[gi] = exp2f(m_own[gi] - mn);
             m_own[gi] = mn;
             l_own[gi] *= alpha[gi];
@@ -393,9 +481,21 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         for (int j = 0; j < T::NJ; ++j) {
           const int t = j * T::TPS + tis;
           const int row = row0 + t;
+          float dv[T::NBP];
+          if constexpr (VB != 16) {
+            const __half* vs = reinterpret_cast<const __half*>(st + T::OFF_VS + row * T::VS_ROW);
+            if constexpr (T::NBP == 4) {
+              const uint2 w = *reinterpret_cast<const uint2*>(vs);
+              const float2 a0 = h2_to_f2(w.x), a1 = h2_to_f2(w.y);
+              dv[0] = a0.x; dv[1] = a0.y; dv[2] = a1.x; dv[3] = a1.y;
+            } else {
+              const float2 a0 = h2_to_f2(*reinterpret_cast<const uint32_t*>(vs));
+              dv[0] = a0.x; dv[1] = a0.y;
+            }
+          }
 #pragma unroll
           for (int gi = 0; gi < T::GPL; ++gi) {
-            const float p = exp2f(sc[j][gi] - m_own[gi]);
+            const float p = exp2f(sc[j][gi] - m_own[gi]);   // 0 for masked tokens
             l_own[gi] += p;
             if (VB == 16) {
               if (rep == 0) pw[t * G + g0 + gi] = make_float2(p, p);
@@ -404,9 +504,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
               for (int bb = 0; bb < T::NBP; bb += T::REP) {
                 const int blk = bb + rep;
                 if (blk < T::NBP) {
-                  const float dv =
-                      __half2float(reinterpret_cast<const __half*>(st + T::OFF_VS + row * T::VS_ROW)[blk]);
-                  const float pv = t < nv_w ? p * dv : 0.f;
+                  const float pv = p * dv[blk < T::NBP ? blk : 0];
                   pw[(t * T::NBP + blk) * G + g0 + gi] = make_float2(pv, pv);
                 }
               }

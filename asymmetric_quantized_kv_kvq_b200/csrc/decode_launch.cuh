@@ -46,9 +46,15 @@ cudaError_t launch_decode_kv(const Layout& L, int layer, const Batch& b, const D
   return cudaErrorInvalidValue;
 }
 
+// Tokens per work chunk of the kernel that runs for (D, G).
 template <int KB, int VB>
-int decode_chunk_tokens_kv(int D) {
-  return D == 128 ? DecodeTraits<KB, VB, 128, 4>::C : DecodeTraits<KB, VB, 64, 4>::C;
+int decode_chunk_tokens_kv(int D, int G) {
+#define KVQ_C(D_, G_) \
+  if (D == D_ && G == G_) return DecodeTraits<KB, VB, D_, G_>::C;
+  KVQ_C(128, 1) KVQ_C(128, 2) KVQ_C(128, 4) KVQ_C(128, 8)
+  KVQ_C(64, 1) KVQ_C(64, 2) KVQ_C(64, 4) KVQ_C(64, 8)
+#undef KVQ_C
+  return 0;
 }
 
 }  // namespace kvq

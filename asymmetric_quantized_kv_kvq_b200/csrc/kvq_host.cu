@@ -414,7 +414,7 @@ kvq_status kvq_decode_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_t
   if (kvq_status s = need_device(c)) return s;
 
   kvq::DecodePlan plan;
-  plan.chunk_tokens = kvq::decode_chunk_tokens(c->L);
+  plan.chunk_tokens = kvq::decode_chunk_tokens(c->L, G);
   const int C = plan.chunk_tokens, H = c->L.n_kv_heads;
   kvq::Batch b;
   b.n = n;

@@ -107,7 +107,7 @@ struct DecodePlan {
 // decode: workspace = partial slots [(max_ctas + n_items)][G][D + 2] fp32
 size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D);
 int decode_max_ctas(int num_sms);
-int decode_chunk_tokens(const Layout& L);
+int decode_chunk_tokens(const Layout& L, int G);
 cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const DecodePlan& plan,
                           int n_q_heads, const void* q, void* out, float scale_log2,
                           void* workspace, cudaStream_t s);
