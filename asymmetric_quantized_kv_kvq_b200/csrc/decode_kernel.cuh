@@ -60,7 +60,7 @@ struct DecodeTraits {
   static constexpr int KS_ROW = KB == 16 ? 0 : NB * 2;
   static constexpr int VS_ROW = VB == 16 ? 0 : NB * 2;
   static constexpr int TOK_BYTES = K_ROW + KS_ROW + V_ROW + VS_ROW;
-  static constexpr int C = TOK_BYTES <= 128 ? 256 : TOK_BYTES <= 320 ? 128 : 64;
+  static constexpr int C = TOK_BYTES <= 320 ? 256 : 64;   // tokens per stage (W = C / NW per warp)
   static constexpr int W = C / NW;
   static constexpr int J = (INT_QK && G <= 4) ? 32 : 16;   // head_dim elements per lane in QK
   static constexpr int LPT = D / J;
@@ -211,6 +211,14 @@ __device__ __forceinline__ void load_v8(const uint8_t* row, int vs, float2 (&vf)
     const uint4 w = *reinterpret_cast<const uint4*>(row + 16 * vs);
     vf[0] = h2_to_f2(w.x); vf[1] = h2_to_f2(w.y); vf[2] = h2_to_f2(w.z); vf[3] = h2_to_f2(w.w);
   }
+}
+
+// Index of the (token, V block) group of G p' pairs in a warp's buffer: the
+// block index is XOR-swizzled by the token so that the p' stores of the tokens
+// of a step fall in different banks.
+template <int NBP>
+__device__ __forceinline__ int pgroup(int t, int blk) {
+  return t * NBP + (blk ^ (t & (NBP - 1)));
 }
 
 // Reduce-scatter of G partial sums over the LPT lanes of one token (lanes
@@ -505,7 +513,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
                 const int blk = bb + rep;
                 if (blk < T::NBP) {
                   const float pv = p * dv[blk < T::NBP ? blk : 0];
-                  pw[(t * T::NBP + blk) * G + g0 + gi] = make_float2(pv, pv);
+                  pw[pgroup<T::NBP>(t, blk) * G + g0 + gi] = make_float2(pv, pv);
                 }
               }
             }
@@ -519,7 +527,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
           if (t < nv_w) {
             float2 vf[4];
             load_v8<VB>(st + T::OFF_VC + (row0 + t) * T::V_ROW, vsl, vf);
-            const float2* pp = pw + (t * T::NBP + v_block<VB>(vsl)) * G;
+            const float2* pp = pw + pgroup<T::NBP>(t, v_block<VB>(vsl)) * G;
 #pragma unroll
             for (int g = 0; g < G; g += 2) {
               float2 p0, p1;
