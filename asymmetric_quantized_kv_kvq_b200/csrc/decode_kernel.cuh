@@ -19,10 +19,13 @@
 //    scales (four contiguous ranges of one page's head block) into a ring of S
 //    shared-memory stages with 1-D TMA bulk copies (cp.async.bulk, L2
 //    evict-first) completing on the stage's "full" mbarrier;
-//  - consumers: warp w takes tokens [w*W, w*W + W) of each stage.
-//      QK on quantized keys: integer dot products.  Each lane owns J head_dim
-//      elements (a whole 32-element block when G <= 4) of every query head of
-//      the group.  The query, pre-scaled by sigma log2 e, is held as two int8
+//  - consumers: the NW warps form NG = G / GW head groups of NTW warps; a
+//    warp holds the state of GW <= 4 query heads (more would not fit its
+//    registers) and takes tokens [tw*W, tw*W + W) of each stage, tw being its
+//    slot in the group, so with 8 query heads per KV head two warps read every
+//    token, each for its 4 heads.
+//      QK on quantized keys: integer dot products.  Each lane owns a whole
+//      32-element block of every query head of the warp.  The query, pre-scaled by sigma log2 e, is held as two int8
 //      digits per element against one fp32 scale per (head, lane slice):
 //      q ~= s * (256 hi + lo), |q - s (256 hi + lo)| <= s / 2 with
 //      s = max|q| / 32512, i.e. 15-bit precision.  dp4a multiplies the stored
@@ -52,7 +55,10 @@ namespace kvq {
 template <int KB, int VB, int D, int G>
 struct DecodeTraits {
   static constexpr bool INT_QK = KB != 16;              // dp4a path for quantized keys
-  static constexpr int NW = G == 8 ? 4 : 8;              // consumer warps (8 heads of state need the registers)
+  static constexpr int GW = G > 4 ? 4 : G;               // query heads whose state one warp holds
+  static constexpr int NG = G / GW;                      // head groups (warps of different groups read the same tokens)
+  static constexpr int NW = 8;                           // consumer warps
+  static constexpr int NTW = NW / NG;                    // warps that split the tokens of a stage
   static constexpr int NT = (NW + 1) * 32;
   static constexpr int NB = D / 32;
   static constexpr int K_ROW = KB == 16 ? 2 * D : KB == 8 ? D : D / 2;
@@ -60,14 +66,14 @@ struct DecodeTraits {
   static constexpr int KS_ROW = KB == 16 ? 0 : NB * 2;
   static constexpr int VS_ROW = VB == 16 ? 0 : NB * 2;
   static constexpr int TOK_BYTES = K_ROW + KS_ROW + V_ROW + VS_ROW;
-  static constexpr int C = TOK_BYTES <= 320 ? 256 : 64;   // tokens per stage (W = C / NW per warp)
-  static constexpr int W = C / NW;
-  static constexpr int J = (INT_QK && G <= 4) ? 32 : 16;   // head_dim elements per lane in QK
+  static constexpr int C = TOK_BYTES <= 320 ? 256 / NG : 64;   // tokens per stage (W = C / NTW per warp)
+  static constexpr int W = C / NTW;
+  static constexpr int J = INT_QK ? 32 : 16;             // head_dim elements per lane in QK
   static constexpr int LPT = D / J;
   static constexpr int TPS = 32 / LPT;
   static constexpr int NJ = W / TPS;
-  static constexpr int GPL = G > LPT ? G / LPT : 1;
-  static constexpr int REP = G < LPT ? LPT / G : 1;
+  static constexpr int GPL = GW > LPT ? GW / LPT : 1;
+  static constexpr int REP = GW < LPT ? LPT / GW : 1;
   static constexpr int LPV = D / 8;
   static constexpr int TPV = 32 / LPV;
   static constexpr int NPV = W / TPV;
@@ -76,9 +82,9 @@ struct DecodeTraits {
   static constexpr int OFF_VC = OFF_KS + C * KS_ROW;
   static constexpr int OFF_VS = OFF_VC + C * V_ROW;
   static constexpr int STAGE_BYTES = OFF_VS + C * VS_ROW;
-  static constexpr int PBUF_BYTES = NW * W * NBP * G * 8;
-  static constexpr int MRG_O_BYTES = NW * G * D * 4;
-  static constexpr int MRG_ML_BYTES = NW * G * 2 * 4;
+  static constexpr int PBUF_BYTES = NW * W * NBP * GW * 8;
+  static constexpr int MRG_O_BYTES = NTW * G * D * 4;
+  static constexpr int MRG_ML_BYTES = NTW * G * 2 * 4;
   static constexpr int BAR_BYTES = 256;
   static constexpr int FIXED = PBUF_BYTES + MRG_O_BYTES + MRG_ML_BYTES + BAR_BYTES;
   static constexpr int SMEM_LIMIT = 227 * 1024;
@@ -250,12 +256,12 @@ template <int KB, int VB, int D, int G>
 __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
     decode_split_kernel(const DecodeArgs a, const __grid_constant__ Batch b) {
   using T = DecodeTraits<KB, VB, D, G>;
-  constexpr int S = T::S, W = T::W, NW = T::NW;
+  constexpr int S = T::S, W = T::W, NW = T::NW, GW = T::GW, NTW = T::NTW;
   extern __shared__ __align__(128) uint8_t smem[];
   uint8_t* stages = smem;
   float2* pbuf = reinterpret_cast<float2*>(smem + S * T::STAGE_BYTES);
   float* mrg_o = reinterpret_cast<float*>(smem + S * T::STAGE_BYTES + T::PBUF_BYTES);
-  float* mrg_ml = mrg_o + NW * G * D;
+  float* mrg_ml = mrg_o + NTW * G * D;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * T::STAGE_BYTES + T::PBUF_BYTES + T::MRG_O_BYTES +
                                                T::MRG_ML_BYTES);
   // bars[0..S) full, [S..2S) empty, [2S] merge-full, [2S+1] merge-free, then the abort flag
@@ -332,6 +338,8 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
   // ------------------------------------------------------------------ consumers
   const int slice = lane % T::LPT, tis = lane / T::LPT;
   const int vsl = lane % T::LPV, tslot = lane / T::LPV;
+  const int hg = warp / NTW, tw = warp % NTW;     // head group, token slot of this warp
+  const int gb = hg * GW;                          // first query head of the group
   const int g0 = (slice / T::REP) * T::GPL;
   const int rep = slice % T::REP;
   const int ct = warp * 32 + lane;
@@ -343,13 +351,13 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
     const int item = sg.bi * H + sg.h;
 
     // q slice in registers, pre-scaled by sigma * log2(e)
-    float2 qp[T::INT_QK ? 1 : G][8];          // fp16-key path: fp32 pairs
-    uint32_t qh[T::INT_QK ? G : 1][T::J / 4], ql[T::INT_QK ? G : 1][T::J / 4];   // integer path: digit words
-    float qsc[G];
-    int qcorr[G];
+    float2 qp[T::INT_QK ? 1 : GW][8];          // fp16-key path: fp32 pairs
+    uint32_t qh[T::INT_QK ? GW : 1][T::J / 4], ql[T::INT_QK ? GW : 1][T::J / 4];   // integer path: digit words
+    float qsc[GW];
+    int qcorr[GW];
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const __half* qrow = a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + g) * D;
+    for (int g = 0; g < GW; ++g) {
+      const __half* qrow = a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + gb + g) * D;
       if constexpr (T::INT_QK) {
         float qv[T::J];
         float amax = 0.f;
@@ -389,9 +397,9 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         qcorr[g] = 0;
       }
     }
-    float2 O[G][4];
+    float2 O[GW][4];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+    for (int g = 0; g < GW; ++g)
 #pragma unroll
       for (int k = 0; k < 4; ++k) O[g][k] = make_float2(0.f, 0.f);
     float m_own[T::GPL], l_own[T::GPL];
@@ -410,47 +418,47 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
       }
       ++it;
       const int nvalid = min(a.chunk, sd.a - k * a.chunk);
-      const int nv_w = min(W, max(0, nvalid - warp * W));
+      const int nv_w = min(W, max(0, nvalid - tw * W));
       if (nv_w > 0) {
         const uint8_t* st = stages + s * T::STAGE_BYTES;
-        const int row0 = warp * W;
+        const int row0 = tw * W;
         // ---- scores
         float sc[T::NJ][T::GPL];
 #pragma unroll
         for (int j = 0; j < T::NJ; ++j) {
           const int t = j * T::TPS + tis;
           const int row = row0 + t;
-          float part[G];
+          float part[GW];
           if constexpr (T::INT_QK) {
             uint32_t cw[T::J / 4];
             load_kcodes<KB, T::J>(st + row * T::K_ROW, slice, cw);
             const float dk = __half2float(
                 reinterpret_cast<const __half*>(st + T::OFF_KS + row * T::KS_ROW)[(slice * T::J) >> 5]);
-            int hs[G], ls[G];
+            int hs[GW], ls[GW];
 #pragma unroll
-            for (int g = 0; g < G; ++g) hs[g] = ls[g] = 0;
+            for (int g = 0; g < GW; ++g) hs[g] = ls[g] = 0;
 #pragma unroll
-            for (int q = 0; q < T::J / 4; ++q) {        // 2G independent dp4a chains, interleaved
+            for (int q = 0; q < T::J / 4; ++q) {        // 2 GW independent dp4a chains, interleaved
 #pragma unroll
-              for (int g = 0; g < G; ++g) {
+              for (int g = 0; g < GW; ++g) {
                 hs[g] = __dp4a(int(cw[q]), int(qh[g][q]), hs[g]);
                 ls[g] = __dp4a(int(cw[q]), int(ql[g][q]), ls[g]);
               }
             }
 #pragma unroll
-            for (int g = 0; g < G; ++g) part[g] = __int2float_rn(hs[g] * 256 + ls[g] - qcorr[g]) * (qsc[g] * dk);
+            for (int g = 0; g < GW; ++g) part[g] = __int2float_rn(hs[g] * 256 + ls[g] - qcorr[g]) * (qsc[g] * dk);
           } else {
             float2 kf[8];
             load_k16<KB, D>(st + row * T::K_ROW, slice, kf);
 #pragma unroll
-            for (int g = 0; g < G; ++g) {
+            for (int g = 0; g < GW; ++g) {
               float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
               for (int i = 0; i < 8; ++i) acc = ffma2(qp[g][i], kf[i], acc);
               part[g] = acc.x + acc.y;
             }
           }
-          reduce_scatter<G, T::LPT>(part, lane);
+          reduce_scatter<GW, T::LPT>(part, lane);
 #pragma unroll
           for (int gi = 0; gi < T::GPL; ++gi) sc[j][gi] = t < nv_w ? part[gi] : -INFINITY;
         }
@@ -477,14 +485,14 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
             l_own[gi] *= alpha[gi];
           }
 #pragma unroll
-          for (int g = 0; g < G; ++g) {
+          for (int g = 0; g < GW; ++g) {
             const float al = __shfl_sync(0xffffffffu, alpha[g % T::GPL], (g / T::GPL) * T::REP);
 #pragma unroll
             for (int k = 0; k < 4; ++k) O[g][k] = fmul2(O[g][k], make_float2(al, al));
           }
         }
         // ---- p and p' = p * d_v (duplicated pairs) into the warp's buffer
-        float2* pw = pbuf + size_t(warp) * W * T::NBP * G;
+        float2* pw = pbuf + size_t(warp) * W * T::NBP * GW;
 #pragma unroll
         for (int j = 0; j < T::NJ; ++j) {
           const int t = j * T::TPS + tis;
@@ -506,14 +514,14 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
             const float p = exp2f(sc[j][gi] - m_own[gi]);   // 0 for masked tokens
             l_own[gi] += p;
             if (VB == 16) {
-              if (rep == 0) pw[t * G + g0 + gi] = make_float2(p, p);
+              if (rep == 0) pw[t * GW + g0 + gi] = make_float2(p, p);
             } else {
 #pragma unroll
               for (int bb = 0; bb < T::NBP; bb += T::REP) {
                 const int blk = bb + rep;
                 if (blk < T::NBP) {
                   const float pv = p * dv[blk < T::NBP ? blk : 0];
-                  pw[pgroup<T::NBP>(t, blk) * G + g0 + gi] = make_float2(pv, pv);
+                  pw[pgroup<T::NBP>(t, blk) * GW + g0 + gi] = make_float2(pv, pv);
                 }
               }
             }
@@ -527,12 +535,12 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
           if (t < nv_w) {
             float2 vf[4];
             load_v8<VB>(st + T::OFF_VC + (row0 + t) * T::V_ROW, vsl, vf);
-            const float2* pp = pw + pgroup<T::NBP>(t, v_block<VB>(vsl)) * G;
+            const float2* pp = pw + pgroup<T::NBP>(t, v_block<VB>(vsl)) * GW;
 #pragma unroll
-            for (int g = 0; g < G; g += 2) {
+            for (int g = 0; g < GW; g += 2) {
               float2 p0, p1;
               (void)p1;
-              if constexpr (G >= 2) {
+              if constexpr (GW >= 2) {
                 const float4 pq = *reinterpret_cast<const float4*>(pp + g);
                 p0 = make_float2(pq.x, pq.y);
                 p1 = make_float2(pq.z, pq.w);
@@ -557,7 +565,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
 #pragma unroll
     for (int o = T::LPV; o < 32; o <<= 1)
 #pragma unroll
-      for (int g = 0; g < G; ++g)
+      for (int g = 0; g < GW; ++g)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           O[g][k].x += __shfl_xor_sync(0xffffffffu, O[g][k].x, o);
@@ -575,18 +583,18 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
     }
     if (tslot == 0) {
 #pragma unroll
-      for (int g = 0; g < G; ++g)
+      for (int g = 0; g < GW; ++g)
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          mrg_o[(warp * G + g) * D + v_elem<VB>(vsl, 2 * k)] = O[g][k].x;
-          mrg_o[(warp * G + g) * D + v_elem<VB>(vsl, 2 * k + 1)] = O[g][k].y;
+          mrg_o[(tw * G + gb + g) * D + v_elem<VB>(vsl, 2 * k)] = O[g][k].x;
+          mrg_o[(tw * G + gb + g) * D + v_elem<VB>(vsl, 2 * k + 1)] = O[g][k].y;
         }
     }
     if (tis == 0 && rep == 0) {
 #pragma unroll
       for (int gi = 0; gi < T::GPL; ++gi) {
-        mrg_ml[(warp * G + g0 + gi) * 2] = m_own[gi];
-        mrg_ml[(warp * G + g0 + gi) * 2 + 1] = l_own[gi];
+        mrg_ml[(tw * G + gb + g0 + gi) * 2] = m_own[gi];
+        mrg_ml[(tw * G + gb + g0 + gi) * 2 + 1] = l_own[gi];
       }
     }
     __syncwarp();
@@ -603,10 +611,10 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
       const int g = e / D, d = e % D;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) M = fmaxf(M, mrg_ml[(w * G + g) * 2]);
+      for (int w = 0; w < NTW; ++w) M = fmaxf(M, mrg_ml[(w * G + g) * 2]);
       float acc = 0.f, L = 0.f;
 #pragma unroll
-      for (int w = 0; w < NW; ++w) {
+      for (int w = 0; w < NTW; ++w) {
         const float f = exp2f(mrg_ml[(w * G + g) * 2] - M);
         acc += f * mrg_o[(w * G + g) * D + d];
         L += f * mrg_ml[(w * G + g) * 2 + 1];
