@@ -14,6 +14,11 @@ cudaError_t launch_decode_kv(const Layout&, int, const Batch&, const DecodePlan&
 template <int KB, int VB>
 int decode_chunk_tokens_kv(int D, int G);
 
+bool decode_tc_supported(const Layout& L, int G);
+int decode_tc_tile_tokens();
+cudaError_t launch_decode_tc(const Layout& L, int layer, const Batch& b, const DecodePlan& plan, int n_q_heads,
+                             const void* q, void* out, float scale_log2, void* ws, cudaStream_t s);
+
 namespace {
 
 __global__ void lse_combine_kernel(const __grid_constant__ Batch b, int H, int G, int D, int n_q_heads, int64_t cpc,
@@ -55,6 +60,7 @@ size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D) {
 
 static int stage_tokens(const Layout& L, int G) {
   const int kb = L.k_bits, vb = L.v_bits, D = L.head_dim;
+  if (decode_tc_supported(L, G)) return decode_tc_tile_tokens();
   if (kb == 16) return decode_chunk_tokens_kv<16, 16>(D, G);
   if (kb == 8 && vb == 8) return decode_chunk_tokens_kv<8, 8>(D, G);
   if (kb == 8 && vb == 4) return decode_chunk_tokens_kv<8, 4>(D, G);
@@ -78,7 +84,9 @@ cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const Deco
                           const void* q, void* out, float scale_log2, void* ws, cudaStream_t s) {
   const int kb = L.k_bits, vb = L.v_bits;
   cudaError_t e;
-  if (kb == 16) e = launch_decode_kv<16, 16>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  if (decode_tc_supported(L, n_q_heads / L.n_kv_heads))
+    e = launch_decode_tc(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  else if (kb == 16) e = launch_decode_kv<16, 16>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
   else if (kb == 8 && vb == 8) e = launch_decode_kv<8, 8>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
   else if (kb == 8 && vb == 4) e = launch_decode_kv<8, 4>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
   else if (kb == 4 && vb == 4) e = launch_decode_kv<4, 4>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);

@@ -183,6 +183,7 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
   const int P = c->cfg.page_tokens, D = c->cfg.head_dim, H = c->cfg.n_kv_heads;
   kvq::Layout& L = c->L;
   L.n_kv_heads = H;
+  L.n_layers = c->cfg.n_layers;
   L.page_tokens = P;
   L.head_dim = D;
   L.k_bits = c->cfg.k_bits;

@@ -37,6 +37,7 @@ struct Layout {
   const int32_t* page_table;           // [max_seqs][max_pages_per_seq], -1 = unmapped
   uint32_t* err;                       // device error word
   int64_t head_block;                  // bytes per (layer, page, head)
+  int32_t n_layers;
   int32_t n_pages;                     // pages in the pool
   int32_t max_pages_per_seq;
   int32_t n_kv_heads;

@@ -40,6 +40,7 @@
 #include "kvq_internal.cuh"
 #include "sm100_util.cuh"
 #include "tcgen05_util.cuh"
+#include "tma_host.h"
 
 namespace kvq {
 namespace {
@@ -426,28 +427,6 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 // ------------------------------------------------------------------ host
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
-  return fn;
-}
-
-bool make_map(CUtensorMap* m, void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides,
-              const cuuint32_t* box) {
-  auto fn = encode_fn();
-  if (!fn) return false;
-  cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, rank, base, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // Batch sorted by decreasing length (heavy work first), with tile and query-tile offsets.
 PrefillBatch plan(const Layout& L, const Batch& in, int n_q_heads, int64_t* n_tiles_total, int64_t* n_qtiles) {
   PrefillBatch b{};
@@ -497,20 +476,20 @@ cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_
     cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(n_q_heads), cuuint64_t(total_q)};
     cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(n_q_heads) * D * 2};
     cuuint32_t box[3] = {64, cuuint32_t(G), cuuint32_t(kQT / G)};
-    if (!make_map(&mq, const_cast<void*>(q), 3, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&mq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, const_cast<void*>(q), 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
     cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(n_tiles) * kKT};
     cuuint64_t strides[1] = {cuuint64_t(D) * 2};
     cuuint32_t box[2] = {64, kKT};
-    if (!make_map(&mkh, khi, 2, dims, strides, box)) return cudaErrorInvalidValue;
-    if (!make_map(&mkl, klo, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&mkh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, khi, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&mkl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, klo, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   {
     cuuint64_t dims[2] = {cuuint64_t(kKT), cuuint64_t(n_tiles) * D};
     cuuint64_t strides[1] = {cuuint64_t(kKT) * 2};
     cuuint32_t box[2] = {64, cuuint32_t(D)};
-    if (!make_map(&mv, vws, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    if (!make_tensor_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, vws, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   using T = PTraits<D>;
   static bool configured = false;

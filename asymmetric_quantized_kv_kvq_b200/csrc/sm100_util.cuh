@@ -75,6 +75,27 @@ __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Named barrier over `threads` threads that also reduces a predicate: every
+// participant gets the OR (resp. AND) of all participants' `p`.
+__device__ __forceinline__ bool bar_red_or(int id, int threads, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n bar.red.or.pred b, %2, %3, a;\n selp.u32 %0, 1, 0, b;\n}\n"
+      : "=r"(r)
+      : "r"(uint32_t(p)), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool bar_red_and(int id, int threads, bool p) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred a, b;\n setp.ne.u32 a, %1, 0;\n bar.red.and.pred b, %2, %3, a;\n selp.u32 %0, 1, 0, b;\n}\n"
+      : "=r"(r)
+      : "r"(uint32_t(p)), "r"(id), "r"(threads)
+      : "memory");
+  return r != 0;
+}
+
 // ---- packed fp32 pairs (sm_100 f32x2) ----
 __device__ __forceinline__ unsigned long long f2_bits(float2 a) {
   return (static_cast<unsigned long long>(__float_as_uint(a.y)) << 32) | __float_as_uint(a.x);
