@@ -639,7 +639,7 @@ cudaError_t launch_tc(const CUtensorMap& tm, const DecodeArgs& a, const Batch& b
 }  // namespace
 
 bool decode_tc_supported(const Layout& L, int G) {
-  return L.k_bits == 8 && (L.v_bits == 4 || L.v_bits == 8) && L.head_dim == kD &&
+  return L.decode_tc && L.k_bits == 8 && (L.v_bits == 4 || L.v_bits == 8) && L.head_dim == kD &&
          (G == 1 || G == 2 || G == 4 || G == 8) &&
          int64_t(L.n_layers) * L.n_pages * L.n_kv_heads < (int64_t(1) << 31);
 }

@@ -64,7 +64,7 @@ kvq_status check_config(const kvq_cache_config* c) {
   if (c->max_tokens < 1) return fail(KVQ_ERR_INVALID_ARG, "max_tokens must be >= 1");
   int64_t mst = c->max_seq_tokens ? c->max_seq_tokens : c->max_tokens;
   if (mst < 1 || mst > (int64_t(1) << 30)) return fail(KVQ_ERR_INVALID_ARG, "max_seq_tokens out of range (<= 2^30)");
-  if (c->flags & ~KVQ_CACHE_HOST_ONLY) return fail(KVQ_ERR_INVALID_ARG, "unknown flags");
+  if (c->flags & ~(KVQ_CACHE_HOST_ONLY | KVQ_CACHE_DECODE_TENSOR_CORES)) return fail(KVQ_ERR_INVALID_ARG, "unknown flags");
   int64_t pages = (c->max_tokens + P - 1) / P;
   if (pages > (int64_t(1) << 30)) return fail(KVQ_ERR_INVALID_ARG, "max_tokens too large");
   int64_t mpps = (mst + P - 1) / P;
@@ -184,6 +184,7 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
   kvq::Layout& L = c->L;
   L.n_kv_heads = H;
   L.n_layers = c->cfg.n_layers;
+  L.decode_tc = (cfg->flags & KVQ_CACHE_DECODE_TENSOR_CORES) ? 1 : 0;
   L.page_tokens = P;
   L.head_dim = D;
   L.k_bits = c->cfg.k_bits;

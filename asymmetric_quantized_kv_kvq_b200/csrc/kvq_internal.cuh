@@ -47,6 +47,7 @@ struct Layout {
   int32_t k_row, v_row;                // code bytes per token
   int32_t s_row;                       // scale bytes per token (D/32 * 2), 0 for 16-bit
   int32_t k_scales_off, v_codes_off, v_scales_off;   // byte offsets inside a head block
+  int32_t decode_tc;                   // KVQ_CACHE_DECODE_TENSOR_CORES was set
 
   __host__ __device__ __forceinline__ uint8_t* head_ptr(int layer, int page, int head) const {
     return pool + ((int64_t(layer) * n_pages + page) * n_kv_heads + head) * head_block;

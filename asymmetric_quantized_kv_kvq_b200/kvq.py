@@ -19,6 +19,7 @@ STATUS_NAMES = {
     4: "KVQ_ERR_CAPACITY", 5: "KVQ_ERR_CUDA", 6: "KVQ_ERR_DEVICE_CHECK", 7: "KVQ_ERR_WORKSPACE",
 }
 KVQ_CACHE_HOST_ONLY = 1
+KVQ_CACHE_DECODE_TENSOR_CORES = 2
 KVQ_MAX_BATCH = 256
 KVQ_NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -116,9 +117,10 @@ def _dev_fp16(t, name: str, shape: Optional[tuple] = None):
 
 
 def make_config(n_layers, n_kv_heads, head_dim, k_bits, v_bits, max_seqs, max_tokens,
-                page_tokens=256, max_seq_tokens=0, host_only=False) -> CacheConfig:
+                page_tokens=256, max_seq_tokens=0, host_only=False, decode_tc=False) -> CacheConfig:
+    flags = (KVQ_CACHE_HOST_ONLY if host_only else 0) | (KVQ_CACHE_DECODE_TENSOR_CORES if decode_tc else 0)
     return CacheConfig(n_layers, n_kv_heads, head_dim, k_bits, v_bits, page_tokens, max_seqs,
-                       KVQ_CACHE_HOST_ONLY if host_only else 0, max_tokens, max_seq_tokens)
+                       flags, max_tokens, max_seq_tokens)
 
 
 def footprint_bytes(n_layers, n_kv_heads, head_dim, k_bits, v_bits, n_tokens, page_tokens=256):
@@ -134,10 +136,10 @@ class Cache:
 
     def __init__(self, n_layers: int, n_kv_heads: int, head_dim: int, k_bits: int, v_bits: int,
                  max_seqs: int, max_tokens: int, page_tokens: int = 256, max_seq_tokens: int = 0,
-                 host_only: bool = False):
+                 host_only: bool = False, decode_tc: bool = False):
         self._lib = load_library()
         self.cfg = make_config(n_layers, n_kv_heads, head_dim, k_bits, v_bits, max_seqs, max_tokens,
-                               page_tokens, max_seq_tokens, host_only)
+                               page_tokens, max_seq_tokens, host_only, decode_tc)
         self.n_layers, self.n_kv_heads, self.head_dim = n_layers, n_kv_heads, head_dim
         self.k_bits, self.v_bits = k_bits, v_bits
         self.host_only = host_only

@@ -62,10 +62,10 @@ def kernel_source_sha() -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(workload: str, precision: str):
+def ncu_traffic(workload: str, precision: str, kernel: str = "decode_split"):
     """DRAM bytes per launch of the decode kernel from the committed ncu summary
     of this workload, if it was captured on the current kernel source."""
-    path = os.path.join(PROFILE_DIR, f"decode_split_{precision.lower()}_{workload}.txt")
+    path = os.path.join(PROFILE_DIR, f"{kernel}_{precision.lower()}_{workload}.txt")
     if not os.path.exists(path):
         return None
     vals = {}
@@ -131,7 +131,7 @@ class ClockSampler:
 class DecodeRun:
     """A resident cache of the workload plus one decode step's inputs."""
 
-    def __init__(self, wl, kb: int, vb: int, capacity_extra: int, device):
+    def __init__(self, wl, kb: int, vb: int, capacity_extra: int, device, decode_tc: bool = False):
         import torch
         from asymmetric_quantized_kv_kvq_b200 import kvq
         from asymmetric_quantized_kv_kvq_b200.inputs import gen_kv, gen_q, GEN_CHUNK
@@ -139,7 +139,8 @@ class DecodeRun:
         L, B, H, D, T = wl.n_layers, wl.batch, wl.n_kv_heads, wl.head_dim, wl.cached
         P = 256
         cap = T + capacity_extra
-        self.cache = kvq.Cache(L, H, D, kb, vb, max_seqs=B, max_tokens=B * (-(-cap // P)) * P, max_seq_tokens=cap)
+        self.cache = kvq.Cache(L, H, D, kb, vb, max_seqs=B, max_tokens=B * (-(-cap // P)) * P, max_seq_tokens=cap,
+                               decode_tc=decode_tc)
         self.ids = list(range(B))
         # fill: chunk by chunk, every layer (the order a model's prefill writes the cache)
         for c in range(-(-T // GEN_CHUNK)):
@@ -199,7 +200,7 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
     torch.cuda.set_device(dev)
     extra = args.warmup + 2 * args.steps + 8
     t0 = time.time()
-    run = DecodeRun(wl, kb, vb, extra, dev)
+    run = DecodeRun(wl, kb, vb, extra, dev, decode_tc=args.decode_tc)
     setup_s = time.time() - t0
     L = wl.n_layers
     lens0 = run.lengths()
@@ -576,6 +577,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--decode-tc", action="store_true",
+                    help="decode on the tensor-core kernel (cache flag KVQ_CACHE_DECODE_TENSOR_CORES) "
+                         "instead of the default CUDA-core kernel")
     a = ap.parse_args()
     if a.warmup < 3 and a.impl == "ours":
         ap.error("--warmup must be >= 3")
@@ -659,14 +663,17 @@ def main():
         peaks = measured_peaks()
         achieved = res["kern_bytes_per_launch"] / (res["kern_ms_per_launch"] * 1e-3) / 1e9
         in_step = res["dec_bytes_per_launch"] / (res["dec_ms_per_launch"] * 1e-3) / 1e9
-        traffic = ncu_traffic(wl.name, precision)
+        tc = args.decode_tc and kb == 8 and vb in (4, 8) and wl.head_dim == 128
+        traffic = ncu_traffic(wl.name, precision, "decode_tc" if tc else "decode_split")
         line = {
             "metric": METRIC, "value": res["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": config_of(wl, precision, world, res["flush"]),
+            "config": dict(config_of(wl, precision, world, res["flush"]),
+                           decode_kernel="tensor cores (opt-in)" if tc else "CUDA cores"),
             "decode_tokens_per_s": res["decode_tokens_per_s"],
-            "roofline": {"bound": "hbm", "kernel": "decode split kernel + lse_combine_kernel",
+            "roofline": {"bound": "hbm",
+                         "kernel": ("decode_tc_kernel" if tc else "decode_split_kernel") + " + lse_combine_kernel",
                          "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
                          "frac_of_8tbs_nominal": achieved / 8000.0,

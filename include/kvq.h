@@ -99,6 +99,14 @@ typedef struct {
  * GPU (no device memory); calls that would launch work then return
  * KVQ_ERR_UNSUPPORTED.  Used to test the host logic on machines without a GPU. */
 #define KVQ_CACHE_HOST_ONLY 1
+/* KVQ_CACHE_DECODE_TENSOR_CORES runs kvq_decode_attn on the tcgen05 tensor
+ * cores where a kernel for the shape exists (8-bit keys, 4- or 8-bit values,
+ * head_dim 128, 1 / 2 / 4 / 8 query heads per KV head): scores as int8 MMAs on
+ * the stored key codes, PV as fp16 MMAs on values dequantised once per token.
+ * Other shapes, and caches without the flag, use the CUDA-core kernel that
+ * dequantises K and V in registers.  Results agree within the attention
+ * tolerance; the flag only changes speed. */
+#define KVQ_CACHE_DECODE_TENSOR_CORES 2
 
 /* Most sequences one append / decode / prefill call may name. */
 #define KVQ_MAX_BATCH 256

@@ -191,3 +191,22 @@ def test_decode_workspace_is_length_independent(kvq):
 
 def test_destroy_null_is_noop(kvq):
     assert kvq.load_library().kvq_cache_destroy(None) == 0
+
+
+def test_cache_flags(kvq):
+    """The header's flag values, and unknown bits refused before anything is allocated."""
+    with open(os.path.join(ROOT, "include", "kvq.h")) as f:
+        text = f.read()
+    assert re.search(r"#define KVQ_CACHE_HOST_ONLY 1\b", text)
+    assert re.search(r"#define KVQ_CACHE_DECODE_TENSOR_CORES 2\b", text)
+    assert kvq.KVQ_CACHE_HOST_ONLY == 1 and kvq.KVQ_CACHE_DECODE_TENSOR_CORES == 2
+    lib = kvq.load_library()
+    cfg = kvq.make_config(1, 8, 128, 8, 4, 2, 4096, host_only=True, decode_tc=True)
+    assert cfg.flags == 3
+    h = ctypes.c_void_p()
+    assert lib.kvq_cache_create(ctypes.byref(cfg), ctypes.byref(h)) == 0
+    assert lib.kvq_cache_destroy(h) == 0
+    cfg.flags = 1 | 4
+    h = ctypes.c_void_p()
+    assert lib.kvq_cache_create(ctypes.byref(cfg), ctypes.byref(h)) == 1      # KVQ_ERR_INVALID_ARG
+    assert b"unknown flags" in lib.kvq_last_error()
