@@ -19,16 +19,23 @@
 //     128-row query tile: a 4096-token chunk with 4 query heads per KV head
 //     has 128 of them.)  Positions past the end are zero.
 //  2. prefill_attn_kernel: one CTA per (query tile of 128 rows = 128/G tokens
-//     x G query heads of one KV head).  Warp 0 streams Q once and the K_hi /
-//     K_lo / V tiles through a three-stage ring with 2-D / 3-D TMA tensor
-//     loads (128-byte swizzle); warp 1 owns TMEM (S double buffer + O
-//     accumulator) and issues tcgen05.mma kind::f16 (fp16 x fp16 -> fp32):
-//        S_j = Q K_hi,j^T + Q K_lo,j^T into TMEM, O += P_j V_j from shared memory;
-//     warps 2-5 (one per TMEM lane quadrant, one thread per row) read S with
-//     tcgen05.ld, apply sigma log2 e and the causal mask, run the online softmax
-//     (running max moved only when it grows by more than 2^8; then O is
-//     rescaled in TMEM), write P as fp16 in the swizzled K-major layout, and at
-//     the end normalise O and store it.  Every wait is bounded.
+//     x G query heads of one KV head).  Warp 0 streams Q once, then 128-key
+//     tiles (two pass-1 tiles) with 2-D / 3-D TMA tensor loads (128-byte
+//     swizzle): lane 0 fills a ring of K_hi / K_lo slots, lane 1 a separate
+//     ring of V^T slots, so a key slot refills as soon as its scores are done.
+//     Warp 1 owns all 512 TMEM columns (S double buffer, O, P double buffer)
+//     and issues tcgen05.mma kind::f16 (fp16 x fp16 -> fp32):
+//        S_j = Q K_hi,j^T + Q K_lo,j^T   (M 128, N 128: 2 x D/16 MMAs per 128 keys)
+//        O  += P_j V_j                   (A = P read from TMEM, 8 MMAs per 128 keys).
+//     A tcgen05.mma costs roughly the same time for N up to 128, so wide key
+//     tiles halve the instruction count of 64-key ones.  Warps 2-9 run the
+//     softmax, two per TMEM lane quadrant (one thread per row, 64 keys each):
+//     one tcgen05.ld of the raw scores, the row max exchanged between the two
+//     halves through shared memory at a named barrier, sigma log2 e and the
+//     causal mask applied, the online softmax (running max moved only when it
+//     grows by more than 2^8; then O is rescaled in TMEM), and P stored as fp16
+//     pairs into TMEM (tcgen05.st), where the PV MMA takes its A operand.  At
+//     the end they normalise O and store it.  Every wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -164,31 +171,36 @@ __global__ void __launch_bounds__(256) dequant_tiles_kernel(const Layout L, int 
 }
 
 // ------------------------------------------------------------------ pass 2: attention
+constexpr int kKV = 128;     // key / value tokens per stage: N of S, K of P V (two pass-1 tiles)
+
 template <int D>
 struct PTraits {
   static constexpr int CB = D / 64;                      // 128-byte column blocks of a Q / K row
-  static constexpr int NSTAGE = 3;
   static constexpr int Q_BYTES = kQT * D * 2;            // CB blocks of [128 rows][128 B]
-  static constexpr int K_BYTES = kKT * D * 2;            // CB blocks of [64 rows][128 B]
-  static constexpr int V_BYTES = D * kKT * 2;            // one block of [D rows][128 B]
-  static constexpr int STAGE = 2 * K_BYTES + V_BYTES;    // K_hi, K_lo, V^T
+  static constexpr int K_BYTES = kKV * D * 2;            // CB blocks of [128 rows][128 B]
+  static constexpr int V_BYTES = D * kKV * 2;            // two blocks (64 tokens each) of [D rows][128 B]
+  static constexpr int KSLOT = 2 * K_BYTES;              // K_hi, K_lo of one 128-key tile
+  static constexpr int NSTAGE = D == 128 ? 2 : 3;        // slots of each ring (keys and values separately,
+                                                         // so a key slot is refilled as soon as S is done)
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_KV = OFF_Q + Q_BYTES;
-  static constexpr int OFF_P = OFF_KV + NSTAGE * STAGE;
-  static constexpr int P_BYTES = kQT * kKT * 2;          // one block of [128 rows][128 B]
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_V = OFF_K + NSTAGE * KSLOT;
+  static constexpr int OFF_BAR = OFF_V + NSTAGE * V_BYTES;
   // + alignment slack; never less than ~116 KB so that a second CTA cannot
   // share the SM and wait in tcgen05.alloc
-  static constexpr int SMEM_NEED = OFF_BAR + 256 + 1024;
+  static constexpr int SMEM_NEED = OFF_BAR + 256 + 2 * 128 * 4 + 1024;   // barriers, TMEM slot, row maxima
   static constexpr int SMEM = SMEM_NEED > 118 * 1024 ? SMEM_NEED : 118 * 1024;
-  static constexpr int NT = 192;                         // 6 warps
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t S_COL0 = 0, O_COL = 128;     // S double buffer [0, 128), O [128, 128 + D)
-  static_assert(O_COL + D <= TMEM_COLS, "TMEM");
-  static_assert(OFF_KV % 1024 == 0 && STAGE % 1024 == 0 && OFF_P % 1024 == 0, "swizzle atoms");
+  static constexpr int NT = 320;                         // 10 warps: copies, MMAs, 2 x 4 softmax
+  static constexpr uint32_t TMEM_COLS = 512;
+  // S double buffer [0, 256) (fp32, 128 keys each), O [256, 256 + D), P double buffer [384, 512)
+  // (fp16 pairs, 64 columns = 128 keys each)
+  static constexpr uint32_t S_COL0 = 0, O_COL = 256, P_COL0 = 384;
+  static_assert(O_COL + D <= P_COL0 && P_COL0 + 2 * kKV / 2 <= TMEM_COLS, "TMEM");
+  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && KSLOT % 1024 == 0 && V_BYTES % 1024 == 0,
+                "swizzle atoms");
+  static_assert(SMEM <= 227 * 1024, "shared memory");
 };
 
-// barriers: 0 q_full | 1..3 kv_full | 4..6 kv_empty | 7..8 s_full | 9 p_full | 10 pv_done | 11 mma_done
 struct PrefillArgs {
   float scale_log2;
   __half* out;
@@ -196,7 +208,7 @@ struct PrefillArgs {
 };
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_khi,
                         const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
                         const PrefillArgs a, const __grid_constant__ PrefillBatch b) {
@@ -209,10 +221,12 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::OFF_BAR);
   const uint32_t bar0 = smem_u32(bars);
   auto bar = [&](int i) { return bar0 + 8u * i; };
-  constexpr int B_Q = 0, B_FULL = 1, B_EMPTY = 1 + NS, B_S = 1 + 2 * NS, B_P = 3 + 2 * NS, B_PV = 4 + 2 * NS,
-                B_DONE = 5 + 2 * NS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+  // barriers: q_full | k_full[NS] | k_empty[NS] | v_full[NS] | v_empty[NS] | s_full[2] | p_full | pv_done | done
+  constexpr int B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + NS, B_VFULL = 1 + 2 * NS, B_VEMPTY = 1 + 3 * NS,
+                B_S = 1 + 4 * NS, B_P = 3 + 4 * NS, B_PV = 4 + 4 * NS, B_DONE = 5 + 4 * NS;
+  static_assert(B_DONE < 24, "barrier area");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 25);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int si = find_seq_by(b, blockIdx.x, false);
@@ -224,11 +238,11 @@ __global__ void __launch_bounds__(192, 1)
   const int tok0 = qt * TT;                                // first chunk row of this tile
   const int qpos0 = sq.len - sq.q_len + tok0;              // absolute position of row 0
   const int qpos_last = sq.len - sq.q_len + min(tok0 + TT, sq.q_len) - 1;
-  const int n_kv = qpos_last / kKT + 1;
-  const int tile_base = sq.tile_base + h * sq.n_tiles;
+  const int n_kv = qpos_last / kKV + 1;
+  const int tile_base = sq.tile_base + h * sq.n_tiles;     // first 64-token pass-1 tile of this head
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i <= B_DONE; ++i) mbar_init(bar(i), i == B_P ? 128u : 1u);
+    for (int i = 0; i <= B_DONE; ++i) mbar_init(bar(i), i == B_P ? 256u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -239,7 +253,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producers: lane 0 Q and keys, lane 1 values
     if (lane == 0) {
       uint32_t issued = 0;
       mbar_arrive_expect_tx(bar(B_Q), T::Q_BYTES);
@@ -247,63 +261,90 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_3d(base + T::OFF_Q + cb * kQT * 128, &tm_q, cb * 64, h * G, sq.q_off + tok0, bar(B_Q));
       for (int j = 0; j < n_kv; ++j) {
         const int s = j % NS;
-        if (!mbar_wait(bar(B_EMPTY + s), ((j / NS) & 1) ^ 1, abort_flag)) {
+        if (!mbar_wait(bar(B_KEMPTY + s), ((j / NS) & 1) ^ 1, abort_flag)) {
           record_error(a.err, kErrWaitTimeout | 0x11);
           *abort_flag = 1;
           break;
         }
-        const uint32_t full = bar(B_FULL + s);
-        mbar_arrive_expect_tx(full, T::STAGE);
-        const uint32_t st = base + T::OFF_KV + s * T::STAGE;
-        const int row = (tile_base + j) * kKT;
+        const uint32_t full = bar(B_KFULL + s);
+        mbar_arrive_expect_tx(full, T::KSLOT);
+        const uint32_t st = base + T::OFF_K + s * T::KSLOT;
+        const int t64 = tile_base + 2 * j;                   // two consecutive pass-1 tiles
         for (int cb = 0; cb < T::CB; ++cb) {
-          tma_load_2d(st + cb * kKT * 128, &tm_khi, cb * 64, row, full);
-          tma_load_2d(st + T::K_BYTES + cb * kKT * 128, &tm_klo, cb * 64, row, full);
+          tma_load_2d(st + cb * kKV * 128, &tm_khi, cb * 64, t64 * 64, full);
+          tma_load_2d(st + T::K_BYTES + cb * kKV * 128, &tm_klo, cb * 64, t64 * 64, full);
         }
-        tma_load_2d(st + 2 * T::K_BYTES, &tm_v, 0, (tile_base + j) * D, full);
         ++issued;
       }
       // no copy may outlive the CTA
       mbar_wait(bar(B_Q), 0, nullptr);
       for (uint32_t j = issued > uint32_t(NS) ? issued - NS : 0; j < issued; ++j)
-        mbar_wait(bar(B_FULL + j % NS), (j / NS) & 1, nullptr);
+        mbar_wait(bar(B_KFULL + j % NS), (j / NS) & 1, nullptr);
+    } else if (lane == 1) {
+      uint32_t issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(bar(B_VEMPTY + s), ((j / NS) & 1) ^ 1, abort_flag)) {
+          record_error(a.err, kErrWaitTimeout | 0x15);
+          *abort_flag = 1;
+          break;
+        }
+        const uint32_t full = bar(B_VFULL + s);
+        mbar_arrive_expect_tx(full, T::V_BYTES);
+        const uint32_t st = base + T::OFF_V + s * T::V_BYTES;
+        const int t64 = tile_base + 2 * j;
+        tma_load_2d(st, &tm_v, 0, t64 * D, full);
+        tma_load_2d(st + D * 128, &tm_v, 0, (t64 + 1) * D, full);
+        ++issued;
+      }
+      for (uint32_t j = issued > uint32_t(NS) ? issued - NS : 0; j < issued; ++j)
+        mbar_wait(bar(B_VFULL + j % NS), (j / NS) & 1, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_f16_f32(kQT, kKT);
+      constexpr uint32_t idS = idesc_f16_f32(kQT, kKV);
       constexpr uint32_t idO = idesc_f16_f32(kQT, D);
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
+      // S_j = Q K_hi^T + Q K_lo^T into S buffer j & 1, issued once the softmax has turned S_(j-2) into
+      // P_(j-2) (p_full) and PV(j - 2) is queued.
       auto issue_s = [&](int j) -> bool {
         const int s = j % NS;
-        if (!mbar_wait(bar(B_FULL + s), (j / NS) & 1, abort_flag)) return false;
+        if (!mbar_wait(bar(B_KFULL + s), (j / NS) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t qa = base + T::OFF_Q, ka = base + T::OFF_KV + s * T::STAGE;
-        const uint32_t dst = tmem + T::S_COL0 + (j & 1) * kKT;
+        const uint32_t qa = base + T::OFF_Q, ka = base + T::OFF_K + s * T::KSLOT;
+        const uint32_t dst = tmem + T::S_COL0 + (j & 1) * kKV;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {          // K_hi then K_lo, accumulated
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t qoff = (k >> 2) * kQT * 128 + (k & 3) * 32;
-            const uint32_t koff = part * T::K_BYTES + (k >> 2) * kKT * 128 + (k & 3) * 32;
+            const uint32_t koff = part * T::K_BYTES + (k >> 2) * kKV * 128 + (k & 3) * 32;
             umma_f16(dst, sdesc_k_sw128(qa + qoff), sdesc_k_sw128(ka + koff), idS, (part | k) != 0);
           }
         }
         umma_commit(bar(B_S + (j & 1)));
+        umma_commit(bar(B_KEMPTY + s));                 // the key slot refills once S_j is done
         return true;
       };
       if (ok) ok = issue_s(0);
       if (ok && n_kv > 1) ok = issue_s(1);
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % NS;
-        if (!mbar_wait(bar(B_P), j & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(bar(B_P), j & 1, abort_flag) || !mbar_wait(bar(B_VFULL + s), (j / NS) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t pa = base + T::OFF_P, va = base + T::OFF_KV + s * T::STAGE + 2 * T::K_BYTES;
+        // O += P V: A = P in TMEM (16 keys = 8 columns per step), B = V^T [D][128 keys] in two 64-key blocks
+        const uint32_t pa = tmem + T::P_COL0 + (j & 1) * (kKV / 2);
+        const uint32_t va = base + T::OFF_V + s * T::V_BYTES;
 #pragma unroll
-        for (int k = 0; k < kKT / 16; ++k)
-          umma_f16(tmem + T::O_COL, sdesc_k_sw128(pa + k * 32), sdesc_k_sw128(va + k * 32), idO, (j > 0 || k > 0));
+        for (int k = 0; k < kKV / 16; ++k)
+          umma_f16_ta(tmem + T::O_COL, pa + 8 * k, sdesc_k_sw128(va + (k >> 2) * D * 128 + (k & 3) * 32), idO,
+                      (j > 0 || k > 0));
         umma_commit(bar(B_PV));
-        umma_commit(bar(B_EMPTY + s));
+        umma_commit(bar(B_VEMPTY + s));
         if (j + 2 < n_kv) ok = issue_s(j + 2);
       }
       if (!ok) {
@@ -315,107 +356,136 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(bar(B_DONE), 0, nullptr);
     }
   } else {
-    // ------------------------------------------------------------ softmax (warps 2..5)
-    const int quad = warp & 3;
+    // ------------------------------------------------------------ softmax (warps 2..9)
+    // Two warps per TMEM lane quadrant: `half` 0 takes keys [0, 64) of each tile and head_dim
+    // columns [0, D/2) of O, half 1 keys [64, 128) and columns [D/2, D).  The row max is exchanged
+    // through shared memory at a 256-thread named barrier that also makes every exit uniform.
+    constexpr int BAR_MAX = 1, BAR_L = 2, BAR_MAX_READ = 3, NTH = 256;
+    const int quad = warp & 3, half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + (uint32_t(quad * 32) << 16);
     const int qpos = qpos0 + row / G;
+    float* redmax = reinterpret_cast<float*>(bars + 32);        // [2 halves][128 rows]
     float m_used = -INFINITY, l = 0.f;
-    uint8_t* P = smem + T::OFF_P;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      if (!mbar_wait(bar(B_S + (j & 1)), (j >> 1) & 1, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      float sv[kKT];
-#pragma unroll
-      for (int c = 0; c < kKT / 32; ++c) {
-        uint32_t r32[32];
-        tmem_ld32(lane_addr + T::S_COL0 + (j & 1) * kKT + 32 * c, r32);
+    bool wok = true;
+    int j = 0;
+    for (; j < n_kv; ++j) {
+      bool w = __all_sync(0xffffffffu, mbar_wait(bar(B_S + (j & 1)), (j >> 1) & 1, abort_flag));
+      const uint32_t sbuf = lane_addr + T::S_COL0 + (j & 1) * kKV + 64 * half;
+      const int kpos0 = j * kKV + 64 * half;
+      // pass 1: this half's 64 raw scores into registers (one TMEM read) and their max (sigma log2 e > 0
+      // keeps the order); only 32-key chunks that reach past the first row's position need the causal mask
+      uint32_t sv[64];
+      float mx = -INFINITY;
+      if (w) {
+        tc_fence_after();
+        tmem_ld32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+        tmem_ld32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sv[32 * c + i] = __uint_as_float(r32[i]) * a.scale_log2;
-      }
-      const int kpos0 = j * kKT;
-      float mx = -INFINITY;
-      if (kpos0 + kKT - 1 > qpos0) {      // tile reaches past the diagonal of row 0: mask
+        for (int c = 0; c < 2; ++c) {
+          if (kpos0 + 32 * c + 31 > qpos0) {
 #pragma unroll
-        for (int i = 0; i < kKT; ++i) {
-          if (kpos0 + i > qpos) sv[i] = -INFINITY;
-          mx = fmaxf(mx, sv[i]);
+            for (int i = 0; i < 32; ++i)
+              if (kpos0 + 32 * c + i <= qpos) mx = fmaxf(mx, __uint_as_float(sv[32 * c + i]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[32 * c + i]));
+          }
         }
       } else {
 #pragma unroll
-        for (int i = 0; i < kKT; ++i) mx = fmaxf(mx, sv[i]);
+        for (int i = 0; i < 64; ++i) sv[i] = 0u;
       }
-      // previous P consumed and O stable before either is touched
-      if (j > 0 && !mbar_wait(bar(B_PV), (j - 1) & 1, abort_flag)) { ok = false; break; }
+      redmax[half * 128 + row] = mx;
+      if (!bar_red_and(BAR_MAX, NTH, w && wok)) break;
+      mx = fmaxf(mx, redmax[(half ^ 1) * 128 + row]) * a.scale_log2;
+      named_barrier(BAR_MAX_READ, NTH);                          // redmax is rewritten next tile
+      // O stable (PV of the previous tile done) before it may be rescaled or P_(j-2)'s buffer reused
+      if (j > 0) wok = __all_sync(0xffffffffu, mbar_wait(bar(B_PV), (j - 1) & 1, abort_flag));
+      if (!wok) *abort_flag = 1;
       const bool need = mx > m_used + 8.f;
       if (__any_sync(0xffffffffu, need)) {
         const float mnew = need ? mx : m_used;
         const float alpha = exp2f(m_used - mnew);   // 0 when m_used = -inf
         l *= alpha;
         m_used = mnew;
-        if (j > 0) {
+        if (j > 0 && wok) {
           tc_fence_after();
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+#pragma unroll 1
+          for (int c = 0; c < D / 64; ++c) {
             uint32_t r32[32];
-            tmem_ld32(lane_addr + T::O_COL + 32 * c, r32);
+            const uint32_t oc = lane_addr + T::O_COL + (D / 2) * half + 32 * c;
+            tmem_ld32(oc, r32);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i) r32[i] = __float_as_uint(__uint_as_float(r32[i]) * alpha);
-            tmem_st32(lane_addr + T::O_COL + 32 * c, r32);
+            tmem_st32(oc, r32);
           }
           tmem_wait_st();
         }
       }
-      // P = 2^(s - m) in fp16: one K-major 128-byte-swizzled row of 64 tokens
+      // pass 2: P = 2^(sigma log2 e s - m) as fp16 pairs into P buffer j & 1 (this half's 32 columns)
+      const float neg_m = -m_used;
+      const uint32_t pbuf = lane_addr + T::P_COL0 + (j & 1) * (kKV / 2) + 32 * half;
 #pragma unroll
-      for (int c = 0; c < kKT / 8; ++c) {
-        uint32_t w[4];
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+        const bool masked = kpos0 + 32 * c + 31 > qpos0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float p0 = exp2f(sv[8 * c + 2 * i] - m_used), p1 = exp2f(sv[8 * c + 2 * i + 1] - m_used);
+        for (int i = 0; i < 16; ++i) {
+          float p0 = exp2f(fmaf(__uint_as_float(sv[32 * c + 2 * i]), a.scale_log2, neg_m));
+          float p1 = exp2f(fmaf(__uint_as_float(sv[32 * c + 2 * i + 1]), a.scale_log2, neg_m));
+          if (masked) {
+            const int k0 = kpos0 + 32 * c + 2 * i;
+            p0 = k0 > qpos ? 0.f : p0;
+            p1 = k0 + 1 > qpos ? 0.f : p1;
+          }
           l += p0 + p1;
           __half2 hp = __floats2half2_rn(p0, p1);
-          w[i] = *reinterpret_cast<uint32_t*>(&hp);
+          pk[i] = *reinterpret_cast<uint32_t*>(&hp);
         }
-        *reinterpret_cast<uint4*>(P + row * 128 + ((c ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        if (wok) tmem_st16(pbuf + 16 * c, pk);
       }
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_P));
     }
-    if (!ok) {
+    const bool done = j == n_kv;
+    bool fin = done && wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV), (n_kv - 1) & 1, abort_flag));
+    // the l of both halves of each row; every thread takes part so the barrier is uniform
+    if (done) {
+      redmax[half * 128 + row] = l;                  // every tile's max was read before BAR_MAX_READ
+      fin = bar_red_and(BAR_L, NTH, fin);
+    }
+    if (!done || !fin) {
       record_error(a.err, kErrWaitTimeout | 0x13);
       *abort_flag = 1;
-    } else if (mbar_wait(bar(B_PV), (n_kv - 1) & 1, abort_flag)) {
+    } else {
+      l += redmax[(half ^ 1) * 128 + row];
       tc_fence_after();
       const int t = tok0 + row / G;
       const float inv = 1.f / l;
-      __half* orow = a.out + (int64_t(sq.q_off + t) * b.Hq + h * G + row % G) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      __half* orow = a.out + (int64_t(sq.q_off + t) * b.Hq + h * G + row % G) * D + (D / 2) * half;
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t r32[32];
-        tmem_ld32(lane_addr + T::O_COL + 32 * c, r32);
+        tmem_ld32(lane_addr + T::O_COL + (D / 2) * half + 32 * c, r32);
         tmem_wait_ld();
         if (t < sq.q_len) {
 #pragma unroll
           for (int i = 0; i < 32; i += 8) {
-            uint32_t w[4];
+            uint32_t w4[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
               __half2 hv = __floats2half2_rn(__uint_as_float(r32[i + 2 * k]) * inv,
                                              __uint_as_float(r32[i + 2 * k + 1]) * inv);
-              w[k] = *reinterpret_cast<uint32_t*>(&hv);
+              w4[k] = *reinterpret_cast<uint32_t*>(&hv);
             }
-            *reinterpret_cast<uint4*>(orow + 32 * c + i) = make_uint4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<uint4*>(orow + 32 * c + i) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
       }
-    } else {
-      record_error(a.err, kErrWaitTimeout | 0x14);
-      *abort_flag = 1;
     }
   }
   tc_fence_before();
@@ -481,7 +551,7 @@ cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_
   {
     cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(n_tiles) * kKT};
     cuuint64_t strides[1] = {cuuint64_t(D) * 2};
-    cuuint32_t box[2] = {64, kKT};
+    cuuint32_t box[2] = {64, kKV};
     if (!make_tensor_map(&mkh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, khi, 2, dims, strides, box)) return cudaErrorInvalidValue;
     if (!make_tensor_map(&mkl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, klo, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
