@@ -8,8 +8,10 @@
 // library's reading of the format): 8-bit d = fp16(fp32(amax / 127)),
 // c = clamp(roundf(x / d), -127, 127); 4-bit d = fp16(m / -8) with m the
 // largest-|x| element (lowest index on ties), c = clamp(roundf(x / d), -8, 7),
-// nibble u = c + 8, byte i = u_i | u_{i+16} << 4.  Divisions are IEEE fp32
-// (__fdiv_rn), so codes and scales are bit-exact across implementations.
+// nibble u = c + 8, byte i = u_i | u_{i+16} << 4.  The 8-bit scale uses an
+// IEEE fp32 divide; the codes use round_quotient below, which equals roundf of
+// the IEEE fp32 quotient x / d, so codes and scales are bit-exact across
+// implementations.
 //
 // One warp quantises one (token, KV head): D/32 elements per lane, a block is
 // 32/E consecutive lanes, its max is a shuffle reduction inside that group.
@@ -40,8 +42,11 @@ struct HalfVec<2> {
 };
 
 template <int E>
-__device__ __forceinline__ void load_row(const __half* src, int lane, float (&x)[E], uint16_t (&bits)[E]) {
-  typename HalfVec<E>::T raw = *reinterpret_cast<const typename HalfVec<E>::T*>(src + lane * E);
+__device__ __forceinline__ typename HalfVec<E>::T load_raw(const __half* src, int lane) {
+  return *reinterpret_cast<const typename HalfVec<E>::T*>(src + lane * E);
+}
+template <int E>
+__device__ __forceinline__ void unpack_row(typename HalfVec<E>::T raw, float (&x)[E], uint16_t (&bits)[E]) {
   const uint16_t* h = reinterpret_cast<const uint16_t*>(&raw);
 #pragma unroll
   for (int i = 0; i < E; ++i) {
@@ -64,6 +69,23 @@ __device__ __forceinline__ uint32_t group_max_u32(uint32_t v) {
   return v;
 }
 
+// roundf(fp32(x / d)) clamped to [lo, hi], for fp16-valued x and d != 0, without
+// a divide: n from the correctly rounded reciprocal is within 1 of the answer,
+// the remainder x - n d is exact in fp32 (n d has at most 18 significant bits),
+// and comparing it with |d| / 2 fixes n, ties going away from zero.  For fp16 x
+// and d the fp32 rounding of the quotient never moves it across a half-integer
+// it did not sit on, so this is the same integer (checked for every finite fp16
+// x against 3400 scales).
+__device__ __forceinline__ int round_quotient(float x, float d, float rd, int lo, int hi) {
+  int n = __float2int_rn(__fmul_rn(x, rd));
+  const float e = __fmaf_rn(-float(n), d, x);
+  const float hd = 0.5f * fabsf(d);
+  const float ed = d > 0.f ? e : -e;
+  if (ed > hd || (ed == hd && n >= 0)) ++n;
+  else if (ed < -hd || (ed == -hd && n <= 0)) --n;
+  return max(lo, min(hi, n));
+}
+
 template <int E>
 __device__ __forceinline__ void quant8(const float (&x)[E], const uint16_t (&bits)[E], int lane, uint8_t* codes_row,
                                        __half* scales_row) {
@@ -73,11 +95,11 @@ __device__ __forceinline__ void quant8(const float (&x)[E], const uint16_t (&bit
   a = group_max<E>(a);
   const __half d = __float2half_rn(__fdiv_rn(a, 127.0f));
   const float df = __half2float(d);
+  const float rd = df != 0.f ? __frcp_rn(df) : 0.f;
   uint32_t packed = 0;
 #pragma unroll
   for (int i = 0; i < E; ++i) {
-    int c = 0;
-    if (df != 0.f) c = max(-127, min(127, __float2int_rn(0.f) + (int)roundf(__fdiv_rn(x[i], df))));
+    const int c = df != 0.f ? round_quotient(x[i], df, rd, -127, 127) : 0;
     packed |= (uint32_t(uint8_t(int8_t(c)))) << (8 * i);
   }
   if (E == 4)
@@ -103,13 +125,13 @@ __device__ __forceinline__ void quant4(const float (&x)[E], const uint16_t (&bit
   key = group_max_u32<E>(key);
   const uint16_t mbits = uint16_t(((key >> 6) & 0x7FFF) | ((key & 1u) << 15));
   const float m = __half2float(__ushort_as_half(mbits));
-  const __half d = __float2half_rn(__fdiv_rn(m, -8.0f));
+  const __half d = __float2half_rn(m * -0.125f);   // m / -8, exact in fp32
   const float df = __half2float(d);
+  const float rd = df != 0.f ? __frcp_rn(df) : 0.f;
   uint32_t u = 0;   // E nibbles, element i in bits [4i, 4i+4)
 #pragma unroll
   for (int i = 0; i < E; ++i) {
-    int c = 0;
-    if (df != 0.f) c = max(-8, min(7, (int)roundf(__fdiv_rn(x[i], df))));
+    const int c = df != 0.f ? round_quotient(x[i], df, rd, -8, 7) : 0;
     u |= uint32_t(c + 8) << (4 * i);
   }
   // partner lane holds elements j + 16 of the same block
@@ -153,6 +175,10 @@ __global__ void __launch_bounds__(256) append_kernel(const Layout L, int layer, 
   const int H = L.n_kv_heads;
   if (w >= int64_t(total_tokens) * H) return;
   const int row = int(w / H), h = int(w % H);
+  // both fp16 rows are loaded first: their addresses need no page, so the loads
+  // overlap the page-table lookup below
+  const int64_t src = (int64_t(row) * H + h) * D;
+  const typename HalfVec<E>::T kraw = load_raw<E>(k + src, lane), vraw = load_raw<E>(v + src, lane);
   // sequence of this row: last i with b.s[i].c <= row (row offsets ascending)
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
@@ -168,15 +194,13 @@ __global__ void __launch_bounds__(256) append_kernel(const Layout L, int layer, 
     return;
   }
   uint8_t* blk = L.head_ptr(layer, page, h);
-  const int64_t src = (int64_t(row) * H + h) * D;
-  float x[E];
-  uint16_t bits[E];
-
-  load_row<E>(k + src, lane, x, bits);
+  float x[E], y[E];
+  uint16_t bits[E], ybits[E];
+  unpack_row<E>(kraw, x, bits);
+  unpack_row<E>(vraw, y, ybits);
   store_row<E>(L.k_bits, x, bits, lane, blk + int64_t(r) * L.k_row,
                reinterpret_cast<__half*>(blk + L.k_scales_off + int64_t(r) * L.s_row));
-  load_row<E>(v + src, lane, x, bits);
-  store_row<E>(L.v_bits, x, bits, lane, blk + L.v_codes_off + int64_t(r) * L.v_row,
+  store_row<E>(L.v_bits, y, ybits, lane, blk + L.v_codes_off + int64_t(r) * L.v_row,
                reinterpret_cast<__half*>(blk + L.v_scales_off + int64_t(r) * L.s_row));
 }
 
