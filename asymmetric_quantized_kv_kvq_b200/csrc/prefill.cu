@@ -190,7 +190,7 @@ struct PTraits {
   // share the SM and wait in tcgen05.alloc
   static constexpr int SMEM_NEED = OFF_BAR + 256 + 2 * 128 * 4 + 1024;   // barriers, TMEM slot, row maxima
   static constexpr int SMEM = SMEM_NEED > 118 * 1024 ? SMEM_NEED : 118 * 1024;
-  static constexpr int NT = 320;                         // 10 warps: copies, MMAs, 2 x 4 softmax
+  static constexpr int NT = 352;                         // 11 warps: copies, score MMAs, 2 x 4 softmax, PV MMAs
   static constexpr uint32_t TMEM_COLS = 512;
   // S double buffer [0, 256) (fp32, 128 keys each), O [256, 256 + D), P double buffer [384, 512)
   // (fp16 pairs, 64 columns = 128 keys each)
@@ -208,7 +208,7 @@ struct PrefillArgs {
 };
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     prefill_attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_khi,
                         const __grid_constant__ CUtensorMap tm_klo, const __grid_constant__ CUtensorMap tm_v,
                         const PrefillArgs a, const __grid_constant__ PrefillBatch b) {
@@ -223,8 +223,9 @@ __global__ void __launch_bounds__(320, 1)
   auto bar = [&](int i) { return bar0 + 8u * i; };
   // barriers: q_full | k_full[NS] | k_empty[NS] | v_full[NS] | v_empty[NS] | s_full[2] | p_full | pv_done | done
   constexpr int B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + NS, B_VFULL = 1 + 2 * NS, B_VEMPTY = 1 + 3 * NS,
-                B_S = 1 + 4 * NS, B_P = 3 + 4 * NS, B_PV = 4 + 4 * NS, B_DONE = 5 + 4 * NS;
-  static_assert(B_DONE < 24, "barrier area");
+                B_S = 1 + 4 * NS, B_SFREE = 3 + 4 * NS, B_P = 5 + 4 * NS, B_PV = 7 + 4 * NS, B_DONE = 9 + 4 * NS,
+                B_DONE2 = 10 + 4 * NS;   // S, SFREE, P, PV: one barrier per buffer parity
+  static_assert(B_DONE2 < 24, "barrier area");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 25);
 
@@ -242,7 +243,8 @@ __global__ void __launch_bounds__(320, 1)
   const int tile_base = sq.tile_base + h * sq.n_tiles;     // first 64-token pass-1 tile of this head
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i <= B_DONE; ++i) mbar_init(bar(i), i == B_P ? 256u : 1u);
+    for (int i = 0; i <= B_DONE2; ++i)
+      mbar_init(bar(i), (i == B_P || i == B_P + 1 || i == B_SFREE || i == B_SFREE + 1) ? 256u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -301,18 +303,21 @@ __global__ void __launch_bounds__(320, 1)
         mbar_wait(bar(B_VFULL + j % NS), (j / NS) & 1, nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ score MMAs
+    // A tcgen05.mma keeps its issuing thread busy for ~100 cycles whatever its shape (measured), so the
+    // score MMAs and the PV MMAs are issued by two warps; they touch disjoint TMEM columns.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16_f32(kQT, kKV);
-      constexpr uint32_t idO = idesc_f16_f32(kQT, D);
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
-      // S_j = Q K_hi^T + Q K_lo^T into S buffer j & 1, issued once the softmax has turned S_(j-2) into
-      // P_(j-2) (p_full) and PV(j - 2) is queued.
-      auto issue_s = [&](int j) -> bool {
+      const uint64_t qd0 = sdesc_k_sw128(base + T::OFF_Q);
+      for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % NS;
-        if (!mbar_wait(bar(B_KFULL + s), (j / NS) & 1, abort_flag)) return false;
+        // S buffer j & 1 was read by the softmax of tile j - 2; the key slot is full
+        if (j >= 2) ok = mbar_wait(bar(B_SFREE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag);
+        if (ok) ok = mbar_wait(bar(B_KFULL + s), (j / NS) & 1, abort_flag);
+        if (!ok) break;
         tc_fence_after();
-        const uint32_t qa = base + T::OFF_Q, ka = base + T::OFF_K + s * T::KSLOT;
+        const uint64_t kd0 = sdesc_k_sw128(base + T::OFF_K + s * T::KSLOT);
         const uint32_t dst = tmem + T::S_COL0 + (j & 1) * kKV;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {          // K_hi then K_lo, accumulated
@@ -320,32 +325,11 @@ __global__ void __launch_bounds__(320, 1)
           for (int k = 0; k < D / 16; ++k) {
             const uint32_t qoff = (k >> 2) * kQT * 128 + (k & 3) * 32;
             const uint32_t koff = part * T::K_BYTES + (k >> 2) * kKV * 128 + (k & 3) * 32;
-            umma_f16(dst, sdesc_k_sw128(qa + qoff), sdesc_k_sw128(ka + koff), idS, (part | k) != 0);
+            umma_f16(dst, qd0 + (qoff >> 4), kd0 + (koff >> 4), idS, (part | k) != 0);
           }
         }
         umma_commit(bar(B_S + (j & 1)));
         umma_commit(bar(B_KEMPTY + s));                 // the key slot refills once S_j is done
-        return true;
-      };
-      if (ok) ok = issue_s(0);
-      if (ok && n_kv > 1) ok = issue_s(1);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        const int s = j % NS;
-        if (!mbar_wait(bar(B_P), j & 1, abort_flag) || !mbar_wait(bar(B_VFULL + s), (j / NS) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // O += P V: A = P in TMEM (16 keys = 8 columns per step), B = V^T [D][128 keys] in two 64-key blocks
-        const uint32_t pa = tmem + T::P_COL0 + (j & 1) * (kKV / 2);
-        const uint32_t va = base + T::OFF_V + s * T::V_BYTES;
-#pragma unroll
-        for (int k = 0; k < kKV / 16; ++k)
-          umma_f16_ta(tmem + T::O_COL, pa + 8 * k, sdesc_k_sw128(va + (k >> 2) * D * 128 + (k & 3) * 32), idO,
-                      (j > 0 || k > 0));
-        umma_commit(bar(B_PV));
-        umma_commit(bar(B_VEMPTY + s));
-        if (j + 2 < n_kv) ok = issue_s(j + 2);
       }
       if (!ok) {
         record_error(a.err, kErrWaitTimeout | 0x12);
@@ -354,6 +338,36 @@ __global__ void __launch_bounds__(320, 1)
       // every MMA issued by this thread has completed before TMEM is released
       umma_commit(bar(B_DONE));
       mbar_wait(bar(B_DONE), 0, nullptr);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ PV MMAs
+    if (lane == 0) {
+      constexpr uint32_t idO = idesc_f16_f32(kQT, D);
+      bool ok = true;
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(bar(B_P + (j & 1)), (j >> 1) & 1, abort_flag) ||
+            !mbar_wait(bar(B_VFULL + s), (j / NS) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // O += P V: A = P in TMEM (16 keys = 8 columns per step), B = V^T [D][128 keys] in two 64-key blocks
+        const uint32_t pa = tmem + T::P_COL0 + (j & 1) * (kKV / 2);
+        const uint64_t vd0 = sdesc_k_sw128(base + T::OFF_V + s * T::V_BYTES);
+#pragma unroll
+        for (int k = 0; k < kKV / 16; ++k)
+          umma_f16_ta(tmem + T::O_COL, pa + 8 * k, vd0 + (((k >> 2) * D * 128 + (k & 3) * 32) >> 4), idO,
+                      (j > 0 || k > 0));
+        umma_commit(bar(B_PV + (j & 1)));
+        umma_commit(bar(B_VEMPTY + s));
+      }
+      if (!ok) {
+        record_error(a.err, kErrWaitTimeout | 0x16);
+        *abort_flag = 1;
+      }
+      umma_commit(bar(B_DONE2));
+      mbar_wait(bar(B_DONE2), 0, nullptr);
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 2..9)
@@ -382,6 +396,8 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
         tmem_ld32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(bar(B_SFREE + (j & 1)));           // S buffer j & 1 may be overwritten by S_(j+2)
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           if (kpos0 + 32 * c + 31 > qpos0) {
@@ -401,8 +417,8 @@ __global__ void __launch_bounds__(320, 1)
       if (!bar_red_and(BAR_MAX, NTH, w && wok)) break;
       mx = fmaxf(mx, redmax[(half ^ 1) * 128 + row]) * a.scale_log2;
       named_barrier(BAR_MAX_READ, NTH);                          // redmax is rewritten next tile
-      // O stable (PV of the previous tile done) before it may be rescaled or P_(j-2)'s buffer reused
-      if (j > 0) wok = __all_sync(0xffffffffu, mbar_wait(bar(B_PV), (j - 1) & 1, abort_flag));
+      // P buffer j & 1 was read by PV(j - 2); PV(j - 1) may still run
+      if (j > 1) wok = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV + (j & 1)), ((j - 2) >> 1) & 1, abort_flag));
       if (!wok) *abort_flag = 1;
       const bool need = mx > m_used + 8.f;
       if (__any_sync(0xffffffffu, need)) {
@@ -410,6 +426,8 @@ __global__ void __launch_bounds__(320, 1)
         const float alpha = exp2f(m_used - mnew);   // 0 when m_used = -inf
         l *= alpha;
         m_used = mnew;
+        // O is rescaled once every PV issued so far (up to PV(j - 1)) is done
+        if (j > 0) wok = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag));
         if (j > 0 && wok) {
           tc_fence_after();
 #pragma unroll 1
@@ -449,10 +467,11 @@ __global__ void __launch_bounds__(320, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_P));
+      mbar_arrive(bar(B_P + (j & 1)));
     }
     const bool done = j == n_kv;
-    bool fin = done && wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV), (n_kv - 1) & 1, abort_flag));
+    bool fin = done && wok &&
+               __all_sync(0xffffffffu, mbar_wait(bar(B_PV + ((n_kv - 1) & 1)), ((n_kv - 1) >> 1) & 1, abort_flag));
     // the l of both halves of each row; every thread takes part so the barrier is uniform
     if (done) {
       redmax[half * 128 + row] = l;                  // every tile's max was read before BAR_MAX_READ
