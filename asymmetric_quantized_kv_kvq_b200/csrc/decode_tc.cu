@@ -33,10 +33,10 @@
 //          fp32 accumulation in TMEM (M = head_dim 128, N = 16 >= G, K = 16
 //          tokens per instruction, 8 per tile).
 //
-// CTA = 10 warps, one CTA per SM (persistent): warp 0 streams each chunk
+// CTA = 11 warps, one CTA per SM (persistent): warp 0 streams each chunk
 // (TMA tensor load of the key codes, bulk copies of key scales, value codes
 // and value scales) into a ring of stages; warp 1 owns TMEM and issues the
-// MMAs; warps 2-5 (one per TMEM lane quadrant) run the softmax and the
+// score MMAs, warp 10 the PV MMAs; warps 2-5 (one per TMEM lane quadrant) run the softmax and the
 // per-item epilogue; warps 6-9 convert V.  TMEM: two 64-column score tiles
 // and two 16-column O accumulators (by item parity).  Every wait is bounded
 // (2 s): on expiry the kernel records an error code, raises a CTA-wide abort
@@ -86,7 +86,7 @@ struct TcTraits {
   static constexpr int NS = NS_FIT > 6 ? 6 : NS_FIT;
   static constexpr int OFF_MISC = OFF_STAGE + NS * STAGE;
   static constexpr int SMEM = OFF_MISC + MISC + 1024;    // + slack for the 1024-B alignment
-  static constexpr int NT = 320;
+  static constexpr int NT = 352;
   static constexpr uint32_t TMEM_COLS = 256;
   static constexpr uint32_t S_COL = 0;                   // two 64-column score tiles
   static constexpr uint32_t O_COL = 128;                 // two 16-column O^T accumulators
@@ -195,13 +195,13 @@ __device__ __forceinline__ void dequant_v_row(const uint8_t* st, int row, bool v
 }
 
 template <int VB, int G>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_k, const DecodeArgs a, const __grid_constant__ Batch b) {
   using T = TcTraits<VB>;
   constexpr int NS = T::NS;
   constexpr int B_FULL = 0, B_EMPTY = NS, B_SFULL = 2 * NS, B_SFREE = 2 * NS + 2, B_PFULL = 2 * NS + 4,
                 B_VFULL = 2 * NS + 6, B_PVDONE = 2 * NS + 8, B_QFULL = 2 * NS + 10, B_OFULL = 2 * NS + 12,
-                B_OFREE = 2 * NS + 14, B_DONE = 2 * NS + 16, NBAR = 2 * NS + 17;
+                B_OFREE = 2 * NS + 14, B_DONE = 2 * NS + 16, B_DONE2 = 2 * NS + 17, NBAR = 2 * NS + 18;
   static_assert(NBAR * 8 <= 256, "barrier area");
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -288,49 +288,30 @@ __global__ void __launch_bounds__(320, 1)
       for (uint32_t j = it > uint32_t(NS) ? it - NS : 0; j < it; ++j) mbar_wait(bar(B_FULL + j % NS), (j / NS) & 1, nullptr);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ score MMAs
+    // A tcgen05.mma keeps its issuing thread ~100 cycles whatever its shape (measured; two issuing warps
+    // double the rate), so score MMAs (this warp) and PV MMAs (warp 10) come from different warps.
     if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_s8_s32(kTT, 16);
-      constexpr uint32_t ID_PV = idesc_f16_f32_amn(kD, 16);
       uint32_t it = 0, j = 0, ii = 0;
       bool ok = true;
       for (int64_t x = x0; x < x1 && ok; ++ii) {
         const DecodeSeg sg = decode_find_seg(b, x, x1);
-        const uint32_t ip = ii & 1;
-        const uint32_t qd = base + T::OFF_QD + ip * T::QD_BYTES;
-        const uint32_t o_tm = tmem + T::O_COL + 16 * ip;
-        auto issue_pv = [&](uint32_t jj, bool first) -> bool {
-          if (!mbar_wait(bar(B_PFULL + (jj & 1)), (jj >> 1) & 1, abort_flag)) return false;
-          if (!mbar_wait(bar(B_VFULL + (jj & 1)), (jj >> 1) & 1, abort_flag)) return false;
-          tc_fence_after();
-          const uint32_t vh = base + T::OFF_VH + (jj & 1) * T::VH_BYTES;
-          const uint32_t pb = base + T::OFF_P + (jj & 1) * T::P_BYTES;
-#pragma unroll
-          for (int kk = 0; kk < kTT / 16; ++kk)
-            umma_f16(o_tm, sdesc_mn_sw128(vh + kk * 2048, kTT * 128, 1024),
-                     sdesc_k_sw128(pb + (kk >> 2) * 2048 + (kk & 3) * 32), ID_PV, (first && kk == 0) ? 0u : 1u);
-          umma_commit(bar(B_PVDONE + (jj & 1)));
-          return true;
-        };
-        ok = mbar_wait(bar(B_QFULL + ip), (ii >> 1) & 1, abort_flag) &&
-             mbar_wait(bar(B_OFREE + ip), ((ii >> 1) & 1) ^ 1, abort_flag);
+        const uint64_t qd0 = sdesc_k_sw128(base + T::OFF_QD + (ii & 1) * T::QD_BYTES);
+        ok = mbar_wait(bar(B_QFULL + (ii & 1)), (ii >> 1) & 1, abort_flag);
         for (int k = 0; k < sg.n && ok; ++k, ++it, ++j) {
           const int s = it % NS;
           ok = mbar_wait(bar(B_FULL + s), (it / NS) & 1, abort_flag) &&
                mbar_wait(bar(B_SFREE + (j & 1)), ((j >> 1) & 1) ^ 1, abort_flag);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t kt = base + T::OFF_STAGE + s * T::STAGE;
+          const uint64_t kd0 = sdesc_k_sw128(base + T::OFF_STAGE + s * T::STAGE);
           const uint32_t s_tm = tmem + T::S_COL + 64 * (j & 1);
 #pragma unroll
-          for (int bb = 0; bb < kNB; ++bb)
-            umma_i8(s_tm + 16 * bb, sdesc_k_sw128(kt + 32 * bb), sdesc_k_sw128(qd + 32 * bb), ID_QK, 0u);
+          for (int bb = 0; bb < kNB; ++bb) umma_i8(s_tm + 16 * bb, kd0 + 2 * bb, qd0 + 2 * bb, ID_QK, 0u);
           umma_commit(bar(B_SFULL + (j & 1)));
           umma_commit(bar(B_EMPTY + s));
-          if (k > 0) ok = issue_pv(j - 1, k == 1);    // PV of the previous tile behind this tile's scores
         }
-        if (ok) ok = issue_pv(j - 1, sg.n == 1);
-        if (ok) umma_commit(bar(B_OFULL + ip));
         x += sg.n;
       }
       if (!ok) {
@@ -340,6 +321,40 @@ __global__ void __launch_bounds__(320, 1)
       // every MMA issued by this thread has completed before TMEM is released
       umma_commit(bar(B_DONE));
       mbar_wait(bar(B_DONE), 0, nullptr);
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ PV MMAs
+    if (lane == 0) {
+      constexpr uint32_t ID_PV = idesc_f16_f32_amn(kD, 16);
+      uint32_t j = 0, ii = 0;
+      bool ok = true;
+      for (int64_t x = x0; x < x1 && ok; ++ii) {
+        const DecodeSeg sg = decode_find_seg(b, x, x1);
+        const uint32_t ip = ii & 1;
+        const uint32_t o_tm = tmem + T::O_COL + 16 * ip;
+        ok = mbar_wait(bar(B_OFREE + ip), ((ii >> 1) & 1) ^ 1, abort_flag);
+        for (int k = 0; k < sg.n && ok; ++k, ++j) {
+          ok = mbar_wait(bar(B_PFULL + (j & 1)), (j >> 1) & 1, abort_flag) &&
+               mbar_wait(bar(B_VFULL + (j & 1)), (j >> 1) & 1, abort_flag);
+          if (!ok) break;
+          tc_fence_after();
+          const uint64_t vd0 = sdesc_mn_sw128(base + T::OFF_VH + (j & 1) * T::VH_BYTES, kTT * 128, 1024);
+          const uint64_t pd0 = sdesc_k_sw128(base + T::OFF_P + (j & 1) * T::P_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kTT / 16; ++kk)
+            umma_f16(o_tm, vd0 + kk * (2048 >> 4), pd0 + (((kk >> 2) * 2048 + (kk & 3) * 32) >> 4), ID_PV,
+                     (k == 0 && kk == 0) ? 0u : 1u);
+          umma_commit(bar(B_PVDONE + (j & 1)));
+        }
+        if (ok) umma_commit(bar(B_OFULL + ip));
+        x += sg.n;
+      }
+      if (!ok) {
+        record_error(a.L.err, kErrWaitTimeout | 0x25);
+        *abort_flag = 1;
+      }
+      umma_commit(bar(B_DONE2));
+      mbar_wait(bar(B_DONE2), 0, nullptr);
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ softmax + epilogue (warps 2..5)
