@@ -470,7 +470,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         }
         __syncwarp();
         // ---- O += p' v
-#pragma unroll 2
+#pragma unroll 4
         for (int j2 = 0; j2 < T::NPV; ++j2) {
           const int t = j2 * T::TPV + tslot;
           if (t < nv_w) {
