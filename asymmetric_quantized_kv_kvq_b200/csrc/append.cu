@@ -9,14 +9,12 @@
 // c = clamp(roundf(x / d), -127, 127); 4-bit d = fp16(m / -8) with m the
 // largest-|x| element (lowest index on ties), c = clamp(roundf(x / d), -8, 7),
 // nibble u = c + 8, byte i = u_i | u_{i+16} << 4.  The 8-bit scale uses an
-// IEEE fp32 divide; the codes use round_quotient below, which equals roundf of
-// the IEEE fp32 quotient x / d, so codes and scales are bit-exact across
+// IEEE fp32 divide; the codes use round_code below, which equals roundf of the
+// IEEE fp32 quotient x / d, so codes and scales are bit-exact across
 // implementations.
 //
-// One warp quantises one (token, KV head): D/32 elements per lane, a block is
-// 32/E consecutive lanes, its max is a shuffle reduction inside that group.
-// Loads and stores are lane-contiguous (one 8-B fp16 load, one 4-B code store
-// per lane for D = 128), so the kernel streams HBM at full width.
+// One thread quantises one 32-element block of a K or V row (see
+// append_kernel); a warp's loads and stores are contiguous 16-byte accesses.
 #include <cuda_fp16.h>
 
 #include "kvq_internal.cuh"
@@ -29,157 +27,133 @@ __global__ void pt_update_kernel(int32_t* table, const __grid_constant__ PtUpdat
   if (i < u.n) table[u.idx[i]] = u.val[i];
 }
 
-// Element i of this lane is row element lane * E + i.
-template <int E>
-struct HalfVec;
-template <>
-struct HalfVec<4> {
-  using T = uint2;
+// Code rounding without a divide and without integer conversions, for
+// fp16-valued x and d != 0: c = clamp(roundf(fp32(x / d)), -cn, cp) as an exact
+// small integer in a float.  With t = |x| / |d|, n = floor(fma(|x|, 1/|d|, 0.5))
+// is within 1 of floor(t + 1/2); the remainder e = |x| - n |d| is exact in fp32
+// (n |d| has at most 18 significant bits) and moves n up when e >= |d|/2 and down
+// when e < -|d|/2, ties going away from zero; the sign of x / d is applied last.
+// For fp16 x and d the fp32 rounding of the quotient never moves it across a
+// half-integer it did not sit on, so this is the same integer as roundf of the
+// IEEE quotient (checked for every finite fp16 x against 3400 scales, both
+// clamp ranges).
+struct RoundCtx {
+  float ad, ra, hd;   // |d|, fp32(1 / |d|), |d| / 2
+  bool dneg;
 };
-template <>
-struct HalfVec<2> {
-  using T = uint32_t;
-};
-
-template <int E>
-__device__ __forceinline__ typename HalfVec<E>::T load_raw(const __half* src, int lane) {
-  return *reinterpret_cast<const typename HalfVec<E>::T*>(src + lane * E);
+__device__ __forceinline__ RoundCtx round_ctx(float d) {
+  RoundCtx r;
+  r.ad = fabsf(d);
+  r.ra = __frcp_rn(r.ad);
+  r.hd = 0.5f * r.ad;
+  r.dneg = d < 0.f;
+  return r;
 }
-template <int E>
-__device__ __forceinline__ void unpack_row(typename HalfVec<E>::T raw, float (&x)[E], uint16_t (&bits)[E]) {
-  const uint16_t* h = reinterpret_cast<const uint16_t*>(&raw);
+__device__ __forceinline__ float round_code(float x, const RoundCtx& r, float cn, float cp) {
+  const float ax = fabsf(x);
+  float n = floorf(__fmaf_rn(ax, r.ra, 0.5f));
+  const float e = __fmaf_rn(-n, r.ad, ax);
+  n += e >= r.hd ? 1.f : 0.f;
+  n -= e < -r.hd ? 1.f : 0.f;
+  return ((x < 0.f) != r.dneg) ? -fminf(n, cn) : fminf(n, cp);
+}
+// Low byte of an exact integer v in [-128, 255] held in a float (two's complement for v < 0).
+__device__ __forceinline__ uint32_t float_int_bits(float v) { return __float_as_uint(v + 12582912.0f); }
+// Bytes 0 of a, b, c, e -> one word.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t e) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, e, 0x0040), 0x5410);
+}
+
+// One thread quantises one 32-element block of one K or V row: it loads the
+// block's 64 bytes with four 16-byte loads, takes the block max in registers
+// (no shuffles, one scale and one reciprocal per block), rounds the 32 codes on
+// the FMA pipe and writes them with 16-byte stores.  A warp covers 32
+// consecutive blocks, so loads and stores stay contiguous.
+__device__ __forceinline__ void load_block(const __half* src, float (&x)[32]) {
+  const uint4* p = reinterpret_cast<const uint4*>(src);
 #pragma unroll
-  for (int i = 0; i < E; ++i) {
-    bits[i] = h[i];
-    x[i] = __half2float(__ushort_as_half(h[i]));
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w = p[c];
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ws[i]));
+      x[8 * c + 2 * i] = f.x;
+      x[8 * c + 2 * i + 1] = f.y;
+    }
   }
 }
 
-// Reduce over the G = 32/E lanes of one block (aligned groups of consecutive lanes).
-template <int E>
-__device__ __forceinline__ float group_max(float v) {
-#pragma unroll
-  for (int o = 1; o < 32 / E; o <<= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-template <int E>
-__device__ __forceinline__ uint32_t group_max_u32(uint32_t v) {
-#pragma unroll
-  for (int o = 1; o < 32 / E; o <<= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
-// roundf(fp32(x / d)) clamped to [lo, hi], for fp16-valued x and d != 0, without
-// a divide: n from the correctly rounded reciprocal is within 1 of the answer,
-// the remainder x - n d is exact in fp32 (n d has at most 18 significant bits),
-// and comparing it with |d| / 2 fixes n, ties going away from zero.  For fp16 x
-// and d the fp32 rounding of the quotient never moves it across a half-integer
-// it did not sit on, so this is the same integer (checked for every finite fp16
-// x against 3400 scales).
-__device__ __forceinline__ int round_quotient(float x, float d, float rd, int lo, int hi) {
-  int n = __float2int_rn(__fmul_rn(x, rd));
-  const float e = __fmaf_rn(-float(n), d, x);
-  const float hd = 0.5f * fabsf(d);
-  const float ed = d > 0.f ? e : -e;
-  if (ed > hd || (ed == hd && n >= 0)) ++n;
-  else if (ed < -hd || (ed == -hd && n <= 0)) --n;
-  return max(lo, min(hi, n));
-}
-
-template <int E>
-__device__ __forceinline__ void quant8(const float (&x)[E], const uint16_t (&bits)[E], int lane, uint8_t* codes_row,
-                                       __half* scales_row) {
+// 8-bit: d = fp16(fp32(amax / 127)), c = clamp(roundf(x / d), -127, 127).
+__device__ __forceinline__ void quant8_block(const float (&x)[32], uint8_t* codes, __half* scale) {
   float a = 0.f;
 #pragma unroll
-  for (int i = 0; i < E; ++i) a = fmaxf(a, fabsf(x[i]));
-  a = group_max<E>(a);
+  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(x[i]));
   const __half d = __float2half_rn(__fdiv_rn(a, 127.0f));
   const float df = __half2float(d);
-  const float rd = df != 0.f ? __frcp_rn(df) : 0.f;
-  uint32_t packed = 0;
+  uint32_t w[8];
+  if (df != 0.f) {
+    const RoundCtx r = round_ctx(df);
 #pragma unroll
-  for (int i = 0; i < E; ++i) {
-    const int c = df != 0.f ? round_quotient(x[i], df, rd, -127, 127) : 0;
-    packed |= (uint32_t(uint8_t(int8_t(c)))) << (8 * i);
-  }
-  if (E == 4)
-    *reinterpret_cast<uint32_t*>(codes_row + lane * 4) = packed;
-  else
-    *reinterpret_cast<uint16_t*>(codes_row + lane * 2) = uint16_t(packed);
-  if ((lane & (32 / E - 1)) == 0) scales_row[lane / (32 / E)] = d;
-}
-
-template <int E>
-__device__ __forceinline__ void quant4(const float (&x)[E], const uint16_t (&bits)[E], int lane, uint8_t* codes_row,
-                                       __half* scales_row) {
-  constexpr int LPB = 32 / E;           // lanes per block
-  const int jbase = (lane % LPB) * E;   // index of this lane's first element inside its block
-  // key = |x| bits (15) << 6 | (31 - j) << 1 | sign: the max is the largest
-  // magnitude, lowest index on ties; the sign rides along in bit 0.
-  uint32_t key = 0;
-#pragma unroll
-  for (int i = 0; i < E; ++i) {
-    const uint32_t k = (uint32_t(bits[i] & 0x7FFF) << 6) | (uint32_t(31 - (jbase + i)) << 1) | (bits[i] >> 15);
-    key = max(key, k);
-  }
-  key = group_max_u32<E>(key);
-  const uint16_t mbits = uint16_t(((key >> 6) & 0x7FFF) | ((key & 1u) << 15));
-  const float m = __half2float(__ushort_as_half(mbits));
-  const __half d = __float2half_rn(m * -0.125f);   // m / -8, exact in fp32
-  const float df = __half2float(d);
-  const float rd = df != 0.f ? __frcp_rn(df) : 0.f;
-  uint32_t u = 0;   // E nibbles, element i in bits [4i, 4i+4)
-#pragma unroll
-  for (int i = 0; i < E; ++i) {
-    const int c = df != 0.f ? round_quotient(x[i], df, rd, -8, 7) : 0;
-    u |= uint32_t(c + 8) << (4 * i);
-  }
-  // partner lane holds elements j + 16 of the same block
-  const uint32_t hi = __shfl_xor_sync(0xffffffffu, u, LPB / 2);
-  if ((lane % LPB) < LPB / 2) {
-    uint32_t out = 0;
-#pragma unroll
-    for (int i = 0; i < E; ++i) out |= (((u >> (4 * i)) & 0xF) | (((hi >> (4 * i)) & 0xF) << 4)) << (8 * i);
-    uint8_t* dst = codes_row + (lane / LPB) * 16 + (lane % LPB) * E;
-    if (E == 4)
-      *reinterpret_cast<uint32_t*>(dst) = out;
-    else
-      *reinterpret_cast<uint16_t*>(dst) = uint16_t(out);
-  }
-  if ((lane & (LPB - 1)) == 0) scales_row[lane / LPB] = d;
-}
-
-template <int E>
-__device__ __forceinline__ void store_row(int bits_w, const float (&x)[E], const uint16_t (&bits)[E], int lane,
-                                          uint8_t* codes_row, __half* scales_row) {
-  if (bits_w == 8) {
-    quant8<E>(x, bits, lane, codes_row, scales_row);
-  } else if (bits_w == 4) {
-    quant4<E>(x, bits, lane, codes_row, scales_row);
+    for (int k = 0; k < 8; ++k)
+      w[k] = pack_low_bytes(float_int_bits(round_code(x[4 * k], r, 127.f, 127.f)),
+                            float_int_bits(round_code(x[4 * k + 1], r, 127.f, 127.f)),
+                            float_int_bits(round_code(x[4 * k + 2], r, 127.f, 127.f)),
+                            float_int_bits(round_code(x[4 * k + 3], r, 127.f, 127.f)));
   } else {
-    typename HalfVec<E>::T raw;
-    uint16_t* h = reinterpret_cast<uint16_t*>(&raw);
 #pragma unroll
-    for (int i = 0; i < E; ++i) h[i] = bits[i];
-    *reinterpret_cast<typename HalfVec<E>::T*>(codes_row + lane * E * 2) = raw;
+    for (int k = 0; k < 8; ++k) w[k] = 0u;
   }
+  reinterpret_cast<uint4*>(codes)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  reinterpret_cast<uint4*>(codes)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  *scale = d;
+}
+
+// 4-bit: m = the largest-|x| element (lowest index on ties), d = fp16(m / -8),
+// c = clamp(roundf(x / d), -8, 7), u = c + 8, byte i = u_i | u_{i+16} << 4.
+__device__ __forceinline__ void quant4_block(const float (&x)[32], uint8_t* codes, __half* scale) {
+  float m = x[0];
+#pragma unroll
+  for (int i = 1; i < 32; ++i)
+    if (fabsf(x[i]) > fabsf(m)) m = x[i];                  // strict: the lowest index wins ties
+  const __half d = __float2half_rn(m * -0.125f);            // m / -8, exact in fp32
+  const float df = __half2float(d);
+  uint32_t w[4];
+  if (df != 0.f) {
+    const RoundCtx r = round_ctx(df);
+    uint32_t by[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      // u_j + 16 u_{j+16} = c_j + 16 c_{j+16} + 136, an exact integer in [0, 255]
+      const float c0 = round_code(x[j], r, 8.f, 7.f), c1 = round_code(x[j + 16], r, 8.f, 7.f);
+      by[j] = float_int_bits(__fmaf_rn(c1, 16.f, c0) + 136.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = pack_low_bytes(by[4 * k], by[4 * k + 1], by[4 * k + 2], by[4 * k + 3]);
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = 0x88888888u;         // all codes 0: u = 8 in both nibbles
+  }
+  reinterpret_cast<uint4*>(codes)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  *scale = d;
 }
 
 template <int D>
 __global__ void __launch_bounds__(256) append_kernel(const Layout L, int layer, const __grid_constant__ Batch b,
                                                      int total_tokens, const __half* __restrict__ k,
                                                      const __half* __restrict__ v) {
-  constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  const int64_t w = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
+  constexpr int NB = D / 32;                       // blocks per row
+  const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int H = L.n_kv_heads;
-  if (w >= int64_t(total_tokens) * H) return;
-  const int row = int(w / H), h = int(w % H);
-  // both fp16 rows are loaded first: their addresses need no page, so the loads
-  // overlap the page-table lookup below
-  const int64_t src = (int64_t(row) * H + h) * D;
-  const typename HalfVec<E>::T kraw = load_raw<E>(k + src, lane), vraw = load_raw<E>(v + src, lane);
-  // sequence of this row: last i with b.s[i].c <= row (row offsets ascending)
+  const int64_t n_rows = int64_t(total_tokens) * H;
+  if (t >= n_rows * 2 * NB) return;
+  const int64_t rr = t / (2 * NB);                 // (token, head) row
+  const int kv = int(t / NB) & 1, blk = int(t % NB);
+  const __half* src = (kv ? v : k) + rr * D + blk * 32;
+  float x[32];
+  load_block(src, x);                              // issued before the page lookup it does not need
+  const int row = int(rr / H), h = int(rr % H);
+  // sequence of this row: last s with b.s[s].c <= row (row offsets ascending)
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
@@ -187,21 +161,26 @@ __global__ void __launch_bounds__(256) append_kernel(const Layout L, int layer, 
   }
   const SeqDesc sd = b.s[lo];
   const int pos = sd.a + (row - sd.c);
-  const int lp = pos / L.page_tokens, r = pos % L.page_tokens;
-  const int page = L.page_table[int64_t(sd.seq_id) * L.max_pages_per_seq + lp];
+  const int page = L.page_table[int64_t(sd.seq_id) * L.max_pages_per_seq + pos / L.page_tokens];
   if (page < 0 || page >= L.n_pages) {
-    if (lane == 0) record_error(L.err, kErrBadPage);
+    record_error(L.err, kErrBadPage);
     return;
   }
-  uint8_t* blk = L.head_ptr(layer, page, h);
-  float x[E], y[E];
-  uint16_t bits[E], ybits[E];
-  unpack_row<E>(kraw, x, bits);
-  unpack_row<E>(vraw, y, ybits);
-  store_row<E>(L.k_bits, x, bits, lane, blk + int64_t(r) * L.k_row,
-               reinterpret_cast<__half*>(blk + L.k_scales_off + int64_t(r) * L.s_row));
-  store_row<E>(L.v_bits, y, ybits, lane, blk + L.v_codes_off + int64_t(r) * L.v_row,
-               reinterpret_cast<__half*>(blk + L.v_scales_off + int64_t(r) * L.s_row));
+  const int r = pos % L.page_tokens;
+  uint8_t* hb = L.head_ptr(layer, page, h);
+  const int bitsw = kv ? L.v_bits : L.k_bits;
+  uint8_t* codes_row = hb + (kv ? L.v_codes_off : 0) + int64_t(r) * (kv ? L.v_row : L.k_row);
+  __half* scales_row = reinterpret_cast<__half*>(hb + (kv ? L.v_scales_off : L.k_scales_off) + int64_t(r) * L.s_row);
+  if (bitsw == 8) {
+    quant8_block(x, codes_row + blk * 32, scales_row + blk);
+  } else if (bitsw == 4) {
+    quant4_block(x, codes_row + blk * 16, scales_row + blk);
+  } else {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(codes_row + blk * 64);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) d4[c] = s4[c];
+  }
 }
 
 // Canonical export: one warp per (token, head) copies that row's code and
@@ -242,8 +221,8 @@ cudaError_t launch_pt_update(int32_t* table, const PtUpdate& u, cudaStream_t s) 
 
 cudaError_t launch_append(const Layout& L, int layer, const Batch& b, int total_tokens, const void* k, const void* v,
                           cudaStream_t s) {
-  const int64_t warps = int64_t(total_tokens) * L.n_kv_heads;
-  const unsigned grid = unsigned((warps + 7) / 8);
+  const int64_t threads = int64_t(total_tokens) * L.n_kv_heads * 2 * (L.head_dim / 32);
+  const unsigned grid = unsigned((threads + 255) / 256);
   if (L.head_dim == 128)
     append_kernel<128><<<grid, 256, 0, s>>>(L, layer, b, total_tokens, static_cast<const __half*>(k),
                                             static_cast<const __half*>(v));
