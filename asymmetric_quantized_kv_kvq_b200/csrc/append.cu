@@ -29,14 +29,14 @@ __global__ void pt_update_kernel(int32_t* table, const __grid_constant__ PtUpdat
 
 // Code rounding without a divide and without integer conversions, for
 // fp16-valued x and d != 0: c = clamp(roundf(fp32(x / d)), -cn, cp) as an exact
-// small integer in a float.  With t = |x| / |d|, n = floor(fma(|x|, 1/|d|, 0.5))
-// is within 1 of floor(t + 1/2); the remainder e = |x| - n |d| is exact in fp32
-// (n |d| has at most 18 significant bits) and moves n up when e >= |d|/2 and down
-// when e < -|d|/2, ties going away from zero; the sign of x / d is applied last.
-// For fp16 x and d the fp32 rounding of the quotient never moves it across a
-// half-integer it did not sit on, so this is the same integer as roundf of the
-// IEEE quotient (checked for every finite fp16 x against 3400 scales, both
-// clamp ranges).
+// small integer in a float.  With t = |x| / |d|, n = rint(|x| * fp32(1/|d|)) (one
+// FMA against 1.5 * 2^23) is within 1 of floor(t + 1/2); the remainder
+// e = |x| - n |d| is exact in fp32 (n |d| has at most 18 significant bits) and
+// moves n up when e >= |d|/2 and down when e < -|d|/2, ties going away from
+// zero; the sign of x / d is applied last.  For fp16 x and d the fp32 rounding of
+// the quotient never moves it across a half-integer it did not sit on, so this
+// is the same integer as roundf of the IEEE quotient (checked for every finite
+// fp16 x against 3400 scales, both clamp ranges).
 struct RoundCtx {
   float ad, ra, hd;   // |d|, fp32(1 / |d|), |d| / 2
   bool dneg;
@@ -49,13 +49,20 @@ __device__ __forceinline__ RoundCtx round_ctx(float d) {
   r.dneg = d < 0.f;
   return r;
 }
-__device__ __forceinline__ float round_code(float x, const RoundCtx& r, float cn, float cp) {
+__device__ __forceinline__ float round_mag(float x, const RoundCtx& r) {
   const float ax = fabsf(x);
-  float n = floorf(__fmaf_rn(ax, r.ra, 0.5f));
+  float n = __fadd_rn(__fmaf_rn(ax, r.ra, 12582912.0f), -12582912.0f);
   const float e = __fmaf_rn(-n, r.ad, ax);
-  n += e >= r.hd ? 1.f : 0.f;
-  n -= e < -r.hd ? 1.f : 0.f;
+  n += (e >= r.hd ? 1.f : 0.f) - (e < -r.hd ? 1.f : 0.f);
+  return n;
+}
+__device__ __forceinline__ float round_code(float x, const RoundCtx& r, float cn, float cp) {
+  const float n = round_mag(x, r);
   return ((x < 0.f) != r.dneg) ? -fminf(n, cn) : fminf(n, cp);
+}
+// 8-bit: d > 0, symmetric clamp
+__device__ __forceinline__ float round_code8(float x, const RoundCtx& r) {
+  return copysignf(fminf(round_mag(x, r), 127.f), x);
 }
 // Low byte of an exact integer v in [-128, 255] held in a float (two's complement for v < 0).
 __device__ __forceinline__ uint32_t float_int_bits(float v) { return __float_as_uint(v + 12582912.0f); }
@@ -96,10 +103,8 @@ __device__ __forceinline__ void quant8_block(const float (&x)[32], uint8_t* code
     const RoundCtx r = round_ctx(df);
 #pragma unroll
     for (int k = 0; k < 8; ++k)
-      w[k] = pack_low_bytes(float_int_bits(round_code(x[4 * k], r, 127.f, 127.f)),
-                            float_int_bits(round_code(x[4 * k + 1], r, 127.f, 127.f)),
-                            float_int_bits(round_code(x[4 * k + 2], r, 127.f, 127.f)),
-                            float_int_bits(round_code(x[4 * k + 3], r, 127.f, 127.f)));
+      w[k] = pack_low_bytes(float_int_bits(round_code8(x[4 * k], r)), float_int_bits(round_code8(x[4 * k + 1], r)),
+                            float_int_bits(round_code8(x[4 * k + 2], r)), float_int_bits(round_code8(x[4 * k + 3], r)));
   } else {
 #pragma unroll
     for (int k = 0; k < 8; ++k) w[k] = 0u;
