@@ -39,8 +39,10 @@
 //      Softmax: online, per warp, with lazy rescaling (the running max is only
 //      moved when a score exceeds it by more than 2^8).
 //      PV: 8 head_dim elements per lane; p' = p * d_v is precomputed per
-//      (token, block, head) into a warp-private buffer as a duplicated pair,
-//      so the inner loop is one f32x2 FMA per two elements and head.
+//      (token, block, head) into a warp-private buffer (stored twice, so two
+//      heads' values arrive in one 16-byte load), and the inner loop is one
+//      scalar FMA per element and head: scalar FMAs overlap with the byte
+//      permutes of the V conversion, f32x2 FMAs do not.
 //  - every wait is bounded (2 s); on expiry the kernel records an error code,
 //    raises a CTA-wide abort flag, drains its own copies and returns.
 #pragma once
@@ -166,6 +168,12 @@ __device__ __forceinline__ void load_k16(const uint8_t* row, int slice, float2 (
 template <int NBP>
 __device__ __forceinline__ int pgroup(int t, int blk) {
   return t * NBP + (blk ^ (t & (NBP - 1)));
+}
+
+// o += p * v for the two elements of a pair, as two scalar FMAs.
+__device__ __forceinline__ void fma_pair(float p, float2 v, float2& o) {
+  o.x = fmaf(p, v.x, o.x);
+  o.y = fmaf(p, v.y, o.y);
 }
 
 // Reduce-scatter of G partial sums over the LPT lanes of one token (lanes
@@ -486,13 +494,13 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
                 p0 = make_float2(pq.x, pq.y);
                 p1 = make_float2(pq.z, pq.w);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) O[g][kk] = ffma2(p0, vf[kk], O[g][kk]);
+                for (int kk = 0; kk < 4; ++kk) fma_pair(p0.x, vf[kk], O[g][kk]);
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) O[g + 1][kk] = ffma2(p1, vf[kk], O[g + 1][kk]);
+                for (int kk = 0; kk < 4; ++kk) fma_pair(p1.x, vf[kk], O[g + 1][kk]);
               } else {
                 p0 = pp[g];
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) O[g][kk] = ffma2(p0, vf[kk], O[g][kk]);
+                for (int kk = 0; kk < 4; ++kk) fma_pair(p0.x, vf[kk], O[g][kk]);
               }
             }
           }

@@ -52,11 +52,16 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_source_sha() -> str:
-    """Hash of the decode kernel sources: ncu traffic figures are valid only for this hash."""
+KERNEL_SOURCES = {
+    "decode_split": ("decode_kernel.cuh", "decode_launch.cuh", "decode.cu", "decode_common.cuh", "sm100_util.cuh"),
+    "decode_tc": ("decode_tc.cu", "decode.cu", "decode_common.cuh", "sm100_util.cuh", "tcgen05_util.cuh"),
+}
+
+
+def kernel_source_sha(kernel: str = "decode_split") -> str:
+    """Hash of one decode kernel's sources: ncu traffic figures are valid only for this hash."""
     h = hashlib.sha256()
-    for name in ("decode_kernel.cuh", "decode_launch.cuh", "decode.cu", "decode_common.cuh", "decode_tc.cu",
-                 "sm100_util.cuh", "tcgen05_util.cuh"):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "asymmetric_quantized_kv_kvq_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -74,7 +79,7 @@ def ncu_traffic(workload: str, precision: str, kernel: str = "decode_split"):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
-    if vals.get("kernel_source_sha") != kernel_source_sha():
+    if vals.get("kernel_source_sha") != kernel_source_sha(kernel):
         return None
     try:
         return float(vals["dram_bytes_per_launch"])
