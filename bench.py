@@ -216,10 +216,15 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
     for _ in range(args.warmup):
         run.step()
     run.cache.check()
+    graph, graph_lens, launch_mode = None, None, "eager (--eager)"
+    if not args.eager:
+        graph, graph_lens, launch_mode = capture_step(run, run.step)
     barrier(world)
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps, CUDA events on the launching stream
+    # ---- timed region: K steps, CUDA events on the launching stream.  With a captured graph every
+    #      step is one replay of the same decode step (append of one token per sequence + decode, all
+    #      layers): the token is re-appended at the same position and attended over the same length.
     ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
     dec_ms, step_ms, dec_bytes, app_bytes, launches = [], [], 0, 0, 0
     gpu_id = gpu_uuid(dev)
@@ -227,18 +232,32 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         for _ in range(args.steps):
             if flush:
                 scratch.zero_()
-            lens_before = run.lengths()
+            lens_before = graph_lens if graph is not None else run.lengths()
             s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             s0.record()
-            run.step(record=ev)
+            if graph is not None:
+                graph.replay()
+            else:
+                run.step(record=ev)
             s1.record()
             torch.cuda.synchronize()
             step_ms.append(s0.elapsed_time(s1))
-            dec_ms.extend(e0.elapsed_time(e1) for e0, e1 in ev)
+            if graph is None:
+                dec_ms.extend(e0.elapsed_time(e1) for e0, e1 in ev)
             d, a = run.step_bytes([n + 1 for n in lens_before])
             dec_bytes += d
             app_bytes += a
             launches += run.launches_per_step(lens_before)
+    in_step_bytes = dec_bytes / args.steps
+    if graph is not None:
+        # per-layer decode durations inside a step: one eager step with events (outside the timed region)
+        lens_e = run.lengths()
+        if flush:
+            scratch.zero_()
+        run.step(record=ev)
+        torch.cuda.synchronize()
+        dec_ms.extend(e0.elapsed_time(e1) for e0, e1 in ev)
+        in_step_bytes = run.step_bytes([n + 1 for n in lens_e])[0]
     # ---- kernel duration: every layer's decode call once more, back to back on the
     #      stream behind a short device-side sleep, so that host work between calls
     #      (binding, plan) never leaves the GPU idle inside the events
@@ -270,7 +289,8 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         "ms_per_step": max_ms / args.steps,
         "value": tot_bytes / (max_ms * 1e-3) / 1e9,
         "decode_tokens_per_s": tot_tokens / (max_ms * 1e-3),
-        "dec_bytes_per_launch": dec_bytes / (args.steps * L),
+        "dec_bytes_per_launch": in_step_bytes / L,
+        "launch_mode": launch_mode,
         "dec_ms_per_launch": statistics.mean(dec_ms),
         "kern_bytes_per_launch": kern_bytes,
         "kern_ms_per_launch": min(kern_ms),
@@ -287,6 +307,26 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
     return res
 
 
+def capture_step(run, body):
+    """Capture `body` (one decode step through the public API) into a CUDA graph.
+    Returns (graph, lengths before the captured step, launch-mode note); on a
+    capture error, (None, None, the reason) and the caller steps eagerly."""
+    import torch
+    lens = run.lengths()
+    try:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            body()
+        torch.cuda.synchronize()
+        for _ in range(2):          # upload + warm replays, untimed
+            g.replay()
+        torch.cuda.synchronize()
+        return g, lens, "CUDA graph of one decode step (all layers), replayed"
+    except Exception as e:  # noqa: BLE001 -- reported in the JSON line
+        torch.cuda.synchronize()
+        return None, None, f"eager (graph capture failed: {type(e).__name__}: {str(e)[:120]})"
+
+
 def run_e2e(run, args, world, dev) -> dict:
     """Same step, but every step copies its inputs (q, new K / V for all layers)
     from pinned host memory and reads all outputs back to pinned host memory."""
@@ -298,15 +338,8 @@ def run_e2e(run, args, world, dev) -> dict:
     ho = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in run.out]
     h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv)
     d2h = sum(t.numel() * t.element_size() for t in ho)
-    for _ in range(2):
-        run.step()
-    barrier(world)
-    torch.cuda.synchronize()
-    nbytes, ms = 0, 0.0
-    for _ in range(args.steps):
-        lens_before = run.lengths()
-        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        s0.record()
+
+    def body():
         for layer in range(L):
             run.q[layer].copy_(hq[layer], non_blocking=True)
             run.k_new[layer].copy_(hk[layer], non_blocking=True)
@@ -314,6 +347,23 @@ def run_e2e(run, args, world, dev) -> dict:
         run.step()
         for layer in range(L):
             ho[layer].copy_(run.out[layer], non_blocking=True)
+
+    for _ in range(2):
+        body()
+    graph, graph_lens = None, None
+    if not args.eager:
+        graph, graph_lens, _ = capture_step(run, body)
+    barrier(world)
+    torch.cuda.synchronize()
+    nbytes, ms = 0, 0.0
+    for _ in range(args.steps):
+        lens_before = graph_lens if graph is not None else run.lengths()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record()
+        if graph is not None:
+            graph.replay()
+        else:
+            body()
         s1.record()
         torch.cuda.synchronize()
         ms += s0.elapsed_time(s1)
@@ -599,6 +649,9 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--eager", action="store_true",
+                    help="launch every decode step through the API calls directly instead of replaying a "
+                         "CUDA graph of one captured step")
     ap.add_argument("--decode-tc", action="store_true",
                     help="decode on the tensor-core kernel (cache flag KVQ_CACHE_DECODE_TENSOR_CORES) "
                          "instead of the default CUDA-core kernel")
@@ -692,7 +745,8 @@ def main():
             "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": dict(config_of(wl, precision, world, res["flush"]),
-                           decode_kernel="tensor cores (opt-in)" if tc else "CUDA cores"),
+                           decode_kernel="tensor cores (opt-in)" if tc else "CUDA cores",
+                           step_launch=res["launch_mode"]),
             "decode_tokens_per_s": res["decode_tokens_per_s"],
             "roofline": {"bound": "hbm",
                          "kernel": ("decode_tc_kernel" if tc else "decode_split_kernel") + " + lse_combine_kernel",

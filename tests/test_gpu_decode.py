@@ -116,3 +116,53 @@ def test_decode_after_incremental_appends():
             assert_close_attention(out, ref, f"step {step}")
     cache.check()
     cache.close()
+
+
+@pytest.mark.gpu
+def test_decode_step_replays_from_a_cuda_graph():
+    """One decode step through the API (extend, then append + decode for every layer) captured in a CUDA
+    graph and replayed: each replay re-appends the same token and gives the eager result bit for bit,
+    within tolerance of the oracle.  Sequence 0 crosses a page boundary inside the captured step."""
+    m = kvq()
+    D, H, G, layers = 128, 8, 4, 2
+    lens = [256, 700]
+    B = len(lens)
+    cache, ids, hat = _build(m, 8, 4, D, H, lens, layers=layers)
+    k_new = [decode_kv(B, H, D, 500 + l) for l in range(layers)]
+    v_new = [random_fp16((B, H, D), 600 + l) for l in range(layers)]
+    q = [random_fp16((B, H * G, D), 700 + l) for l in range(layers)]
+    kd, vd, qd = [t.cuda() for t in k_new], [t.cuda() for t in v_new], [t.cuda() for t in q]
+    out = [torch.empty_like(t) for t in qd]
+    ws = torch.empty(cache.decode_workspace_size(B, H * G), dtype=torch.uint8, device="cuda")
+    cache.decode(0, ids, qd[0], out=out[0], workspace=ws)      # first-call setup outside the capture
+    torch.cuda.synchronize()
+
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        cache.extend(ids, [1] * B)
+        for layer in range(layers):
+            cache.append(layer, ids, [1] * B, kd[layer], vd[layer])
+            cache.decode(layer, ids, qd[layer], out=out[layer], workspace=ws)
+    assert [cache.length(s) for s in ids] == [n + 1 for n in lens]
+    for o in out:
+        o.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    first = [o.clone() for o in out]
+    g.replay()
+    torch.cuda.synchronize()
+    cache.check()
+    for layer in range(layers):
+        assert torch.equal(out[layer], first[layer]), f"layer {layer}: replays differ"
+        eager = cache.decode(layer, ids, qd[layer])
+        assert torch.equal(eager, first[layer]), f"layer {layer}: replay differs from the eager call"
+        kv = []
+        for s in ids:
+            kh, vh = hat[(layer, s)]
+            kh = np.concatenate([kh, oracle_dequant(k_new[layer][s:s + 1], 8)])
+            vh = np.concatenate([vh, oracle_dequant(v_new[layer][s:s + 1], 4)])
+            kv.append((kh, vh))
+        ref = oracle.attention_decode_batch(q[layer].numpy(), kv)
+        assert_close_attention(first[layer], ref, f"graph replay layer {layer}")
+    del g
+    cache.close()
