@@ -72,6 +72,20 @@ struct PrefillBatch {
   PrefillSeq s[kMaxBatch];
 };
 
+// Softmax arithmetic of the attention kernel: three-input max, and 2^x by the
+// MUFU approximation with subnormal results flushed (p < 2^-126 contributes
+// nothing visible once P is rounded to fp16 for the PV MMA).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float ex2_ftz(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ int find_seq_by(const PrefillBatch& b, int x, bool by_tiles) {
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
@@ -406,7 +420,8 @@ __global__ void __launch_bounds__(352, 1)
               if (kpos0 + 32 * c + i <= qpos) mx = fmaxf(mx, __uint_as_float(sv[32 * c + i]));
           } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sv[32 * c + i]));
+            for (int i = 0; i < 32; i += 2)
+              mx = fmax3(mx, __uint_as_float(sv[32 * c + i]), __uint_as_float(sv[32 * c + i + 1]));
           }
         }
       } else {
@@ -444,7 +459,9 @@ __global__ void __launch_bounds__(352, 1)
         }
       }
       // pass 2: P = 2^(sigma log2 e s - m) as fp16 pairs into P buffer j & 1 (this half's 32 columns)
-      const float neg_m = -m_used;
+      // (pairs: one f32x2 FMA scales and shifts two scores, one f32x2 add sums two p)
+      const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_used, -m_used);
+      float2 l2 = make_float2(0.f, 0.f);
       const uint32_t pbuf = lane_addr + T::P_COL0 + (j & 1) * (kKV / 2) + 32 * half;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -452,19 +469,22 @@ __global__ void __launch_bounds__(352, 1)
         const bool masked = kpos0 + 32 * c + 31 > qpos0;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          float p0 = exp2f(fmaf(__uint_as_float(sv[32 * c + 2 * i]), a.scale_log2, neg_m));
-          float p1 = exp2f(fmaf(__uint_as_float(sv[32 * c + 2 * i + 1]), a.scale_log2, neg_m));
+          const float2 x = ffma2(make_float2(__uint_as_float(sv[32 * c + 2 * i]),
+                                             __uint_as_float(sv[32 * c + 2 * i + 1])), sc2, nm2);
+          float p0 = ex2_ftz(x.x);
+          float p1 = ex2_ftz(x.y);
           if (masked) {
             const int k0 = kpos0 + 32 * c + 2 * i;
             p0 = k0 > qpos ? 0.f : p0;
             p1 = k0 + 1 > qpos ? 0.f : p1;
           }
-          l += p0 + p1;
+          l2 = fadd2(l2, make_float2(p0, p1));
           __half2 hp = __floats2half2_rn(p0, p1);
           pk[i] = *reinterpret_cast<uint32_t*>(&hp);
         }
         if (wok) tmem_st16(pbuf + 16 * c, pk);
       }
+      l += l2.x + l2.y;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(B_P + (j & 1)));

@@ -163,7 +163,8 @@ KVQ_API kvq_status kvq_seq_page(const kvq_cache* cache, int32_t seq_id, int32_t 
  * i.e. positions [len - n_new[i], len).  k, v: device fp16
  * [sum_i n_new[i], n_kv_heads, head_dim], sequences' rows in call order.
  * Quantises every 32-element block along head_dim to the cache's K / V bit
- * widths (format above) and stores codes and scales into the sequence's pages. */
+ * widths (format above) and stores codes and scales into the sequence's pages.
+ * k and v must be 16-byte aligned (KVQ_ERR_INVALID_ARG otherwise). */
 KVQ_API kvq_status kvq_append(kvq_cache* cache, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
                       const int32_t* n_new, const void* k, const void* v, kvq_stream_t stream);
 
@@ -179,7 +180,12 @@ KVQ_API kvq_status kvq_decode_workspace_size(const kvq_cache* cache, int32_t n_s
  * q, out: device fp16 [n_seqs, n_q_heads, head_dim].  Split-KV flash-decoding:
  * partial (O, max, sum) per slice of the cache in `workspace` (device,
  * ws_bytes >= kvq_decode_workspace_size), merged by a log-sum-exp combine.
- * Every named sequence must have len >= 1. */
+ * Every named sequence must have len >= 1.  q, out and workspace must be
+ * 16-byte aligned (KVQ_ERR_INVALID_ARG otherwise).
+ * kvq_seq_extend, kvq_append, kvq_decode_attn and kvq_prefill_attn only
+ * validate on the host and enqueue kernels on `stream` (no allocation, no
+ * synchronisation), so a decode step made of them can be captured in a CUDA
+ * graph and replayed. */
 KVQ_API kvq_status kvq_decode_attn(kvq_cache* cache, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
                            int32_t n_q_heads, const void* q, void* out, float softmax_scale,
                            void* workspace, size_t ws_bytes, kvq_stream_t stream);
@@ -216,8 +222,10 @@ KVQ_API kvq_status kvq_prefill_workspace_size(const kvq_cache* cache, int32_t n_
  * appended to the cache); row r attends causally to positions
  * 0 .. len - q_lens[i] + r, i.e. the cached tokens and the chunk up to itself,
  * all dequantised.  q, out: device fp16 [sum_i q_lens[i], n_q_heads, head_dim].
- * Tensor cores (tcgen05) compute Q K^T and P V in fp16 with fp32 accumulation;
- * the dequantised K / V are rounded to fp16 first. */
+ * Tensor cores (tcgen05) compute Q K^T and P V from fp16 operands with fp32
+ * accumulation: the dequantised K enters as two fp16 terms (its fp16 rounding
+ * and the remainder, about 22 bits together), V and P are rounded to fp16.
+ * q, out and workspace must be 16-byte aligned. */
 KVQ_API kvq_status kvq_prefill_attn(kvq_cache* cache, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
                             const int32_t* q_lens, int32_t n_q_heads, const void* q, void* out,
                             float softmax_scale, void* workspace, size_t ws_bytes,
