@@ -21,9 +21,16 @@ cudaError_t launch_decode_tc(const Layout& L, int layer, const Batch& b, const D
 
 namespace {
 
-__global__ void lse_combine_kernel(const __grid_constant__ Batch b, int H, int G, int D, int n_q_heads, int64_t cpc,
+// One warp per (item, query head).  The lanes share the item's partial slots:
+// each lane reads the (m, l) of slots lane, lane + 32, ... for the warp-wide max
+// M and sum L, then the warp walks the slots once, every lane accumulating its
+// D / 32 contiguous elements of O (one vector load per slot, weights broadcast
+// by shuffle), so the loads of successive slots are independent.
+template <int D>
+__global__ void lse_combine_kernel(const __grid_constant__ Batch b, int H, int G, int n_q_heads, int64_t cpc,
                                    const float* __restrict__ ws_o, const float* __restrict__ ws_ml,
                                    __half* __restrict__ out) {
+  constexpr int E = D / 32;   // elements per lane: 2 (D = 64) or 4 (D = 128)
   const int lane = threadIdx.x & 31;
   const int64_t wid = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (wid >= int64_t(b.n) * H * G) return;
@@ -33,20 +40,42 @@ __global__ void lse_combine_kernel(const __grid_constant__ Batch b, int H, int G
   const int64_t off = int64_t(b.s[bi].b) + int64_t(h) * nch;
   const int64_t c0 = off / cpc, c1 = (off + nch - 1) / cpc;
   if (c0 == c1) return;   // written directly by the split kernel
+  const int n = int(c1 - c0 + 1);
+  const float* ml = ws_ml + ((c0 + item) * G + g) * 2;          // slot c0 + i at ml[2 * G * i]
   float M = -INFINITY;
-  for (int64_t c = c0; c <= c1; ++c) M = fmaxf(M, ws_ml[((c + item) * G + g) * 2]);
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[int64_t(2) * G * i]);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float L = 0.f;
-  for (int64_t c = c0; c <= c1; ++c) {
-    const float* ml = ws_ml + ((c + item) * G + g) * 2;
-    L += exp2f(ml[0] - M) * ml[1];
+  for (int i = lane; i < n; i += 32) L += exp2f(ml[int64_t(2) * G * i] - M) * ml[int64_t(2) * G * i + 1];
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  const float* o0 = ws_o + ((c0 + item) * G + g) * D + E * lane;  // slot c0 + i at o0[G * D * i]
+  for (int base = 0; base < n; base += 32) {
+    const int i = base + lane;
+    const float w = i < n ? exp2f(ml[int64_t(2) * G * i] - M) : 0.f;
+    const int cnt = min(32, n - base);
+#pragma unroll 4
+    for (int k = 0; k < cnt; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, k);
+      const float* src = o0 + int64_t(G) * D * (base + k);
+      if constexpr (E == 4) {
+        const float4 v = *reinterpret_cast<const float4*>(src);
+        acc[0] = fmaf(wk, v.x, acc[0]); acc[1] = fmaf(wk, v.y, acc[1]);
+        acc[2] = fmaf(wk, v.z, acc[2]); acc[3] = fmaf(wk, v.w, acc[3]);
+      } else {
+        const float2 v = *reinterpret_cast<const float2*>(src);
+        acc[0] = fmaf(wk, v.x, acc[0]); acc[1] = fmaf(wk, v.y, acc[1]);
+      }
+    }
   }
   const float inv = 1.f / L;
-  for (int d = lane; d < D; d += 32) {
-    float acc = 0.f;
-    for (int64_t c = c0; c <= c1; ++c)
-      acc += exp2f(ws_ml[((c + item) * G + g) * 2] - M) * ws_o[((c + item) * G + g) * D + d];
-    out[(int64_t(bi) * n_q_heads + h * G + g) * D + d] = __float2half_rn(acc * inv);
-  }
+  __half* dst = out + (int64_t(bi) * n_q_heads + h * G + g) * D + E * lane;
+#pragma unroll
+  for (int e = 0; e < E; e += 2) *reinterpret_cast<__half2*>(dst + e) = __floats2half2_rn(acc[e] * inv, acc[e + 1] * inv);
 }
 
 }  // namespace
@@ -99,8 +128,13 @@ cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const Deco
     const float* ws_o = static_cast<const float*>(ws);
     const float* ws_ml = ws_o + slots * G * D;
     const int64_t warps = int64_t(plan.n_items) * G;
-    lse_combine_kernel<<<unsigned((warps + 7) / 8), 256, 0, s>>>(b, H, G, D, n_q_heads, plan.chunks_per_cta, ws_o,
-                                                                 ws_ml, static_cast<__half*>(out));
+    const unsigned blocks = unsigned((warps + 7) / 8);
+    if (D == 128)
+      lse_combine_kernel<128><<<blocks, 256, 0, s>>>(b, H, G, n_q_heads, plan.chunks_per_cta, ws_o, ws_ml,
+                                                     static_cast<__half*>(out));
+    else
+      lse_combine_kernel<64><<<blocks, 256, 0, s>>>(b, H, G, n_q_heads, plan.chunks_per_cta, ws_o, ws_ml,
+                                                    static_cast<__half*>(out));
     e = cudaGetLastError();
   }
   return e;
