@@ -10,10 +10,11 @@
 //
 // Two passes:
 //  1. dequant_tiles_kernel: every (sequence, KV head) of the batch is
-//     dequantised once, in 64-token tiles of a workspace: K as two fp16 tiles
-//     K_hi = fp16(k^) and K_lo = fp16(k^ - K_hi) [64 tokens][D] (fp16 alone
-//     would round the x10 outlier key channels by up to 2^-12 relative, which
-//     moves the softmax by ~0.2%; hi + lo keeps ~22 bits), and V transposed
+//     dequantised once, in 64-token tiles of a workspace: K as K_hi = fp16(k^)
+//     [64 tokens][D] plus the remainder K_lo = k^ - K_hi (fp16 alone would
+//     round the x10 outlier key channels by up to 2^-12 relative, which moves
+//     the softmax by ~0.2%), stored as e5m2 x 2^8 at head_dim 128 (k^ to
+//     ~2^-15) and as fp16 at head_dim 64 (~22 bits), and V transposed
 //     [D][64 tokens] in fp16, so both MMAs read K-major operands.
 //     (Dequantising inside the attention kernel would redo it for every
 //     128-row query tile: a 4096-token chunk with 4 query heads per KV head
@@ -24,9 +25,13 @@
 //     swizzle): lane 0 fills a ring of K_hi / K_lo slots, lane 1 a separate
 //     ring of V^T slots, so a key slot refills as soon as its scores are done.
 //     Warp 1 owns all 512 TMEM columns (S double buffer, O, P double buffer)
-//     and issues tcgen05.mma kind::f16 (fp16 x fp16 -> fp32):
-//        S_j = Q K_hi,j^T + Q K_lo,j^T   (M 128, N 128: 2 x D/16 MMAs per 128 keys)
-//        O  += P_j V_j                   (A = P read from TMEM, 8 MMAs per 128 keys).
+//     and issues the score MMAs, warp 10 the PV MMAs (fp32 accumulators):
+//        S_j = Q K_hi,j^T + Q8 K_lo,j^T  (M 128, N 128: D/16 kind::f16 MMAs and, at
+//                                         head_dim 128, D/32 kind::f8f6f4 MMAs on e5m2
+//                                         operands, Q8 = e5m2(Q 2^-8) converted once
+//                                         per CTA by the softmax warps; at head_dim 64
+//                                         K_lo is fp16 and Q K_lo^T takes D/16 more)
+//        O  += P_j V_j                   (kind::f16, A = P read from TMEM, 8 MMAs per 128 keys).
 //     A tcgen05.mma costs roughly the same time for N up to 128, so wide key
 //     tiles halve the instruction count of 64-key ones.  Warps 2-9 run the
 //     softmax, two per TMEM lane quadrant (one thread per row, 64 keys each):
@@ -86,6 +91,23 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   return y;
 }
 
+// The remainder K_lo = k^ - fp16(k^) enters the scores at head_dim 128 as e5m2
+// (2 mantissa bits, scaled by 2^8) against an e5m2 copy of Q scaled by 2^-8,
+// through a kind::f8f6f4 MMA (K = 32 per instruction, twice the fp16 rate):
+// the correction term is then exact to ~2^-3 of itself, i.e. k^ to ~2^-15.
+// At head_dim 64 K_lo stays fp16.
+template <int D>
+constexpr bool kLo8 = D == 128;
+constexpr float kLoScale = 256.f, kQ8Scale = 1.f / 256.f;
+
+// two fp32 -> e5m2 (round to nearest even, saturating to the largest finite);
+// `first` lands in the low byte
+__device__ __forceinline__ uint32_t e5m2x2(float first, float second) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
+  return r;
+}
+
 __device__ __forceinline__ int find_seq_by(const PrefillBatch& b, int x, bool by_tiles) {
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
@@ -100,7 +122,7 @@ __device__ __forceinline__ int find_seq_by(const PrefillBatch& b, int x, bool by
 template <int D>
 __global__ void __launch_bounds__(256) dequant_tiles_kernel(const Layout L, int layer,
                                                             const __grid_constant__ PrefillBatch b,
-                                                            __half* __restrict__ khi, __half* __restrict__ klo,
+                                                            __half* __restrict__ khi, void* __restrict__ klo,
                                                             __half* __restrict__ vws) {
   __shared__ __align__(16) __half vt[kKT][D + 8];
   const int gt = blockIdx.x;
@@ -162,12 +184,23 @@ __global__ void __launch_bounds__(256) dequant_tiles_kernel(const Layout L, int 
     __half hi[8], lo[8];
     deq(L.k_bits, blk, blk + L.k_scales_off, e0, x);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      hi[i] = __float2half_rn(x[i]);
-      lo[i] = __float2half_rn(x[i] - __half2float(hi[i]));
-    }
+    for (int i = 0; i < 8; ++i) hi[i] = __float2half_rn(x[i]);
     *reinterpret_cast<uint4*>(khi + tile_off + t * D + e0) = *reinterpret_cast<uint4*>(hi);
-    *reinterpret_cast<uint4*>(klo + tile_off + t * D + e0) = *reinterpret_cast<uint4*>(lo);
+    if constexpr (kLo8<D>) {
+      // x - fp16(x) is exact in fp32 (x has at most 19 significant bits), and so is the 2^8 scaling
+      uint32_t w[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+        w[i] = e5m2x2((x[4 * i] - __half2float(hi[4 * i])) * kLoScale,
+                      (x[4 * i + 1] - __half2float(hi[4 * i + 1])) * kLoScale) |
+               (e5m2x2((x[4 * i + 2] - __half2float(hi[4 * i + 2])) * kLoScale,
+                       (x[4 * i + 3] - __half2float(hi[4 * i + 3])) * kLoScale) << 16);
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(klo) + tile_off + t * D + e0) = make_uint2(w[0], w[1]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) lo[i] = __float2half_rn(x[i] - __half2float(hi[i]));
+      *reinterpret_cast<uint4*>(static_cast<__half*>(klo) + tile_off + t * D + e0) = *reinterpret_cast<uint4*>(lo);
+    }
     deq(L.v_bits, blk + L.v_codes_off, blk + L.v_scales_off, e0, x);
 #pragma unroll
     for (int i = 0; i < 8; ++i) hi[i] = __float2half_rn(x[i]);
@@ -193,11 +226,15 @@ struct PTraits {
   static constexpr int Q_BYTES = kQT * D * 2;            // CB blocks of [128 rows][128 B]
   static constexpr int K_BYTES = kKV * D * 2;            // CB blocks of [128 rows][128 B]
   static constexpr int V_BYTES = D * kKV * 2;            // two blocks (64 tokens each) of [D rows][128 B]
-  static constexpr int KSLOT = 2 * K_BYTES;              // K_hi, K_lo of one 128-key tile
+  static constexpr bool LO8 = kLo8<D>;
+  static constexpr int KLO_BYTES = LO8 ? kKV * D : K_BYTES;   // e5m2: one block of [128 rows][128 B]
+  static constexpr int Q8_BYTES = LO8 ? kQT * D : 0;          // e5m2 copy of Q, [128 rows][128 B]
+  static constexpr int KSLOT = K_BYTES + KLO_BYTES;      // K_hi, K_lo of one 128-key tile
   static constexpr int NSTAGE = D == 128 ? 2 : 3;        // slots of each ring (keys and values separately,
                                                          // so a key slot is refilled as soon as S is done)
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_Q8 = OFF_Q + Q_BYTES;
+  static constexpr int OFF_K = OFF_Q8 + Q8_BYTES;
   static constexpr int OFF_V = OFF_K + NSTAGE * KSLOT;
   static constexpr int OFF_BAR = OFF_V + NSTAGE * V_BYTES;
   // + alignment slack; never less than ~116 KB so that a second CTA cannot
@@ -210,7 +247,8 @@ struct PTraits {
   // (fp16 pairs, 64 columns = 128 keys each)
   static constexpr uint32_t S_COL0 = 0, O_COL = 256, P_COL0 = 384;
   static_assert(O_COL + D <= P_COL0 && P_COL0 + 2 * kKV / 2 <= TMEM_COLS, "TMEM");
-  static_assert(OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && KSLOT % 1024 == 0 && V_BYTES % 1024 == 0,
+  static_assert(OFF_Q8 % 1024 == 0 && OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && KSLOT % 1024 == 0 &&
+                    K_BYTES % 1024 == 0 && V_BYTES % 1024 == 0,
                 "swizzle atoms");
   static_assert(SMEM <= 227 * 1024, "shared memory");
 };
@@ -238,8 +276,8 @@ __global__ void __launch_bounds__(352, 1)
   // barriers: q_full | k_full[NS] | k_empty[NS] | v_full[NS] | v_empty[NS] | s_full[2] | p_full | pv_done | done
   constexpr int B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + NS, B_VFULL = 1 + 2 * NS, B_VEMPTY = 1 + 3 * NS,
                 B_S = 1 + 4 * NS, B_SFREE = 3 + 4 * NS, B_P = 5 + 4 * NS, B_PV = 7 + 4 * NS, B_DONE = 9 + 4 * NS,
-                B_DONE2 = 10 + 4 * NS;   // S, SFREE, P, PV: one barrier per buffer parity
-  static_assert(B_DONE2 < 24, "barrier area");
+                B_DONE2 = 10 + 4 * NS, B_Q8 = 11 + 4 * NS;   // S, SFREE, P, PV: one barrier per buffer parity
+  static_assert(B_Q8 < 24, "barrier area");
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 25);
 
@@ -257,8 +295,8 @@ __global__ void __launch_bounds__(352, 1)
   const int tile_base = sq.tile_base + h * sq.n_tiles;     // first 64-token pass-1 tile of this head
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i <= B_DONE2; ++i)
-      mbar_init(bar(i), (i == B_P || i == B_P + 1 || i == B_SFREE || i == B_SFREE + 1) ? 256u : 1u);
+    for (int i = 0; i <= B_Q8; ++i)
+      mbar_init(bar(i), (i == B_P || i == B_P + 1 || i == B_SFREE || i == B_SFREE + 1 || i == B_Q8) ? 256u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -288,8 +326,9 @@ __global__ void __launch_bounds__(352, 1)
         const int t64 = tile_base + 2 * j;                   // two consecutive pass-1 tiles
         for (int cb = 0; cb < T::CB; ++cb) {
           tma_load_2d(st + cb * kKV * 128, &tm_khi, cb * 64, t64 * 64, full);
-          tma_load_2d(st + T::K_BYTES + cb * kKV * 128, &tm_klo, cb * 64, t64 * 64, full);
+          if (!T::LO8) tma_load_2d(st + T::K_BYTES + cb * kKV * 128, &tm_klo, cb * 64, t64 * 64, full);
         }
+        if (T::LO8) tma_load_2d(st + T::K_BYTES, &tm_klo, 0, t64 * 64, full);
         ++issued;
       }
       // no copy may outlive the CTA
@@ -322,8 +361,10 @@ __global__ void __launch_bounds__(352, 1)
     // score MMAs and the PV MMAs are issued by two warps; they touch disjoint TMEM columns.
     if (lane == 0) {
       constexpr uint32_t idS = idesc_f16_f32(kQT, kKV);
+      constexpr uint32_t idS8 = idesc_e5m2_f32(kQT, kKV);
       bool ok = mbar_wait(bar(B_Q), 0, abort_flag);
       const uint64_t qd0 = sdesc_k_sw128(base + T::OFF_Q);
+      const uint64_t q8d0 = sdesc_k_sw128(base + T::OFF_Q8);
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % NS;
         // S buffer j & 1 was read by the softmax of tile j - 2; the key slot is full
@@ -333,13 +374,31 @@ __global__ void __launch_bounds__(352, 1)
         tc_fence_after();
         const uint64_t kd0 = sdesc_k_sw128(base + T::OFF_K + s * T::KSLOT);
         const uint32_t dst = tmem + T::S_COL0 + (j & 1) * kKV;
+        if constexpr (T::LO8) {
 #pragma unroll
-        for (int part = 0; part < 2; ++part) {          // K_hi then K_lo, accumulated
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
+          for (int k = 0; k < D / 16; ++k) {          // Q K_hi^T (fp16)
             const uint32_t qoff = (k >> 2) * kQT * 128 + (k & 3) * 32;
-            const uint32_t koff = part * T::K_BYTES + (k >> 2) * kKV * 128 + (k & 3) * 32;
-            umma_f16(dst, qd0 + (qoff >> 4), kd0 + (koff >> 4), idS, (part | k) != 0);
+            const uint32_t koff = (k >> 2) * kKV * 128 + (k & 3) * 32;
+            umma_f16(dst, qd0 + (qoff >> 4), kd0 + (koff >> 4), idS, k != 0);
+          }
+          // + Q8 K_lo8^T (e5m2, 32 elements = 32 B per MMA); Q8 is written by the softmax warps once
+          if (j == 0 && !mbar_wait(bar(B_Q8), 0, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k)
+            umma_f8(dst, q8d0 + ((k * 32) >> 4), kd0 + ((T::K_BYTES + k * 32) >> 4), idS8, 1);
+        } else {
+#pragma unroll
+          for (int part = 0; part < 2; ++part) {        // K_hi then K_lo, accumulated
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint32_t qoff = (k >> 2) * kQT * 128 + (k & 3) * 32;
+              const uint32_t koff = part * T::K_BYTES + (k >> 2) * kKV * 128 + (k & 3) * 32;
+              umma_f16(dst, qd0 + (qoff >> 4), kd0 + (koff >> 4), idS, (part | k) != 0);
+            }
           }
         }
         umma_commit(bar(B_S + (j & 1)));
@@ -396,6 +455,30 @@ __global__ void __launch_bounds__(352, 1)
     float* redmax = reinterpret_cast<float*>(bars + 32);        // [2 halves][128 rows]
     float m_used = -INFINITY, l = 0.f;
     bool wok = true;
+    if constexpr (T::LO8) {
+      // Q8 = e5m2(Q 2^-8): thread (row r, half hf) converts elements [64 hf, 64 hf + 64) of row r from
+      // the fp16 tile (column block hf, 128-byte swizzle) into the e5m2 tile (one column block)
+      const int st = threadIdx.x - 64, r = st >> 1, hf = st & 1;
+      if (mbar_wait(bar(B_Q), 0, abort_flag)) {
+        const uint8_t* src = smem + T::OFF_Q + hf * kQT * 128 + r * 128;
+        uint8_t* dq = smem + T::OFF_Q8 + r * 128;
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint4 w = *reinterpret_cast<const uint4*>(src + ((c8 ^ (r & 7)) << 4));
+          const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+          uint32_t o[2];
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const float2 f0 = h2_to_f2(ws[2 * i]), f1 = h2_to_f2(ws[2 * i + 1]);
+            o[i] = e5m2x2(f0.x * kQ8Scale, f0.y * kQ8Scale) | (e5m2x2(f1.x * kQ8Scale, f1.y * kQ8Scale) << 16);
+          }
+          const int x = 64 * hf + 8 * c8;                         // byte = element index in the e5m2 row
+          *reinterpret_cast<uint2*>(dq + ((((x >> 4) ^ (r & 7)) << 4) | (x & 8))) = make_uint2(o[0], o[1]);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
+      mbar_arrive(bar(B_Q8));
+    }
     int j = 0;
     for (; j < n_kv; ++j) {
       bool w = __all_sync(0xffffffffu, mbar_wait(bar(B_S + (j & 1)), (j >> 1) & 1, abort_flag));
@@ -573,7 +656,7 @@ cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_
   const PrefillBatch b = plan(L, in, n_q_heads, &n_tiles, &n_qt);
   const int64_t per = n_tiles * kKT * D;
   __half* khi = static_cast<__half*>(ws);
-  __half* klo = khi + per;
+  __half* klo = khi + per;          // fp16 [tokens][D], or e5m2 [tokens][D] in its first half (head_dim 128)
   __half* vws = klo + per;
   dequant_tiles_kernel<D><<<unsigned(n_tiles), 256, 0, s>>>(L, layer, b, khi, klo, vws);
   cudaError_t e = cudaGetLastError();
@@ -592,7 +675,13 @@ cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_
     cuuint64_t strides[1] = {cuuint64_t(D) * 2};
     cuuint32_t box[2] = {64, kKV};
     if (!make_tensor_map(&mkh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, khi, 2, dims, strides, box)) return cudaErrorInvalidValue;
-    if (!make_tensor_map(&mkl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, klo, 2, dims, strides, box)) return cudaErrorInvalidValue;
+    if (kLo8<D>) {
+      cuuint64_t strides8[1] = {cuuint64_t(D)};
+      cuuint32_t box8[2] = {cuuint32_t(D), kKV};
+      if (!make_tensor_map(&mkl, CU_TENSOR_MAP_DATA_TYPE_UINT8, klo, 2, dims, strides8, box8)) return cudaErrorInvalidValue;
+    } else if (!make_tensor_map(&mkl, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, klo, 2, dims, strides, box)) {
+      return cudaErrorInvalidValue;
+    }
   }
   {
     cuuint64_t dims[2] = {cuuint64_t(kKT), cuuint64_t(n_tiles) * D};

@@ -63,6 +63,13 @@ __host__ __device__ constexpr uint32_t idesc_f16_f32_amn(int M, int N) {
   return (1u << 4) | (1u << 15) | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f8f6f4: e5m2 A and B, fp32 accumulator, both K-major.
+__host__ __device__ constexpr uint32_t idesc_e5m2_f32(int M, int N) {
+  return (1u << 4)                       // D format: f32
+         | (1u << 7) | (1u << 10)        // A, B format: e5m2
+         | (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
+}
+
 // Instruction descriptor, kind::f16: fp16 A and B, fp32 accumulator, both K-major.
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4)                       // D format: f32
@@ -83,6 +90,14 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 // D[tmem] (+)= A[smem] * B[smem]^T with signed 8-bit operands and s32 accumulation.
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate) {
   asm volatile(

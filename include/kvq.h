@@ -223,8 +223,9 @@ KVQ_API kvq_status kvq_prefill_workspace_size(const kvq_cache* cache, int32_t n_
  * 0 .. len - q_lens[i] + r, i.e. the cached tokens and the chunk up to itself,
  * all dequantised.  q, out: device fp16 [sum_i q_lens[i], n_q_heads, head_dim].
  * Tensor cores (tcgen05) compute Q K^T and P V from fp16 operands with fp32
- * accumulation: the dequantised K enters as two fp16 terms (its fp16 rounding
- * and the remainder, about 22 bits together), V and P are rounded to fp16.
+ * accumulation: the dequantised K enters as its fp16 rounding plus the
+ * remainder (an e5m2 term against an e5m2 copy of q at head_dim 128, k to about
+ * 2^-15; an fp16 term at head_dim 64, about 22 bits), V and P are rounded to fp16.
  * q, out and workspace must be 16-byte aligned. */
 KVQ_API kvq_status kvq_prefill_attn(kvq_cache* cache, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
                             const int32_t* q_lens, int32_t n_q_heads, const void* q, void* out,
