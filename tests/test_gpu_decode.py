@@ -166,3 +166,22 @@ def test_decode_step_replays_from_a_cuda_graph():
         assert_close_attention(first[layer], ref, f"graph replay layer {layer}")
     del g
     cache.close()
+
+
+@pytest.mark.gpu
+def test_decode_at_the_maximum_batch():
+    """KVQ_MAX_BATCH sequences in one call (the batch descriptors travel as kernel parameters), with
+    lengths from 1 to a few pages; every output checked against the oracle."""
+    m = kvq()
+    D, H, G = 64, 2, 4
+    B = m.KVQ_MAX_BATCH
+    rng = np.random.default_rng(11)
+    lens = [int(x) for x in rng.integers(1, 700, size=B)]
+    lens[0], lens[-1] = 1, 256
+    cache, ids, hat = _build(m, 8, 4, D, H, lens)
+    q = random_fp16((B, H * G, D), 21)
+    out = cache.decode(0, ids, q.cuda())
+    cache.check()
+    ref = oracle.attention_decode_batch(q.numpy(), [hat[(0, s)] for s in ids])
+    assert_close_attention(out, ref, "max batch")
+    cache.close()
