@@ -53,7 +53,8 @@ __device__ __forceinline__ float round_mag(float x, const RoundCtx& r) {
   const float ax = fabsf(x);
   float n = __fadd_rn(__fmaf_rn(ax, r.ra, 12582912.0f), -12582912.0f);
   const float e = __fmaf_rn(-n, r.ad, ax);
-  n += (e >= r.hd ? 1.f : 0.f) - (e < -r.hd ? 1.f : 0.f);
+  if (e >= r.hd) n += 1.f;           // rare: two compares and predicated adds
+  if (e < -r.hd) n -= 1.f;
   return n;
 }
 __device__ __forceinline__ float round_code(float x, const RoundCtx& r, float cn, float cp) {
@@ -63,6 +64,12 @@ __device__ __forceinline__ float round_code(float x, const RoundCtx& r, float cn
 // 8-bit: d > 0, symmetric clamp
 __device__ __forceinline__ float round_code8(float x, const RoundCtx& r) {
   return copysignf(fminf(round_mag(x, r), 127.f), x);
+}
+// max(a, b, c) in one instruction
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 // Low byte of an exact integer v in [-128, 255] held in a float (two's complement for v < 0).
 __device__ __forceinline__ uint32_t float_int_bits(float v) { return __float_as_uint(v + 12582912.0f); }
@@ -95,7 +102,7 @@ __device__ __forceinline__ void load_block(const __half* src, float (&x)[32]) {
 __device__ __forceinline__ void quant8_block(const float (&x)[32], uint8_t* codes, __half* scale) {
   float a = 0.f;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(x[i]));
+  for (int i = 0; i < 32; i += 2) a = fmax3(a, fabsf(x[i]), fabsf(x[i + 1]));
   const __half d = __float2half_rn(__fdiv_rn(a, 127.0f));
   const float df = __half2float(d);
   uint32_t w[8];

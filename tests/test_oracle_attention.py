@@ -164,3 +164,51 @@ def test_keys_are_the_sensitive_half():
 
     assert err(4, 8) > 2 * err(8, 4)
     assert err(8, 8) < err(8, 4) < err(4, 4)
+
+
+def _e5m2(x):
+    """Round to the nearest e5m2 value (2 mantissa bits, ties to even, subnormals below 2^-14)."""
+    x = np.asarray(x, np.float64)
+    e = np.floor(np.log2(np.where(x != 0, np.abs(x), 1.0)))
+    ulp = 2.0 ** (np.maximum(e, -14) - 2)
+    return np.round(x / ulp) * ulp
+
+
+def test_prefill_score_split_keeps_attention_within_tolerance():
+    """The prefill kernel's reading of the scores at head_dim 128: s = q . fp16(k^) +
+    e5m2(2^-8 q) . e5m2(2^8 (k^ - fp16(k^))), with P and v^ rounded to fp16 for the PV product.
+    Emulated here in float64 on x10 outlier key channels, it stays within the tolerance of the
+    exact oracle with margin, while fp16(k^) alone uses several times more of it."""
+    rng = np.random.default_rng(3)
+    T, C, D = 1024, 16, 128
+    k = rng.standard_normal((T, 1, D)).astype(np.float16)
+    k[:, :, [5, 77]] *= np.float16(10)
+    v = rng.standard_normal((T, 1, D)).astype(np.float16)
+    kh = dequantize_kv(*quantize_kv(k, 8), 8)[:, 0, :]
+    vh = dequantize_kv(*quantize_kv(v, 4), 4)[:, 0, :]
+    q = rng.standard_normal((C, 1, D)).astype(np.float16).astype(np.float64)
+    ref = attention_prefill(q, kh[:, None, :], vh[:, None, :], T - C)[:, 0, :]
+
+    def f16(a):
+        return np.asarray(a).astype(np.float16).astype(np.float64)
+
+    hi = f16(kh)
+    lo8 = _e5m2((kh - hi) * 256.0)
+    sigma = 1.0 / math.sqrt(D)
+
+    def attend(scores):
+        out = np.empty((C, D))
+        for i in range(C):
+            n = T - C + i + 1
+            s = scores[i, :n] * sigma
+            p = np.exp(s - s.max())
+            out[i] = f16(p) @ f16(vh[:n]) / p.sum()
+        return out
+
+    split = attend(q[:, 0] @ hi.T + _e5m2(q[:, 0] / 256.0) @ lo8.T)
+    fp16_only = attend(q[:, 0] @ hi.T)
+    bound = 2e-3 + 1e-2 * np.abs(ref)
+    used_split = (np.abs(split - ref) / bound).max()
+    used_fp16 = (np.abs(fp16_only - ref) / bound).max()
+    assert used_split < 0.5, used_split
+    assert used_fp16 > 2 * used_split, (used_fp16, used_split)
