@@ -55,6 +55,7 @@ def measured_peaks() -> dict:
 KERNEL_SOURCES = {
     "decode_split": ("decode_kernel.cuh", "decode_launch.cuh", "decode.cu", "decode_common.cuh", "sm100_util.cuh"),
     "decode_tc": ("decode_tc.cu", "decode.cu", "decode_common.cuh", "sm100_util.cuh", "tcgen05_util.cuh"),
+    "append": ("append.cu", "kvq_internal.cuh"),
 }
 
 
@@ -794,7 +795,8 @@ def prefill_main(args, wl, precision, kb, vb, rank, world):
                             "ms_per_launch": res["append_kernel_ms"],
                             "timing": "CUDA events around 8 back-to-back appends of the chunk queued behind a "
                                       "device sleep",
-                            "achieved_in_step": res["append_gbs_in_step"]},
+                            "achieved_in_step": res["append_gbs_in_step"],
+                            "traffic": ncu_traffic(wl.name, precision, "append")},
         "roofline": {"bound": "tensor", "kernel": "dequant_tiles_kernel + prefill_attn_kernel",
                      "achieved": res["prefill_tflops"], "peak": peak["value"], "unit": "TFLOP/s",
                      "frac": res["prefill_tflops"] / peak["value"], "peak_source": peak["source"],
