@@ -81,8 +81,10 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint3
 // One thread quantises one 32-element block of one K or V row: it loads the
 // block's 64 bytes with four 16-byte loads, takes the block max in registers
 // (no shuffles, one scale and one reciprocal per block), rounds the 32 codes on
-// the FMA pipe and writes them with 16-byte stores.  A warp covers 32
-// consecutive blocks, so loads and stores stay contiguous.
+// the FMA pipe and writes them with 16-byte stores.  A warp covers the 32
+// consecutive blocks of 32 / (D / 32) rows of K only or of V only (warps
+// alternate), so its loads and stores stay contiguous and its lanes never
+// diverge between the 8-bit and the 4-bit code paths.
 __device__ __forceinline__ void load_block(const __half* src, float (&x)[32]) {
   const uint4* p = reinterpret_cast<const uint4*>(src);
 #pragma unroll
@@ -155,16 +157,20 @@ __global__ void __launch_bounds__(256) append_kernel(const Layout L, int layer, 
                                                      int total_tokens, const __half* __restrict__ k,
                                                      const __half* __restrict__ v) {
   constexpr int NB = D / 32;                       // blocks per row
+  constexpr int RPW = 32 / NB;                     // rows per warp
   const int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   const int H = L.n_kv_heads;
   const int64_t n_rows = int64_t(total_tokens) * H;
-  if (t >= n_rows * 2 * NB) return;
-  const int64_t rr = t / (2 * NB);                 // (token, head) row
-  const int kv = int(t / NB) & 1, blk = int(t % NB);
-  const __half* src = (kv ? v : k) + rr * D + blk * 32;
+  const int64_t gw = t >> 5;                       // warp pair gw / 2 covers rows [RPW (gw / 2), + RPW)
+  const int lane = int(t & 31);
+  const int kv = int(gw & 1), blk = lane % NB;
+  const int64_t rr64 = (gw >> 1) * RPW + lane / NB;
+  if (rr64 >= n_rows) return;
+  const int rr = int(rr64);                        // (token, head) row; < 2^31 for any input that fits in HBM
+  const __half* src = (kv ? v : k) + int64_t(rr) * D + blk * 32;
   float x[32];
   load_block(src, x);                              // issued before the page lookup it does not need
-  const int row = int(rr / H), h = int(rr % H);
+  const int row = rr / H, h = rr % H;
   // sequence of this row: last s with b.s[s].c <= row (row offsets ascending)
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
@@ -233,7 +239,8 @@ cudaError_t launch_pt_update(int32_t* table, const PtUpdate& u, cudaStream_t s) 
 
 cudaError_t launch_append(const Layout& L, int layer, const Batch& b, int total_tokens, const void* k, const void* v,
                           cudaStream_t s) {
-  const int64_t threads = int64_t(total_tokens) * L.n_kv_heads * 2 * (L.head_dim / 32);
+  const int64_t rows = int64_t(total_tokens) * L.n_kv_heads, rpw = 32 / (L.head_dim / 32);
+  const int64_t threads = (rows + rpw - 1) / rpw * 64;            // one K warp and one V warp per rpw rows
   const unsigned grid = unsigned((threads + 255) / 256);
   if (L.head_dim == 128)
     append_kernel<128><<<grid, 256, 0, s>>>(L, layer, b, total_tokens, static_cast<const __half*>(k),
