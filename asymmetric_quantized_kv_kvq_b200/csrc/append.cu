@@ -33,20 +33,18 @@ __global__ void pt_update_kernel(int32_t* table, const __grid_constant__ PtUpdat
 // FMA against 1.5 * 2^23) is within 1 of floor(t + 1/2); the remainder
 // e = |x| - n |d| is exact in fp32 (n |d| has at most 18 significant bits) and
 // moves n up when e >= |d|/2 and down when e < -|d|/2, ties going away from
-// zero; the sign of x / d is applied last.  For fp16 x and d the fp32 rounding of
-// the quotient never moves it across a half-integer it did not sit on, so this
-// is the same integer as roundf of the IEEE quotient (checked for every finite
-// fp16 x against 3400 scales, both clamp ranges).
+// zero; the sign of x / d is applied last, then the clamp.  For fp16 x and d
+// the fp32 rounding of the quotient never moves it across a half-integer it did
+// not sit on, so this is the same integer as roundf of the IEEE quotient
+// (checked for every finite fp16 x against 3400 scales, both clamp ranges).
 struct RoundCtx {
   float ad, ra, hd;   // |d|, fp32(1 / |d|), |d| / 2
-  bool dneg;
 };
 __device__ __forceinline__ RoundCtx round_ctx(float d) {
   RoundCtx r;
   r.ad = fabsf(d);
   r.ra = __frcp_rn(r.ad);
   r.hd = 0.5f * r.ad;
-  r.dneg = d < 0.f;
   return r;
 }
 __device__ __forceinline__ float round_mag(float x, const RoundCtx& r) {
@@ -57,18 +55,26 @@ __device__ __forceinline__ float round_mag(float x, const RoundCtx& r) {
   if (e < -r.hd) n -= 1.f;
   return n;
 }
-__device__ __forceinline__ float round_code(float x, const RoundCtx& r, float cn, float cp) {
+// 4-bit (d of either sign): the sign of x / d set on the magnitude with one bit
+// operation, then the asymmetric clamp to [-8, 7].
+__device__ __forceinline__ float round_code4(float x, const RoundCtx& r, uint32_t dbits) {
   const float n = round_mag(x, r);
-  return ((x < 0.f) != r.dneg) ? -fminf(n, cn) : fminf(n, cp);
+  const float c = __uint_as_float(__float_as_uint(n) | ((__float_as_uint(x) ^ dbits) & 0x80000000u));
+  return fmaxf(fminf(c, 7.f), -8.f);
 }
 // 8-bit: d > 0, symmetric clamp
 __device__ __forceinline__ float round_code8(float x, const RoundCtx& r) {
   return copysignf(fminf(round_mag(x, r), 127.f), x);
 }
-// max(a, b, c) in one instruction
+// max(a, b, c) and min(a, b, c) in one instruction each
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
 // Low byte of an exact integer v in [-128, 255] held in a float (two's complement for v < 0).
@@ -126,20 +132,34 @@ __device__ __forceinline__ void quant8_block(const float (&x)[32], uint8_t* code
 // 4-bit: m = the largest-|x| element (lowest index on ties), d = fp16(m / -8),
 // c = clamp(roundf(x / d), -8, 7), u = c + 8, byte i = u_i | u_{i+16} << 4.
 __device__ __forceinline__ void quant4_block(const float (&x)[32], uint8_t* codes, __half* scale) {
-  float m = x[0];
+  // the largest-|x| element is max(x) or min(x); only when max(x) == -min(x) (a +- tie, or a zero
+  // block) does the index decide, by a scan in which the lowest index wins
+  float mx = x[0], mn = x[0];
 #pragma unroll
-  for (int i = 1; i < 32; ++i)
-    if (fabsf(x[i]) > fabsf(m)) m = x[i];                  // strict: the lowest index wins ties
+  for (int i = 1; i < 31; i += 2) {
+    mx = fmax3(mx, x[i], x[i + 1]);
+    mn = fmin3(mn, x[i], x[i + 1]);
+  }
+  mx = fmaxf(mx, x[31]);
+  mn = fminf(mn, x[31]);
+  float m = mx > -mn ? mx : mn;
+  if (mx == -mn) {
+    m = x[0];
+#pragma unroll                                               // registers only: no dynamic index into x
+    for (int i = 1; i < 32; ++i)
+      if (fabsf(x[i]) > fabsf(m)) m = x[i];                // strict: the lowest index wins ties
+  }
   const __half d = __float2half_rn(m * -0.125f);            // m / -8, exact in fp32
   const float df = __half2float(d);
   uint32_t w[4];
   if (df != 0.f) {
     const RoundCtx r = round_ctx(df);
+    const uint32_t dbits = __float_as_uint(df);
     uint32_t by[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       // u_j + 16 u_{j+16} = c_j + 16 c_{j+16} + 136, an exact integer in [0, 255]
-      const float c0 = round_code(x[j], r, 8.f, 7.f), c1 = round_code(x[j + 16], r, 8.f, 7.f);
+      const float c0 = round_code4(x[j], r, dbits), c1 = round_code4(x[j + 16], r, dbits);
       by[j] = float_int_bits(__fmaf_rn(c1, 16.f, c0) + 136.f);
     }
 #pragma unroll
