@@ -239,7 +239,7 @@ struct PTraits {
   static constexpr int OFF_BAR = OFF_V + NSTAGE * V_BYTES;
   // + alignment slack; never less than ~116 KB so that a second CTA cannot
   // share the SM and wait in tcgen05.alloc
-  static constexpr int SMEM_NEED = OFF_BAR + 256 + 2 * 128 * 4 + 1024;   // barriers, TMEM slot, row maxima
+  static constexpr int SMEM_NEED = OFF_BAR + 256 + 2 * 2 * 128 * 4 + 1024;   // barriers, TMEM slot, row maxima
   static constexpr int SMEM = SMEM_NEED > 118 * 1024 ? SMEM_NEED : 118 * 1024;
   static constexpr int NT = 352;                         // 11 warps: copies, score MMAs, 2 x 4 softmax, PV MMAs
   static constexpr uint32_t TMEM_COLS = 512;
@@ -447,12 +447,14 @@ __global__ void __launch_bounds__(352, 1)
     // Two warps per TMEM lane quadrant: `half` 0 takes keys [0, 64) of each tile and head_dim
     // columns [0, D/2) of O, half 1 keys [64, 128) and columns [D/2, D).  The row max is exchanged
     // through shared memory at a 256-thread named barrier that also makes every exit uniform.
-    constexpr int BAR_MAX = 1, BAR_L = 2, BAR_MAX_READ = 3, NTH = 256;
+    constexpr int BAR_MAX = 1, BAR_L = 2, NTH = 256;
     const int quad = warp & 3, half = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + (uint32_t(quad * 32) << 16);
     const int qpos = qpos0 + row / G;
-    float* redmax = reinterpret_cast<float*>(bars + 32);        // [2 halves][128 rows]
+    // [2 tile parities][2 halves][128 rows]: a buffer is rewritten two tiles later, after every thread
+    // has passed the next tile's BAR_MAX, so no second barrier guards the reads
+    float* redmax = reinterpret_cast<float*>(bars + 32);
     float m_used = -INFINITY, l = 0.f;
     bool wok = true;
     if constexpr (T::LO8) {
@@ -511,10 +513,10 @@ __global__ void __launch_bounds__(352, 1)
 #pragma unroll
         for (int i = 0; i < 64; ++i) sv[i] = 0u;
       }
-      redmax[half * 128 + row] = mx;
+      float* rm = redmax + (j & 1) * 256;
+      rm[half * 128 + row] = mx;
       if (!bar_red_and(BAR_MAX, NTH, w && wok)) break;
-      mx = fmaxf(mx, redmax[(half ^ 1) * 128 + row]) * a.scale_log2;
-      named_barrier(BAR_MAX_READ, NTH);                          // redmax is rewritten next tile
+      mx = fmaxf(mx, rm[(half ^ 1) * 128 + row]) * a.scale_log2;
       // P buffer j & 1 was read by PV(j - 2); PV(j - 1) may still run
       if (j > 1) wok = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV + (j & 1)), ((j - 2) >> 1) & 1, abort_flag));
       if (!wok) *abort_flag = 1;
@@ -577,14 +579,14 @@ __global__ void __launch_bounds__(352, 1)
                __all_sync(0xffffffffu, mbar_wait(bar(B_PV + ((n_kv - 1) & 1)), ((n_kv - 1) >> 1) & 1, abort_flag));
     // the l of both halves of each row; every thread takes part so the barrier is uniform
     if (done) {
-      redmax[half * 128 + row] = l;                  // every tile's max was read before BAR_MAX_READ
+      redmax[(n_kv & 1) * 256 + half * 128 + row] = l;   // the buffer last read two tiles back
       fin = bar_red_and(BAR_L, NTH, fin);
     }
     if (!done || !fin) {
       record_error(a.err, kErrWaitTimeout | 0x13);
       *abort_flag = 1;
     } else {
-      l += redmax[(half ^ 1) * 128 + row];
+      l += redmax[(n_kv & 1) * 256 + (half ^ 1) * 128 + row];
       tc_fence_after();
       const int t = tok0 + row / G;
       const float inv = 1.f / l;
