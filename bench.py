@@ -10,6 +10,9 @@ for each layer the new token's K / V are quantised into the paged cache
 split-KV kernel + log-sum-exp combine).  Metric: algorithmic KV bytes moved
 per second (cache codes + scales read by decode, fp16 q / out, the appended
 token's fp16 read and quantised write), and decode tokens/s = batch / step.
+By default one step is captured in a CUDA graph after the warm-up and every
+timed step replays it (the same token re-appended at the same position, the
+same length attended); --eager makes the API calls directly each step.
 
 Multi-GPU (torchrun): every rank holds an independent replica of the workload
 (sequences are independent, so the batch shards with no collective); value =
