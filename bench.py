@@ -692,7 +692,7 @@ def main():
             r = oracle_prefill_rows(wl, kb, vb, budget_s=0.0)
             vals = [oracle_prefill_rows(wl, kb, vb, budget_s=1.0) for _ in range(args.steps)]
             val = statistics.mean(v["value"] for v in vals)
-            line = {"metric": PREFILL_METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference", "n_gpus": 0,
+            line = {"metric": PREFILL_METRIC, "value": val, "unit": "TFLOP/s", "impl": "reference", "n_gpus": world, "device": "host cores (oracle)",
                     "steps": args.steps, "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True,
                     "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                     "config": {"workload": wl.name, "precision": precision},
@@ -705,7 +705,7 @@ def main():
         times = [time_oracle_slice(sl, kb, vb) for _ in range(args.warmup + args.steps)][args.warmup:]
         secs = sum(times)
         val = args.steps * slice_bytes(wl, kb, vb) / secs / 1e9
-        line = {"metric": METRIC, "value": val, "unit": "GB/s", "impl": "reference", "n_gpus": 0,
+        line = {"metric": METRIC, "value": val, "unit": "GB/s", "impl": "reference", "n_gpus": world, "device": "host cores (oracle)",
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / args.steps,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
                 "data": "synthetic", "config": config_of(wl, precision, 1, False),
