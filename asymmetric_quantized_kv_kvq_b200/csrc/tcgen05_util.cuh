@@ -1,6 +1,7 @@
-// sm_100a tensor-core helpers: TMEM allocation, tcgen05.mma (kind::f16, both
-// operands in shared memory), commits to mbarriers, TMEM loads / stores, the
-// UMMA shared-memory and instruction descriptors, and 2-D / 3-D TMA tensor loads.
+// sm_100a tensor-core helpers: TMEM allocation, tcgen05.mma (kind::f16 with A
+// in shared memory or in TMEM, kind::i8, kind::f8f6f4), commits to mbarriers,
+// TMEM loads / stores, the UMMA shared-memory and instruction descriptors, and
+// 2-D / 3-D TMA tensor loads.
 #pragma once
 
 #include <cstdint>
