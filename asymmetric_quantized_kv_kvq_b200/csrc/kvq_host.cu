@@ -93,7 +93,8 @@ struct kvq_cache {
   std::vector<int64_t> len;          // tokens per sequence
   std::vector<int32_t> mapped;       // pages mapped per sequence
   std::vector<int32_t> free_pages;   // stack; back() is handed out next
-  int64_t mapped_pages = 0;
+  std::vector<int32_t> refs;         // sequences mapping each physical page (0 = free)
+  int64_t mapped_pages = 0;          // physical pages in use (each counted once)
 };
 
 namespace {
@@ -123,6 +124,23 @@ kvq_status check_ids(const kvq_cache* c, int32_t n, const int32_t* ids) {
 kvq_status check_layer(const kvq_cache* c, int32_t layer) {
   if (layer < 0 || layer >= c->cfg.n_layers) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
   return KVQ_OK;
+}
+
+// Physical page bookkeeping: a page leaves the free stack with one reference,
+// gains one per sequence that shares it (kvq_seq_fork) and returns to the stack
+// when its last reference is dropped.
+int32_t take_page(kvq_cache* c) {
+  const int32_t page = c->free_pages.back();
+  c->free_pages.pop_back();
+  c->refs[page] = 1;
+  c->mapped_pages++;
+  return page;
+}
+void drop_page(kvq_cache* c, int32_t page) {
+  if (--c->refs[page] == 0) {
+    c->free_pages.push_back(page);
+    c->mapped_pages--;
+  }
 }
 
 kvq_status need_device(const kvq_cache* c) {
@@ -207,6 +225,7 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
     c->len.assign(c->cfg.max_seqs, 0);
     c->mapped.assign(c->cfg.max_seqs, 0);
     c->free_pages.resize(L.n_pages);
+    c->refs.assign(L.n_pages, 0);
   } catch (...) {
     delete c;
     return fail(KVQ_ERR_OUT_OF_MEMORY, "host bookkeeping allocation failed");
@@ -292,6 +311,13 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
   if (kvq_status s = check_ids(c, n, ids)) return s;
   if (!n_new) return fail(KVQ_ERR_INVALID_ARG, "n_new is NULL");
   const int P = c->L.page_tokens;
+  // a sequence whose last page is partly filled and shared with another sequence
+  // (kvq_seq_fork) gets a private copy of that page before new tokens land in it
+  auto shared_tail = [&](int32_t id) -> int32_t {
+    if (c->len[id] % P == 0) return -1;
+    const int32_t p = int32_t(c->len[id] / P);
+    return c->refs[c->table[size_t(id) * c->L.max_pages_per_seq + p]] > 1 ? p : -1;
+  };
   int64_t need = 0;
   for (int i = 0; i < n; ++i) {
     if (n_new[i] < 0) return fail(KVQ_ERR_INVALID_ARG, "n_new[%d] < 0", i);
@@ -299,6 +325,7 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
     if (nl > c->cfg.max_seq_tokens)
       return fail(KVQ_ERR_CAPACITY, "sequence %d would hold %lld tokens > max_seq_tokens", ids[i], (long long)nl);
     need += (nl + P - 1) / P - c->mapped[ids[i]];
+    if (n_new[i] > 0 && shared_tail(ids[i]) >= 0) ++need;
   }
   if (need > int64_t(c->free_pages.size()))
     return fail(KVQ_ERR_CAPACITY, "need %lld pages, %zu free", (long long)need, c->free_pages.size());
@@ -315,13 +342,31 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
     const int32_t id = ids[i];
     const int64_t nl = c->len[id] + n_new[i];
     const int32_t want = int32_t((nl + P - 1) / P);
+    const int32_t tail = n_new[i] > 0 ? shared_tail(id) : -1;
+    if (tail >= 0) {
+      const int32_t slot = id * c->L.max_pages_per_seq + tail;
+      const int32_t from = c->table[slot], to = take_page(c);
+      if (!c->host_only) {
+        // the page's head blocks of one layer are contiguous: one copy per layer
+        const int64_t bytes = int64_t(c->L.n_kv_heads) * c->L.head_block;
+        for (int32_t layer = 0; layer < c->cfg.n_layers; ++layer) {
+          const cudaError_t e = cudaMemcpyAsync(c->L.head_ptr(layer, to, 0), c->L.head_ptr(layer, from, 0),
+                                                size_t(bytes), cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+          if (e != cudaSuccess) return cuda_fail(e, "copy of a shared page");
+        }
+      }
+      drop_page(c, from);
+      c->table[slot] = to;
+      upd.idx[upd.n] = slot;
+      upd.val[upd.n] = to;
+      if (++upd.n == kvq::kMaxPtUpdates)
+        if (kvq_status s = flush()) return s;
+    }
     while (c->mapped[id] < want) {
-      const int32_t page = c->free_pages.back();
-      c->free_pages.pop_back();
+      const int32_t page = take_page(c);
       const int32_t slot = id * c->L.max_pages_per_seq + c->mapped[id];
       c->table[slot] = page;
       c->mapped[id]++;
-      c->mapped_pages++;
       upd.idx[upd.n] = slot;
       upd.val[upd.n] = page;
       if (++upd.n == kvq::kMaxPtUpdates)
@@ -337,10 +382,9 @@ kvq_status kvq_seq_release(kvq_cache* c, int32_t id) {
   if (kvq_status s = check_seq(c, id)) return s;
   for (int32_t p = c->mapped[id] - 1; p >= 0; --p) {
     int32_t& slot = c->table[size_t(id) * c->L.max_pages_per_seq + p];
-    c->free_pages.push_back(slot);
+    drop_page(c, slot);
     slot = -1;
   }
-  c->mapped_pages -= c->mapped[id];
   c->mapped[id] = 0;
   c->len[id] = 0;
   return KVQ_OK;
@@ -355,12 +399,44 @@ kvq_status kvq_seq_truncate(kvq_cache* c, int32_t id, int64_t new_len) {
   const int32_t keep = int32_t((new_len + P - 1) / P);
   for (int32_t p = c->mapped[id] - 1; p >= keep; --p) {
     int32_t& slot = c->table[size_t(id) * c->L.max_pages_per_seq + p];
-    c->free_pages.push_back(slot);
+    drop_page(c, slot);
     slot = -1;
   }
-  c->mapped_pages -= c->mapped[id] - keep;
   c->mapped[id] = keep;
   c->len[id] = new_len;
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_fork(kvq_cache* c, int32_t src, int32_t dst, int64_t n_tokens, kvq_stream_t stream) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_seq(c, src)) return s;
+  if (kvq_status s = check_seq(c, dst)) return s;
+  if (src == dst) return fail(KVQ_ERR_INVALID_ARG, "fork of sequence %d onto itself", src);
+  if (c->len[dst] != 0 || c->mapped[dst] != 0) return fail(KVQ_ERR_INVALID_ARG, "sequence %d is not empty", dst);
+  if (n_tokens < 0 || n_tokens > c->len[src])
+    return fail(KVQ_ERR_INVALID_ARG, "n_tokens %lld outside [0, len = %lld]", (long long)n_tokens,
+                (long long)c->len[src]);
+  const int P = c->L.page_tokens;
+  const int32_t pages = int32_t((n_tokens + P - 1) / P);
+  kvq::PtUpdate upd;
+  upd.n = 0;
+  for (int32_t p = 0; p < pages; ++p) {
+    const int32_t page = c->table[size_t(src) * c->L.max_pages_per_seq + p];
+    const int32_t slot = dst * c->L.max_pages_per_seq + p;
+    c->table[slot] = page;
+    c->refs[page]++;
+    upd.idx[upd.n] = slot;
+    upd.val[upd.n] = page;
+    if (++upd.n == kvq::kMaxPtUpdates || p == pages - 1) {
+      if (!c->host_only)
+        if (kvq_status s = launched(kvq::launch_pt_update(c->d_page_table, upd, (cudaStream_t)stream),
+                                    "page-table update"))
+          return s;
+      upd.n = 0;
+    }
+  }
+  c->mapped[dst] = pages;
+  c->len[dst] = n_tokens;
   return KVQ_OK;
 }
 

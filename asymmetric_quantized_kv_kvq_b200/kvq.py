@@ -54,6 +54,7 @@ SIGNATURES = {
     "kvq_seq_extend": (_i32, [_p, _i32, _pi32, _pi32, _p]),
     "kvq_seq_release": (_i32, [_p, _i32]),
     "kvq_seq_truncate": (_i32, [_p, _i32, _i64]),
+    "kvq_seq_fork": (_i32, [_p, _i32, _i32, _i64, _p]),
     "kvq_seq_length": (_i32, [_p, _i32, _pi64]),
     "kvq_seq_page": (_i32, [_p, _i32, _i32, _pi32]),
     "kvq_append": (_i32, [_p, _i32, _i32, _pi32, _pi32, _p, _p, _p]),
@@ -183,6 +184,12 @@ class Cache:
 
     def truncate(self, seq_id: int, new_len: int) -> None:
         _check(self._lib.kvq_seq_truncate(self._h, seq_id, new_len))
+
+    def fork(self, src: int, dst: int, n_tokens: Optional[int] = None, stream=None) -> None:
+        """Empty sequence `dst` shares the first n_tokens (default: all) positions of `src`."""
+        n = self.length(src) if n_tokens is None else n_tokens
+        s = None if self.host_only else _stream(stream)
+        _check(self._lib.kvq_seq_fork(self._h, src, dst, n, s))
 
     def length(self, seq_id: int) -> int:
         n = ctypes.c_int64()

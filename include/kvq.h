@@ -136,7 +136,9 @@ KVQ_API kvq_status kvq_cache_footprint(const kvq_cache* cache, int64_t* pool_byt
  * token positions at its end, mapping free pages as needed (host arrays).
  * Page-table updates are enqueued on `stream`.  The new positions hold no data
  * until kvq_append writes them, layer by layer.  All-or-nothing: on
- * KVQ_ERR_CAPACITY no sequence changes.  A sequence id may appear once. */
+ * KVQ_ERR_CAPACITY no sequence changes (the capacity check counts one page for
+ * every shared partly filled last page it may have to copy).  A sequence id may
+ * appear once. */
 KVQ_API kvq_status kvq_seq_extend(kvq_cache* cache, int32_t n_seqs, const int32_t* seq_ids,
                           const int32_t* n_new, kvq_stream_t stream);
 
@@ -150,6 +152,22 @@ KVQ_API kvq_status kvq_seq_release(kvq_cache* cache, int32_t seq_id);
  * Whole pages past new_len return to the pool.  Host bookkeeping only: the
  * caller orders it after device work that still reads the dropped positions. */
 KVQ_API kvq_status kvq_seq_truncate(kvq_cache* cache, int32_t seq_id, int64_t new_len);
+
+/* Share a prefix: empty sequence dst becomes the first n_tokens <= len(src)
+ * positions of src, in every layer, by mapping the same physical pages
+ * (reference-counted; no data is copied).  A page stays shared while neither
+ * sequence writes into it; when kvq_seq_extend is about to add positions to a
+ * partly filled page that another sequence still maps, it first copies that
+ * page (all layers) to a private page on `stream` (copy-on-write), so appends
+ * never change what the other sequence reads.  Release and truncate drop one
+ * reference; a page returns to the pool with its last one.  This is the
+ * keep-the-cache reuse of "Reutilizacao de Cache KV para Conversas Longas no
+ * Apple Silicon" ("Principais Descobertas e Benchmarks") extended to several
+ * conversations that start from one cached prefix.  Page-table updates are
+ * enqueued on `stream`.  KVQ_ERR_INVALID_ARG if src == dst, dst is not empty or
+ * n_tokens is outside [0, len(src)]. */
+KVQ_API kvq_status kvq_seq_fork(kvq_cache* cache, int32_t src_seq, int32_t dst_seq, int64_t n_tokens,
+                                kvq_stream_t stream);
 
 /* Current length (token positions) of a sequence. */
 KVQ_API kvq_status kvq_seq_length(const kvq_cache* cache, int32_t seq_id, int64_t* len);

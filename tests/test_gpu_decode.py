@@ -185,3 +185,54 @@ def test_decode_at_the_maximum_batch():
     ref = oracle.attention_decode_batch(q.numpy(), [hat[(0, s)] for s in ids])
     assert_close_attention(out, ref, "max batch")
     cache.close()
+
+
+@pytest.mark.gpu
+def test_fork_shares_a_prefix_and_copies_on_write():
+    """kvq_seq_fork: two sequences started from one cached prefix read the same pages; new tokens appended
+    to each afterwards (the shared, partly filled last page is copied first) leave the other intact."""
+    m = kvq()
+    D, H, G, layers = 128, 2, 4, 2
+    T = 300
+    cache = m.Cache(n_layers=layers, n_kv_heads=H, head_dim=D, k_bits=8, v_bits=4, max_seqs=4, max_tokens=4096)
+    cache.extend([0], [T])
+    base = {}
+    for layer in range(layers):
+        k = decode_kv(T, H, D, 40 + layer)
+        v = random_fp16((T, H, D), 50 + layer)
+        cache.append(layer, [0], [T], k.cuda(), v.cuda())
+        base[layer] = (k, v)
+    cache.fork(0, 1)                 # all 300 positions
+    cache.fork(0, 2, 200)            # a prefix ending inside the first page
+    assert cache.page(1, 1) == cache.page(0, 1) and cache.page(2, 0) == cache.page(0, 0)
+    q = [random_fp16((3, H * G, D), 60 + layer) for layer in range(layers)]
+    same = cache.decode(0, [0, 1], q[0][:1].repeat(2, 1, 1).cuda())     # one query for both sequences
+    assert torch.equal(same[0], same[1])
+    cache.extend([0, 1, 2], [1, 1, 1])
+    assert cache.page(0, 1) != cache.page(1, 1) and cache.page(2, 0) != cache.page(0, 0)
+    new = {}
+    for layer in range(layers):
+        k = decode_kv(3, H, D, 70 + layer)
+        v = random_fp16((3, H, D), 80 + layer)
+        cache.append(layer, [0, 1, 2], [1, 1, 1], k.cuda(), v.cuda())
+        new[layer] = (k, v)
+    cache.check()
+    prefix = {0: T, 1: T, 2: 200}
+    for layer in range(layers):
+        out = cache.decode(layer, [0, 1, 2], q[layer].cuda())
+        kv = []
+        for s in range(3):
+            k = torch.cat([base[layer][0][:prefix[s]], new[layer][0][s:s + 1]])
+            v = torch.cat([base[layer][1][:prefix[s]], new[layer][1][s:s + 1]])
+            kv.append((oracle_dequant(k, 8), oracle_dequant(v, 4)))
+        ref = oracle.attention_decode_batch(q[layer].numpy(), kv)
+        assert_close_attention(out, ref, f"fork layer {layer}")
+    cache.release(0)
+    cache.release(2)
+    out1 = cache.decode(0, [1], q[0][1:2].cuda())       # seq 1 still reads its pages
+    k = torch.cat([base[0][0], new[0][0][1:2]])
+    v = torch.cat([base[0][1], new[0][1][1:2]])
+    ref = oracle.attention_decode_batch(q[0][1:2].numpy(), [(oracle_dequant(k, 8), oracle_dequant(v, 4))])
+    assert_close_attention(out1, ref, "fork after release")
+    cache.check()
+    cache.close()

@@ -116,6 +116,59 @@ def test_truncate_returns_whole_pages(kvq):
     c.close()
 
 
+def test_fork_shares_pages_and_copies_a_shared_tail_before_writing(kvq):
+    c = _host_cache(kvq, max_tokens=2048)                 # 8 pages
+    per_page = 2 * 2 * (64 + 4 + 32 + 4) * 256
+    c.extend([0], [300])                                  # pages 0, 1 (page 1 partly filled)
+    c.fork(0, 1)                                          # seq 1 = all 300 positions of seq 0
+    assert c.length(1) == 300 and [c.page(1, i) for i in range(2)] == [0, 1]
+    assert c.footprint()[1] == 2 * per_page               # shared pages count once
+    c.extend([0, 1], [1, 1])                              # both write into page 1: seq 0 copies it first
+    assert c.page(0, 0) == 0 and c.page(1, 0) == 0        # the full page stays shared
+    assert c.page(0, 1) == 2 and c.page(1, 1) == 1        # seq 1 is now the only user of page 1
+    assert c.footprint()[1] == 3 * per_page
+    c.fork(0, 2, 256)                                     # a page-aligned prefix: nothing to copy later
+    c.extend([2], [10])
+    assert c.page(2, 0) == 0 and c.page(2, 1) == 3
+    c.fork(1, 3, 100)                                     # a prefix ending inside shared page 0
+    c.extend([3], [1])                                    # page 0 is copied for seq 3 before the write
+    assert c.page(3, 0) == 4 and c.page(0, 0) == 0 and c.length(3) == 101
+    c.release(0)
+    c.release(2)
+    assert c.page(1, 0) == 0                              # still held by seq 1
+    c.release(1)
+    c.release(3)
+    assert c.footprint()[1] == 0
+    c.extend([0], [2048])                                 # every page is free again
+    with pytest.raises(kvq.KvqError) as e:
+        c.fork(0, 0)
+    assert e.value.name == "KVQ_ERR_INVALID_ARG"
+    c.extend([1], [0])
+    with pytest.raises(kvq.KvqError):
+        c.fork(0, 1, 2049)                                # longer than the source
+    c.close()
+
+
+def test_fork_respects_the_capacity_check(kvq):
+    c = _host_cache(kvq, max_tokens=768)                  # 3 pages
+    c.extend([0], [300])                                  # pages 0, 1; one free
+    c.fork(0, 1)
+    with pytest.raises(kvq.KvqError) as e:
+        c.extend([0, 1], [1, 1])
+    # a copy is counted for each sequence whose last page is shared, although the second one would find
+    # the page private by then: the check is conservative, and nothing changes
+    assert e.value.name == "KVQ_ERR_CAPACITY"
+    assert c.length(0) == 300 and c.length(1) == 300 and c.page(0, 1) == c.page(1, 1) == 1
+    c.extend([1], [1])                                    # one copy fits
+    assert c.page(1, 1) == 2 and c.page(0, 1) == 1 and c.length(1) == 301
+    with pytest.raises(kvq.KvqError) as e:                # no page left for a copy
+        c.fork(1, 2)
+        c.fork(1, 3)
+        c.extend([2], [1])
+    assert e.value.name == "KVQ_ERR_CAPACITY"
+    c.close()
+
+
 def test_max_seq_tokens_bound(kvq):
     c = _host_cache(kvq, max_seq_tokens=300)
     c.extend([0], [300])
