@@ -142,15 +142,17 @@ KVQ_API kvq_status kvq_cache_footprint(const kvq_cache* cache, int64_t* pool_byt
 KVQ_API kvq_status kvq_seq_extend(kvq_cache* cache, int32_t n_seqs, const int32_t* seq_ids,
                           const int32_t* n_new, kvq_stream_t stream);
 
-/* Drop a sequence: its pages return to the pool and its length becomes 0. */
+/* Drop a sequence: its length becomes 0 and each of its pages returns to the
+ * pool unless another sequence still maps it (kvq_seq_fork). */
 KVQ_API kvq_status kvq_seq_release(kvq_cache* cache, int32_t seq_id);
 
 /* Shorten a sequence to new_len <= its length (rewind a chunk, or keep a
  * session's prefix and drop its last turn, as in reusing a conversation's
  * cache and processing only the new tokens: "Reutilizacao de Cache KV para
  * Conversas Longas no Apple Silicon", "Principais Descobertas e Benchmarks").
- * Whole pages past new_len return to the pool.  Host bookkeeping only: the
- * caller orders it after device work that still reads the dropped positions. */
+ * Whole pages past new_len are dropped (returned to the pool unless another
+ * sequence still maps them).  Host bookkeeping only: the caller orders it after
+ * device work that still reads the dropped positions. */
 KVQ_API kvq_status kvq_seq_truncate(kvq_cache* cache, int32_t seq_id, int64_t new_len);
 
 /* Share a prefix: empty sequence dst becomes the first n_tokens <= len(src)
