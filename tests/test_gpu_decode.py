@@ -1,6 +1,5 @@
 """GPU parity: split-KV decode attention against the oracle's float64 softmax
 attention over its own dequantisation of the same fp16 inputs."""
-import math
 
 import numpy as np
 import pytest
