@@ -5,6 +5,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <string>
@@ -221,6 +222,10 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
   c->pool_bytes = int64_t(c->cfg.n_layers) * L.n_pages * H * L.head_block;
 
   try {
+    // host-side fault injection for tests: the environment variable
+    // KVQ_INJECT_ALLOC_FAILURE=1 makes this allocation fail, through the same
+    // cleanup as a real one
+    if (const char* f = std::getenv("KVQ_INJECT_ALLOC_FAILURE"); f && f[0] == '1') throw std::bad_alloc();
     c->table.assign(size_t(c->cfg.max_seqs) * L.max_pages_per_seq, -1);
     c->len.assign(c->cfg.max_seqs, 0);
     c->mapped.assign(c->cfg.max_seqs, 0);

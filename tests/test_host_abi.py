@@ -263,3 +263,17 @@ def test_cache_flags(kvq):
     h = ctypes.c_void_p()
     assert lib.kvq_cache_create(ctypes.byref(cfg), ctypes.byref(h)) == 1      # KVQ_ERR_INVALID_ARG
     assert b"unknown flags" in lib.kvq_last_error()
+
+
+def test_injected_allocation_failure_is_reported_and_cleaned_up(kvq, monkeypatch):
+    """Host-side fault injection: a failed bookkeeping allocation returns KVQ_ERR_OUT_OF_MEMORY with no
+    cache created, and the next creation succeeds."""
+    monkeypatch.setenv("KVQ_INJECT_ALLOC_FAILURE", "1")
+    with pytest.raises(kvq.KvqError) as e:
+        _host_cache(kvq)
+    assert e.value.name == "KVQ_ERR_OUT_OF_MEMORY"
+    monkeypatch.delenv("KVQ_INJECT_ALLOC_FAILURE")
+    c = _host_cache(kvq)
+    c.extend([0], [10])
+    assert c.length(0) == 10
+    c.close()
