@@ -37,3 +37,17 @@ def test_reference_arm_prefill_line():
     assert KEYS <= set(d), KEYS - set(d)
     assert d["unit"] == "TFLOP/s" and d["value"] > 0
     assert d["config"]["workload"] == "prefill-16x4096"
+
+
+def test_reference_arm_under_torchrun_prints_one_line_from_rank_0():
+    """Two ranks launched as the driver launches them: rank 0 alone times the oracle and prints one
+    line with n_gpus = 2; the other rank exits 0 without work."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", "29731", "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "1", "--warmup", "1"]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
