@@ -43,9 +43,12 @@ extern "C" KVQ_API kvq_status kvq_decode_attn_noalloc(kvq_cache* cache, int32_t 
                                "kvq_decode_attn_noalloc: this batch needs more scratch than the fixed "
                                "KVQ_NOALLOC_SCRATCH_BYTES (8 MiB); split the batch or call kvq_decode_attn "
                                "with a caller-owned workspace");
+  // a host-only cache, or a current device other than the cache's, is refused
+  // before the scratch address is looked up (which would touch the device)
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-    return kvq::set_last_error(KVQ_ERR_CUDA, "kvq_decode_attn_noalloc: no usable current CUDA device");
+  if (kvq_status s = kvq::launch_device(cache, &dev)) return s;
+  if (dev < 0 || dev >= kMaxDevices)
+    return kvq::set_last_error(KVQ_ERR_UNSUPPORTED, "kvq_decode_attn_noalloc: device index out of range");
   void* ptr = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_mu);

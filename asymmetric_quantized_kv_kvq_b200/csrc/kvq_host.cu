@@ -127,27 +127,127 @@ kvq_status check_layer(const kvq_cache* c, int32_t layer) {
   return KVQ_OK;
 }
 
+// Host-side fault injection for tests: with KVQ_INJECT_PT_FAILURE=k (k >= 1) in
+// the environment, the k-th page-table enqueue of every kvq_seq_extend /
+// kvq_seq_fork call fails as if the launch had failed (also for host-only
+// caches, which enqueue nothing), so the rollback below runs on the CPU.
+bool injected_pt_failure(int nth) {
+  const char* f = std::getenv("KVQ_INJECT_PT_FAILURE");
+  return f && std::atoi(f) == nth;
+}
+
+// Undo log of one kvq_seq_extend / kvq_seq_fork.  Those calls change the host
+// bookkeeping as they go and enqueue page copies and page-table updates; if an
+// enqueue fails part way, every change is put back in reverse order (and the
+// page-table entries already enqueued are restored on the stream, best effort),
+// so the call is all-or-nothing for the caller.
+struct Journal {
+  enum Kind : int32_t { kTake, kDrop, kRef, kSlot, kLen, kMapped };
+  struct Op {
+    Kind kind;
+    int32_t a;     // page, table slot or sequence id
+    int64_t old;   // previous value (slot entry, length, mapped pages)
+  };
+  std::vector<Op> ops;
+  void add(Kind k, int32_t a, int64_t old = 0) { ops.push_back({k, a, old}); }
+};
+
 // Physical page bookkeeping: a page leaves the free stack with one reference,
 // gains one per sequence that shares it (kvq_seq_fork) and returns to the stack
 // when its last reference is dropped.
-int32_t take_page(kvq_cache* c) {
+int32_t take_page(kvq_cache* c, Journal* j = nullptr) {
   const int32_t page = c->free_pages.back();
   c->free_pages.pop_back();
   c->refs[page] = 1;
   c->mapped_pages++;
+  if (j) j->add(Journal::kTake, page);
   return page;
 }
-void drop_page(kvq_cache* c, int32_t page) {
+void drop_page(kvq_cache* c, int32_t page, Journal* j = nullptr) {
   if (--c->refs[page] == 0) {
     c->free_pages.push_back(page);
     c->mapped_pages--;
   }
+  if (j) j->add(Journal::kDrop, page);
+}
+void set_slot(kvq_cache* c, size_t slot, int32_t val, Journal* j) {
+  j->add(Journal::kSlot, int32_t(slot), c->table[slot]);
+  c->table[slot] = val;
+}
+
+// Puts the host bookkeeping back as it was before the journal's first change.
+void undo(kvq_cache* c, const Journal& j) {
+  for (auto it = j.ops.rbegin(); it != j.ops.rend(); ++it) {
+    switch (it->kind) {
+      case Journal::kTake:            // the page was popped from the free stack with one reference
+        c->refs[it->a] = 0;
+        c->mapped_pages--;
+        c->free_pages.push_back(it->a);
+        break;
+      case Journal::kDrop:            // a reference was dropped; the last one pushed the page back
+        if (c->refs[it->a] == 0) {
+          c->free_pages.pop_back();
+          c->mapped_pages++;
+        }
+        c->refs[it->a]++;
+        break;
+      case Journal::kRef: c->refs[it->a]--; break;
+      case Journal::kSlot: c->table[size_t(it->a)] = int32_t(it->old); break;
+      case Journal::kLen: c->len[it->a] = it->old; break;
+      case Journal::kMapped: c->mapped[it->a] = int32_t(it->old); break;
+    }
+  }
+}
+
+// Undo after a failed enqueue: the host bookkeeping goes back, and the
+// page-table entries of the first `flushed` journal entries, already enqueued,
+// are set back to their old values on the stream (best effort: the enqueue
+// that failed may fail again, which kvq_cache_check then reports).
+void rollback(kvq_cache* c, const Journal& j, size_t flushed, kvq_stream_t stream) {
+  if (!c->host_only && flushed) {
+    kvq::PtUpdate upd;
+    upd.n = 0;
+    for (size_t i = flushed; i-- > 0;) {
+      const Journal::Op& op = j.ops[i];
+      if (op.kind != Journal::kSlot) continue;
+      upd.idx[upd.n] = op.a;
+      upd.val[upd.n] = int32_t(op.old);
+      if (++upd.n == kvq::kMaxPtUpdates) {
+        (void)kvq::launch_pt_update(c->d_page_table, upd, (cudaStream_t)stream);
+        upd.n = 0;
+      }
+    }
+    (void)kvq::launch_pt_update(c->d_page_table, upd, (cudaStream_t)stream);
+  }
+  undo(c, j);
+}
+
+// Work is enqueued on the caller's stream with the caller's current device:
+// that device must be the one the cache lives on.
+kvq_status same_device(const kvq_cache* c) {
+  if (c->host_only) return KVQ_OK;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVQ_ERR_CUDA, "cudaGetDevice failed");
+  if (dev != c->device)
+    return fail(KVQ_ERR_INVALID_ARG, "the current CUDA device is %d but the cache lives on device %d", dev, c->device);
+  return KVQ_OK;
 }
 
 kvq_status need_device(const kvq_cache* c) {
   if (c->host_only) return fail(KVQ_ERR_UNSUPPORTED, "cache was created host-only");
+  return same_device(c);
+}
+
+}  // namespace
+
+kvq_status kvq::launch_device(const kvq_cache* c, int* device) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = need_device(c)) return s;
+  *device = c->device;
   return KVQ_OK;
 }
+
+namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
@@ -315,6 +415,7 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
   if (kvq_status s = check_cache(c)) return s;
   if (kvq_status s = check_ids(c, n, ids)) return s;
   if (!n_new) return fail(KVQ_ERR_INVALID_ARG, "n_new is NULL");
+  if (kvq_status s = same_device(c)) return s;
   const int P = c->L.page_tokens;
   // a sequence whose last page is partly filled and shared with another sequence
   // (kvq_seq_fork) gets a private copy of that page before new tokens land in it
@@ -335,51 +436,66 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
   if (need > int64_t(c->free_pages.size()))
     return fail(KVQ_ERR_CAPACITY, "need %lld pages, %zu free", (long long)need, c->free_pages.size());
 
+  Journal j;
   kvq::PtUpdate upd;
   upd.n = 0;
+  size_t flushed = 0;   // journal entries whose page-table updates were enqueued
+  int n_flush = 0;
   auto flush = [&]() -> kvq_status {
-    if (upd.n == 0 || c->host_only) { upd.n = 0; return KVQ_OK; }
-    cudaError_t e = kvq::launch_pt_update(c->d_page_table, upd, (cudaStream_t)stream);
+    if (upd.n == 0) return KVQ_OK;
+    if (injected_pt_failure(++n_flush)) {
+      upd.n = 0;
+      return fail(KVQ_ERR_CUDA, "page-table update: injected failure (KVQ_INJECT_PT_FAILURE)");
+    }
+    if (c->host_only) { upd.n = 0; flushed = j.ops.size(); return KVQ_OK; }
+    const cudaError_t e = kvq::launch_pt_update(c->d_page_table, upd, (cudaStream_t)stream);
     upd.n = 0;
+    if (e == cudaSuccess) flushed = j.ops.size();
     return launched(e, "page-table update");
   };
-  for (int i = 0; i < n; ++i) {
+  auto queue = [&](size_t slot, int32_t page) -> kvq_status {
+    set_slot(c, slot, page, &j);
+    upd.idx[upd.n] = int32_t(slot);
+    upd.val[upd.n] = page;
+    return ++upd.n == kvq::kMaxPtUpdates ? flush() : KVQ_OK;
+  };
+  kvq_status st = KVQ_OK;
+  for (int i = 0; i < n && st == KVQ_OK; ++i) {
     const int32_t id = ids[i];
     const int64_t nl = c->len[id] + n_new[i];
     const int32_t want = int32_t((nl + P - 1) / P);
     const int32_t tail = n_new[i] > 0 ? shared_tail(id) : -1;
     if (tail >= 0) {
-      const int32_t slot = id * c->L.max_pages_per_seq + tail;
-      const int32_t from = c->table[slot], to = take_page(c);
+      const size_t slot = size_t(id) * c->L.max_pages_per_seq + tail;
+      const int32_t from = c->table[slot], to = take_page(c, &j);
       if (!c->host_only) {
         // the page's head blocks of one layer are contiguous: one copy per layer
         const int64_t bytes = int64_t(c->L.n_kv_heads) * c->L.head_block;
-        for (int32_t layer = 0; layer < c->cfg.n_layers; ++layer) {
+        for (int32_t layer = 0; layer < c->cfg.n_layers && st == KVQ_OK; ++layer) {
           const cudaError_t e = cudaMemcpyAsync(c->L.head_ptr(layer, to, 0), c->L.head_ptr(layer, from, 0),
                                                 size_t(bytes), cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
-          if (e != cudaSuccess) return cuda_fail(e, "copy of a shared page");
+          if (e != cudaSuccess) st = cuda_fail(e, "copy of a shared page");
         }
+        if (st != KVQ_OK) break;
       }
-      drop_page(c, from);
-      c->table[slot] = to;
-      upd.idx[upd.n] = slot;
-      upd.val[upd.n] = to;
-      if (++upd.n == kvq::kMaxPtUpdates)
-        if (kvq_status s = flush()) return s;
+      drop_page(c, from, &j);
+      st = queue(slot, to);
     }
-    while (c->mapped[id] < want) {
-      const int32_t page = take_page(c);
-      const int32_t slot = id * c->L.max_pages_per_seq + c->mapped[id];
-      c->table[slot] = page;
+    while (st == KVQ_OK && c->mapped[id] < want) {
+      const int32_t page = take_page(c, &j);
+      const size_t slot = size_t(id) * c->L.max_pages_per_seq + c->mapped[id];
+      j.add(Journal::kMapped, id, c->mapped[id]);
       c->mapped[id]++;
-      upd.idx[upd.n] = slot;
-      upd.val[upd.n] = page;
-      if (++upd.n == kvq::kMaxPtUpdates)
-        if (kvq_status s = flush()) return s;
+      st = queue(slot, page);
     }
-    c->len[id] = nl;
+    if (st == KVQ_OK) {
+      j.add(Journal::kLen, id, c->len[id]);
+      c->len[id] = nl;
+    }
   }
-  return flush();
+  if (st == KVQ_OK) st = flush();
+  if (st != KVQ_OK) rollback(c, j, flushed, stream);
+  return st;
 }
 
 kvq_status kvq_seq_release(kvq_cache* c, int32_t id) {
@@ -421,24 +537,35 @@ kvq_status kvq_seq_fork(kvq_cache* c, int32_t src, int32_t dst, int64_t n_tokens
   if (n_tokens < 0 || n_tokens > c->len[src])
     return fail(KVQ_ERR_INVALID_ARG, "n_tokens %lld outside [0, len = %lld]", (long long)n_tokens,
                 (long long)c->len[src]);
+  if (kvq_status s = same_device(c)) return s;
   const int P = c->L.page_tokens;
   const int32_t pages = int32_t((n_tokens + P - 1) / P);
+  Journal j;
   kvq::PtUpdate upd;
   upd.n = 0;
-  for (int32_t p = 0; p < pages; ++p) {
+  size_t flushed = 0;
+  int n_flush = 0;
+  kvq_status st = KVQ_OK;
+  for (int32_t p = 0; p < pages && st == KVQ_OK; ++p) {
     const int32_t page = c->table[size_t(src) * c->L.max_pages_per_seq + p];
-    const int32_t slot = dst * c->L.max_pages_per_seq + p;
-    c->table[slot] = page;
+    const size_t slot = size_t(dst) * c->L.max_pages_per_seq + p;
+    set_slot(c, slot, page, &j);
     c->refs[page]++;
-    upd.idx[upd.n] = slot;
+    j.add(Journal::kRef, page);
+    upd.idx[upd.n] = int32_t(slot);
     upd.val[upd.n] = page;
     if (++upd.n == kvq::kMaxPtUpdates || p == pages - 1) {
-      if (!c->host_only)
-        if (kvq_status s = launched(kvq::launch_pt_update(c->d_page_table, upd, (cudaStream_t)stream),
-                                    "page-table update"))
-          return s;
+      if (injected_pt_failure(++n_flush))
+        st = fail(KVQ_ERR_CUDA, "page-table update: injected failure (KVQ_INJECT_PT_FAILURE)");
+      else if (!c->host_only)
+        st = launched(kvq::launch_pt_update(c->d_page_table, upd, (cudaStream_t)stream), "page-table update");
+      if (st == KVQ_OK) flushed = j.ops.size();
       upd.n = 0;
     }
+  }
+  if (st != KVQ_OK) {
+    rollback(c, j, flushed, stream);
+    return st;
   }
   c->mapped[dst] = pages;
   c->len[dst] = n_tokens;
@@ -591,6 +718,7 @@ kvq_status kvq_cache_check(kvq_cache* c, kvq_stream_t stream, uint32_t* detail) 
   if (kvq_status s = check_cache(c)) return s;
   if (detail) *detail = 0;
   if (c->host_only) return KVQ_OK;
+  if (kvq_status s = same_device(c)) return s;
   KVQ_CUDA(cudaStreamSynchronize((cudaStream_t)stream), "cudaStreamSynchronize");
   KVQ_CUDA(cudaGetLastError(), "earlier launch");
   uint32_t code = 0;

@@ -85,6 +85,11 @@ __device__ __forceinline__ void record_error(uint32_t* err, uint32_t code) {
 // Sets the text kvq_last_error() returns on this thread; returns `s`.
 kvq_status set_last_error(kvq_status s, const char* msg);
 
+// For calls that launch work: KVQ_ERR_UNSUPPORTED for a host-only cache,
+// KVQ_ERR_INVALID_ARG when the current CUDA device is not the cache's;
+// otherwise *device = the cache's device.
+kvq_status launch_device(const kvq_cache* c, int* device);
+
 // ---------------------------------------------------------------------------
 // launchers (defined in the kernel translation units)
 // ---------------------------------------------------------------------------

@@ -277,3 +277,51 @@ def test_injected_allocation_failure_is_reported_and_cleaned_up(kvq, monkeypatch
     c.extend([0], [10])
     assert c.length(0) == 10
     c.close()
+
+
+def _allocator_state(c, ids, pages):
+    return ([c.length(i) for i in ids], [[c.page(i, p) for p in range(pages)] for i in ids], c.footprint())
+
+
+@pytest.mark.parametrize("nth", [1, 2])
+def test_extend_is_all_or_nothing_when_a_page_table_enqueue_fails(kvq, monkeypatch, nth):
+    """Host-side fault injection: the nth page-table enqueue of kvq_seq_extend fails (the first one after
+    1024 updates, or the final one).  The call returns KVQ_ERR_CUDA and no sequence, page or reference
+    changes; the same extend then succeeds and hands out the pages a fresh cache would."""
+    c = kvq.Cache(n_layers=1, n_kv_heads=2, head_dim=64, k_bits=8, v_bits=4, max_seqs=3,
+                  max_tokens=64 * 3000, page_tokens=64, host_only=True)
+    c.extend([0], [100])
+    c.fork(0, 2, 70)                                    # a shared, partly filled tail page (copy-on-write)
+    before = _allocator_state(c, [0, 1, 2], 1200)
+    monkeypatch.setenv("KVQ_INJECT_PT_FAILURE", str(nth))
+    with pytest.raises(kvq.KvqError) as e:
+        c.extend([2, 1], [5, 64 * 1100])                # 1 copy-on-write page + 1100 new pages
+    assert e.value.name == "KVQ_ERR_CUDA" and "injected" in str(e.value)
+    assert _allocator_state(c, [0, 1, 2], 1200) == before
+    monkeypatch.delenv("KVQ_INJECT_PT_FAILURE")
+    c.extend([2, 1], [5, 64 * 1100])
+    fresh = kvq.Cache(n_layers=1, n_kv_heads=2, head_dim=64, k_bits=8, v_bits=4, max_seqs=3,
+                      max_tokens=64 * 3000, page_tokens=64, host_only=True)
+    fresh.extend([0], [100])
+    fresh.fork(0, 2, 70)
+    fresh.extend([2, 1], [5, 64 * 1100])
+    assert _allocator_state(c, [0, 1, 2], 1200) == _allocator_state(fresh, [0, 1, 2], 1200)
+    c.close()
+    fresh.close()
+
+
+def test_fork_is_all_or_nothing_when_a_page_table_enqueue_fails(kvq, monkeypatch):
+    """A fork of 1100 pages whose second page-table enqueue fails leaves both sequences and every
+    reference count as they were: releasing the source afterwards frees all its pages."""
+    c = kvq.Cache(n_layers=1, n_kv_heads=2, head_dim=64, k_bits=8, v_bits=4, max_seqs=2,
+                  max_tokens=64 * 1200, page_tokens=64, host_only=True)
+    c.extend([0], [64 * 1100])
+    before = _allocator_state(c, [0, 1], 1100)
+    monkeypatch.setenv("KVQ_INJECT_PT_FAILURE", "2")
+    with pytest.raises(kvq.KvqError):
+        c.fork(0, 1)
+    monkeypatch.delenv("KVQ_INJECT_PT_FAILURE")
+    assert _allocator_state(c, [0, 1], 1100) == before
+    c.release(0)
+    assert c.footprint()[1] == 0                        # no page kept alive by a leaked reference
+    c.close()
