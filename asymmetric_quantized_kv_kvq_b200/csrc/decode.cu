@@ -9,8 +9,8 @@
 namespace kvq {
 
 template <int KB, int VB>
-cudaError_t launch_decode_kv(const Layout&, int, const Batch&, const DecodePlan&, int, const void*, void*, float,
-                             void*, cudaStream_t);
+cudaError_t launch_decode_kv(const Layout&, int, const Batch&, const DecodePlan&, int, const void*, void*, const void*,
+                             const void*, float, void*, cudaStream_t, bool*);
 template <int KB, int VB>
 int decode_chunk_tokens_kv(int D, int G);
 
@@ -110,19 +110,26 @@ int decode_chunk_tokens(const Layout& L, int G) {
 }
 
 cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const DecodePlan& plan, int n_q_heads,
-                          const void* q, void* out, float scale_log2, void* ws, cudaStream_t s) {
+                          const void* q, void* out, const void* k_new, const void* v_new, float scale_log2, void* ws,
+                          cudaStream_t s) {
   const int kb = L.k_bits, vb = L.v_bits;
   cudaError_t e;
+  bool combined = false;
   if (decode_tc_supported(L, n_q_heads / L.n_kv_heads))
     e = launch_decode_tc(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
-  else if (kb == 16) e = launch_decode_kv<16, 16>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
-  else if (kb == 8 && vb == 8) e = launch_decode_kv<8, 8>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
-  else if (kb == 8 && vb == 4) e = launch_decode_kv<8, 4>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
-  else if (kb == 4 && vb == 4) e = launch_decode_kv<4, 4>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
-  else e = launch_decode_kv<4, 8>(L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, s);
+  else if (kb == 16)
+    e = launch_decode_kv<16, 16>(L, layer, b, plan, n_q_heads, q, out, k_new, v_new, scale_log2, ws, s, &combined);
+  else if (kb == 8 && vb == 8)
+    e = launch_decode_kv<8, 8>(L, layer, b, plan, n_q_heads, q, out, k_new, v_new, scale_log2, ws, s, &combined);
+  else if (kb == 8 && vb == 4)
+    e = launch_decode_kv<8, 4>(L, layer, b, plan, n_q_heads, q, out, k_new, v_new, scale_log2, ws, s, &combined);
+  else if (kb == 4 && vb == 4)
+    e = launch_decode_kv<4, 4>(L, layer, b, plan, n_q_heads, q, out, k_new, v_new, scale_log2, ws, s, &combined);
+  else
+    e = launch_decode_kv<4, 8>(L, layer, b, plan, n_q_heads, q, out, k_new, v_new, scale_log2, ws, s, &combined);
   if (e != cudaSuccess) return e;
-  // combine only when some item spans several CTAs
-  if (plan.n_cta > 1 || plan.n_items > 1) {
+  // separate combine only for the kernels that leave split items' partials in the workspace
+  if (!combined && (plan.n_cta > 1 || plan.n_items > 1)) {
     const int H = L.n_kv_heads, G = n_q_heads / H, D = L.head_dim;
     const int64_t slots = int64_t(plan.max_ctas) + plan.n_items;
     const float* ws_o = static_cast<const float*>(ws);
@@ -138,6 +145,11 @@ cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const Deco
     e = cudaGetLastError();
   }
   return e;
+}
+
+// True when launch_decode quantises k_new / v_new itself (fused append).
+bool decode_fuses_append(const Layout& L, int G) {
+  return L.k_bits != 16 && L.v_bits != 16 && !decode_tc_supported(L, G);
 }
 
 }  // namespace kvq

@@ -1,8 +1,8 @@
-// Split-KV decode kernels for K16V16 caches.
+// Split-KV decode kernels for FP16 caches.
 #include "decode_launch.cuh"
 
 namespace kvq {
 template cudaError_t launch_decode_kv<16, 16>(const Layout&, int, const Batch&, const DecodePlan&, int, const void*,
-                                              void*, float, void*, cudaStream_t);
+                                              void*, const void*, const void*, float, void*, cudaStream_t, bool*);
 template int decode_chunk_tokens_kv<16, 16>(int, int);
 }  // namespace kvq

@@ -223,9 +223,9 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
   const int64_t x0 = int64_t(blockIdx.x) * a.cpc;
   const int64_t x1 = min(a.total_chunks, x0 + a.cpc);
 
-  // stage ring starts zeroed so rows never written by a copy stay finite
-  for (int i = threadIdx.x; i < S * T::STAGE_BYTES / 16; i += T::NT)
-    reinterpret_cast<uint4*>(stages)[i] = make_uint4(0, 0, 0, 0);
+  // the stage ring is not cleared: rows past a sequence's end (never copied, or
+  // stale) only reach scores that are replaced by -inf with a select, and the PV
+  // loop skips them, so their contents never matter
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(full0 + 8 * s, 1);

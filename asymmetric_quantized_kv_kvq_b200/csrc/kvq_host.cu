@@ -90,6 +90,7 @@ struct kvq_cache {
   int64_t bytes_per_token_layer = 0;
   int32_t* d_page_table = nullptr;
   uint32_t* d_err = nullptr;
+  int32_t* d_counters = nullptr;     // decode split-item counters, [KVQ_MAX_BATCH * n_kv_heads]
   std::vector<int32_t> table;        // host mirror of the page table
   std::vector<int64_t> len;          // tokens per sequence
   std::vector<int32_t> mapped;       // pages mapped per sequence
@@ -348,9 +349,11 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
       if (L.pool) cudaFree(L.pool);
       if (c->d_page_table) cudaFree(c->d_page_table);
       if (c->d_err) cudaFree(c->d_err);
+      if (c->d_counters) cudaFree(c->d_counters);
       delete c;
       return cuda_fail(err, what);
     };
+    const size_t counter_bytes = size_t(kvq::kMaxBatch) * H * sizeof(int32_t);
     if ((e = cudaMalloc(&L.pool, size_t(c->pool_bytes))) != cudaSuccess) return cleanup(e, "cudaMalloc(page pool)");
     if ((e = cudaMalloc(&c->d_page_table, c->table.size() * sizeof(int32_t))) != cudaSuccess)
       return cleanup(e, "cudaMalloc(page table)");
@@ -359,9 +362,12 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
     if ((e = cudaMemset(c->d_page_table, 0xFF, c->table.size() * sizeof(int32_t))) != cudaSuccess)
       return cleanup(e, "cudaMemset(page table)");
     if ((e = cudaMemset(c->d_err, 0, sizeof(uint32_t))) != cudaSuccess) return cleanup(e, "cudaMemset(err)");
+    if ((e = cudaMalloc(&c->d_counters, counter_bytes)) != cudaSuccess) return cleanup(e, "cudaMalloc(counters)");
+    if ((e = cudaMemset(c->d_counters, 0, counter_bytes)) != cudaSuccess) return cleanup(e, "cudaMemset(counters)");
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cleanup(e, "cudaDeviceSynchronize");
     L.page_table = c->d_page_table;
     L.err = c->d_err;
+    L.counters = c->d_counters;
   }
   *out = c;
   return KVQ_OK;
@@ -376,6 +382,7 @@ kvq_status kvq_cache_destroy(kvq_cache* c) {
     cudaFree(c->L.pool);
     cudaFree(c->d_page_table);
     cudaFree(c->d_err);
+    cudaFree(c->d_counters);
   }
   delete c;
   return st;
@@ -605,9 +612,16 @@ kvq_status kvq_decode_workspace_size(const kvq_cache* c, int32_t n, int32_t n_q_
   return KVQ_OK;
 }
 
-kvq_status kvq_decode_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, int32_t n_q_heads,
-                           const void* q, void* out, float softmax_scale, void* ws, size_t ws_bytes,
-                           kvq_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// kvq_decode_attn, and with k_new / v_new the appending variant: position
+// len - 1 of every named sequence is quantised first (fused into the decode
+// kernel for quantized caches, a separate append launch otherwise).
+kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, int32_t n_q_heads, const void* q,
+                       const void* k_new, const void* v_new, void* out, float softmax_scale, void* ws,
+                       size_t ws_bytes, kvq_stream_t stream) {
   if (kvq_status s = check_cache(c)) return s;
   if (kvq_status s = check_layer(c, layer)) return s;
   if (kvq_status s = check_ids(c, n, ids)) return s;
@@ -616,6 +630,10 @@ kvq_status kvq_decode_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_t
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KVQ_ERR_UNSUPPORTED, "GQA group %d not built (1, 2, 4, 8)", G);
   if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q or out is NULL");
   if (!aligned16(q) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
+  const bool appending = k_new || v_new;
+  if (appending && (!k_new || !v_new)) return fail(KVQ_ERR_INVALID_ARG, "k_new and v_new must both be given");
+  if (appending && (!aligned16(k_new) || !aligned16(v_new)))
+    return fail(KVQ_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
   if (ws && !aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return fail(KVQ_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   size_t need = 0;
@@ -645,8 +663,34 @@ kvq_status kvq_decode_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_t
   if (flat >= (int64_t(1) << 31)) return fail(KVQ_ERR_INVALID_ARG, "batch too large");
   const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(c->L.head_dim));
   const float scale_log2 = sigma * 1.4426950408889634f;
-  return launched(kvq::launch_decode(c->L, layer, b, plan, n_q_heads, q, out, scale_log2, ws, (cudaStream_t)stream),
+  const bool fused = appending && kvq::decode_fuses_append(c->L, G);
+  if (appending && !fused) {
+    kvq::Batch ab;
+    ab.n = n;
+    for (int i = 0; i < n; ++i) ab.s[i] = {ids[i], int32_t(c->len[ids[i]] - 1), 1, i};
+    if (kvq_status s = launched(kvq::launch_append(c->L, layer, ab, n, k_new, v_new, (cudaStream_t)stream), "append"))
+      return s;
+  }
+  return launched(kvq::launch_decode(c->L, layer, b, plan, n_q_heads, q, out, fused ? k_new : nullptr,
+                                     fused ? v_new : nullptr, scale_log2, ws, (cudaStream_t)stream),
                   "decode");
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kvq_decode_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, int32_t n_q_heads,
+                           const void* q, void* out, float softmax_scale, void* ws, size_t ws_bytes,
+                           kvq_stream_t stream) {
+  return decode_impl(c, layer, n, ids, n_q_heads, q, nullptr, nullptr, out, softmax_scale, ws, ws_bytes, stream);
+}
+
+kvq_status kvq_decode_append_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, int32_t n_q_heads,
+                                  const void* q, const void* k_new, const void* v_new, void* out,
+                                  float softmax_scale, void* ws, size_t ws_bytes, kvq_stream_t stream) {
+  if (!k_new || !v_new) return fail(KVQ_ERR_INVALID_ARG, "k_new or v_new is NULL");
+  return decode_impl(c, layer, n, ids, n_q_heads, q, k_new, v_new, out, softmax_scale, ws, ws_bytes, stream);
 }
 
 kvq_status kvq_prefill_workspace_size(const kvq_cache* c, int32_t n, const int32_t* ids, const int32_t* q_lens,
@@ -726,6 +770,9 @@ kvq_status kvq_cache_check(kvq_cache* c, kvq_stream_t stream, uint32_t* detail) 
   if (code) {
     if (detail) *detail = code;
     KVQ_CUDA(cudaMemset(c->d_err, 0, sizeof code), "clear device error word");
+    // a kernel that gave up may have left split-item counters raised
+    KVQ_CUDA(cudaMemset(c->d_counters, 0, size_t(kvq::kMaxBatch) * c->L.n_kv_heads * sizeof(int32_t)),
+             "clear decode counters");
     return fail(KVQ_ERR_DEVICE_CHECK, "device check failed, code 0x%x", code);
   }
   return KVQ_OK;

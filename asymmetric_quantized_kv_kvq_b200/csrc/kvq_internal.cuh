@@ -48,6 +48,7 @@ struct Layout {
   int32_t s_row;                       // scale bytes per token (D/32 * 2), 0 for 16-bit
   int32_t k_scales_off, v_codes_off, v_scales_off;   // byte offsets inside a head block
   int32_t decode_tc;                   // KVQ_CACHE_DECODE_TENSOR_CORES was set
+  int32_t* counters;                   // [kMaxBatch * n_kv_heads] split-item counters of the decode kernel (zero at rest)
 
   __host__ __device__ __forceinline__ uint8_t* head_ptr(int layer, int page, int head) const {
     return pool + ((int64_t(layer) * n_pages + page) * n_kv_heads + head) * head_block;
@@ -115,9 +116,12 @@ struct DecodePlan {
 size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D);
 int decode_max_ctas(int num_sms);
 int decode_chunk_tokens(const Layout& L, int G);
+// k_new / v_new: fp16 [B, Hkv, D] rows of position len - 1 to quantise into the
+// cache first (nullptr: plain decode); only when decode_fuses_append(L, G).
 cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const DecodePlan& plan,
-                          int n_q_heads, const void* q, void* out, float scale_log2,
-                          void* workspace, cudaStream_t s);
+                          int n_q_heads, const void* q, void* out, const void* k_new, const void* v_new,
+                          float scale_log2, void* workspace, cudaStream_t s);
+bool decode_fuses_append(const Layout& L, int G);
 
 size_t prefill_workspace_bytes(const Layout& L, const Batch& b);
 cudaError_t launch_prefill(const Layout& L, int layer, const Batch& b, int total_q, int n_q_heads,

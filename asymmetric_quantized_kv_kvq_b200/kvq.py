@@ -61,6 +61,7 @@ SIGNATURES = {
     "kvq_decode_workspace_size": (_i32, [_p, _i32, _i32, _psz]),
     "kvq_decode_attn": (_i32, [_p, _i32, _i32, _pi32, _i32, _p, _p, _f32, _p, _sz, _p]),
     "kvq_decode_attn_noalloc": (_i32, [_p, _i32, _i32, _pi32, _i32, _p, _p, _f32, _p]),
+    "kvq_decode_append_attn": (_i32, [_p, _i32, _i32, _pi32, _i32, _p, _p, _p, _p, _f32, _p, _sz, _p]),
     "kvq_prefill_workspace_size": (_i32, [_p, _i32, _pi32, _pi32, _i32, _psz]),
     "kvq_prefill_attn": (_i32, [_p, _i32, _i32, _pi32, _pi32, _i32, _p, _p, _f32, _p, _sz, _p]),
     "kvq_export": (_i32, [_p, _i32, _i32, _i64, _i64, _p, _p, _p, _p, _p]),
@@ -238,6 +239,28 @@ class Cache:
         _check(self._lib.kvq_decode_attn(self._h, layer, B, _i32_array(seq_ids), Hq, q.data_ptr(),
                                          out.data_ptr(), softmax_scale, ws.data_ptr(),
                                          ws.numel() * ws.element_size(), _stream(stream)))
+        return out
+
+    def decode_append(self, layer: int, seq_ids: Sequence[int], q, k_new, v_new, out=None,
+                      softmax_scale: float = 0.0, workspace=None, stream=None):
+        """kvq_decode_append_attn: quantise k_new / v_new (fp16 [B, Hkv, D]) into position len - 1
+        of each sequence, then decode q over positions 0 .. len - 1 (one launch for quantized caches)."""
+        import torch
+        B = len(seq_ids)
+        if q.dim() != 3 or q.shape[0] != B or q.shape[2] != self.head_dim:
+            raise KvqError(1, f"q has shape {tuple(q.shape)}, expected [{B}, Hq, {self.head_dim}]")
+        Hq = q.shape[1]
+        _dev_fp16(q, "q")
+        kp = _dev_fp16(k_new, "k_new", (B, self.n_kv_heads, self.head_dim))
+        vp = _dev_fp16(v_new, "v_new", (B, self.n_kv_heads, self.head_dim))
+        if out is None:
+            out = torch.empty_like(q)
+        _dev_fp16(out, "out", tuple(q.shape))
+        need = self.decode_workspace_size(B, Hq)
+        ws = workspace if workspace is not None else self._workspace(need, q.device)
+        _check(self._lib.kvq_decode_append_attn(self._h, layer, B, _i32_array(seq_ids), Hq, q.data_ptr(), kp, vp,
+                                                out.data_ptr(), softmax_scale, ws.data_ptr(),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
         return out
 
     def decode_noalloc(self, layer: int, seq_ids: Sequence[int], q, out=None, softmax_scale: float = 0.0,

@@ -5,14 +5,20 @@
     python bench.py --impl reference ...      # the CPU oracle on host cores
 
 One step = one decode step of the workload: every sequence gains one token;
-for each layer the new token's K / V are quantised into the paged cache
-(kvq_append) and the query attends to the whole cache (kvq_decode_attn:
-split-KV kernel + log-sum-exp combine).  Metric: algorithmic KV bytes moved
-per second (cache codes + scales read by decode, fp16 q / out, the appended
+for each layer the new token's K / V are quantised into the paged cache and
+the query attends to the whole cache.  For quantized caches that is one
+kvq_decode_append_attn launch per layer (append, split-KV attention and the
+log-sum-exp combine in one kernel); fp16 caches (and --separate) call
+kvq_append then kvq_decode_attn.  Metric: algorithmic KV bytes moved per
+second (cache codes + scales read by decode, fp16 q / out, the appended
 token's fp16 read and quantised write), and decode tokens/s = batch / step.
 By default one step is captured in a CUDA graph after the warm-up and every
 timed step replays it (the same token re-appended at the same position, the
 same length attended); --eager makes the API calls directly each step.
+
+The default run (no --workload) also measures, as compact "extra" records with
+their own clocks, the 70B-shaped single-sequence decode (K8V4 and FP16) and
+the ragged chunked prefill (prefill TFLOP/s and append GB/s).
 
 Multi-GPU (torchrun): every rank holds an independent replica of the workload
 (sequences are independent, so the batch shards with no collective); value =
@@ -56,8 +62,10 @@ def measured_peaks() -> dict:
 
 KERNEL_SOURCES = {
     "decode_split": ("decode_kernel.cuh", "decode_launch.cuh", "decode.cu", "decode_common.cuh", "sm100_util.cuh"),
+    "decode_q": ("decode_q.cuh", "decode_launch.cuh", "decode.cu", "decode_common.cuh", "sm100_util.cuh",
+                 "quant_block.cuh"),
     "decode_tc": ("decode_tc.cu", "decode.cu", "decode_common.cuh", "sm100_util.cuh", "tcgen05_util.cuh"),
-    "append": ("append.cu", "kvq_internal.cuh"),
+    "append": ("append.cu", "quant_block.cuh", "kvq_internal.cuh"),
 }
 
 
@@ -139,7 +147,8 @@ class ClockSampler:
 class DecodeRun:
     """A resident cache of the workload plus one decode step's inputs."""
 
-    def __init__(self, wl, kb: int, vb: int, capacity_extra: int, device, decode_tc: bool = False):
+    def __init__(self, wl, kb: int, vb: int, capacity_extra: int, device, decode_tc: bool = False,
+                 separate: bool = False):
         import torch
         from asymmetric_quantized_kv_kvq_b200 import kvq
         from asymmetric_quantized_kv_kvq_b200.inputs import gen_kv, gen_q, GEN_CHUNK
@@ -174,6 +183,8 @@ class DecodeRun:
         self.ws = torch.empty(self.cache.decode_workspace_size(B, wl.n_q_heads), dtype=torch.uint8, device=device)
         self.ones = [1] * B
         self.ev = None
+        # one launch per layer (append fused into the decode kernel) for quantized caches on CUDA cores
+        self.fused = kb != 16 and not decode_tc and not separate
 
     def lengths(self):
         return [self.cache.length(b) for b in self.ids]
@@ -189,15 +200,28 @@ class DecodeRun:
 
     def launches_per_step(self, lens_before) -> int:
         pt = 1 if any(n % 256 == 0 for n in lens_before) else 0
-        return pt + self.wl.n_layers * 3   # append, decode split, combine
+        if self.fused:
+            return pt + self.wl.n_layers                 # one decode kernel (append + split + combine)
+        combine = 0 if (self.kb != 16 and not self.cache_tc) else 1
+        return pt + self.wl.n_layers * (2 + combine)    # append, decode[, combine]
+
+    @property
+    def cache_tc(self) -> bool:
+        return self.cache.cfg.flags & 2 != 0 and self.kb == 8 and self.wl.head_dim == 128
 
     def step(self, record=None):
         self.cache.extend(self.ids, self.ones)
         for layer in range(self.wl.n_layers):
-            self.cache.append(layer, self.ids, self.ones, self.k_new[layer], self.v_new[layer])
-            if record is not None:
-                record[layer][0].record()
-            self.cache.decode(layer, self.ids, self.q[layer], out=self.out[layer], workspace=self.ws)
+            if self.fused:
+                if record is not None:
+                    record[layer][0].record()
+                self.cache.decode_append(layer, self.ids, self.q[layer], self.k_new[layer], self.v_new[layer],
+                                         out=self.out[layer], workspace=self.ws)
+            else:
+                self.cache.append(layer, self.ids, self.ones, self.k_new[layer], self.v_new[layer])
+                if record is not None:
+                    record[layer][0].record()
+                self.cache.decode(layer, self.ids, self.q[layer], out=self.out[layer], workspace=self.ws)
             if record is not None:
                 record[layer][1].record()
 
@@ -208,7 +232,7 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
     torch.cuda.set_device(dev)
     extra = args.warmup + 2 * args.steps + 8
     t0 = time.time()
-    run = DecodeRun(wl, kb, vb, extra, dev, decode_tc=args.decode_tc)
+    run = DecodeRun(wl, kb, vb, extra, dev, decode_tc=args.decode_tc, separate=args.separate)
     setup_s = time.time() - t0
     L = wl.n_layers
     lens0 = run.lengths()
@@ -251,7 +275,7 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
             dec_bytes += d
             app_bytes += a
             launches += run.launches_per_step(lens_before)
-    in_step_bytes = dec_bytes / args.steps
+    in_step_bytes = (dec_bytes + (app_bytes if run.fused else 0)) / args.steps
     if graph is not None:
         # per-layer decode durations inside a step: one eager step with events (outside the timed region)
         lens_e = run.lengths()
@@ -260,12 +284,14 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         run.step(record=ev)
         torch.cuda.synchronize()
         dec_ms.extend(e0.elapsed_time(e1) for e0, e1 in ev)
-        in_step_bytes = run.step_bytes([n + 1 for n in lens_e])[0]
+        d_e, a_e = run.step_bytes([n + 1 for n in lens_e])
+        in_step_bytes = d_e + (a_e if run.fused else 0)
     # ---- kernel duration: every layer's decode call once more, back to back on the
     #      stream behind a short device-side sleep, so that host work between calls
     #      (binding, plan) never leaves the GPU idle inside the events
     lens_k = run.lengths()
-    kern_bytes = run.step_bytes(lens_k)[0] / L
+    kd, ka = run.step_bytes(lens_k)
+    kern_bytes = (kd + (ka if run.fused else 0)) / L
     reps = max(L, 8)
     kern_ms = []
     for _ in range(2):
@@ -276,7 +302,11 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         k0.record()
         for i in range(reps):
             lay = i % L
-            run.cache.decode(lay, run.ids, run.q[lay], out=run.out[lay], workspace=run.ws)
+            if run.fused:        # re-appends the last token at the same position, as a replayed step does
+                run.cache.decode_append(lay, run.ids, run.q[lay], run.k_new[lay], run.v_new[lay], out=run.out[lay],
+                                        workspace=run.ws)
+            else:
+                run.cache.decode(lay, run.ids, run.q[lay], out=run.out[lay], workspace=run.ws)
         k1.record()
         torch.cuda.synchronize()
         kern_ms.append(k0.elapsed_time(k1) / reps)
@@ -301,11 +331,18 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         "clocks": clk.summary(),
         "flush": flush,
         "setup_s": setup_s,
+        "fused": run.fused,
+        "step_only_decode": run.fused and graph is not None,
+        "step_bytes": (dec_bytes + app_bytes) / args.steps,
     }
 
-    # ---- end to end through the public API with host buffers
+    # ---- end to end through the public API with host buffers: replaying the captured step (the
+    #      default launch mode) and, beside it, calling the API eagerly every step
     if not args.no_e2e:
-        res["e2e"] = run_e2e(run, args, world, dev)
+        res["e2e"] = run_e2e(run, args, world, dev, eager=args.eager)
+        if not args.eager:
+            res["e2e_eager"] = run_e2e(run, args, world, dev, eager=True)
+    del graph
     run.cache.close()
     return res
 
@@ -330,9 +367,11 @@ def capture_step(run, body):
         return None, None, f"eager (graph capture failed: {type(e).__name__}: {str(e)[:120]})"
 
 
-def run_e2e(run, args, world, dev) -> dict:
+def run_e2e(run, args, world, dev, eager: bool) -> dict:
     """Same step, but every step copies its inputs (q, new K / V for all layers)
-    from pinned host memory and reads all outputs back to pinned host memory."""
+    from pinned host memory and reads all outputs back to pinned host memory;
+    the step is a replayed graph of the copies + calls, or (eager) the host
+    calls themselves, binding and validation included."""
     import torch
     L = run.wl.n_layers
     hq = [t.cpu().pin_memory() for t in run.q]
@@ -354,7 +393,7 @@ def run_e2e(run, args, world, dev) -> dict:
     for _ in range(2):
         body()
     graph, graph_lens = None, None
-    if not args.eager:
+    if not eager:
         graph, graph_lens, _ = capture_step(run, body)
     barrier(world)
     torch.cuda.synchronize()
@@ -375,8 +414,9 @@ def run_e2e(run, args, world, dev) -> dict:
     barrier(world)
     max_ms = all_reduce_max(ms, world, dev)
     tot = all_reduce_sum(float(nbytes), world, dev)
+    del graph
     return {"value": tot / (max_ms * 1e-3) / 1e9, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h}
+            "d2h_bytes_per_step": d2h, "launch": "eager API calls" if eager else "replayed CUDA graph"}
 
 
 PREFILL_METRIC = "K8V4 chunked-prefill TFLOP/s (causal FLOPs) and quantise-on-append GB/s"
@@ -644,7 +684,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=list(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=list(WORKLOADS), default=None,
+                    help=f"default {DEFAULT_WORKLOAD} (plus the extra records)")
     ap.add_argument("--precision", default=None, help="K8V4, K8V8, K4V4, K4V8 or FP16 (default: first of the workload)")
     ap.add_argument("--layers", type=int, default=0, help="override the workload's layer count (profiling)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiling)")
@@ -655,6 +696,11 @@ def parse():
     ap.add_argument("--eager", action="store_true",
                     help="launch every decode step through the API calls directly instead of replaying a "
                          "CUDA graph of one captured step")
+    ap.add_argument("--separate", action="store_true",
+                    help="quantized caches: kvq_append + kvq_decode_attn per layer instead of the fused "
+                         "kvq_decode_append_attn launch")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="default run: skip the 70B-shaped decode and the prefill sub-records")
     ap.add_argument("--decode-tc", action="store_true",
                     help="decode on the tensor-core kernel (cache flag KVQ_CACHE_DECODE_TENSOR_CORES) "
                          "instead of the default CUDA-core kernel")
@@ -674,6 +720,8 @@ def config_of(wl, precision, world, flush) -> dict:
 def main():
     args = parse()
     from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS, parse_precision
+    default_run = args.workload is None
+    args.workload = args.workload or DEFAULT_WORKLOAD
     wl = WORKLOADS[args.workload]
     if args.layers or args.batch or args.cached:
         import dataclasses
@@ -737,39 +785,107 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = oracle_decode_slices(wl, kb, vb, args.cpu_seconds)
+    extras = []
+    if default_run and world == 1 and not args.no_extras:
+        extras = run_extras(args)
     if rank == 0:
-        peaks = measured_peaks()
-        achieved = res["kern_bytes_per_launch"] / (res["kern_ms_per_launch"] * 1e-3) / 1e9
-        in_step = res["dec_bytes_per_launch"] / (res["dec_ms_per_launch"] * 1e-3) / 1e9
-        tc = args.decode_tc and kb == 8 and vb in (4, 8) and wl.head_dim == 128
-        traffic = ncu_traffic(wl.name, precision, "decode_tc" if tc else "decode_split")
-        line = {
-            "metric": METRIC, "value": res["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": dict(config_of(wl, precision, world, res["flush"]),
-                           decode_kernel="tensor cores (opt-in)" if tc else "CUDA cores",
-                           step_launch=res["launch_mode"]),
-            "decode_tokens_per_s": res["decode_tokens_per_s"],
-            "roofline": {"bound": "hbm",
-                         "kernel": ("decode_tc_kernel" if tc else "decode_split_kernel") + " + lse_combine_kernel",
-                         "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
-                         "frac_of_8tbs_nominal": achieved / 8000.0,
-                         "bytes_per_launch": res["kern_bytes_per_launch"],
-                         "ms_per_launch": res["kern_ms_per_launch"],
-                         "timing": f"CUDA events around {max(wl.n_layers, 8)} back-to-back decode calls "
-                                   f"(one per layer) queued behind a device sleep; best of 2",
-                         "achieved_in_step": in_step, "traffic": traffic},
-            "cpu_baseline": None if cpu is None else {k: cpu[k] for k in ("value", "unit", "cores", "kind", "sample")},
-            "e2e": res.get("e2e"),
-            "clocks": res["clocks"],
-            "gpu_launches": res["launches"],
-        }
+        line = decode_line(args, wl, precision, kb, vb, res, world)
+        line["cpu_baseline"] = None if cpu is None else {k: cpu[k] for k in ("value", "unit", "cores", "kind",
+                                                                             "sample")}
+        if extras:
+            line["extra"] = extras
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def decode_line(args, wl, precision, kb, vb, res, world) -> dict:
+    """The JSON line of a decode run.  The roofline's dominant kernel is the decode
+    kernel; for the fused one-launch step the replayed step is nothing but those
+    launches, so its bytes / the step's own CUDA-event time is the kernel's
+    achieved bandwidth (same basis as ms_per_step)."""
+    peaks = measured_peaks()
+    L = wl.n_layers
+    isolated = res["kern_bytes_per_launch"] / (res["kern_ms_per_launch"] * 1e-3) / 1e9
+    in_step = res["dec_bytes_per_launch"] / (res["dec_ms_per_launch"] * 1e-3) / 1e9
+    tc = args.decode_tc and kb == 8 and vb in (4, 8) and wl.head_dim == 128
+    if res["step_only_decode"]:
+        achieved = res["value"]
+        ms_launch = res["ms_per_step"] / L
+        timing = (f"CUDA events around each replayed step = {L} back-to-back decode launches (one per layer, "
+                  f"append and combine fused); ms_per_launch = ms_per_step / {L}")
+        kernel = "decode_q_kernel (append + split-KV + combine)"
+        bytes_launch = res["step_bytes"] / L
+    else:
+        achieved = isolated
+        ms_launch = res["kern_ms_per_launch"]
+        timing = (f"CUDA events around {max(L, 8)} back-to-back decode calls (one per layer) queued behind a "
+                  f"device sleep; best of 2")
+        if tc:
+            kernel = "decode_tc_kernel + lse_combine_kernel"
+        elif kb == 16:
+            kernel = "decode_split_kernel + lse_combine_kernel"
+        else:
+            kernel = "decode_q_kernel (split-KV + combine)"
+        bytes_launch = res["kern_bytes_per_launch"]
+    traffic_kernel = "decode_tc" if tc else ("decode_split" if kb == 16 else "decode_q")
+    line = {
+        "metric": METRIC, "value": res["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(config_of(wl, precision, world, res["flush"]),
+                       decode_kernel="tensor cores (opt-in)" if tc else "CUDA cores",
+                       step_launch=res["launch_mode"] + ("; one fused append+decode launch per layer"
+                                                         if res["fused"] else "")),
+        "decode_tokens_per_s": res["decode_tokens_per_s"],
+        "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+                     "frac_of_8tbs_nominal": achieved / 8000.0, "bytes_per_launch": bytes_launch,
+                     "ms_per_launch": ms_launch, "timing": timing,
+                     "achieved_isolated": isolated, "achieved_in_eager_step": in_step,
+                     "traffic": ncu_traffic(wl.name, precision, traffic_kernel)},
+        "cpu_baseline": None,
+        "e2e": res.get("e2e"),
+        "e2e_eager": res.get("e2e_eager"),
+        "clocks": res["clocks"],
+        "gpu_launches": res["launches"],
+    }
+    return line
+
+
+def run_extras(args) -> list:
+    """Compact records of the other gate workloads, measured in the same run: the
+    70B-shaped 128K-token decode in K8V4 and FP16, and the ragged chunked prefill."""
+    import argparse as _ap
+    import torch
+    from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS, parse_precision
+    out = []
+    sub = _ap.Namespace(**vars(args))
+    sub.steps, sub.warmup, sub.no_e2e, sub.decode_tc, sub.separate = 5, 3, True, False, False
+    for name, prec in (("llama70b-b1-128k", "K8V4"), ("llama70b-b1-128k", "FP16")):
+        wl = WORKLOADS[name]
+        kb, vb = parse_precision(prec)
+        torch.cuda.empty_cache()
+        r = run_decode_bench(sub, wl, kb, vb, 0, 1)
+        line = decode_line(sub, wl, prec, kb, vb, r, 1)
+        out.append({"workload": name, "precision": prec, "metric": "decode KV GB/s", "value": r["value"],
+                    "unit": "GB/s", "ms_per_step": r["ms_per_step"], "steps": sub.steps,
+                    "decode_tokens_per_s": r["decode_tokens_per_s"],
+                    "roofline_frac": line["roofline"]["frac"], "kernel": line["roofline"]["kernel"],
+                    "step_launch": line["config"]["step_launch"], "gpu_launches": r["launches"],
+                    "clocks": r["clocks"]})
+    wl = WORKLOADS["prefill-16x4096"]
+    kb, vb = parse_precision("K8V4")
+    torch.cuda.empty_cache()
+    r = run_prefill_bench(sub, wl, kb, vb, 0, 1)
+    peak = measured_tensor_peak()
+    out.append({"workload": wl.name, "precision": "K8V4", "metric": PREFILL_METRIC, "value": r["value"],
+                "unit": "TFLOP/s", "ms_per_step": r["ms_per_step"], "steps": sub.steps,
+                "prefill_tflops": r["prefill_tflops"], "prefill_frac": r["prefill_tflops"] / peak["value"],
+                "append_gbs": r["append_gbs"], "append_frac": r["append_gbs"] / measured_peaks()["hbm_gbs"],
+                "gpu_launches": r["launches"], "clocks": r["clocks"]})
+    return out
 
 
 def prefill_main(args, wl, precision, kb, vb, rank, world):

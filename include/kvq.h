@@ -199,7 +199,10 @@ KVQ_API kvq_status kvq_decode_workspace_size(const kvq_cache* cache, int32_t n_s
  * K, V, sigma = softmax_scale (0 selects 1/sqrt(head_dim)).
  * q, out: device fp16 [n_seqs, n_q_heads, head_dim].  Split-KV flash-decoding:
  * partial (O, max, sum) per slice of the cache in `workspace` (device,
- * ws_bytes >= kvq_decode_workspace_size), merged by a log-sum-exp combine.
+ * ws_bytes >= kvq_decode_workspace_size), merged by a log-sum-exp combine (for
+ * quantized caches inside the same kernel, by the last CTA that finishes a
+ * sequence's KV head; for fp16 caches and the tensor-core kernel, by a second
+ * kernel).  The merge order is fixed, so results are deterministic.
  * Every named sequence must have len >= 1.  q, out and workspace must be
  * 16-byte aligned (KVQ_ERR_INVALID_ARG otherwise).
  * kvq_seq_extend, kvq_append, kvq_decode_attn and kvq_prefill_attn only
@@ -209,6 +212,24 @@ KVQ_API kvq_status kvq_decode_workspace_size(const kvq_cache* cache, int32_t n_s
 KVQ_API kvq_status kvq_decode_attn(kvq_cache* cache, int32_t layer, int32_t n_seqs, const int32_t* seq_ids,
                            int32_t n_q_heads, const void* q, void* out, float softmax_scale,
                            void* workspace, size_t ws_bytes, kvq_stream_t stream);
+
+/* One decode step of one layer: quantise-on-append of the token at position
+ * len - 1 of every named sequence, then decode attention of its query over
+ * positions 0 .. len - 1 (which include that token).  Same result as
+ * kvq_append (n_new = 1 for each sequence) followed by kvq_decode_attn, in one
+ * kernel launch for quantized caches (the CTA that streams the chunk holding
+ * position len - 1 quantises the new row into the page just before copying
+ * that chunk), two launches for fp16 caches and the tensor-core kernel.  The
+ * positions must already exist (kvq_seq_extend), as for kvq_append.
+ * k_new, v_new: device fp16 [n_seqs, n_kv_heads, head_dim], 16-byte aligned.
+ * The KVSplit page quantises the cache at run time as tokens are processed
+ * (Hacker News reply on .gguf files); the pages' small-model workloads
+ * (22-layer table, "Principais resultados de benchmark") are one such step per
+ * layer.  Other arguments, workspace and errors as kvq_decode_attn. */
+KVQ_API kvq_status kvq_decode_append_attn(kvq_cache* cache, int32_t layer, int32_t n_seqs,
+                                          const int32_t* seq_ids, int32_t n_q_heads, const void* q,
+                                          const void* k_new, const void* v_new, void* out, float softmax_scale,
+                                          void* workspace, size_t ws_bytes, kvq_stream_t stream);
 
 /* Size of the scratch array compiled into the library for
  * kvq_decode_attn_noalloc (8 MiB per GPU that loads the library). */
