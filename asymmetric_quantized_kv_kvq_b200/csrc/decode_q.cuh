@@ -266,7 +266,7 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
   const int item = sg.bi * H + sg.h;
   __syncwarp();
   if (lane == 0) mbar_arrive(sm.mfull);
-  if (!mbar_wait(sm.mfull, itm & 1, sm.abort_flag)) {
+  if (!mbar_wait(sm.mfull, itm & 1, sm.abort_flag, a.L.wait_ns)) {
     if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 6);
     *sm.abort_flag = 1;
     return false;
@@ -307,7 +307,7 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.mws);
     if (ct == 0) {
-      const bool ok = mbar_wait(sm.mws, itw & 1, sm.abort_flag);
+      const bool ok = mbar_wait(sm.mws, itw & 1, sm.abort_flag, a.L.wait_ns);
       int last = 0;
       if (ok) {
         __threadfence();
@@ -321,7 +321,7 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
       *sm.last_flag = last;
       mbar_arrive(sm.mlast);
     }
-    if (!mbar_wait(sm.mlast, itw & 1, sm.abort_flag)) {
+    if (!mbar_wait(sm.mlast, itw & 1, sm.abort_flag, a.L.wait_ns)) {
       if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 8);
       *sm.abort_flag = 1;
       return false;
@@ -369,7 +369,7 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
     const SeqDesc sd = b.s[sg.bi];
     for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
       const int s = it % S;
-      if (!mbar_wait(sm.empty0 + 8 * s, ((it / S) & 1) ^ 1, sm.abort_flag)) {
+      if (!mbar_wait(sm.empty0 + 8 * s, ((it / S) & 1) ^ 1, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 1);
         *sm.abort_flag = 1;
         ok = false;
@@ -407,7 +407,10 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
         }
         __syncwarp();
       }
-      if (lane == 0) {
+      // test hook (cache created with KVQ_TEST_WITHHOLD_ARRIVAL set): CTA 0 never fills its
+      // first stage, so its consumers' bounded waits run out and report kErrWaitTimeout
+      const bool withhold = a.L.test_withhold && blockIdx.x == 0 && it == 0;
+      if (lane == 0 && !withhold) {
         const uint32_t bar = sm.full0 + 8 * s;
         const uint32_t dst = smem_u32(sm.stages + s * T::STAGE);
         mbar_arrive_expect_tx(bar, uint32_t(ncopy * T::TOK_BYTES));
@@ -422,7 +425,7 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
   }
   // no copy may outlive the CTA: wait (bounded) for the last fills to land
   if (lane == 0)
-    for (uint32_t j = it > uint32_t(S) ? it - S : 0; j < it; ++j) mbar_wait(sm.full0 + 8 * (j % S), (j / S) & 1, nullptr);
+    for (uint32_t j = it > uint32_t(S) ? it - S : 0; j < it; ++j) mbar_wait(sm.full0 + 8 * (j % S), (j / S) & 1, nullptr, a.L.wait_ns);
 }
 
 // Score warp: q . k over its partition's tokens, online softmax, p' = p d_v.
@@ -508,7 +511,7 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
     for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
       const int s = it % S, par = it & 1;
       const uint32_t pph = (it >> 1) & 1;
-      if (!mbar_wait(sm.full0 + 8 * s, (it / S) & 1, sm.abort_flag)) {
+      if (!mbar_wait(sm.full0 + 8 * s, (it / S) & 1, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 2);
         *sm.abort_flag = 1;
         return;
@@ -555,7 +558,7 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
         for (int j = 0; j < NF; ++j) need |= sc[ps][j] > m_own[j] + 8.f;
       const bool any = __any_sync(FULL, need);
       // the value warps must be done with this buffer (two stages back) before it is rewritten
-      if (!mbar_wait(sm.free0 + 8 * (part * 2 + par), pph ^ 1, sm.abort_flag)) {
+      if (!mbar_wait(sm.free0 + 8 * (part * 2 + par), pph ^ 1, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 3);
         *sm.abort_flag = 1;
         return;
@@ -615,7 +618,7 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
       ++it;
     }
     // ---- publish (m, l) of this partition's heads, then merge
-    if (!mbar_wait(sm.mfree, (itm & 1) ^ 1, sm.abort_flag)) {
+    if (!mbar_wait(sm.mfree, (itm & 1) ^ 1, sm.abort_flag, a.L.wait_ns)) {
       if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 5);
       *sm.abort_flag = 1;
       return;
@@ -661,8 +664,8 @@ __device__ __forceinline__ void value_role(const DecodeQArgs& a, const Batch& b,
     for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
       const int s = it % S, par = it & 1;
       const uint32_t pph = (it >> 1) & 1;
-      if (!mbar_wait(sm.full0 + 8 * s, (it / S) & 1, sm.abort_flag) ||
-          !mbar_wait(sm.ready0 + 8 * (part * 2 + par), pph, sm.abort_flag)) {
+      if (!mbar_wait(sm.full0 + 8 * s, (it / S) & 1, sm.abort_flag, a.L.wait_ns) ||
+          !mbar_wait(sm.ready0 + 8 * (part * 2 + par), pph, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 4);
         *sm.abort_flag = 1;
         return;
@@ -747,7 +750,7 @@ __device__ __forceinline__ void value_role(const DecodeQArgs& a, const Batch& b,
       ++it;
     }
     // ---- publish this warp's O (summed over its token lanes), then merge
-    if (!mbar_wait(sm.mfree, (itm & 1) ^ 1, sm.abort_flag)) {
+    if (!mbar_wait(sm.mfree, (itm & 1) ^ 1, sm.abort_flag, a.L.wait_ns)) {
       if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 5);
       *sm.abort_flag = 1;
       return;

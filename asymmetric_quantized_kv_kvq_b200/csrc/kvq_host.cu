@@ -12,6 +12,7 @@
 #include <vector>
 
 #include "kvq_internal.cuh"
+#include "sm100_util.cuh"
 
 namespace {
 
@@ -52,13 +53,24 @@ int64_t bytes_per_token_head(int bits, int D) {
   return int64_t(D / 32) * 18;
 }
 
+// Bit widths of one layer: the per-layer arrays when given, else the cache-wide pair.
+int layer_k_bits(const kvq_cache_config* c, int layer) { return c->layer_k_bits ? c->layer_k_bits[layer] : c->k_bits; }
+int layer_v_bits(const kvq_cache_config* c, int layer) { return c->layer_v_bits ? c->layer_v_bits[layer] : c->v_bits; }
+
 kvq_status check_config(const kvq_cache_config* c) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "config is NULL");
   if (c->n_layers < 1 || c->n_kv_heads < 1) return fail(KVQ_ERR_INVALID_ARG, "n_layers and n_kv_heads must be >= 1");
+  if (c->n_layers > 4096) return fail(KVQ_ERR_INVALID_ARG, "n_layers must be <= 4096");
   if (c->head_dim <= 0 || c->head_dim % 32) return fail(KVQ_ERR_INVALID_ARG, "head_dim must be a positive multiple of 32");
-  if (!bits_ok(c->k_bits) || !bits_ok(c->v_bits)) return fail(KVQ_ERR_INVALID_ARG, "k_bits and v_bits must be 16, 8 or 4");
+  if (!c->layer_k_bits != !c->layer_v_bits)
+    return fail(KVQ_ERR_INVALID_ARG, "layer_k_bits and layer_v_bits must both be given or both be NULL");
+  for (int l = 0; l < c->n_layers; ++l) {
+    const int kb = layer_k_bits(c, l), vb = layer_v_bits(c, l);
+    if (!bits_ok(kb) || !bits_ok(vb)) return fail(KVQ_ERR_INVALID_ARG, "layer %d: k_bits and v_bits must be 16, 8 or 4", l);
+    if (!pair_supported(kb, vb)) return fail(KVQ_ERR_UNSUPPORTED, "layer %d: K%dV%d not built", l, kb, vb);
+    if (!c->layer_k_bits) break;
+  }
   if (c->head_dim != 64 && c->head_dim != 128) return fail(KVQ_ERR_UNSUPPORTED, "head_dim %d not built (64, 128)", c->head_dim);
-  if (!pair_supported(c->k_bits, c->v_bits)) return fail(KVQ_ERR_UNSUPPORTED, "K%dV%d not built", c->k_bits, c->v_bits);
   int P = c->page_tokens ? c->page_tokens : 256;
   if (P < 64 || P > 4096 || P % 64) return fail(KVQ_ERR_INVALID_ARG, "page_tokens must be a multiple of 64 in [64, 4096]");
   if (c->max_seqs < 1 || c->max_seqs > (1 << 22)) return fail(KVQ_ERR_INVALID_ARG, "max_seqs out of range");
@@ -85,9 +97,12 @@ struct kvq_cache {
   bool host_only = false;
   int device = 0;
   int num_sms = 148;
-  kvq::Layout L{};
+  kvq::Layout L{};                   // cache-wide fields (pool = start of layer 0)
+  std::vector<kvq::Layout> layers;   // per-layer views: pool = the layer's region, that layer's bits
+  std::vector<int32_t> k_bits, v_bits;
   int64_t pool_bytes = 0;
-  int64_t bytes_per_token_layer = 0;
+  int64_t bytes_per_token = 0;       // all layers, K + V codes and scales
+  int64_t bytes_per_page = 0;        // all layers, all heads
   int32_t* d_page_table = nullptr;
   uint32_t* d_err = nullptr;
   int32_t* d_counters = nullptr;     // decode split-item counters, [KVQ_MAX_BATCH * n_kv_heads]
@@ -281,11 +296,13 @@ kvq_status kvq_footprint_bytes(const kvq_cache_config* cfg, int64_t n_tokens, in
   if (kvq_status s = check_config(cfg)) return s;
   if (n_tokens < 0) return fail(KVQ_ERR_INVALID_ARG, "n_tokens must be >= 0");
   int P = cfg->page_tokens ? cfg->page_tokens : 256;
-  int64_t per = int64_t(cfg->n_kv_heads) *
-                (bytes_per_token_head(cfg->k_bits, cfg->head_dim) + bytes_per_token_head(cfg->v_bits, cfg->head_dim));
+  int64_t per = 0;   // bytes of one token over all layers
+  for (int l = 0; l < cfg->n_layers; ++l)
+    per += int64_t(cfg->n_kv_heads) * (bytes_per_token_head(layer_k_bits(cfg, l), cfg->head_dim) +
+                                       bytes_per_token_head(layer_v_bits(cfg, l), cfg->head_dim));
   int64_t pages = (n_tokens + P - 1) / P;
-  if (allocated) *allocated = int64_t(cfg->n_layers) * pages * P * per;
-  if (used) *used = int64_t(cfg->n_layers) * n_tokens * per;
+  if (allocated) *allocated = pages * P * per;
+  if (used) *used = n_tokens * per;
   return KVQ_OK;
 }
 
@@ -305,24 +322,52 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
   L.n_kv_heads = H;
   L.n_layers = c->cfg.n_layers;
   L.decode_tc = (cfg->flags & KVQ_CACHE_DECODE_TENSOR_CORES) ? 1 : 0;
+  // Device-side fault injection for tests: with KVQ_TEST_WITHHOLD_ARRIVAL=1 in the
+  // environment when the cache is created, the quantized decode kernel's CTA 0
+  // never fills its first stage and every wait of the kernel gives up after
+  // 1 ms instead of 2 s, so the bounded wait runs out, the kernel records
+  // kErrWaitTimeout and returns, and kvq_cache_check reports it.  No wait is
+  // unbounded, so nothing hangs.
+  if (const char* f = std::getenv("KVQ_TEST_WITHHOLD_ARRIVAL"); f && f[0] == '1') {
+    L.test_withhold = 1;
+    L.wait_ns = 1000000ull;
+  } else {
+    L.test_withhold = 0;
+    L.wait_ns = kvq::kWaitLimitNs;
+  }
   L.page_tokens = P;
   L.head_dim = D;
-  L.k_bits = c->cfg.k_bits;
-  L.v_bits = c->cfg.v_bits;
-  L.k_row = kvq::code_row_bytes(L.k_bits, D);
-  L.v_row = kvq::code_row_bytes(L.v_bits, D);
   L.s_row = (D / kvq::QK) * 2;
-  const int ks = L.k_bits == 16 ? 0 : L.s_row, vs = L.v_bits == 16 ? 0 : L.s_row;
-  L.k_scales_off = P * L.k_row;
-  L.v_codes_off = L.k_scales_off + P * ks;
-  L.v_scales_off = L.v_codes_off + P * L.v_row;
-  L.head_block = int64_t(L.v_scales_off) + int64_t(P) * vs;
   L.n_pages = int32_t((c->cfg.max_tokens + P - 1) / P);
   L.max_pages_per_seq = int32_t((c->cfg.max_seq_tokens + P - 1) / P);
-  c->bytes_per_token_layer = int64_t(H) * (L.k_row + ks + L.v_row + vs);
-  c->pool_bytes = int64_t(c->cfg.n_layers) * L.n_pages * H * L.head_block;
 
   try {
+    // per-layer views of the pool: pool[layer] is n_pages * H head blocks of that layer's format
+    // (the per-layer bit widths of the KVSplit page's roadmap, "Configuracao recomendada e roadmap")
+    c->layers.assign(c->cfg.n_layers, L);
+    c->k_bits.resize(c->cfg.n_layers);
+    c->v_bits.resize(c->cfg.n_layers);
+    for (int l = 0; l < c->cfg.n_layers; ++l) {
+      kvq::Layout& V = c->layers[l];
+      c->k_bits[l] = V.k_bits = layer_k_bits(cfg, l);
+      c->v_bits[l] = V.v_bits = layer_v_bits(cfg, l);
+      V.k_row = kvq::code_row_bytes(V.k_bits, D);
+      V.v_row = kvq::code_row_bytes(V.v_bits, D);
+      const int ks = V.k_bits == 16 ? 0 : V.s_row, vs = V.v_bits == 16 ? 0 : V.s_row;
+      V.k_scales_off = P * V.k_row;
+      V.v_codes_off = V.k_scales_off + P * ks;
+      V.v_scales_off = V.v_codes_off + P * V.v_row;
+      V.head_block = int64_t(V.v_scales_off) + int64_t(P) * vs;
+      V.n_layers = 1;
+      c->bytes_per_token += int64_t(H) * (V.k_row + ks + V.v_row + vs);
+      c->bytes_per_page += int64_t(H) * V.head_block;
+    }
+    c->cfg.layer_k_bits = nullptr;   // the caller's arrays are not kept
+    c->cfg.layer_v_bits = nullptr;
+    L.k_bits = c->k_bits[0];
+    L.v_bits = c->v_bits[0];
+    c->pool_bytes = int64_t(L.n_pages) * c->bytes_per_page;
+
     // host-side fault injection for tests: the environment variable
     // KVQ_INJECT_ALLOC_FAILURE=1 makes this allocation fail, through the same
     // cleanup as a real one
@@ -368,6 +413,14 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
     L.page_table = c->d_page_table;
     L.err = c->d_err;
     L.counters = c->d_counters;
+    int64_t base = 0;
+    for (kvq::Layout& V : c->layers) {
+      V.pool = L.pool + base;
+      V.page_table = L.page_table;
+      V.err = L.err;
+      V.counters = L.counters;
+      base += int64_t(L.n_pages) * H * V.head_block;
+    }
   }
   *out = c;
   return KVQ_OK;
@@ -391,12 +444,11 @@ kvq_status kvq_cache_destroy(kvq_cache* c) {
 kvq_status kvq_cache_footprint(const kvq_cache* c, int64_t* pool, int64_t* mapped, int64_t* used) {
   if (kvq_status s = check_cache(c)) return s;
   if (pool) *pool = c->pool_bytes;
-  if (mapped)
-    *mapped = c->mapped_pages * int64_t(c->cfg.n_layers) * c->L.n_kv_heads * c->L.head_block;
+  if (mapped) *mapped = c->mapped_pages * c->bytes_per_page;
   if (used) {
     int64_t t = 0;
     for (int64_t x : c->len) t += x;
-    *used = t * c->bytes_per_token_layer * c->cfg.n_layers;
+    *used = t * c->bytes_per_token;
   }
   return KVQ_OK;
 }
@@ -477,10 +529,11 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
       const int32_t from = c->table[slot], to = take_page(c, &j);
       if (!c->host_only) {
         // the page's head blocks of one layer are contiguous: one copy per layer
-        const int64_t bytes = int64_t(c->L.n_kv_heads) * c->L.head_block;
         for (int32_t layer = 0; layer < c->cfg.n_layers && st == KVQ_OK; ++layer) {
-          const cudaError_t e = cudaMemcpyAsync(c->L.head_ptr(layer, to, 0), c->L.head_ptr(layer, from, 0),
-                                                size_t(bytes), cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
+          const kvq::Layout& V = c->layers[layer];
+          const int64_t bytes = int64_t(V.n_kv_heads) * V.head_block;
+          const cudaError_t e = cudaMemcpyAsync(V.head_ptr(0, to, 0), V.head_ptr(0, from, 0), size_t(bytes),
+                                                cudaMemcpyDeviceToDevice, (cudaStream_t)stream);
           if (e != cudaSuccess) st = cuda_fail(e, "copy of a shared page");
         }
         if (st != KVQ_OK) break;
@@ -599,7 +652,7 @@ kvq_status kvq_append(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids
   if (!k || !v) return fail(KVQ_ERR_INVALID_ARG, "k or v is NULL");
   if (!aligned16(k) || !aligned16(v)) return fail(KVQ_ERR_INVALID_ARG, "k and v must be 16-byte aligned");
   if (kvq_status s = need_device(c)) return s;
-  return launched(kvq::launch_append(c->L, layer, b, int(total), k, v, (cudaStream_t)stream), "append");
+  return launched(kvq::launch_append(c->layers[layer], 0, b, int(total), k, v, (cudaStream_t)stream), "append");
 }
 
 kvq_status kvq_decode_workspace_size(const kvq_cache* c, int32_t n, int32_t n_q_heads, size_t* bytes) {
@@ -642,7 +695,8 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   if (kvq_status s = need_device(c)) return s;
 
   kvq::DecodePlan plan;
-  plan.chunk_tokens = kvq::decode_chunk_tokens(c->L, G);
+  const kvq::Layout& LV = c->layers[layer];
+  plan.chunk_tokens = kvq::decode_chunk_tokens(LV, G);
   const int C = plan.chunk_tokens, H = c->L.n_kv_heads;
   kvq::Batch b;
   b.n = n;
@@ -663,15 +717,15 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   if (flat >= (int64_t(1) << 31)) return fail(KVQ_ERR_INVALID_ARG, "batch too large");
   const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(c->L.head_dim));
   const float scale_log2 = sigma * 1.4426950408889634f;
-  const bool fused = appending && kvq::decode_fuses_append(c->L, G);
+  const bool fused = appending && kvq::decode_fuses_append(LV, G);
   if (appending && !fused) {
     kvq::Batch ab;
     ab.n = n;
     for (int i = 0; i < n; ++i) ab.s[i] = {ids[i], int32_t(c->len[ids[i]] - 1), 1, i};
-    if (kvq_status s = launched(kvq::launch_append(c->L, layer, ab, n, k_new, v_new, (cudaStream_t)stream), "append"))
+    if (kvq_status s = launched(kvq::launch_append(LV, 0, ab, n, k_new, v_new, (cudaStream_t)stream), "append"))
       return s;
   }
-  return launched(kvq::launch_decode(c->L, layer, b, plan, n_q_heads, q, out, fused ? k_new : nullptr,
+  return launched(kvq::launch_decode(LV, 0, b, plan, n_q_heads, q, out, fused ? k_new : nullptr,
                                      fused ? v_new : nullptr, scale_log2, ws, (cudaStream_t)stream),
                   "decode");
 }
@@ -742,7 +796,7 @@ kvq_status kvq_prefill_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_
     return fail(KVQ_ERR_WORKSPACE, "prefill needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
   if (kvq_status s = need_device(c)) return s;
   const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(c->L.head_dim));
-  return launched(kvq::launch_prefill(c->L, layer, b, int(total), n_q_heads, q, out, sigma, ws, ws_bytes,
+  return launched(kvq::launch_prefill(c->layers[layer], 0, b, int(total), n_q_heads, q, out, sigma, ws, ws_bytes,
                                       c->num_sms, (cudaStream_t)stream),
                   "prefill");
 }
@@ -755,7 +809,7 @@ kvq_status kvq_export(const kvq_cache* c, int32_t layer, int32_t id, int64_t tok
   if (tok0 < 0 || n_tok < 0 || tok0 + n_tok > c->len[id]) return fail(KVQ_ERR_INVALID_ARG, "token range outside the sequence");
   if (n_tok == 0) return KVQ_OK;
   if (kvq_status s = need_device(c)) return s;
-  return launched(kvq::launch_export(c->L, layer, id, tok0, n_tok, kc, ks, vc, vs, (cudaStream_t)stream), "export");
+  return launched(kvq::launch_export(c->layers[layer], 0, id, tok0, n_tok, kc, ks, vc, vs, (cudaStream_t)stream), "export");
 }
 
 kvq_status kvq_cache_check(kvq_cache* c, kvq_stream_t stream, uint32_t* detail) {

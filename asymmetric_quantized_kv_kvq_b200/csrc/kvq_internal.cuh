@@ -49,6 +49,8 @@ struct Layout {
   int32_t k_scales_off, v_codes_off, v_scales_off;   // byte offsets inside a head block
   int32_t decode_tc;                   // KVQ_CACHE_DECODE_TENSOR_CORES was set
   int32_t* counters;                   // [kMaxBatch * n_kv_heads] split-item counters of the decode kernel (zero at rest)
+  uint64_t wait_ns;                    // limit of every bounded wait of the decode kernel
+  int32_t test_withhold;               // test hook: the decode kernel withholds one stage's arrival
 
   __host__ __device__ __forceinline__ uint8_t* head_ptr(int layer, int page, int head) const {
     return pool + ((int64_t(layer) * n_pages + page) * n_kv_heads + head) * head_block;

@@ -36,7 +36,8 @@ class CacheConfig(ctypes.Structure):
         ("n_layers", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
         ("k_bits", ctypes.c_int32), ("v_bits", ctypes.c_int32), ("page_tokens", ctypes.c_int32),
         ("max_seqs", ctypes.c_int32), ("flags", ctypes.c_int32), ("max_tokens", ctypes.c_int64),
-        ("max_seq_tokens", ctypes.c_int64),
+        ("max_seq_tokens", ctypes.c_int64), ("layer_k_bits", ctypes.POINTER(ctypes.c_int32)),
+        ("layer_v_bits", ctypes.POINTER(ctypes.c_int32)),
     ]
 
 
@@ -119,15 +120,26 @@ def _dev_fp16(t, name: str, shape: Optional[tuple] = None):
 
 
 def make_config(n_layers, n_kv_heads, head_dim, k_bits, v_bits, max_seqs, max_tokens,
-                page_tokens=256, max_seq_tokens=0, host_only=False, decode_tc=False) -> CacheConfig:
+                page_tokens=256, max_seq_tokens=0, host_only=False, decode_tc=False,
+                layer_bits: Optional[Sequence[tuple]] = None) -> CacheConfig:
+    """layer_bits: optional [(k_bits, v_bits)] per layer, replacing k_bits / v_bits layer by layer."""
     flags = (KVQ_CACHE_HOST_ONLY if host_only else 0) | (KVQ_CACHE_DECODE_TENSOR_CORES if decode_tc else 0)
-    return CacheConfig(n_layers, n_kv_heads, head_dim, k_bits, v_bits, page_tokens, max_seqs,
-                       flags, max_tokens, max_seq_tokens)
+    cfg = CacheConfig(n_layers, n_kv_heads, head_dim, k_bits, v_bits, page_tokens, max_seqs,
+                      flags, max_tokens, max_seq_tokens, None, None)
+    if layer_bits is not None:
+        if len(layer_bits) != n_layers:
+            raise KvqError(1, f"layer_bits has {len(layer_bits)} entries for {n_layers} layers")
+        cfg._lk = _i32_array([kb for kb, _ in layer_bits])      # kept alive with the config
+        cfg._lv = _i32_array([vb for _, vb in layer_bits])
+        cfg.layer_k_bits = ctypes.cast(cfg._lk, ctypes.POINTER(ctypes.c_int32))
+        cfg.layer_v_bits = ctypes.cast(cfg._lv, ctypes.POINTER(ctypes.c_int32))
+    return cfg
 
 
-def footprint_bytes(n_layers, n_kv_heads, head_dim, k_bits, v_bits, n_tokens, page_tokens=256):
+def footprint_bytes(n_layers, n_kv_heads, head_dim, k_bits, v_bits, n_tokens, page_tokens=256, layer_bits=None):
     """(allocated, used) bytes of one sequence of n_tokens (library closed form)."""
-    cfg = make_config(n_layers, n_kv_heads, head_dim, k_bits, v_bits, 1, max(1, n_tokens), page_tokens)
+    cfg = make_config(n_layers, n_kv_heads, head_dim, k_bits, v_bits, 1, max(1, n_tokens), page_tokens,
+                      layer_bits=layer_bits)
     a, u = ctypes.c_int64(), ctypes.c_int64()
     _check(load_library().kvq_footprint_bytes(ctypes.byref(cfg), n_tokens, ctypes.byref(a), ctypes.byref(u)))
     return a.value, u.value
@@ -138,12 +150,15 @@ class Cache:
 
     def __init__(self, n_layers: int, n_kv_heads: int, head_dim: int, k_bits: int, v_bits: int,
                  max_seqs: int, max_tokens: int, page_tokens: int = 256, max_seq_tokens: int = 0,
-                 host_only: bool = False, decode_tc: bool = False):
+                 host_only: bool = False, decode_tc: bool = False, layer_bits: Optional[Sequence[tuple]] = None):
+        """layer_bits: optional [(k_bits, v_bits)] per layer (per-layer precision); k_bits / v_bits
+        then only name the default."""
         self._lib = load_library()
         self.cfg = make_config(n_layers, n_kv_heads, head_dim, k_bits, v_bits, max_seqs, max_tokens,
-                               page_tokens, max_seq_tokens, host_only, decode_tc)
+                               page_tokens, max_seq_tokens, host_only, decode_tc, layer_bits)
         self.n_layers, self.n_kv_heads, self.head_dim = n_layers, n_kv_heads, head_dim
         self.k_bits, self.v_bits = k_bits, v_bits
+        self.layer_bits = [tuple(x) for x in layer_bits] if layer_bits is not None else [(k_bits, v_bits)] * n_layers
         self.host_only = host_only
         h = ctypes.c_void_p()
         _check(self._lib.kvq_cache_create(ctypes.byref(self.cfg), ctypes.byref(h)))
@@ -316,9 +331,10 @@ class Cache:
                 return torch.empty((n_tok, H, D), dtype=torch.int8, device=device)
             return torch.empty((n_tok, H, D // 2), dtype=torch.uint8, device=device)
 
-        kc, vc = codes(self.k_bits), codes(self.v_bits)
-        ks = torch.empty((n_tok, H, D // 32), dtype=torch.float16, device=device) if self.k_bits != 16 else None
-        vs = torch.empty((n_tok, H, D // 32), dtype=torch.float16, device=device) if self.v_bits != 16 else None
+        kb, vb = self.layer_bits[layer]
+        kc, vc = codes(kb), codes(vb)
+        ks = torch.empty((n_tok, H, D // 32), dtype=torch.float16, device=device) if kb != 16 else None
+        vs = torch.empty((n_tok, H, D // 32), dtype=torch.float16, device=device) if vb != 16 else None
         ptr = lambda t: None if t is None else t.data_ptr()
         _check(self._lib.kvq_export(self._h, layer, seq_id, tok0, n_tok, ptr(kc), ptr(ks), ptr(vc), ptr(vs),
                                     _stream(stream)))

@@ -81,7 +81,13 @@ typedef enum {
  * page_tokens a multiple of 64 in [64, 4096] (0 selects 256); sequences are
  * named by ids 0 .. max_seqs-1; max_tokens is the pool capacity in tokens over
  * all sequences (rounded up to whole pages); max_seq_tokens (0 = max_tokens)
- * bounds one sequence's length and sizes its page-table row. */
+ * bounds one sequence's length and sizes its page-table row.
+ * Per-layer precision (the "Layer-Specific Quantization" item of the KVSplit
+ * page's "Configuracao recomendada e roadmap"): layer_k_bits / layer_v_bits,
+ * when not NULL, are host arrays of n_layers bit widths that replace k_bits /
+ * v_bits layer by layer (both or neither; read by kvq_cache_create and
+ * kvq_footprint_bytes only, not kept).  Each layer is either fp16 for K and V
+ * or quantized for both. */
 typedef struct {
   int32_t n_layers;
   int32_t n_kv_heads;
@@ -93,6 +99,8 @@ typedef struct {
   int32_t flags;            /* KVQ_CACHE_* bits */
   int64_t max_tokens;
   int64_t max_seq_tokens;
+  const int32_t* layer_k_bits;   /* NULL or [n_layers] */
+  const int32_t* layer_v_bits;   /* NULL or [n_layers] */
 } kvq_cache_config;
 
 /* flags: KVQ_CACHE_HOST_ONLY creates the page bookkeeping without touching a

@@ -42,10 +42,11 @@ import math
 import numpy as np
 
 __all__ = [
-    "QK", "MIB", "block_bytes", "kv_bytes_per_token_layer", "footprint_bytes", "used_bytes",
+    "QK", "MIB", "block_bytes", "kv_bytes_per_token_layer", "footprint_bytes", "footprint_bytes_layers",
+    "used_bytes",
     "q8_scale", "q4_scale", "round_half_away", "quantize_q8", "quantize_q4",
     "dequantize_q8", "dequantize_q4", "unpack_q4", "quantize_kv", "dequantize_kv",
-    "attention_decode", "attention_prefill", "attention_decode_batch", "lse_merge",
+    "attention_decode", "attention_decode_window", "attention_prefill", "attention_decode_batch", "lse_merge",
 ]
 
 QK = 32            # elements per quantisation block
@@ -91,6 +92,16 @@ def footprint_bytes(n_layers, n_kv_heads, head_dim, k_bits, v_bits, n_tokens,
     """
     pages = -(-n_tokens // page_tokens)
     return used_bytes(n_layers, n_kv_heads, head_dim, k_bits, v_bits, pages * page_tokens)
+
+
+def footprint_bytes_layers(n_kv_heads, head_dim, layer_bits, n_tokens, page_tokens: int = 256) -> int:
+    """Allocated bytes of a cache whose layers have their own (k_bits, v_bits)
+    ([KVSplit] "Configuracao recomendada e roadmap": layer-specific quantisation,
+    different precisions per layer).  Every layer holds the same tokens in whole
+    pages, so the footprint is the sum of the single-layer footprints.
+    Pinned by the printed table: a 22-layer cache half K8V4, half K4V4 holds
+    (71.50 + 49.50) / 2 MB at 8192 tokens."""
+    return sum(footprint_bytes(1, n_kv_heads, head_dim, kb, vb, n_tokens, page_tokens) for kb, vb in layer_bits)
 
 
 # ---------------------------------------------------------------------------
@@ -233,6 +244,22 @@ def attention_decode(q, k_hat, v_hat, scale=None) -> np.ndarray:
         p = np.exp(s - s.max())
         out[h] = (p @ v_hat[:, g, :]) / p.sum()
     return out
+
+
+def attention_decode_window(q, k_hat, v_hat, window: int, scale=None) -> np.ndarray:
+    """Decode over a rotating cache of `window` tokens ([Reuse] "O Que Nao Funcionou":
+    rotating the KV cache at 8192 tokens keeps only the most recent tokens, which
+    gave the best tokens/s but lost the earlier context): the query at position
+    T-1 sees only tokens max(0, T - window) .. T-1.  window = 0 means no window.
+    Pinned by: window >= T gives attention_decode; window 1 gives the last
+    token's value; brute force over the kept tokens on tiny inputs."""
+    k_hat = np.asarray(k_hat, dtype=np.float64)
+    v_hat = np.asarray(v_hat, dtype=np.float64)
+    T = k_hat.shape[0]
+    if window < 0:
+        raise ValueError("window must be >= 0")
+    lo = max(0, T - window) if window else 0
+    return attention_decode(q, k_hat[lo:], v_hat[lo:], scale)
 
 
 def attention_decode_batch(q, caches, scale=None) -> np.ndarray:

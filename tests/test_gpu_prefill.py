@@ -40,10 +40,11 @@ def _run(m, kb, vb, D, H, G, cached, chunk, seed=0, page_tokens=256):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("kb,vb", [(8, 4), (16, 16), (8, 8), (4, 4)])
-def test_prefill_matches_oracle_ragged(kb, vb):
+@pytest.mark.parametrize("kb,vb", [(8, 4), (16, 16), (8, 8), (4, 4), (4, 8)])
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_matches_oracle_ragged(kb, vb, D):
     m = kvq()
-    _run(m, kb, vb, D=128, H=2, G=4, cached=[0, 100, 300, 129], chunk=[64, 200, 129, 1])
+    _run(m, kb, vb, D=D, H=2, G=4, cached=[0, 100, 300, 129], chunk=[64, 200, 129, 1])
 
 
 @pytest.mark.gpu

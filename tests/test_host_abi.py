@@ -8,7 +8,7 @@ import re
 import pytest
 
 from asymmetric_quantized_kv_kvq_b200 import build as kbuild
-from oracle import footprint_bytes as oracle_footprint
+from oracle import footprint_bytes as oracle_footprint, footprint_bytes_layers
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -325,3 +325,30 @@ def test_fork_is_all_or_nothing_when_a_page_table_enqueue_fails(kvq, monkeypatch
     c.release(0)
     assert c.footprint()[1] == 0                        # no page kept alive by a leaked reference
     c.close()
+
+
+@pytest.mark.parametrize("tokens", [1, 255, 256, 8192, 100000])
+def test_per_layer_precision_footprint_matches_oracle(kvq, tokens):
+    bits = [(8, 4), (4, 8), (16, 16), (8, 8), (4, 4), (8, 4)]
+    alloc, used = kvq.footprint_bytes(6, 4, 64, 8, 4, tokens, layer_bits=bits)
+    assert alloc == footprint_bytes_layers(4, 64, bits, tokens)
+    c = kvq.Cache(6, 4, 64, 8, 4, max_seqs=2, max_tokens=tokens + 512, host_only=True, layer_bits=bits)
+    c.extend([0], [tokens])
+    pool, mapped, used_c = c.footprint()
+    assert mapped == alloc and used_c == used
+    c.close()
+
+
+def test_per_layer_precision_validation(kvq):
+    lib = kvq.load_library()
+    cfg = kvq.make_config(3, 2, 64, 8, 4, 2, 1024, host_only=True, layer_bits=[(8, 4), (16, 8), (4, 4)])
+    h = ctypes.c_void_p()
+    assert lib.kvq_cache_create(ctypes.byref(cfg), ctypes.byref(h)) == 2      # K16V8 not built
+    assert b"layer 1" in lib.kvq_last_error()
+    cfg = kvq.make_config(3, 2, 64, 8, 4, 2, 1024, host_only=True, layer_bits=[(8, 4), (8, 3), (4, 4)])
+    assert lib.kvq_cache_create(ctypes.byref(cfg), ctypes.byref(h)) == 1
+    cfg = kvq.make_config(3, 2, 64, 8, 4, 2, 1024, host_only=True)
+    cfg.layer_k_bits = (ctypes.c_int32 * 3)(8, 8, 8)                           # one array without the other
+    assert lib.kvq_cache_create(ctypes.byref(cfg), ctypes.byref(h)) == 1
+    with pytest.raises(kvq.KvqError):
+        kvq.make_config(3, 2, 64, 8, 4, 2, 1024, layer_bits=[(8, 4)])

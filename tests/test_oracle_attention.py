@@ -6,8 +6,8 @@ import math
 import numpy as np
 import pytest
 
-from oracle import (attention_decode, attention_prefill, attention_decode_batch, lse_merge,
-                    quantize_kv, dequantize_kv)
+from oracle import (attention_decode, attention_decode_window, attention_prefill, attention_decode_batch,
+                    lse_merge, quantize_kv, dequantize_kv)
 
 
 def _brute(q, k, v, scale):
@@ -212,3 +212,39 @@ def test_prefill_score_split_keeps_attention_within_tolerance():
     used_fp16 = (np.abs(fp16_only - ref) / bound).max()
     assert used_split < 0.5, used_split
     assert used_fp16 > 2 * used_split, (used_fp16, used_split)
+
+
+@pytest.mark.parametrize("T,window", [(6, 2), (6, 3), (5, 5), (9, 4)])
+def test_window_decode_matches_brute_force_over_the_last_tokens(T, window):
+    """Brute force over the kept tokens: positions T - window .. T-1 only."""
+    rng = np.random.default_rng(T * 10 + window)
+    Hq, Hkv, D = 4, 2, 32
+    q = rng.standard_normal((Hq, D))
+    k = rng.standard_normal((T, Hkv, D)) * 2
+    v = rng.standard_normal((T, Hkv, D))
+    got = attention_decode_window(q, k, v, window)
+    for h in range(Hq):
+        g = h // 2
+        want = _brute(q[h].tolist(), k[T - window:, g].tolist(), v[T - window:, g].tolist(), 1 / math.sqrt(D))
+        assert np.allclose(got[h], want, rtol=1e-12, atol=1e-13)
+
+
+def test_window_special_cases():
+    rng = np.random.default_rng(5)
+    T, Hq, Hkv, D = 7, 4, 2, 32
+    q = rng.standard_normal((Hq, D))
+    k = rng.standard_normal((T, Hkv, D))
+    v = rng.standard_normal((T, Hkv, D))
+    # a window at least as long as the sequence (or no window) is plain decode
+    for w in (0, T, T + 5):
+        assert np.array_equal(attention_decode_window(q, k, v, w), attention_decode(q, k, v))
+    # a one-token window returns the last token's value exactly
+    one = attention_decode_window(q, k, v, 1)
+    assert np.array_equal(one, np.repeat(v[-1], Hq // Hkv, axis=0))
+    # a dominant key just outside the window has no effect; inside, it takes over
+    k2 = k.copy()
+    k2[T - 4] = 50 * q[0][None, :] / np.linalg.norm(q[0])
+    assert np.allclose(attention_decode_window(q, k2, v, 3), attention_decode_window(q, k, v, 3), rtol=0, atol=0)
+    assert not np.allclose(attention_decode_window(q, k2, v, 4)[0], attention_decode_window(q, k, v, 4)[0])
+    with pytest.raises(ValueError):
+        attention_decode_window(q, k, v, -1)

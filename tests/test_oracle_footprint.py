@@ -3,7 +3,7 @@ import os
 
 import pytest
 
-from oracle import footprint_bytes, used_bytes, kv_bytes_per_token_layer, block_bytes, MIB
+from oracle import footprint_bytes, footprint_bytes_layers, used_bytes, kv_bytes_per_token_layer, block_bytes, MIB
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 BITS = {"FP16": (16, 16), "K8V8": (8, 8), "K8V4": (8, 4), "K4V8": (4, 8), "K4V4": (4, 4)}
@@ -69,3 +69,33 @@ def test_printed_reductions():
             assert int(fp16 / q * 10) / 10 == float(val)
         else:
             assert round(100 * (1 - q / fp16)) == int(val)
+
+
+def _table_mib(cfg, tokens):
+    for c, t, mib in _rows("kvsplit_memory_table.txt"):
+        if c == cfg and int(t) == tokens:
+            return float(mib)
+    raise KeyError((cfg, tokens))
+
+
+@pytest.mark.parametrize("mix", [("K8V4", "K4V4"), ("K8V8", "FP16"), ("K8V4", "K4V8")])
+@pytest.mark.parametrize("tokens", [8192, 4096])
+def test_per_layer_footprint_is_the_layer_share_of_the_printed_rows(mix, tokens):
+    """A 22-layer cache with 11 layers of each format holds half of each printed row (exact at whole
+    pages): per-layer precision changes bytes layer by layer and nothing else."""
+    try:
+        want = (_table_mib(mix[0], tokens) + _table_mib(mix[1], tokens)) / 2
+    except KeyError:
+        pytest.skip("row not printed at this length")
+    bits = [BITS[mix[0]]] * 11 + [BITS[mix[1]]] * 11
+    got = footprint_bytes_layers(SHAPE["n_kv_heads"], SHAPE["head_dim"], bits, tokens)
+    assert got == want * MIB
+    # the order of the layers does not matter
+    assert footprint_bytes_layers(SHAPE["n_kv_heads"], SHAPE["head_dim"], bits[::-1], tokens) == got
+
+
+def test_per_layer_footprint_of_uniform_layers_is_the_uniform_closed_form():
+    for cfg, kbvb in BITS.items():
+        for tokens in (1, 128, 257, 8192):
+            assert footprint_bytes_layers(4, 64, [kbvb] * 22, tokens) == footprint_bytes(k_bits=kbvb[0], v_bits=kbvb[1],
+                                                                                         n_tokens=tokens, **SHAPE)
