@@ -62,7 +62,7 @@ __global__ void __launch_bounds__(256) append_kernel(const Layout L, int layer, 
   }
   const SeqDesc sd = b.s[lo];
   const int pos = sd.a + (row - sd.c);
-  const int page = L.page_table[int64_t(sd.seq_id) * L.max_pages_per_seq + pos / L.page_tokens];
+  const int page = L.page_table[int64_t(sd.seq_id) * L.max_pages_per_seq + page_slot(pos / L.page_tokens, sd.ring)];
   if (page < 0 || page >= L.n_pages) {
     record_error(L.err, kErrBadPage);
     return;
@@ -86,8 +86,8 @@ __global__ void __launch_bounds__(256) append_kernel(const Layout L, int layer, 
 
 // Canonical export: one warp per (token, head) copies that row's code and
 // scale bytes to [n_tok, Hkv, row] destinations.
-__global__ void export_kernel(const Layout L, int layer, int seq_id, int64_t tok0, int64_t n_tok, uint8_t* kc,
-                              uint8_t* ks, uint8_t* vc, uint8_t* vs) {
+__global__ void export_kernel(const Layout L, int layer, int seq_id, int ring, int64_t tok0, int64_t n_tok,
+                              uint8_t* kc, uint8_t* ks, uint8_t* vc, uint8_t* vs) {
   const int lane = threadIdx.x & 31;
   const int64_t w = int64_t(blockIdx.x) * (blockDim.x / 32) + (threadIdx.x >> 5);
   const int H = L.n_kv_heads;
@@ -95,7 +95,7 @@ __global__ void export_kernel(const Layout L, int layer, int seq_id, int64_t tok
   const int64_t t = w / H;
   const int h = int(w % H);
   const int64_t pos = tok0 + t;
-  const int page = L.page_table[int64_t(seq_id) * L.max_pages_per_seq + pos / L.page_tokens];
+  const int page = L.page_table[int64_t(seq_id) * L.max_pages_per_seq + page_slot(int(pos / L.page_tokens), ring)];
   if (page < 0 || page >= L.n_pages) {
     if (lane == 0) record_error(L.err, kErrBadPage);
     return;
@@ -134,10 +134,10 @@ cudaError_t launch_append(const Layout& L, int layer, const Batch& b, int total_
   return cudaGetLastError();
 }
 
-cudaError_t launch_export(const Layout& L, int layer, int seq_id, int64_t tok0, int64_t n_tok, void* kc, void* ks,
-                          void* vc, void* vs, cudaStream_t s) {
+cudaError_t launch_export(const Layout& L, int layer, int seq_id, int ring, int64_t tok0, int64_t n_tok, void* kc,
+                          void* ks, void* vc, void* vs, cudaStream_t s) {
   const int64_t warps = n_tok * L.n_kv_heads;
-  export_kernel<<<unsigned((warps + 7) / 8), 256, 0, s>>>(L, layer, seq_id, tok0, n_tok, static_cast<uint8_t*>(kc),
+  export_kernel<<<unsigned((warps + 7) / 8), 256, 0, s>>>(L, layer, seq_id, ring, tok0, n_tok, static_cast<uint8_t*>(kc),
                                                           static_cast<uint8_t*>(ks), static_cast<uint8_t*>(vc),
                                                           static_cast<uint8_t*>(vs));
   return cudaGetLastError();

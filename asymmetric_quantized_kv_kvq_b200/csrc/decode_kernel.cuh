@@ -256,10 +256,11 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
           ok = false;
           break;
         }
-        const int tok0 = k * a.chunk;
+        const int tok0 = sd.lo / a.chunk * a.chunk + k * a.chunk;   // chunks start at the window's first chunk
         const int ntok = min(a.chunk, sd.a - tok0);
         const int ncopy = min(a.chunk, (ntok + 15) & ~15);
-        const int page = a.L.page_table[int64_t(sd.seq_id) * a.L.max_pages_per_seq + tok0 / a.L.page_tokens];
+        const int page =
+            a.L.page_table[int64_t(sd.seq_id) * a.L.max_pages_per_seq + page_slot(tok0 / a.L.page_tokens, sd.ring)];
         if (page < 0 || page >= a.L.n_pages) {
           record_error(a.L.err, kErrBadPage);
           *abort_flag = 1;
@@ -366,9 +367,13 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         return;
       }
       ++it;
-      const int nvalid = min(a.chunk, sd.a - k * a.chunk);
-      const int nv_w = min(W, max(0, nvalid - tw * W));
-      if (nv_w > 0) {
+      // valid rows of the stage: [rv0, rv1) (rv0 > 0 only in the first chunk of a rotating window);
+      // of this warp's W rows: [lo_w, nv_w)
+      const int tok0 = sd.lo / a.chunk * a.chunk + k * a.chunk;
+      const int rv0 = max(0, sd.lo - tok0), rv1 = min(a.chunk, sd.a - tok0);
+      const int nv_w = min(W, max(0, rv1 - tw * W));
+      const int lo_w = max(0, rv0 - tw * W);
+      if (nv_w > lo_w) {
         const uint8_t* st = stages + s * T::STAGE_BYTES;
         const int row0 = tw * W;
         // ---- scores
@@ -409,7 +414,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
           }
           reduce_scatter<GW, T::LPT>(part, lane);
 #pragma unroll
-          for (int gi = 0; gi < T::GPL; ++gi) sc[j][gi] = t < nv_w ? part[gi] : -INFINITY;
+          for (int gi = 0; gi < T::GPL; ++gi) sc[j][gi] = (t >= lo_w && t < nv_w) ? part[gi] : -INFINITY;
         }
         // ---- online softmax, max moved lazily: a vote decides whether any score
         //      exceeds the running max by more than 2^8; only then is the exact
@@ -481,7 +486,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
 #pragma unroll 4
         for (int j2 = 0; j2 < T::NPV; ++j2) {
           const int t = j2 * T::TPV + tslot;
-          if (t < nv_w) {
+          if (t >= lo_w && t < nv_w) {
             float2 vf[4];
             load_v8<VB>(st + T::OFF_VC + (row0 + t) * T::V_ROW, vsl, vf);
             const float2* pp = pw + pgroup<T::NBP>(t, v_block<VB>(vsl)) * GW;

@@ -161,6 +161,14 @@ __device__ __forceinline__ void reduce_scatter_perm(float (&v)[GW]) {
   }
 }
 
+// 2^x on the SFU (ex2.approx.ftz: results below 2^-126 flush to 0, which a
+// softmax weight that small never notices; 2^-inf = 0).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // ---- stored codes -------------------------------------------------------------
 // Score lane's key code words of one 32-element block, digit-word order w = 0..7
 // (element 4w + e of the block for 8-bit codes; for 4-bit codes words 0..3 are
@@ -375,10 +383,11 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
         ok = false;
         break;
       }
-      const int tok0 = k * a.chunk;
+      const int tok0 = sd.lo / a.chunk * a.chunk + k * a.chunk;   // chunks start at the window's first chunk
       const int ntok = min(a.chunk, sd.a - tok0);
       const int ncopy = min(a.chunk, (ntok + 15) & ~15);
-      const int page = a.L.page_table[int64_t(sd.seq_id) * a.L.max_pages_per_seq + tok0 / a.L.page_tokens];
+      const int page =
+          a.L.page_table[int64_t(sd.seq_id) * a.L.max_pages_per_seq + page_slot(tok0 / a.L.page_tokens, sd.ring)];
       if (page < 0 || page >= a.L.n_pages) {
         if (lane == 0) record_error(a.L.err, kErrBadPage);
         *sm.abort_flag = 1;
@@ -517,9 +526,10 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
         return;
       }
       const uint8_t* st = sm.stages + s * T::STAGE;
-      const int nvalid = min(a.chunk, sd.a - k * a.chunk);
+      const int tok0 = sd.lo / a.chunk * a.chunk + k * a.chunk;
+      const int rv0 = max(0, sd.lo - tok0), rv1 = min(a.chunk, sd.a - tok0);   // valid rows [rv0, rv1)
       const int row0 = part * W;
-      const bool masked = nvalid < row0 + W;
+      const bool masked = rv0 > row0 || rv1 < row0 + W;
       float sc[T::NPASS][NF];
 #pragma unroll
       for (int ps = 0; ps < T::NPASS; ++ps) {
@@ -547,7 +557,7 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
         for (int j = 0; j < NF; ++j) {
           const float v = ps_[j] * qsc[j];
-          sc[ps][j] = (!masked || row < nvalid) ? v : -INFINITY;
+          sc[ps][j] = (!masked || (row >= rv0 && row < rv1)) ? v : -INFINITY;
         }
       }
       // lazy maximum: moved only when a score passes it by 2^8
@@ -573,7 +583,7 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
           for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
           const float mn = fmaxf(m_own[j], mx);
-          alpha[j] = exp2f(m_own[j] - mn);               // 0 while m_own is -inf
+          alpha[j] = fast_exp2(m_own[j] - mn);           // 0 while m_own is -inf
           m_own[j] = mn;
           l_own[j] *= alpha[j];
         }
@@ -588,11 +598,11 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
       for (int ps = 0; ps < T::NPASS; ++ps) {
         const int t = ps * T::TPP + tl;
-        const bool valid = !masked || row0 + t < nvalid;
+        const bool valid = !masked || (row0 + t >= rv0 && row0 + t < rv1);
         float p[NF];
 #pragma unroll
         for (int j = 0; j < NF; ++j) {
-          const float e2 = exp2f(sc[ps][j] - m_own[j]);
+          const float e2 = fast_exp2(sc[ps][j] - m_own[j]);
           p[j] = valid ? e2 : 0.f;
           l_own[j] += p[j];
         }

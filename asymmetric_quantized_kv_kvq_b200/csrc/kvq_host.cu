@@ -2,6 +2,7 @@
 // page allocator, page-table maintenance and kernel dispatch.  Every check
 // runs before anything is enqueued; a failed check leaves the cache unchanged.
 #include <algorithm>
+#include <array>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -106,11 +107,13 @@ struct kvq_cache {
   int32_t* d_page_table = nullptr;
   uint32_t* d_err = nullptr;
   int32_t* d_counters = nullptr;     // decode split-item counters, [KVQ_MAX_BATCH * n_kv_heads]
+  uint32_t* d_dedup = nullptr;       // page hashes [kDedupBatch][4] + compare flags [kDedupBatch]
   std::vector<int32_t> table;        // host mirror of the page table
   std::vector<int64_t> len;          // tokens per sequence
   std::vector<int32_t> mapped;       // pages mapped per sequence
   std::vector<int32_t> free_pages;   // stack; back() is handed out next
   std::vector<int32_t> refs;         // sequences mapping each physical page (0 = free)
+  std::vector<int64_t> window;       // rotating-window length per sequence (0 = keep every token)
   int64_t mapped_pages = 0;          // physical pages in use (each counted once)
 };
 
@@ -141,6 +144,34 @@ kvq_status check_ids(const kvq_cache* c, int32_t n, const int32_t* ids) {
 kvq_status check_layer(const kvq_cache* c, int32_t layer) {
   if (layer < 0 || layer >= c->cfg.n_layers) return fail(KVQ_ERR_INVALID_ARG, "layer %d out of range", layer);
   return KVQ_OK;
+}
+
+// Rotating window: a sequence with a window of W tokens keeps its pages in a ring
+// of W / page_tokens + 1 page-table slots (logical page p in slot p % ring), which
+// always holds the last W positions; 0 for a linear page table.
+int32_t ring_pages(const kvq_cache* c, int32_t id) {
+  return c->window[id] ? int32_t(c->window[id] / c->L.page_tokens + 1) : 0;
+}
+size_t slot_index(const kvq_cache* c, int32_t id, int64_t page) {
+  return size_t(id) * c->L.max_pages_per_seq + size_t(kvq::page_slot(int(page), ring_pages(c, id)));
+}
+// Slots a sequence of nl positions maps.
+int32_t slots_for(const kvq_cache* c, int32_t id, int64_t nl) {
+  const int P = c->L.page_tokens;
+  const int64_t pages = (nl + P - 1) / P;
+  const int32_t R = ring_pages(c, id);
+  return int32_t(R && pages > R ? R : pages);
+}
+// First position attended by a query at the sequence's end.
+int64_t first_attended(const kvq_cache* c, int32_t id) {
+  const int64_t w = c->window[id], n = c->len[id];
+  return w && n > w ? n - w : 0;
+}
+// True once a windowed sequence has reused a ring slot (its logical pages no longer equal its slots).
+bool wrapped(const kvq_cache* c, int32_t id) {
+  const int32_t R = ring_pages(c, id);
+  const int P = c->L.page_tokens;
+  return R && (c->len[id] + P - 1) / P > R;
 }
 
 // Host-side fault injection for tests: with KVQ_INJECT_PT_FAILURE=k (k >= 1) in
@@ -377,6 +408,7 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
     c->mapped.assign(c->cfg.max_seqs, 0);
     c->free_pages.resize(L.n_pages);
     c->refs.assign(L.n_pages, 0);
+    c->window.assign(c->cfg.max_seqs, 0);
   } catch (...) {
     delete c;
     return fail(KVQ_ERR_OUT_OF_MEMORY, "host bookkeeping allocation failed");
@@ -395,6 +427,7 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
       if (c->d_page_table) cudaFree(c->d_page_table);
       if (c->d_err) cudaFree(c->d_err);
       if (c->d_counters) cudaFree(c->d_counters);
+      if (c->d_dedup) cudaFree(c->d_dedup);
       delete c;
       return cuda_fail(err, what);
     };
@@ -409,6 +442,8 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
     if ((e = cudaMemset(c->d_err, 0, sizeof(uint32_t))) != cudaSuccess) return cleanup(e, "cudaMemset(err)");
     if ((e = cudaMalloc(&c->d_counters, counter_bytes)) != cudaSuccess) return cleanup(e, "cudaMalloc(counters)");
     if ((e = cudaMemset(c->d_counters, 0, counter_bytes)) != cudaSuccess) return cleanup(e, "cudaMemset(counters)");
+    if ((e = cudaMalloc(&c->d_dedup, size_t(kvq::kDedupBatch) * 5 * sizeof(uint32_t))) != cudaSuccess)
+      return cleanup(e, "cudaMalloc(dedup)");
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cleanup(e, "cudaDeviceSynchronize");
     L.page_table = c->d_page_table;
     L.err = c->d_err;
@@ -436,6 +471,7 @@ kvq_status kvq_cache_destroy(kvq_cache* c) {
     cudaFree(c->d_page_table);
     cudaFree(c->d_err);
     cudaFree(c->d_counters);
+    cudaFree(c->d_dedup);
   }
   delete c;
   return st;
@@ -450,6 +486,20 @@ kvq_status kvq_cache_footprint(const kvq_cache* c, int64_t* pool, int64_t* mappe
     for (int64_t x : c->len) t += x;
     *used = t * c->bytes_per_token;
   }
+  return KVQ_OK;
+}
+
+kvq_status kvq_seq_set_window(kvq_cache* c, int32_t id, int64_t window_tokens) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_seq(c, id)) return s;
+  if (c->len[id] != 0 || c->mapped[id] != 0) return fail(KVQ_ERR_INVALID_ARG, "sequence %d is not empty", id);
+  const int P = c->L.page_tokens;
+  if (window_tokens < 0 || window_tokens % P)
+    return fail(KVQ_ERR_INVALID_ARG, "window must be 0 or a positive multiple of page_tokens (%d)", P);
+  if (window_tokens / P + 1 > c->L.max_pages_per_seq)
+    return fail(KVQ_ERR_CAPACITY, "a window of %lld tokens needs %lld page-table slots > %d", (long long)window_tokens,
+                (long long)(window_tokens / P + 1), c->L.max_pages_per_seq);
+  c->window[id] = window_tokens;
   return KVQ_OK;
 }
 
@@ -481,15 +531,18 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
   auto shared_tail = [&](int32_t id) -> int32_t {
     if (c->len[id] % P == 0) return -1;
     const int32_t p = int32_t(c->len[id] / P);
-    return c->refs[c->table[size_t(id) * c->L.max_pages_per_seq + p]] > 1 ? p : -1;
+    return c->refs[c->table[slot_index(c, id, p)]] > 1 ? p : -1;
   };
   int64_t need = 0;
   for (int i = 0; i < n; ++i) {
     if (n_new[i] < 0) return fail(KVQ_ERR_INVALID_ARG, "n_new[%d] < 0", i);
     int64_t nl = c->len[ids[i]] + n_new[i];
-    if (nl > c->cfg.max_seq_tokens)
-      return fail(KVQ_ERR_CAPACITY, "sequence %d would hold %lld tokens > max_seq_tokens", ids[i], (long long)nl);
-    need += (nl + P - 1) / P - c->mapped[ids[i]];
+    // a rotating window reuses its ring of pages: only its positions are bounded (kernels index in int32)
+    const int64_t limit = c->window[ids[i]] ? (int64_t(1) << 30) : c->cfg.max_seq_tokens;
+    if (nl > limit)
+      return fail(KVQ_ERR_CAPACITY, "sequence %d would hold %lld tokens > %lld", ids[i], (long long)nl,
+                  (long long)limit);
+    need += slots_for(c, ids[i], nl) - c->mapped[ids[i]];
     if (n_new[i] > 0 && shared_tail(ids[i]) >= 0) ++need;
   }
   if (need > int64_t(c->free_pages.size()))
@@ -522,10 +575,10 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
   for (int i = 0; i < n && st == KVQ_OK; ++i) {
     const int32_t id = ids[i];
     const int64_t nl = c->len[id] + n_new[i];
-    const int32_t want = int32_t((nl + P - 1) / P);
+    const int32_t want = slots_for(c, id, nl);
     const int32_t tail = n_new[i] > 0 ? shared_tail(id) : -1;
     if (tail >= 0) {
-      const size_t slot = size_t(id) * c->L.max_pages_per_seq + tail;
+      const size_t slot = slot_index(c, id, tail);
       const int32_t from = c->table[slot], to = take_page(c, &j);
       if (!c->host_only) {
         // the page's head blocks of one layer are contiguous: one copy per layer
@@ -541,6 +594,8 @@ kvq_status kvq_seq_extend(kvq_cache* c, int32_t n, const int32_t* ids, const int
       drop_page(c, from, &j);
       st = queue(slot, to);
     }
+    // new slots (a ring's slots are only ever added until the ring is full; after that the
+    // slot of the oldest page, entirely before the window, is written again)
     while (st == KVQ_OK && c->mapped[id] < want) {
       const int32_t page = take_page(c, &j);
       const size_t slot = size_t(id) * c->L.max_pages_per_seq + c->mapped[id];
@@ -576,6 +631,8 @@ kvq_status kvq_seq_truncate(kvq_cache* c, int32_t id, int64_t new_len) {
   if (kvq_status s = check_seq(c, id)) return s;
   if (new_len < 0 || new_len > c->len[id])
     return fail(KVQ_ERR_INVALID_ARG, "new_len %lld outside [0, len = %lld]", (long long)new_len, (long long)c->len[id]);
+  if (wrapped(c, id) && new_len != c->len[id])
+    return fail(KVQ_ERR_UNSUPPORTED, "sequence %d: truncate after its rotating window wrapped", id);
   const int P = c->L.page_tokens;
   const int32_t keep = int32_t((new_len + P - 1) / P);
   for (int32_t p = c->mapped[id] - 1; p >= keep; --p) {
@@ -593,6 +650,7 @@ kvq_status kvq_seq_fork(kvq_cache* c, int32_t src, int32_t dst, int64_t n_tokens
   if (kvq_status s = check_seq(c, src)) return s;
   if (kvq_status s = check_seq(c, dst)) return s;
   if (src == dst) return fail(KVQ_ERR_INVALID_ARG, "fork of sequence %d onto itself", src);
+  if (c->window[src] || c->window[dst]) return fail(KVQ_ERR_UNSUPPORTED, "fork of a rotating-window sequence");
   if (c->len[dst] != 0 || c->mapped[dst] != 0) return fail(KVQ_ERR_INVALID_ARG, "sequence %d is not empty", dst);
   if (n_tokens < 0 || n_tokens > c->len[src])
     return fail(KVQ_ERR_INVALID_ARG, "n_tokens %lld outside [0, len = %lld]", (long long)n_tokens,
@@ -644,7 +702,9 @@ kvq_status kvq_append(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids
   for (int i = 0; i < n; ++i) {
     if (n_new[i] < 0 || n_new[i] > c->len[ids[i]])
       return fail(KVQ_ERR_INVALID_ARG, "n_new[%d] = %d outside [0, len = %lld]", i, n_new[i], (long long)c->len[ids[i]]);
-    b.s[i] = {ids[i], int32_t(c->len[ids[i]] - n_new[i]), n_new[i], int32_t(total)};
+    if (c->window[ids[i]] && n_new[i] > c->window[ids[i]])
+      return fail(KVQ_ERR_INVALID_ARG, "n_new[%d] = %d exceeds the sequence's window", i, n_new[i]);
+    b.s[i] = {ids[i], int32_t(c->len[ids[i]] - n_new[i]), n_new[i], int32_t(total), 0, ring_pages(c, ids[i])};
     total += n_new[i];
     if (total > (int64_t(1) << 30)) return fail(KVQ_ERR_INVALID_ARG, "too many tokens in one append");
   }
@@ -695,7 +755,10 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   if (kvq_status s = need_device(c)) return s;
 
   kvq::DecodePlan plan;
-  const kvq::Layout& LV = c->layers[layer];
+  kvq::Layout LV = c->layers[layer];
+  bool windowed = false;
+  for (int i = 0; i < n; ++i) windowed |= c->window[ids[i]] != 0;
+  if (windowed) LV.decode_tc = 0;       // rotating windows run on the CUDA-core kernels
   plan.chunk_tokens = kvq::decode_chunk_tokens(LV, G);
   const int C = plan.chunk_tokens, H = c->L.n_kv_heads;
   kvq::Batch b;
@@ -704,8 +767,9 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   for (int i = 0; i < n; ++i) {
     const int64_t len = c->len[ids[i]];
     if (len < 1) return fail(KVQ_ERR_INVALID_ARG, "sequence %d is empty", ids[i]);
-    const int32_t nch = int32_t((len + C - 1) / C);
-    b.s[i] = {ids[i], int32_t(len), int32_t(flat), nch};
+    const int64_t lo = first_attended(c, ids[i]), base = lo / C * C;
+    const int32_t nch = int32_t((len - base + C - 1) / C);
+    b.s[i] = {ids[i], int32_t(len), int32_t(flat), nch, int32_t(lo), ring_pages(c, ids[i])};
     flat += int64_t(H) * nch;
   }
   plan.n_items = n * H;
@@ -721,7 +785,7 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   if (appending && !fused) {
     kvq::Batch ab;
     ab.n = n;
-    for (int i = 0; i < n; ++i) ab.s[i] = {ids[i], int32_t(c->len[ids[i]] - 1), 1, i};
+    for (int i = 0; i < n; ++i) ab.s[i] = {ids[i], int32_t(c->len[ids[i]] - 1), 1, i, 0, ring_pages(c, ids[i])};
     if (kvq_status s = launched(kvq::launch_append(LV, 0, ab, n, k_new, v_new, (cudaStream_t)stream), "append"))
       return s;
   }
@@ -787,6 +851,8 @@ kvq_status kvq_prefill_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_
   for (int i = 0; i < n; ++i) {
     const int64_t len = c->len[ids[i]];
     if (q_lens[i] < 1 || q_lens[i] > len) return fail(KVQ_ERR_INVALID_ARG, "q_lens[%d] outside [1, len]", i);
+    if (c->window[ids[i]] && len > c->window[ids[i]])
+      return fail(KVQ_ERR_UNSUPPORTED, "prefill of sequence %d beyond its rotating window", ids[i]);
     b.s[i] = {ids[i], int32_t(len), q_lens[i], int32_t(total)};
     total += q_lens[i];
     if (total > (int64_t(1) << 30)) return fail(KVQ_ERR_INVALID_ARG, "too many query rows");
@@ -801,15 +867,139 @@ kvq_status kvq_prefill_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_
                   "prefill");
 }
 
+kvq_status kvq_cache_dedup(kvq_cache* c, kvq_stream_t stream, int64_t* pages_freed) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (pages_freed) *pages_freed = 0;
+  if (kvq_status s = need_device(c)) return s;
+  const int P = c->L.page_tokens, L = c->cfg.n_layers;
+  const int32_t mpps = c->L.max_pages_per_seq;
+  cudaStream_t st = (cudaStream_t)stream;
+  // candidates: pages every mapping of which is a full page of a sequence without a window
+  std::vector<int8_t> state(c->L.n_pages, 0);                 // 0 unseen, 1 candidate, -1 excluded
+  std::vector<std::vector<int32_t>> slots_of;                  // mapping slots per candidate, filled below
+  for (int32_t id = 0; id < c->cfg.max_seqs; ++id)
+    for (int32_t p = 0; p < c->mapped[id]; ++p) {
+      const int32_t phys = c->table[size_t(id) * mpps + p];
+      const bool full = !c->window[id] && int64_t(p + 1) * P <= c->len[id];
+      if (!full) state[phys] = -1;
+      else if (state[phys] == 0) state[phys] = 1;
+    }
+  std::vector<int32_t> cand;
+  std::vector<int32_t> index(c->L.n_pages, -1);
+  for (int32_t pg = 0; pg < c->L.n_pages; ++pg)
+    if (state[pg] == 1) {
+      index[pg] = int32_t(cand.size());
+      cand.push_back(pg);
+    }
+  if (cand.size() < 2) return KVQ_OK;
+  slots_of.resize(cand.size());
+  for (int32_t id = 0; id < c->cfg.max_seqs; ++id)
+    for (int32_t p = 0; p < c->mapped[id]; ++p) {
+      const size_t slot = size_t(id) * mpps + p;
+      if (index[c->table[slot]] >= 0) slots_of[index[c->table[slot]]].push_back(int32_t(slot));
+    }
+  auto regions = [&](kvq::PageRegion* out, int l0, int nl) {
+    for (int l = 0; l < nl; ++l) {
+      const kvq::Layout& V = c->layers[l0 + l];
+      out[l] = {V.pool, int64_t(V.n_kv_heads) * V.head_block};
+    }
+  };
+  // 128-bit content hashes, kDedupBatch pages at a time
+  std::vector<std::array<uint32_t, 4>> hash(cand.size());
+  uint32_t* d_hash = c->d_dedup;
+  uint32_t* d_diff = c->d_dedup + 4 * kvq::kDedupBatch;
+  kvq::PageList pl;
+  for (size_t b0 = 0; b0 < cand.size(); b0 += kvq::kDedupBatch) {
+    pl.n = int32_t(std::min<size_t>(kvq::kDedupBatch, cand.size() - b0));
+    for (int i = 0; i < pl.n; ++i) pl.page[i] = cand[b0 + i];
+    for (int l0 = 0; l0 < L; l0 += kvq::kDedupLayers) {
+      const int nl = std::min(kvq::kDedupLayers, L - l0);
+      regions(pl.layer, l0, nl);
+      KVQ_CUDA(kvq::launch_page_hash(pl, nl, d_hash, l0 == 0, st), "page hash");
+    }
+    KVQ_CUDA(cudaMemcpyAsync(hash[b0].data(), d_hash, size_t(pl.n) * 16, cudaMemcpyDeviceToHost, st), "read hashes");
+    KVQ_CUDA(cudaStreamSynchronize(st), "page hash");
+  }
+  // equal hashes propose duplicates of the group's first page; a byte comparison decides
+  std::vector<int32_t> order(cand.size());
+  for (size_t i = 0; i < cand.size(); ++i) order[i] = int32_t(i);
+  std::stable_sort(order.begin(), order.end(), [&](int32_t x, int32_t y) { return hash[x] < hash[y]; });
+  std::vector<std::pair<int32_t, int32_t>> pairs;                 // (representative, duplicate) candidate indices
+  for (size_t i = 0; i < order.size();) {
+    size_t j = i + 1;
+    while (j < order.size() && hash[order[j]] == hash[order[i]]) ++j;
+    for (size_t k = i + 1; k < j; ++k) pairs.push_back({order[i], order[k]});
+    i = j;
+  }
+  std::vector<uint8_t> same(pairs.size(), 0);
+  kvq::PagePairs pp;
+  std::vector<uint32_t> diff(kvq::kDedupBatch);
+  for (size_t b0 = 0; b0 < pairs.size(); b0 += kvq::kDedupBatch) {
+    pp.n = int32_t(std::min<size_t>(kvq::kDedupBatch, pairs.size() - b0));
+    for (int i = 0; i < pp.n; ++i) {
+      pp.a[i] = cand[pairs[b0 + i].first];
+      pp.b[i] = cand[pairs[b0 + i].second];
+    }
+    for (int l0 = 0; l0 < L; l0 += kvq::kDedupLayers) {
+      const int nl = std::min(kvq::kDedupLayers, L - l0);
+      regions(pp.layer, l0, nl);
+      KVQ_CUDA(kvq::launch_page_compare(pp, nl, d_diff, l0 == 0, st), "page compare");
+    }
+    KVQ_CUDA(cudaMemcpyAsync(diff.data(), d_diff, size_t(pp.n) * 4, cudaMemcpyDeviceToHost, st), "read compare");
+    KVQ_CUDA(cudaStreamSynchronize(st), "page compare");
+    for (int i = 0; i < pp.n; ++i) same[b0 + i] = diff[i] == 0;
+  }
+  // merge: every slot mapping a duplicate maps its representative instead
+  Journal j;
+  kvq::PtUpdate upd;
+  upd.n = 0;
+  size_t flushed = 0;
+  kvq_status stt = KVQ_OK;
+  int64_t freed = 0;
+  for (size_t k = 0; k < pairs.size() && stt == KVQ_OK; ++k) {
+    if (!same[k]) continue;
+    const int32_t rep = cand[pairs[k].first], dup = cand[pairs[k].second];
+    for (int32_t slot : slots_of[pairs[k].second]) {
+      set_slot(c, size_t(slot), rep, &j);
+      c->refs[rep]++;
+      j.add(Journal::kRef, rep);
+      drop_page(c, dup, &j);
+      upd.idx[upd.n] = slot;
+      upd.val[upd.n] = rep;
+      if (++upd.n == kvq::kMaxPtUpdates) {
+        stt = launched(kvq::launch_pt_update(c->d_page_table, upd, st), "page-table update");
+        if (stt == KVQ_OK) flushed = j.ops.size();
+        upd.n = 0;
+        if (stt != KVQ_OK) break;
+      }
+    }
+    ++freed;
+  }
+  if (stt == KVQ_OK && upd.n) {
+    stt = launched(kvq::launch_pt_update(c->d_page_table, upd, st), "page-table update");
+    if (stt == KVQ_OK) flushed = j.ops.size();
+  }
+  if (stt != KVQ_OK) {
+    rollback(c, j, flushed, stream);
+    return stt;
+  }
+  if (pages_freed) *pages_freed = freed;
+  return KVQ_OK;
+}
+
 kvq_status kvq_export(const kvq_cache* c, int32_t layer, int32_t id, int64_t tok0, int64_t n_tok, void* kc,
                       void* ks, void* vc, void* vs, kvq_stream_t stream) {
   if (kvq_status s = check_cache(c)) return s;
   if (kvq_status s = check_layer(c, layer)) return s;
   if (kvq_status s = check_seq(c, id)) return s;
   if (tok0 < 0 || n_tok < 0 || tok0 + n_tok > c->len[id]) return fail(KVQ_ERR_INVALID_ARG, "token range outside the sequence");
+  if (c->window[id] && tok0 < c->len[id] - c->window[id])
+    return fail(KVQ_ERR_INVALID_ARG, "token range starts before the sequence's rotating window");
   if (n_tok == 0) return KVQ_OK;
   if (kvq_status s = need_device(c)) return s;
-  return launched(kvq::launch_export(c->layers[layer], 0, id, tok0, n_tok, kc, ks, vc, vs, (cudaStream_t)stream), "export");
+  return launched(kvq::launch_export(c->layers[layer], 0, id, ring_pages(c, id), tok0, n_tok, kc, ks, vc, vs,
+                                     (cudaStream_t)stream),
+                  "export");
 }
 
 kvq_status kvq_cache_check(kvq_cache* c, kvq_stream_t stream, uint32_t* detail) {

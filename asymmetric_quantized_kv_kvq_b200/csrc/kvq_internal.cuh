@@ -61,12 +61,19 @@ inline int code_row_bytes(int bits, int D) { return bits == 16 ? 2 * D : bits ==
 
 // One sequence of a batched call.  Field meaning depends on the operation:
 //   append : a = first position written (len - n_new), b = n_new, c = row offset in k/v
-//   decode : a = len, b = flat chunk offset of the sequence's first item, c = chunks per item
+//   decode : a = len, b = flat chunk offset of the sequence's first item, c = chunks per item,
+//            lo = first position attended (len - window for a rotating window, else 0)
 //   prefill: a = len, b = q_len, c = row offset in q/out
+// ring: page-table slots of a rotating-window sequence (logical page p lives in
+// slot p % ring), 0 for a linear page table.
 struct SeqDesc {
   int32_t seq_id;
   int32_t a, b, c;
+  int32_t lo, ring;
 };
+
+// Page-table slot of logical page p of a sequence.
+__host__ __device__ __forceinline__ int page_slot(int p, int ring) { return ring ? p % ring : p; }
 
 struct Batch {
   int32_t n;
@@ -80,6 +87,29 @@ struct PtUpdate {
   int32_t idx[kMaxPtUpdates];
   int32_t val[kMaxPtUpdates];
 };
+
+// Page deduplication: one layer's pool region (page i starts at base + i * bytes,
+// bytes = n_kv_heads head blocks) and page lists passed by value to the kernels.
+constexpr int kDedupBatch = 1024;    // pages (or pairs) per launch
+constexpr int kDedupLayers = 256;    // layers per launch (more layers: several launches, sums add up)
+struct PageRegion {
+  const uint8_t* base;
+  int64_t bytes;
+};
+struct PageList {
+  int32_t n;
+  int32_t page[kDedupBatch];
+  PageRegion layer[kDedupLayers];
+};
+struct PagePairs {
+  int32_t n;
+  int32_t a[kDedupBatch], b[kDedupBatch];
+  PageRegion layer[kDedupLayers];
+};
+// hashes: uint32 [n][4] accumulated over launches (zeroed first when asked); diff: uint32 [n],
+// nonzero where a pair differs (OR-ed over launches).
+cudaError_t launch_page_hash(const PageList& pl, int n_layers, uint32_t* hashes, bool zero_first, cudaStream_t s);
+cudaError_t launch_page_compare(const PagePairs& pp, int n_layers, uint32_t* diff, bool zero_first, cudaStream_t s);
 
 __device__ __forceinline__ void record_error(uint32_t* err, uint32_t code) {
   atomicCAS(err, 0u, code);
@@ -101,7 +131,7 @@ cudaError_t launch_pt_update(int32_t* table, const PtUpdate& u, cudaStream_t s);
 cudaError_t launch_append(const Layout& L, int layer, const Batch& b, int total_tokens,
                           const void* k, const void* v, cudaStream_t s);
 
-cudaError_t launch_export(const Layout& L, int layer, int seq_id, int64_t tok0, int64_t n_tok,
+cudaError_t launch_export(const Layout& L, int layer, int seq_id, int ring, int64_t tok0, int64_t n_tok,
                           void* k_codes, void* k_scales, void* v_codes, void* v_scales,
                           cudaStream_t s);
 

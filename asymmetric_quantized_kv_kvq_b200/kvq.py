@@ -57,6 +57,7 @@ SIGNATURES = {
     "kvq_seq_truncate": (_i32, [_p, _i32, _i64]),
     "kvq_seq_fork": (_i32, [_p, _i32, _i32, _i64, _p]),
     "kvq_seq_length": (_i32, [_p, _i32, _pi64]),
+    "kvq_seq_set_window": (_i32, [_p, _i32, _i64]),
     "kvq_seq_page": (_i32, [_p, _i32, _i32, _pi32]),
     "kvq_append": (_i32, [_p, _i32, _i32, _pi32, _pi32, _p, _p, _p]),
     "kvq_decode_workspace_size": (_i32, [_p, _i32, _i32, _psz]),
@@ -67,6 +68,7 @@ SIGNATURES = {
     "kvq_prefill_attn": (_i32, [_p, _i32, _i32, _pi32, _pi32, _i32, _p, _p, _f32, _p, _sz, _p]),
     "kvq_export": (_i32, [_p, _i32, _i32, _i64, _i64, _p, _p, _p, _p, _p]),
     "kvq_cache_check": (_i32, [_p, _p, _pu32]),
+    "kvq_cache_dedup": (_i32, [_p, _p, _pi64]),
     "kvq_status_string": (ctypes.c_char_p, [_i32]),
     "kvq_last_error": (ctypes.c_char_p, []),
 }
@@ -207,6 +209,10 @@ class Cache:
         s = None if self.host_only else _stream(stream)
         _check(self._lib.kvq_seq_fork(self._h, src, dst, n, s))
 
+    def set_window(self, seq_id: int, window_tokens: int) -> None:
+        """Rotating window: empty sequence `seq_id` keeps (and attends to) only its last window_tokens."""
+        _check(self._lib.kvq_seq_set_window(self._h, seq_id, window_tokens))
+
     def length(self, seq_id: int) -> int:
         n = ctypes.c_int64()
         _check(self._lib.kvq_seq_length(self._h, seq_id, ctypes.byref(n)))
@@ -339,6 +345,12 @@ class Cache:
         _check(self._lib.kvq_export(self._h, layer, seq_id, tok0, n_tok, ptr(kc), ptr(ks), ptr(vc), ptr(vs),
                                     _stream(stream)))
         return {"k_codes": kc, "k_scales": ks, "v_codes": vc, "v_scales": vs}
+
+    def dedup(self, stream=None) -> int:
+        """kvq_cache_dedup: merge full pages with identical bytes; returns the pages freed."""
+        n = ctypes.c_int64()
+        _check(self._lib.kvq_cache_dedup(self._h, _stream(stream), ctypes.byref(n)))
+        return n.value
 
     def check(self, stream=None) -> None:
         """Synchronise and raise on any earlier asynchronous or device-side error."""

@@ -179,6 +179,26 @@ KVQ_API kvq_status kvq_seq_truncate(kvq_cache* cache, int32_t seq_id, int64_t ne
 KVQ_API kvq_status kvq_seq_fork(kvq_cache* cache, int32_t src_seq, int32_t dst_seq, int64_t n_tokens,
                                 kvq_stream_t stream);
 
+/* Rotating window ("Reutilizacao de Cache KV para Conversas Longas no Apple
+ * Silicon", "O Que Nao Funcionou": rotating the KV cache at 8192 tokens, which
+ * gave the best tokens/s at the price of the earlier context).  Sequence seq_id,
+ * which must be empty, keeps only its last window_tokens positions from now
+ * on: its pages form a ring of window_tokens / page_tokens + 1 page-table slots,
+ * so once the ring is full kvq_seq_extend reuses the page of the oldest
+ * positions, which lie entirely before the window, and maps no new page.
+ * kvq_decode_attn / kvq_decode_append_attn attend to positions
+ * max(0, len - window_tokens) .. len - 1 (on the CUDA-core kernels).
+ * window_tokens: 0 (no window, the default) or a positive multiple of
+ * page_tokens with window_tokens / page_tokens + 1 <= the page-table row
+ * (max_seq_tokens / page_tokens), else KVQ_ERR_INVALID_ARG / KVQ_ERR_CAPACITY.
+ * A windowed sequence's length is bounded by 2^30 instead of max_seq_tokens;
+ * one kvq_append may add at most window_tokens positions; kvq_export reads
+ * positions inside the window only; kvq_seq_fork of or onto a windowed
+ * sequence, kvq_seq_truncate after the ring wrapped and kvq_prefill_attn once
+ * len > window_tokens return KVQ_ERR_UNSUPPORTED.  The window survives
+ * kvq_seq_release. */
+KVQ_API kvq_status kvq_seq_set_window(kvq_cache* cache, int32_t seq_id, int64_t window_tokens);
+
 /* Current length (token positions) of a sequence. */
 KVQ_API kvq_status kvq_seq_length(const kvq_cache* cache, int32_t seq_id, int64_t* len);
 
@@ -280,6 +300,22 @@ KVQ_API kvq_status kvq_prefill_attn(kvq_cache* cache, int32_t layer, int32_t n_s
                             const int32_t* q_lens, int32_t n_q_heads, const void* q, void* out,
                             float softmax_scale, void* workspace, size_t ws_bytes,
                             kvq_stream_t stream);
+
+/* Content deduplication of full pages ("KVBoost acelera inferencia de LLMs em
+ * 4,49x com cache reutilizavel", section "Contexto": cached chunks are found
+ * again by a hash of their content).  Among the pages that every sequence
+ * mapping them holds completely (all page_tokens positions below its length;
+ * sequences with a rotating window excluded), pages whose bytes are identical in
+ * every layer are merged: each page-table entry of a duplicate then names one
+ * representative page, whose reference count grows by the duplicate's, and the
+ * duplicate returns to the pool.  Candidates come from a 128-bit content hash
+ * computed on the GPU and are merged only after a byte comparison, so different
+ * contents are never merged.  Full pages are never written again (appends
+ * write positions >= len; a truncate into a shared page leaves it to
+ * copy-on-write), so reads are unchanged.  Synchronises `stream` (hash and
+ * comparison results are read back); page-table updates are enqueued on it.
+ * *pages_freed (may be NULL) receives the number of pages returned. */
+KVQ_API kvq_status kvq_cache_dedup(kvq_cache* cache, kvq_stream_t stream, int64_t* pages_freed);
 
 /* Copy tokens [tok0, tok0 + n_tok) of a sequence in `layer` out in canonical
  * form (device destinations, any may be NULL to skip):

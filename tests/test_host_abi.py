@@ -352,3 +352,64 @@ def test_per_layer_precision_validation(kvq):
     assert lib.kvq_cache_create(ctypes.byref(cfg), ctypes.byref(h)) == 1
     with pytest.raises(kvq.KvqError):
         kvq.make_config(3, 2, 64, 8, 4, 2, 1024, layer_bits=[(8, 4)])
+
+
+def test_rotating_window_keeps_a_ring_of_pages(kvq):
+    """A 256-token window with 64-token pages keeps a ring of 5 page-table slots: after 1000 one-token
+    extends the sequence maps exactly 5 distinct pages in slots 0..4 and nothing beyond; a linear
+    sequence next to it maps all its pages; release returns the ring."""
+    c = kvq.Cache(n_layers=2, n_kv_heads=2, head_dim=64, k_bits=8, v_bits=4, max_seqs=3, max_tokens=64 * 40,
+                  page_tokens=64, max_seq_tokens=64 * 8, host_only=True)
+    c.set_window(0, 256)
+    for _ in range(1000):
+        c.extend([0], [1])
+    assert c.length(0) == 1000
+    ring = [c.page(0, s) for s in range(8)]
+    assert all(p >= 0 for p in ring[:5]) and ring[5:] == [-1, -1, -1] and len(set(ring[:5])) == 5
+    pool, mapped, used = c.footprint()
+    assert mapped == 5 * 64 * 2 * 2 * (68 + 36)                   # 5 pages x 64 tokens x 2 layers x 2 heads
+    c.extend([1], [300])
+    assert c.footprint()[1] == (5 + 5) * 64 * 2 * 2 * (68 + 36)
+    # a multi-token extend across the ring's wrap point reuses slots in order
+    c.extend([0], [200])
+    assert [c.page(0, s) for s in range(5)] == ring[:5]
+    c.release(0)
+    assert c.footprint()[1] == 5 * 64 * 2 * 2 * (68 + 36)
+    c.close()
+
+
+def test_rotating_window_refusals(kvq):
+    c = kvq.Cache(n_layers=1, n_kv_heads=2, head_dim=64, k_bits=8, v_bits=4, max_seqs=3, max_tokens=64 * 40,
+                  page_tokens=64, max_seq_tokens=64 * 8, host_only=True)
+    for bad, name in ((100, "KVQ_ERR_INVALID_ARG"), (-64, "KVQ_ERR_INVALID_ARG"), (512, "KVQ_ERR_CAPACITY")):
+        with pytest.raises(kvq.KvqError) as e:
+            c.set_window(0, bad)
+        assert e.value.name == name
+    c.set_window(0, 128)
+    c.extend([0], [1000])                                         # windowed: not bounded by max_seq_tokens
+    with pytest.raises(kvq.KvqError) as e:
+        c.set_window(0, 256)                                      # only on an empty sequence
+    assert e.value.name == "KVQ_ERR_INVALID_ARG"
+    with pytest.raises(kvq.KvqError) as e:
+        c.fork(0, 1, 10)
+    assert e.value.name == "KVQ_ERR_UNSUPPORTED"
+    with pytest.raises(kvq.KvqError) as e:
+        c.truncate(0, 900)
+    assert e.value.name == "KVQ_ERR_UNSUPPORTED"
+    lib = kvq.load_library()
+    ids = (ctypes.c_int32 * 1)(0)
+    nn = (ctypes.c_int32 * 1)(129)
+    assert lib.kvq_append(c._h, 0, 1, ids, nn, 16, 16, None) == 1    # more than the window in one append
+    with pytest.raises(kvq.KvqError):
+        c.extend([1], [64 * 8 + 1])                               # a linear sequence keeps its bound
+    c.close()
+
+
+def test_dedup_needs_a_device(kvq):
+    c = _host_cache(kvq)
+    c.extend([0], [600])
+    lib = kvq.load_library()
+    n = ctypes.c_int64(-1)
+    assert lib.kvq_cache_dedup(c._h, None, ctypes.byref(n)) == 2     # KVQ_ERR_UNSUPPORTED on a host-only cache
+    assert n.value == 0
+    c.close()
