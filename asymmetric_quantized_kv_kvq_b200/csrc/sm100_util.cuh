@@ -32,6 +32,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait that lets the hardware suspend the thread for up to hint_ns while
+// the phase is incomplete (it resumes as soon as the phase completes), instead
+// of returning at once: a waiting warp then issues no instructions.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -42,16 +54,17 @@ __device__ __forceinline__ uint64_t global_ns() {
 // lost arrival can never hang the GPU: the caller records an error and leaves.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// The wait sleeps in the hardware between checks (up to 20 us per try), so a
+// warp blocked on a barrier costs no issue slots; every try also checks the
+// CTA's abort flag and the time limit.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
                                           uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 31) == 0) {
-      if (abort && *abort) return false;
-      if (global_ns() - t0 > limit_ns) return false;
-    }
+  for (;;) {
+    if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
+    if (abort && *abort) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
 }
 

@@ -336,6 +336,26 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         "step_bytes": (dec_bytes + app_bytes) / args.steps,
     }
 
+    # ---- content dedup pass (kvq_cache_dedup) over the resident cache: every full page is hashed on
+    #      the GPU (the contents differ, so nothing is merged); CUDA events around the call
+    if getattr(args, "dedup_probe", False):
+        P = 256
+        full = sum(n // P for n in run.lengths())
+        page_bytes = wl.n_kv_heads * P * (tok_bytes(kb, wl.head_dim) + tok_bytes(vb, wl.head_dim)) * L
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record()
+        freed = run.cache.dedup()
+        d1.record()
+        torch.cuda.synchronize()
+        ms = d0.elapsed_time(d1)
+        res["dedup"] = {"metric": "content-hash dedup pass GB/s (kvq_cache_dedup over the resident cache)",
+                        "value": full * page_bytes / (ms * 1e-3) / 1e9, "unit": "GB/s", "ms": ms,
+                        "pages_hashed": full, "bytes_hashed": full * page_bytes, "pages_freed": freed,
+                        "timing": "CUDA events around one kvq_cache_dedup call (hash kernels, read-back of the "
+                                  "hashes per 1024 pages, host grouping)"}
+        run.cache.check()
+
     # ---- end to end through the public API with host buffers: replaying the captured step (the
     #      default launch mode) and, beside it, calling the API eagerly every step
     if not args.no_e2e:
@@ -722,6 +742,7 @@ def main():
     from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS, parse_precision
     default_run = args.workload is None
     args.workload = args.workload or DEFAULT_WORKLOAD
+    args.dedup_probe = default_run and not args.no_extras
     wl = WORKLOADS[args.workload]
     if args.layers or args.batch or args.cached:
         import dataclasses
@@ -794,6 +815,8 @@ def main():
                                                                              "sample")}
         if extras:
             line["extra"] = extras
+        if "dedup" in res:
+            line["dedup"] = res["dedup"]
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -863,6 +886,7 @@ def run_extras(args) -> list:
     out = []
     sub = _ap.Namespace(**vars(args))
     sub.steps, sub.warmup, sub.no_e2e, sub.decode_tc, sub.separate = 5, 3, True, False, False
+    sub.dedup_probe = False
     for name, prec in (("llama70b-b1-128k", "K8V4"), ("llama70b-b1-128k", "FP16")):
         wl = WORKLOADS[name]
         kb, vb = parse_precision(prec)

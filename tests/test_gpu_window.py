@@ -44,7 +44,7 @@ def test_windowed_decode_matches_oracle(kb, vb, D, H, G):
             windows[s]) for s in ids])
         assert_close_attention(out, ref, f"step {step} lens {[cache.length(s) for s in ids]}")
         step += int(rng.integers(1, 3))
-    assert cache.length(0) > 4 * 256                              # the ring wrapped several times
+    assert cache.length(0) > 3 * 256                              # the ring wrapped several times
     # one fused step: append + decode in one launch over the window
     cache.extend(ids, [1, 1, 1])
     k1 = decode_kv(3, H, D, 77)
