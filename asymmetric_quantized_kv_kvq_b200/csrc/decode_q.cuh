@@ -16,7 +16,10 @@
 // by the last of those CTAs to finish (a counter per item; no CTA ever waits
 // for another): o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 //
-// CTA = 1 producer warp + NS score warps + NP value warps (warp roles):
+// CTA = 4 warpgroups: score warps (4), value warps (8), the producer warp (+3
+// idle warps); after launch the producer group gives registers back
+// (setmaxnreg) and the score group, whose query digits live in registers, takes
+// them (208 per thread; value warps 120, producer 64):
 //  - producer: streams each chunk's K codes, K scales, V codes and V scales
 //    (four contiguous ranges of one page's head block) into a ring of shared-
 //    memory stages with 1-D TMA bulk copies; with a fused append it first
@@ -28,13 +31,14 @@
 //  - score warps hold the query as two int8 digits per element (15 bits:
 //    q ~= s (256 hi + lo), s = max|q| / 32512 per head) and take dot products
 //    with dp4a directly on the stored key codes (4-bit codes unpacked to
-//    bytes, their +8 offset folded into the accumulator's start); lane
-//    (token, block) sums one 32-element block for GW heads, a reduce-scatter
-//    over the token's lanes leaves each lane the full score of its own
-//    head(s) (the query's register slots are permuted per lane so the
-//    exchange needs no selects); online softmax with a lazily moved maximum
-//    (moved only when a score passes it by 2^8); each lane then publishes
-//    p' = p d_v for its value block and all GW heads (one 16-byte store);
+//    bytes, their +8 offset folded into the accumulator's start); a lane sums
+//    two 32-element blocks of one token for GW heads (16 independent dp4a
+//    chains), and one exchange with the token's other lane (head_dim 128; none
+//    at 64) leaves each lane the full scores of its own heads (the query's
+//    register slots are permuted per lane so the exchange needs no selects);
+//    online softmax with a lazily moved maximum (moved only when a score passes
+//    it by 2^8); each lane then publishes p' = p d_v for its two value blocks
+//    and all GW heads (16-byte stores);
 //  - value warps convert each value code once (a byte placed in the mantissa
 //    of 2^23, then one subtraction per pair) and accumulate O += p' c with one
 //    scalar FMA per element and head; a lane owns E elements of one token, so
@@ -72,7 +76,8 @@ struct DecodeQArgs {
 template <int KB, int VB, int D, int G>
 struct QDec {
   static constexpr int NB = D / 32;                  // 32-element blocks per row
-  static constexpr int LPT = NB;                     // score lanes per token (one block each)
+  static constexpr int SBL = 2;                      // key blocks per score lane
+  static constexpr int LPT = NB / SBL;               // score lanes per token
   static constexpr int TPP = 32 / LPT;               // tokens per score pass
   static constexpr int GW = G > 4 ? 4 : G;           // query heads per score warp
   static constexpr int NHG = G / GW;                 // score warps per partition (head groups)
@@ -82,12 +87,17 @@ struct QDec {
   static constexpr int NPART = NS / NHG;             // token partitions of a stage
   static constexpr int NPP = NP / NPART;             // value warps per partition (split its tokens)
   static constexpr int NCW = NS + NP;                // consumer warps
-  static constexpr int NT = (NCW + 1) * 32;
+  static constexpr int NT = 16 * 32;                 // 4 warpgroups: score, value, value, producer (+3 idle)
+  // registers per thread after the split (setmaxnreg; the block launches with 128 each):
+  // 128 * (REG_S + 2 REG_V + REG_P) <= 65536
+  static constexpr int REG_S = 208, REG_V = 120, REG_P = 64;
+  static_assert(REG_S + 2 * REG_V + REG_P <= 512, "register split");
+  static_assert(NS == 4 && NP == 8, "warp roles are whole warpgroups");
   static constexpr int C = 128;                      // tokens per stage
   static constexpr int W = C / NPART;                // tokens per partition
   static constexpr int NPASS = W / TPP;              // score passes per stage
   static constexpr int WP = W / NPP;                 // tokens per value warp per stage
-  static constexpr int E = (64 / G) < (D / 2) ? (64 / G) : (D / 2);   // value elements per lane
+  static constexpr int E = G >= 4 ? 64 / G : 16;    // value elements per lane (E x G <= 64 accumulators)
   static constexpr int LPV = D / E;                  // value lanes per token
   static constexpr int TPV = 32 / LPV;               // tokens per value pass
   static constexpr int NPV = WP / TPV;               // value passes per stage
@@ -170,30 +180,45 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---- stored codes -------------------------------------------------------------
-// Score lane's key code words of one 32-element block, digit-word order w = 0..7
-// (element 4w + e of the block for 8-bit codes; for 4-bit codes words 0..3 are
-// the low nibbles = elements 4w + e, words 4..7 the high nibbles = elements
-// 16 + 4(w - 4) + e).  `swz` swaps the two 16-byte halves of an 8-bit block so
-// that the lanes of one load spread over all shared-memory banks.
+// A score lane reads the codes of its token's two key blocks (64 bytes of 8-bit
+// codes in four 16-byte chunks, or 32 bytes of 4-bit codes in two), chunk
+// c ^ x at load step c, x depending on the lane's token, so that the 16-byte
+// loads of a warp spread over all shared-memory banks.  The words land in two
+// slots of 8: slot sp holds the lane's key block sp ^ bswap (bswap = x >> 1 for
+// 8-bit, x for 4-bit), words in this order: 8-bit: element
+// 16 ((w >> 2) ^ (x & 1)) + 4 (w & 3) + e of the block for byte e of word w;
+// 4-bit: words 0..3 the low nibbles (elements 4w + e), 4..7 the high nibbles
+// (elements 16 + 4 (w - 4) + e), unpacked to one byte each (0..15).
 template <int KB>
-__device__ __forceinline__ void load_kq(const uint8_t* blk, int swz, uint32_t (&cw)[8]) {
+__device__ __forceinline__ void load_kq2(const uint8_t* span, int x, uint32_t (&cw)[16]) {
   if constexpr (KB == 8) {
-    const uint4 a = *reinterpret_cast<const uint4*>(blk + 16 * swz);
-    const uint4 c = *reinterpret_cast<const uint4*>(blk + 16 * (swz ^ 1));
-    cw[0] = a.x; cw[1] = a.y; cw[2] = a.z; cw[3] = a.w;
-    cw[4] = c.x; cw[5] = c.y; cw[6] = c.z; cw[7] = c.w;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 a = *reinterpret_cast<const uint4*>(span + 16 * (c ^ x));
+      cw[4 * c] = a.x; cw[4 * c + 1] = a.y; cw[4 * c + 2] = a.z; cw[4 * c + 3] = a.w;
+    }
   } else {
-    const uint4 a = *reinterpret_cast<const uint4*>(blk);
-    cw[0] = a.x & 0x0F0F0F0Fu; cw[1] = a.y & 0x0F0F0F0Fu; cw[2] = a.z & 0x0F0F0F0Fu; cw[3] = a.w & 0x0F0F0F0Fu;
-    cw[4] = (a.x >> 4) & 0x0F0F0F0Fu; cw[5] = (a.y >> 4) & 0x0F0F0F0Fu;
-    cw[6] = (a.z >> 4) & 0x0F0F0F0Fu; cw[7] = (a.w >> 4) & 0x0F0F0F0Fu;
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const uint4 a = *reinterpret_cast<const uint4*>(span + 16 * (c ^ x));
+      cw[8 * c] = a.x & 0x0F0F0F0Fu; cw[8 * c + 1] = a.y & 0x0F0F0F0Fu;
+      cw[8 * c + 2] = a.z & 0x0F0F0F0Fu; cw[8 * c + 3] = a.w & 0x0F0F0F0Fu;
+      cw[8 * c + 4] = (a.x >> 4) & 0x0F0F0F0Fu; cw[8 * c + 5] = (a.y >> 4) & 0x0F0F0F0Fu;
+      cw[8 * c + 6] = (a.z >> 4) & 0x0F0F0F0Fu; cw[8 * c + 7] = (a.w >> 4) & 0x0F0F0F0Fu;
+    }
   }
 }
-// Element (within the block) of byte e of digit word w, for the load order above.
+// Element (within its block) of byte e of word w of a slot, for the load order above.
 template <int KB>
-__host__ __device__ constexpr int kq_elem(int w, int e, int swz) {
-  if (KB == 8) return 4 * (w ^ (swz ? 4 : 0)) + e;
+__host__ __device__ constexpr int kq2_elem(int w, int e, int x) {
+  if (KB == 8) return 16 * ((w >> 2) ^ (x & 1)) + 4 * (w & 3) + e;
   return w < 4 ? 4 * w + e : 16 + 4 * (w - 4) + e;
+}
+// Chunk rotation x of a score lane of token tl (see load_kq2) and the block swap it implies.
+template <int KB, int D>
+__device__ __forceinline__ int kq2_rot(int tl) {
+  if (KB == 8) return D == 128 ? (tl & 3) : ((tl >> 1) & 3);
+  return D == 128 ? ((tl >> 1) & 1) : ((tl >> 2) & 1);
 }
 
 // Value lane's codes of one 4-byte word -> 8 exact values (u - 8 or c) as fp32,
@@ -443,26 +468,27 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
                                            int64_t x0, int64_t x1) {
   using T = QDec<KB, VB, D, G>;
   constexpr int S = T::S, W = T::W, NB = T::NB, GW = T::GW, NF = T::NF, LPT = T::LPT, NHG = T::NHG;
+  constexpr int KSPAN = 2 * (T::K_ROW / NB);           // code bytes of the lane's two key blocks
   constexpr uint32_t FULL = 0xffffffffu;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = warp / NHG, hg = warp % NHG;
-  const int tl = lane / LPT, blk = lane % LPT;         // lane = tl * LPT + blk
-  const int fmap = rs_map<LPT, GW>(blk);
-  const int swz = (D == 128 ? tl : tl >> 1) & 1;
-  const int H = a.L.n_kv_heads;
+  const int tl = lane / LPT, half = lane % LPT;        // lane = tl * LPT + half: blocks 2 half, 2 half + 1
+  const int fmap = rs_map<LPT, GW>(half);
+  const int xr = kq2_rot<KB, D>(tl);
+  const int bswap = KB == 8 ? (xr >> 1) : xr;          // slot sp holds block 2 half + (sp ^ bswap)
   uint32_t it = 0, itm = 0, itw = 0;
   for (int64_t x = x0; x < x1;) {
     const DecodeSeg sg = decode_find_seg(b, x, x1);
     const SeqDesc sd = b.s[sg.bi];
-    // ---- query digits in permuted slots: slot j <-> head hg * GW + (j ^ fmap), this lane's block
-    const __half* qbase = a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + hg * GW) * D + 32 * blk;
+    // ---- query digits in permuted slots: slot j <-> head hg * GW + (j ^ fmap), this lane's two blocks
+    const __half* qbase = a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + hg * GW) * D + 64 * half;
     float amax[GW];
 #pragma unroll
     for (int j = 0; j < GW; ++j) {
       const uint4* qr = reinterpret_cast<const uint4*>(qbase + (j ^ fmap) * D);
       float mx = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 8; ++c) {
         const uint4 w4 = qr[c];
         const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
@@ -473,8 +499,8 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
       }
       amax[j] = mx * fabsf(a.scale_log2);
     }
-    // per-head max over the token's block lanes: the lane at lane ^ o holds this
-    // lane's slot-j head in its slot j ^ rs_map(o)
+    // per-head max over the token's lanes: the lane at lane ^ o holds this lane's slot-j head in
+    // its slot j ^ rs_map(o)
 #pragma unroll
     for (int o = 1; o < LPT; o <<= 1) {
       float t[GW];
@@ -483,31 +509,35 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
       for (int j = 0; j < GW; ++j) amax[j] = fmaxf(amax[j], t[j]);
     }
-    uint32_t qh[GW][8], ql[GW][8];
-    int qcorr[GW];
+    uint32_t qh[GW][16], ql[GW][16];
+    int qcorr[GW][2];
 #pragma unroll
     for (int j = 0; j < GW; ++j) {
       const __half* qr = qbase + (j ^ fmap) * D;
       const float inv = amax[j] > 0.f ? 32512.f / amax[j] : 0.f;
-      int corr = 0;
 #pragma unroll
-      for (int w = 0; w < 8; ++w) {
-        uint32_t hw = 0, lw = 0;
+      for (int sp = 0; sp < 2; ++sp) {
+        const __half* qb = qr + 32 * (sp ^ bswap);
+        int corr = 0;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float qv = __half2float(qr[kq_elem<KB>(w, e, 0) ^ (KB == 8 && swz ? 16 : 0)]) * a.scale_log2;
-          int n = __float2int_rn(qv * inv);
-          n = max(-32512, min(32512, n));
-          const int lo = ((n + 128) & 255) - 128;
-          const int hi = (n - lo) >> 8;
-          hw |= uint32_t(hi & 255) << (8 * e);
-          lw |= uint32_t(lo & 255) << (8 * e);
-          corr += n;
+        for (int w = 0; w < 8; ++w) {
+          uint32_t hw = 0, lw = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float qv = __half2float(qb[kq2_elem<KB>(w, e, xr)]) * a.scale_log2;
+            int n = __float2int_rn(qv * inv);
+            n = max(-32512, min(32512, n));
+            const int lo = ((n + 128) & 255) - 128;
+            const int hi = (n - lo) >> 8;
+            hw |= uint32_t(hi & 255) << (8 * e);
+            lw |= uint32_t(lo & 255) << (8 * e);
+            corr += n;
+          }
+          qh[j][8 * sp + w] = hw;
+          ql[j][8 * sp + w] = lw;
         }
-        qh[j][w] = hw;
-        ql[j][w] = lw;
+        qcorr[j][sp] = KB == 4 ? -8 * corr : 0;          // 4-bit codes are read as u = c + 8
       }
-      qcorr[j] = KB == 4 ? -8 * corr : 0;                // 4-bit codes are read as u = c + 8
     }
     float qsc[NF], m_own[NF], l_own[NF];
 #pragma unroll
@@ -534,25 +564,31 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
       for (int ps = 0; ps < T::NPASS; ++ps) {
         const int row = row0 + ps * T::TPP + tl;
-        uint32_t cw[8];
-        load_kq<KB>(st + row * T::K_ROW + blk * (T::K_ROW / NB), swz, cw);
-        const float dk = __half2float(reinterpret_cast<const __half*>(st + T::OFF_KS + row * T::S_ROW)[blk]);
-        int hs[GW], ls[GW];
+        uint32_t cw[16];
+        load_kq2<KB>(st + row * T::K_ROW + half * KSPAN, xr, cw);
+        const float2 dk2 = h2_to_f2(*reinterpret_cast<const uint32_t*>(st + T::OFF_KS + row * T::S_ROW + 4 * half));
+        const float dks0 = bswap ? dk2.y : dk2.x, dks1 = bswap ? dk2.x : dk2.y;
+        int hs[GW][2], ls[GW][2];
 #pragma unroll
         for (int j = 0; j < GW; ++j) {
-          hs[j] = 0;
-          ls[j] = qcorr[j];
+          hs[j][0] = hs[j][1] = 0;
+          ls[j][0] = qcorr[j][0];
+          ls[j][1] = qcorr[j][1];
         }
 #pragma unroll
         for (int w = 0; w < 8; ++w)
 #pragma unroll
-          for (int j = 0; j < GW; ++j) {
-            hs[j] = __dp4a(int(cw[w]), int(qh[j][w]), hs[j]);
-            ls[j] = __dp4a(int(cw[w]), int(ql[j][w]), ls[j]);
-          }
+          for (int sp = 0; sp < 2; ++sp)
+#pragma unroll
+            for (int j = 0; j < GW; ++j) {
+              hs[j][sp] = __dp4a(int(cw[8 * sp + w]), int(qh[j][8 * sp + w]), hs[j][sp]);
+              ls[j][sp] = __dp4a(int(cw[8 * sp + w]), int(ql[j][8 * sp + w]), ls[j][sp]);
+            }
         float ps_[GW];
 #pragma unroll
-        for (int j = 0; j < GW; ++j) ps_[j] = __int2float_rn(hs[j] * 256 + ls[j]) * dk;
+        for (int j = 0; j < GW; ++j)
+          ps_[j] = fmaf(__int2float_rn(hs[j][1] * 256 + ls[j][1]), dks1,
+                        __int2float_rn(hs[j][0] * 256 + ls[j][0]) * dks0);
         reduce_scatter_perm<LPT, GW>(ps_);
 #pragma unroll
         for (int j = 0; j < NF; ++j) {
@@ -593,7 +629,7 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
         }
       }
       if (lane == 0) sm.pflag[(part * 2 + par) * NHG + hg] = any ? 1 : 0;
-      // p, and p' = p d_v of this lane's value block for the group's GW heads
+      // p, and p' = p d_v of this lane's two value blocks for the group's GW heads
       float* pb = sm.pbuf + (part * 2 + par) * (W * NB * G);
 #pragma unroll
       for (int ps = 0; ps < T::NPASS; ++ps) {
@@ -608,16 +644,23 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
         }
         float pa[GW];
 #pragma unroll
-        for (int g = 0; g < GW; ++g) pa[g] = __shfl_sync(FULL, p[g % NF], (lane & ~(LPT - 1)) | rs_lane_of<LPT, GW>(g));
-        const float dv = valid ? __half2float(reinterpret_cast<const __half*>(st + T::OFF_VS + (row0 + t) * T::S_ROW)[blk])
-                               : 0.f;
-        float* dst = pb + (t * NB + blk) * G + hg * GW;
-        if constexpr (GW == 4) {
-          *reinterpret_cast<float4*>(dst) = make_float4(pa[0] * dv, pa[1] * dv, pa[2] * dv, pa[3] * dv);
-        } else if constexpr (GW == 2) {
-          *reinterpret_cast<float2*>(dst) = make_float2(pa[0] * dv, pa[1] * dv);
-        } else {
-          *dst = pa[0] * dv;
+        for (int g = 0; g < GW; ++g) {
+          if constexpr (LPT == 1) pa[g] = p[g];           // this lane holds every head (slot g = head g)
+          else pa[g] = __shfl_sync(FULL, p[g % NF], (lane & ~(LPT - 1)) | rs_lane_of<LPT, GW>(g));
+        }
+        float2 dv2 = h2_to_f2(*reinterpret_cast<const uint32_t*>(st + T::OFF_VS + (row0 + t) * T::S_ROW + 4 * half));
+        if (!valid) dv2 = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const float dv = bb ? dv2.y : dv2.x;
+          float* dst = pb + (t * NB + 2 * half + bb) * G + hg * GW;
+          if constexpr (GW == 4) {
+            *reinterpret_cast<float4*>(dst) = make_float4(pa[0] * dv, pa[1] * dv, pa[2] * dv, pa[3] * dv);
+          } else if constexpr (GW == 2) {
+            *reinterpret_cast<float2*>(dst) = make_float2(pa[0] * dv, pa[1] * dv);
+          } else {
+            *dst = pa[0] * dv;
+          }
         }
       }
       __syncwarp();
@@ -648,7 +691,6 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
     if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw)) return;
     x += sg.n;
   }
-  (void)H;
 }
 
 // Value warp: O += p' c over its share of the partition's tokens.
@@ -809,9 +851,20 @@ __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
   const int warp = threadIdx.x >> 5;
   const int64_t x0 = int64_t(blockIdx.x) * a.cpc;
   const int64_t x1 = min(a.total_chunks, x0 + a.cpc);
-  if (warp == T::NCW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1);
-  else if (warp < T::NS) score_role<KB, VB, D, G>(a, b, sm, x0, x1);
-  else value_role<KB, VB, D, G>(a, b, sm, x0, x1);
+  // register split by warpgroup: the producer group gives registers back first, then the
+  // score group (query digits in registers) takes more; the value groups keep theirs
+  if (warp >= T::NCW) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(T::REG_P));
+    if (warp == T::NCW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1);
+    return;                                                 // the group's other 3 warps have no role
+  }
+  if (warp < T::NS) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(T::REG_S));
+    score_role<KB, VB, D, G>(a, b, sm, x0, x1);
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(T::REG_V));
+    value_role<KB, VB, D, G>(a, b, sm, x0, x1);
+  }
 }
 
 }  // namespace kvq

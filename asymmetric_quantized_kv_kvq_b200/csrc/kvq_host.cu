@@ -108,6 +108,7 @@ struct kvq_cache {
   uint32_t* d_err = nullptr;
   int32_t* d_counters = nullptr;     // decode split-item counters, [KVQ_MAX_BATCH * n_kv_heads]
   uint32_t* d_dedup = nullptr;       // page hashes [kDedupBatch][4] + compare flags [kDedupBatch]
+  kvq::PrefillStreams pstreams{};    // internal streams / events of chunked prefill's waves
   std::vector<int32_t> table;        // host mirror of the page table
   std::vector<int64_t> len;          // tokens per sequence
   std::vector<int32_t> mapped;       // pages mapped per sequence
@@ -118,6 +119,15 @@ struct kvq_cache {
 };
 
 namespace {
+
+void destroy_streams(kvq_cache* c) {
+  for (int k = 0; k < 2; ++k) {
+    if (c->pstreams.s[k]) cudaStreamDestroy(c->pstreams.s[k]);
+    if (c->pstreams.join[k]) cudaEventDestroy(c->pstreams.join[k]);
+  }
+  if (c->pstreams.fork) cudaEventDestroy(c->pstreams.fork);
+  c->pstreams = kvq::PrefillStreams{};
+}
 
 kvq_status check_cache(const kvq_cache* c) {
   if (!c) return fail(KVQ_ERR_INVALID_ARG, "cache is NULL");
@@ -428,6 +438,7 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
       if (c->d_err) cudaFree(c->d_err);
       if (c->d_counters) cudaFree(c->d_counters);
       if (c->d_dedup) cudaFree(c->d_dedup);
+      destroy_streams(c);
       delete c;
       return cuda_fail(err, what);
     };
@@ -444,6 +455,12 @@ kvq_status kvq_cache_create(const kvq_cache_config* cfg, kvq_cache** out) {
     if ((e = cudaMemset(c->d_counters, 0, counter_bytes)) != cudaSuccess) return cleanup(e, "cudaMemset(counters)");
     if ((e = cudaMalloc(&c->d_dedup, size_t(kvq::kDedupBatch) * 5 * sizeof(uint32_t))) != cudaSuccess)
       return cleanup(e, "cudaMalloc(dedup)");
+    for (int k = 0; k < 2; ++k)
+      if ((e = cudaStreamCreateWithFlags(&c->pstreams.s[k], cudaStreamNonBlocking)) != cudaSuccess ||
+          (e = cudaEventCreateWithFlags(&c->pstreams.join[k], cudaEventDisableTiming)) != cudaSuccess)
+        return cleanup(e, "prefill streams");
+    if ((e = cudaEventCreateWithFlags(&c->pstreams.fork, cudaEventDisableTiming)) != cudaSuccess)
+      return cleanup(e, "prefill streams");
     if ((e = cudaDeviceSynchronize()) != cudaSuccess) return cleanup(e, "cudaDeviceSynchronize");
     L.page_table = c->d_page_table;
     L.err = c->d_err;
@@ -472,6 +489,7 @@ kvq_status kvq_cache_destroy(kvq_cache* c) {
     cudaFree(c->d_err);
     cudaFree(c->d_counters);
     cudaFree(c->d_dedup);
+    destroy_streams(c);
   }
   delete c;
   return st;
@@ -863,7 +881,7 @@ kvq_status kvq_prefill_attn(kvq_cache* c, int32_t layer, int32_t n, const int32_
   if (kvq_status s = need_device(c)) return s;
   const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(c->L.head_dim));
   return launched(kvq::launch_prefill(c->layers[layer], 0, b, int(total), n_q_heads, q, out, sigma, ws, ws_bytes,
-                                      c->num_sms, (cudaStream_t)stream),
+                                      c->pstreams, (cudaStream_t)stream),
                   "prefill");
 }
 

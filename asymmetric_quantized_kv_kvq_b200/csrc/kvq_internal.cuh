@@ -155,9 +155,14 @@ cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const Deco
                           float scale_log2, void* workspace, cudaStream_t s);
 bool decode_fuses_append(const Layout& L, int G);
 
+// Two internal streams and events of a cache, on which chunked prefill alternates its waves.
+struct PrefillStreams {
+  cudaStream_t s[2];
+  cudaEvent_t fork, join[2];
+};
 size_t prefill_workspace_bytes(const Layout& L, const Batch& b);
 cudaError_t launch_prefill(const Layout& L, int layer, const Batch& b, int total_q, int n_q_heads,
                            const void* q, void* out, float scale, void* workspace, size_t ws_bytes,
-                           int num_sms, cudaStream_t s);
+                           const PrefillStreams& ps, cudaStream_t s);
 
 }  // namespace kvq

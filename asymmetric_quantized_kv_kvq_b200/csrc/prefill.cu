@@ -19,6 +19,13 @@
 //     (Dequantising inside the attention kernel would redo it for every
 //     128-row query tile: a 4096-token chunk with 4 query heads per KV head
 //     has 128 of them.)  Positions past the end are zero.
+//     The batch runs in waves of (sequences x a range of KV heads) whose
+//     dequantised tiles fit a fixed budget (kWaveTiles, ~60 MB at head_dim
+//     128): each wave is dequantised into one half of a two-buffer workspace
+//     and attended on its own stream, alternating between two internal
+//     streams, so the workspace stays bounded (and mostly in L2) whatever the
+//     cache length, and the next wave's CTAs fill SMs as the previous wave's
+//     finish.
 //  2. prefill_attn_kernel: one CTA per (query tile of 128 rows = 128/G tokens
 //     x G query heads of one KV head).  Warp 0 streams Q once, then 128-key
 //     tiles (two pass-1 tiles) with 2-D / 3-D TMA tensor loads (128-byte
@@ -73,9 +80,15 @@ struct PrefillSeq {
 
 struct PrefillBatch {
   int32_t n;
-  int32_t H, G, Hq;
+  int32_t H, G, Hq;     // H = KV heads of this wave, h0 + [0, H)
+  int32_t h0;
   PrefillSeq s[kMaxBatch];
 };
+
+// Dequantised 64-token tiles per wave: a wave is one or more whole sequences
+// with all KV heads, or one sequence with a range of its heads; a single
+// (sequence, head) larger than this is a wave of its own.
+constexpr int64_t kWaveTiles = 1536;
 
 // Softmax arithmetic of the attention kernel: three-input max, and 2^x by the
 // MUFU approximation with subnormal results flushed (p < 2^-126 contributes
@@ -129,7 +142,7 @@ __global__ void __launch_bounds__(256) dequant_tiles_kernel(const Layout L, int 
   const int si = find_seq_by(b, gt, true);
   const PrefillSeq sq = b.s[si];
   const int rel = gt - sq.tile_base;
-  const int h = rel / sq.n_tiles, j = rel % sq.n_tiles;
+  const int h = b.h0 + rel / sq.n_tiles, j = rel % sq.n_tiles;
   const int tid = threadIdx.x;
   constexpr int NB = D / 32;
   constexpr int TPT = 256 / kKT;                 // threads per token
@@ -287,12 +300,12 @@ __global__ void __launch_bounds__(352, 1)
   const int G = b.G, TT = kQT / G;                        // tokens per query tile
   const int nq = (sq.q_len + TT - 1) / TT;
   const int qt = nq - 1 - (int(blockIdx.x) - sq.qt_begin); // heavy tiles first
-  const int h = blockIdx.y;
+  const int h = b.h0 + blockIdx.y;                        // KV head
   const int tok0 = qt * TT;                                // first chunk row of this tile
   const int qpos0 = sq.len - sq.q_len + tok0;              // absolute position of row 0
   const int qpos_last = sq.len - sq.q_len + min(tok0 + TT, sq.q_len) - 1;
   const int n_kv = qpos_last / kKV + 1;
-  const int tile_base = sq.tile_base + h * sq.n_tiles;     // first 64-token pass-1 tile of this head
+  const int tile_base = sq.tile_base + blockIdx.y * sq.n_tiles;   // first 64-token pass-1 tile of this head
 
   if (threadIdx.x == 0) {
     for (int i = 0; i <= B_Q8; ++i)
@@ -621,20 +634,61 @@ __global__ void __launch_bounds__(352, 1)
 }
 
 // ------------------------------------------------------------------ host
-// Batch sorted by decreasing length (heavy work first), with tile and query-tile offsets.
-PrefillBatch plan(const Layout& L, const Batch& in, int n_q_heads, int64_t* n_tiles_total, int64_t* n_qtiles) {
-  PrefillBatch b{};
-  b.n = in.n;
-  b.H = L.n_kv_heads;
-  b.G = n_q_heads / L.n_kv_heads;
-  b.Hq = n_q_heads;
+// Sequence order: decreasing length (heavy work first).
+std::vector<int> length_order(const Batch& in) {
   std::vector<int> order(in.n);
   std::iota(order.begin(), order.end(), 0);
   std::stable_sort(order.begin(), order.end(), [&](int x, int y) { return in.s[x].a > in.s[y].a; });
+  return order;
+}
+
+struct Wave {
+  int first, count;     // positions in the length order
+  int h0, nh;           // KV heads
+  int64_t tiles;
+};
+
+// Waves over the length order: consecutive whole sequences while they fit kWaveTiles,
+// a sequence that does not fit alone split into head ranges.
+std::vector<Wave> make_waves(const Batch& in, const std::vector<int>& order, int H) {
+  std::vector<Wave> w;
+  auto tiles_of = [&](int i) { return int64_t((in.s[order[i]].a + kKT - 1) / kKT); };
+  int i = 0;
+  while (i < in.n) {
+    const int64_t t0 = tiles_of(i);
+    if (t0 * H > kWaveTiles) {
+      const int nh = int(std::max<int64_t>(1, std::min<int64_t>(H, kWaveTiles / t0)));
+      for (int h0 = 0; h0 < H; h0 += nh) {
+        const int n = std::min(nh, H - h0);
+        w.push_back({i, 1, h0, n, t0 * n});
+      }
+      ++i;
+      continue;
+    }
+    Wave v{i, 0, 0, H, 0};
+    while (i < in.n && v.tiles + tiles_of(i) * H <= kWaveTiles) {
+      v.tiles += tiles_of(i) * H;
+      ++v.count;
+      ++i;
+    }
+    w.push_back(v);
+  }
+  return w;
+}
+
+// Batch of one wave, with tile and query-tile offsets.
+PrefillBatch plan(const Batch& in, const std::vector<int>& order, const Wave& v, int H, int n_q_heads,
+                  int64_t* n_tiles_total, int64_t* n_qtiles) {
+  PrefillBatch b{};
+  b.n = v.count;
+  b.H = v.nh;
+  b.h0 = v.h0;
+  b.G = n_q_heads / H;
+  b.Hq = n_q_heads;
   const int TT = kQT / b.G;
   int64_t tiles = 0, qts = 0;
-  for (int i = 0; i < in.n; ++i) {
-    const SeqDesc& d = in.s[order[i]];
+  for (int i = 0; i < v.count; ++i) {
+    const SeqDesc& d = in.s[order[v.first + i]];
     PrefillSeq& p = b.s[i];
     p.seq_id = d.seq_id;
     p.len = d.a;
@@ -651,11 +705,16 @@ PrefillBatch plan(const Layout& L, const Batch& in, int n_q_heads, int64_t* n_ti
   return b;
 }
 
+int64_t max_wave_tiles(const std::vector<Wave>& w) {
+  int64_t m = 0;
+  for (const Wave& v : w) m = std::max(m, v.tiles);
+  return m;
+}
+
+// One wave: dequantise into ws, then the attention kernel, on stream s.
 template <int D>
-cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_q_heads, const void* q, void* out,
-                float scale, void* ws, cudaStream_t s) {
-  int64_t n_tiles = 0, n_qt = 0;
-  const PrefillBatch b = plan(L, in, n_q_heads, &n_tiles, &n_qt);
+cudaError_t run_wave(const Layout& L, int layer, const PrefillBatch& b, int64_t n_tiles, int64_t n_qt,
+                     const CUtensorMap& mq, const void* out, float scale, void* ws, cudaStream_t s) {
   const int64_t per = n_tiles * kKT * D;
   __half* khi = static_cast<__half*>(ws);
   __half* klo = khi + per;          // fp16 [tokens][D], or e5m2 [tokens][D] in its first half (head_dim 128)
@@ -663,15 +722,7 @@ cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_
   dequant_tiles_kernel<D><<<unsigned(n_tiles), 256, 0, s>>>(L, layer, b, khi, klo, vws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-
-  CUtensorMap mq, mkh, mkl, mv;
-  const int G = b.G;
-  {
-    cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(n_q_heads), cuuint64_t(total_q)};
-    cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(n_q_heads) * D * 2};
-    cuuint32_t box[3] = {64, cuuint32_t(G), cuuint32_t(kQT / G)};
-    if (!make_tensor_map(&mq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, const_cast<void*>(q), 3, dims, strides, box)) return cudaErrorInvalidValue;
-  }
+  CUtensorMap mkh, mkl, mv;
   {
     cuuint64_t dims[2] = {cuuint64_t(D), cuuint64_t(n_tiles) * kKT};
     cuuint64_t strides[1] = {cuuint64_t(D) * 2};
@@ -692,33 +743,73 @@ cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_
     if (!make_tensor_map(&mv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, vws, 2, dims, strides, box)) return cudaErrorInvalidValue;
   }
   using T = PTraits<D>;
-  static bool configured = false;
-  if (!configured) {
-    e = cudaFuncSetAttribute(prefill_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
   PrefillArgs a;
   a.scale_log2 = scale * 1.4426950408889634f;
-  a.out = static_cast<__half*>(out);
+  a.out = static_cast<__half*>(const_cast<void*>(out));
   a.err = L.err;
   dim3 grid(unsigned(n_qt), unsigned(b.H));
   prefill_attn_kernel<D><<<grid, T::NT, T::SMEM, s>>>(mq, mkh, mkl, mv, a, b);
   return cudaGetLastError();
 }
 
+template <int D>
+cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_q_heads, const void* q, void* out,
+                float scale, void* ws, const PrefillStreams& ps, cudaStream_t s) {
+  const int H = L.n_kv_heads, G = n_q_heads / H;
+  const std::vector<int> order = length_order(in);
+  const std::vector<Wave> waves = make_waves(in, order, H);
+  CUtensorMap mq;
+  {
+    cuuint64_t dims[3] = {cuuint64_t(D), cuuint64_t(n_q_heads), cuuint64_t(total_q)};
+    cuuint64_t strides[2] = {cuuint64_t(D) * 2, cuuint64_t(n_q_heads) * D * 2};
+    cuuint32_t box[3] = {64, cuuint32_t(G), cuuint32_t(kQT / G)};
+    if (!make_tensor_map(&mq, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, const_cast<void*>(q), 3, dims, strides, box)) return cudaErrorInvalidValue;
+  }
+  using T = PTraits<D>;
+  static bool configured = false;
+  if (!configured) {
+    const cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const size_t half_bytes = size_t(max_wave_tiles(waves)) * kKT * D * 3 * sizeof(__half);
+  if (waves.size() == 1) {
+    int64_t nt = 0, nq = 0;
+    const PrefillBatch b = plan(in, order, waves[0], H, n_q_heads, &nt, &nq);
+    return run_wave<D>(L, layer, b, nt, nq, mq, out, scale, ws, s);
+  }
+  // several waves: alternate two internal streams and two workspace halves; the caller's
+  // stream is forked to both and joined back, so the call stays ordered (and capturable)
+  cudaError_t e = cudaEventRecord(ps.fork, s);
+  for (int k = 0; k < 2 && e == cudaSuccess; ++k) e = cudaStreamWaitEvent(ps.s[k], ps.fork, 0);
+  for (size_t w = 0; w < waves.size() && e == cudaSuccess; ++w) {
+    int64_t nt = 0, nq = 0;
+    const PrefillBatch b = plan(in, order, waves[w], H, n_q_heads, &nt, &nq);
+    void* half = static_cast<uint8_t*>(ws) + (w & 1) * half_bytes;
+    e = run_wave<D>(L, layer, b, nt, nq, mq, out, scale, half, ps.s[w & 1]);
+  }
+  for (int k = 0; k < 2; ++k) {
+    const cudaError_t e2 = cudaEventRecord(ps.join[k], ps.s[k]);
+    if (e == cudaSuccess) e = e2;
+    const cudaError_t e3 = cudaStreamWaitEvent(s, ps.join[k], 0);
+    if (e == cudaSuccess) e = e3;
+  }
+  return e;
+}
+
 }  // namespace
 
 size_t prefill_workspace_bytes(const Layout& L, const Batch& b) {
-  int64_t tiles = 0;
-  for (int i = 0; i < b.n; ++i) tiles += int64_t((b.s[i].a + kKT - 1) / kKT) * L.n_kv_heads;
-  return size_t(tiles) * kKT * L.head_dim * 3 * sizeof(__half);   // K_hi, K_lo, V^T
+  const std::vector<Wave> waves = make_waves(b, length_order(b), L.n_kv_heads);
+  // K_hi, K_lo, V^T of the largest wave, twice when waves alternate between two halves
+  const size_t half = size_t(max_wave_tiles(waves)) * kKT * L.head_dim * 3 * sizeof(__half);
+  return waves.size() > 1 ? 2 * half : half;
 }
 
 cudaError_t launch_prefill(const Layout& L, int layer, const Batch& b, int total_q, int n_q_heads, const void* q,
-                           void* out, float scale, void* ws, size_t, int, cudaStream_t s) {
-  if (L.head_dim == 128) return run<128>(L, layer, b, total_q, n_q_heads, q, out, scale, ws, s);
-  return run<64>(L, layer, b, total_q, n_q_heads, q, out, scale, ws, s);
+                           void* out, float scale, void* ws, size_t, const PrefillStreams& ps, cudaStream_t s) {
+  if (L.head_dim == 128) return run<128>(L, layer, b, total_q, n_q_heads, q, out, scale, ws, ps, s);
+  return run<64>(L, layer, b, total_q, n_q_heads, q, out, scale, ws, ps, s);
 }
 
 }  // namespace kvq

@@ -81,3 +81,45 @@ def test_prefill_rows_agree_with_decode():
     cache.check()
     assert torch.allclose(a.float(), b.float(), atol=2e-3, rtol=1e-2)
     cache.close()
+
+
+@pytest.mark.gpu
+def test_prefill_in_bounded_waves_matches_oracle_and_replays():
+    """A batch whose dequantised tiles exceed one wave: the long sequence is split into KV-head ranges,
+    the short ones form a wave of their own; waves alternate between two internal streams and two
+    halves of a bounded workspace (smaller than the whole cache in fp16).  Every row matches the oracle,
+    and a CUDA graph of the call (fork / join of the internal streams) replays it bit for bit."""
+    m = kvq()
+    kb, vb, D, H, G = 8, 4, 128, 8, 4
+    cached, chunk = [13000, 3000, 100], [64, 129, 1]
+    n = len(cached)
+    cache = m.Cache(n_layers=1, n_kv_heads=H, head_dim=D, k_bits=kb, v_bits=vb, max_seqs=n,
+                    max_tokens=sum(cached) + sum(chunk) + 256 * n)
+    ids = list(range(n))
+    ks = [decode_kv(c + q, H, D, 300 + s) for s, (c, q) in enumerate(zip(cached, chunk))]
+    vs = [random_fp16((c + q, H, D), 400 + s) for s, (c, q) in enumerate(zip(cached, chunk))]
+    cache.extend(ids, [c + q for c, q in zip(cached, chunk)])
+    cache.append(0, ids, [c + q for c, q in zip(cached, chunk)], torch.cat(ks).cuda(), torch.cat(vs).cuda())
+    ws_need = cache.prefill_workspace_size(ids, chunk, H * G)
+    whole = sum(-(-(c + q) // 64) for c, q in zip(cached, chunk)) * H * 64 * D * 3 * 2
+    assert ws_need < whole                                    # bounded: not the whole cache in fp16
+    q = random_fp16((sum(chunk), H * G, D), 77).cuda()
+    out = cache.prefill(0, ids, chunk, q)
+    cache.check()
+    off = 0
+    for s in ids:
+        ref = oracle.attention_prefill(q[off: off + chunk[s]].cpu().numpy(), oracle_dequant(ks[s], kb),
+                                       oracle_dequant(vs[s], vb), cached[s])
+        assert_close_attention(out[off: off + chunk[s]], ref, f"wave prefill seq {s}")
+        off += chunk[s]
+    ws = torch.empty(ws_need, dtype=torch.uint8, device="cuda")
+    out2 = torch.empty_like(q)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, capture_error_mode="thread_local"):
+        cache.prefill(0, ids, chunk, q, out=out2, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    cache.check()
+    assert torch.equal(out2, out)
+    del g
+    cache.close()
