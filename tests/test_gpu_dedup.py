@@ -40,8 +40,10 @@ def test_dedup_merges_identical_full_pages_only(kb, vb):
     mapped0 = cache.footprint()[1]
     freed = cache.dedup()
     cache.check()
-    # full pages are 0..3 (positions 0..255): seq 1 shares all 4, seq 2 pages 0-1, seq 3 pages 0, 1, 3
-    assert freed == 4 + 2 + 3
+    # full pages are 0..3 (positions 0..255): seq 1 shares all 4 with seq 0, seq 2 pages 0-1 with seq 0
+    # and pages 2-3 with seq 4 (the same tokens), seq 3 pages 0, 1, 3 with seq 0
+    assert freed == 4 + 2 + 2 + 3
+    assert [cache.page(2, p) for p in (2, 3)] == [cache.page(4, p) for p in (2, 3)]
     page_bytes = mapped0 // (5 * 5)
     assert cache.footprint()[1] == mapped0 - freed * page_bytes
     assert [cache.page(1, p) for p in range(4)] == [cache.page(0, p) for p in range(4)]
