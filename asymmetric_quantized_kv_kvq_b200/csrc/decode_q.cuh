@@ -397,11 +397,25 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
   const uint64_t pol = l2_evict_first_policy();
   uint32_t it = 0;
   bool ok = true;
+  // Page ids of the next 32 chunks, one per lane, loaded together once every 32 chunks: the
+  // page-table read (a global load, ~1 us) would otherwise sit in front of every stage's copies.
+  int my_page = -1;
   for (int64_t x = x0; x < x1 && ok;) {
     const DecodeSeg sg = decode_find_seg(b, x, x1);
     const SeqDesc sd = b.s[sg.bi];
     for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
       const int s = it % S;
+      if ((it & 31) == 0) {
+        const int64_t xl = x0 + it + lane;                  // this lane's chunk of the flat list
+        my_page = -1;
+        if (xl < x1) {
+          const DecodeSeg gl = decode_find_seg(b, xl, x1);
+          const SeqDesc dl = b.s[gl.bi];
+          const int t0 = dl.lo / a.chunk * a.chunk + gl.k0 * a.chunk;
+          my_page = a.L.page_table[int64_t(dl.seq_id) * a.L.max_pages_per_seq + page_slot(t0 / a.L.page_tokens, dl.ring)];
+        }
+      }
+      const int page = __shfl_sync(0xffffffffu, my_page, it & 31);
       if (!mbar_wait(sm.empty0 + 8 * s, ((it / S) & 1) ^ 1, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 1);
         *sm.abort_flag = 1;
@@ -411,8 +425,6 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
       const int tok0 = sd.lo / a.chunk * a.chunk + k * a.chunk;   // chunks start at the window's first chunk
       const int ntok = min(a.chunk, sd.a - tok0);
       const int ncopy = min(a.chunk, (ntok + 15) & ~15);
-      const int page =
-          a.L.page_table[int64_t(sd.seq_id) * a.L.max_pages_per_seq + page_slot(tok0 / a.L.page_tokens, sd.ring)];
       if (page < 0 || page >= a.L.n_pages) {
         if (lane == 0) record_error(a.L.err, kErrBadPage);
         *sm.abort_flag = 1;
