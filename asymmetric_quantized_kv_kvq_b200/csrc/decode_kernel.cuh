@@ -241,17 +241,30 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
 
   // ------------------------------------------------------------------ producer
   if (warp == NW) {
-    if (lane != 0) return;
     const uint64_t pol = l2_evict_first_policy();
     uint32_t it = 0;
     bool ok = true;
+    // page ids of the next 32 chunks, one per lane, loaded together once every 32 chunks (a
+    // page-table read in front of every stage would cap the stage rate); lane 0 issues the copies
+    int my_page = -1;
     for (int64_t x = x0; x < x1 && ok;) {
       const DecodeSeg sg = decode_find_seg(b, x, x1);
       const SeqDesc sd = b.s[sg.bi];
       for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
         const int s = it % S;
+        if ((it & 31) == 0) {
+          const int64_t xl = x0 + it + lane;
+          my_page = -1;
+          if (xl < x1) {
+            const DecodeSeg gl = decode_find_seg(b, xl, x1);
+            const SeqDesc dl = b.s[gl.bi];
+            const int t0 = dl.lo / a.chunk * a.chunk + gl.k0 * a.chunk;
+            my_page = a.L.page_table[int64_t(dl.seq_id) * a.L.max_pages_per_seq + page_slot(t0 / a.L.page_tokens, dl.ring)];
+          }
+        }
+        const int page = __shfl_sync(0xffffffffu, my_page, it & 31);
         if (!mbar_wait(empty0 + 8 * s, ((it / S) & 1) ^ 1, abort_flag)) {
-          record_error(a.L.err, kErrWaitTimeout | 1);
+          if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 1);
           *abort_flag = 1;
           ok = false;
           break;
@@ -259,29 +272,30 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         const int tok0 = sd.lo / a.chunk * a.chunk + k * a.chunk;   // chunks start at the window's first chunk
         const int ntok = min(a.chunk, sd.a - tok0);
         const int ncopy = min(a.chunk, (ntok + 15) & ~15);
-        const int page =
-            a.L.page_table[int64_t(sd.seq_id) * a.L.max_pages_per_seq + page_slot(tok0 / a.L.page_tokens, sd.ring)];
         if (page < 0 || page >= a.L.n_pages) {
-          record_error(a.L.err, kErrBadPage);
+          if (lane == 0) record_error(a.L.err, kErrBadPage);
           *abort_flag = 1;
           ok = false;
           break;
         }
-        const int r = tok0 % a.L.page_tokens;
-        const uint8_t* hb = a.L.head_ptr(a.layer, page, sg.h);
-        const uint32_t bar = full0 + 8 * s;
-        const uint32_t dst = smem_u32(stages + s * T::STAGE_BYTES);
-        mbar_arrive_expect_tx(bar, uint32_t(ncopy * T::TOK_BYTES));
-        bulk_g2s(dst, hb + int64_t(r) * T::K_ROW, ncopy * T::K_ROW, bar, pol);
-        if (T::KS_ROW) bulk_g2s(dst + T::OFF_KS, hb + a.L.k_scales_off + int64_t(r) * T::KS_ROW, ncopy * T::KS_ROW, bar, pol);
-        bulk_g2s(dst + T::OFF_VC, hb + a.L.v_codes_off + int64_t(r) * T::V_ROW, ncopy * T::V_ROW, bar, pol);
-        if (T::VS_ROW) bulk_g2s(dst + T::OFF_VS, hb + a.L.v_scales_off + int64_t(r) * T::VS_ROW, ncopy * T::VS_ROW, bar, pol);
+        if (lane == 0) {
+          const int r = tok0 % a.L.page_tokens;
+          const uint8_t* hb = a.L.head_ptr(a.layer, page, sg.h);
+          const uint32_t bar = full0 + 8 * s;
+          const uint32_t dst = smem_u32(stages + s * T::STAGE_BYTES);
+          mbar_arrive_expect_tx(bar, uint32_t(ncopy * T::TOK_BYTES));
+          bulk_g2s(dst, hb + int64_t(r) * T::K_ROW, ncopy * T::K_ROW, bar, pol);
+          if (T::KS_ROW) bulk_g2s(dst + T::OFF_KS, hb + a.L.k_scales_off + int64_t(r) * T::KS_ROW, ncopy * T::KS_ROW, bar, pol);
+          bulk_g2s(dst + T::OFF_VC, hb + a.L.v_codes_off + int64_t(r) * T::V_ROW, ncopy * T::V_ROW, bar, pol);
+          if (T::VS_ROW) bulk_g2s(dst + T::OFF_VS, hb + a.L.v_scales_off + int64_t(r) * T::VS_ROW, ncopy * T::VS_ROW, bar, pol);
+        }
         ++it;
       }
       x += sg.n;
     }
     // no copy may outlive the CTA: wait (bounded) for the last fills to land
-    for (uint32_t j = it > uint32_t(S) ? it - S : 0; j < it; ++j) mbar_wait(full0 + 8 * (j % S), (j / S) & 1, nullptr);
+    if (lane == 0)
+      for (uint32_t j = it > uint32_t(S) ? it - S : 0; j < it; ++j) mbar_wait(full0 + 8 * (j % S), (j / S) & 1, nullptr);
     return;
   }
 
