@@ -116,8 +116,9 @@ struct QDec {
   static constexpr int ALPHA = (NPART * 2 * (G + NHG) * 4 + 15) / 16 * 16;   // rescale factors + flags
   static constexpr int MRG_O = NP * G * D * 4;                   // one partial O per value warp
   static constexpr int MRG_ML = NPART * G * 2 * 4;
+  static constexpr int QBUF = NS * GW * D * 2;                   // each score warp's query rows (fp16)
   static constexpr int BARS = 512;
-  static constexpr int FIXED = PBUF + ALPHA + MRG_O + MRG_ML + BARS;
+  static constexpr int FIXED = PBUF + ALPHA + MRG_O + MRG_ML + QBUF + BARS;
   static constexpr int SMEM_LIMIT = 227 * 1024;
   static constexpr int S_FIT = (SMEM_LIMIT - FIXED) / STAGE;
   static constexpr int S = S_FIT > 8 ? 8 : S_FIT;    // stages in the ring
@@ -127,6 +128,7 @@ struct QDec {
   static_assert(E * G <= 64 && BPL % 4 == 0, "value lane");
   static_assert(STAGE % 16 == 0 && OFF_KS % 16 == 0 && OFF_VC % 16 == 0 && OFF_VS % 16 == 0, "alignment");
   static_assert(S * STAGE % 16 == 0 && PBUF % 16 == 0 && ALPHA % 16 == 0 && MRG_O % 16 == 0, "alignment");
+  static_assert(MRG_ML % 16 == 0 && QBUF % 16 == 0, "alignment");
 };
 
 // ---- the permuted reduce-scatter of the score lanes ------------------------------
@@ -259,7 +261,8 @@ struct QDecSmem {
   int* pflag;           // [part][parity][NHG]       1 when the head group moved its maximum
   float* mrg_o;         // [value warp][G][D]
   float* mrg_ml;        // [part][G][2]
-  uint32_t full0, empty0, ready0, free0, mfull, mfree, mws, mlast;
+  __half* qbuf;         // [score warp][GW][D]
+  uint32_t full0, empty0, ready0, free0, mfull, mfree, mws, mlast, mcomb;
   volatile int* abort_flag;
   volatile int* last_flag;
 
@@ -270,6 +273,7 @@ struct QDecSmem {
     pflag = reinterpret_cast<int*>(palpha + T::NPART * 2 * G);
     mrg_o = reinterpret_cast<float*>(smem + T::S * T::STAGE + T::PBUF + T::ALPHA);
     mrg_ml = mrg_o + T::NP * G * D;
+    qbuf = reinterpret_cast<__half*>(mrg_ml + T::NPART * G * 2);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::S * T::STAGE + T::FIXED - T::BARS);
     full0 = smem_u32(bars);                              // [S]: stage filled (tx bytes)
     empty0 = full0 + 8 * T::S;                           // [S]: stage released by every consumer warp
@@ -279,7 +283,8 @@ struct QDecSmem {
     mfree = mfull + 8;                                   // merge data consumed
     mws = mfull + 16;                                    // partial written to the workspace
     mlast = mfull + 24;                                  // "last CTA of the item" decided
-    abort_flag = reinterpret_cast<volatile int*>(bars + 2 * T::S + 4 * T::NPART + 4);
+    mcomb = mfull + 32;                                  // merge weights of a split item written
+    abort_flag = reinterpret_cast<volatile int*>(bars + 2 * T::S + 4 * T::NPART + 5);
     last_flag = abort_flag + 1;
   }
 };
@@ -291,7 +296,7 @@ struct QDecSmem {
 template <int KB, int VB, int D, int G>
 __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<KB, VB, D, G>& sm,
                                            const DecodeSeg& sg, const SeqDesc& sd, uint32_t& itm,
-                                           uint32_t& itw) {
+                                           uint32_t& itw, uint32_t& itc) {
   using T = QDec<KB, VB, D, G>;
   constexpr int NPART = T::NPART, NPP = T::NPP, NCW = T::NCW;
   const int lane = threadIdx.x & 31;
@@ -363,19 +368,42 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
     if (*sm.last_flag) {
       __threadfence();
       const int n = int(c1 - c0 + 1);
+      // weights 2^(m_i - M) of every partial slot i and 1 / L per head, one warp per head (lanes
+      // share the slots), into the merge area, which this CTA's own merge no longer reads
+      float* wts = sm.mrg_o;                             // [n][G]
+      float* linv = sm.mrg_o + n * G;                    // [G]
+      for (int g = ct >> 5; g < G; g += NCW) {
+        const float* ml = a.ws_ml + ((c0 + item) * G + g) * 2;
+        float M = -INFINITY;
+        for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(ml + int64_t(2) * G * i));
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        float L = 0.f;
+        for (int i = lane; i < n; i += 32) {
+          const float w = exp2f(__ldcg(ml + int64_t(2) * G * i) - M);   // 0 for a slot without tokens
+          wts[i * G + g] = w;
+          L = fmaf(w, __ldcg(ml + int64_t(2) * G * i + 1), L);
+        }
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        if (lane == 0) linv[g] = 1.f / L;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.mcomb);
+      if (!mbar_wait(sm.mcomb, itc & 1, sm.abort_flag, a.L.wait_ns)) {
+        if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 9);
+        *sm.abort_flag = 1;
+        return false;
+      }
+      ++itc;
+      // every output element: the weighted sum of its slots, slots in a fixed order (loads unrolled)
       for (int e = ct; e < G * D; e += NCW * 32) {
         const int g = e / D, d = e % D;
-        const float* ml = a.ws_ml + ((c0 + item) * G + g) * 2;
         const float* o0 = a.ws_o + ((c0 + item) * G + g) * D + d;
-        float M = -INFINITY;
-        for (int i = 0; i < n; ++i) M = fmaxf(M, __ldcg(ml + int64_t(2) * G * i));
-        float acc = 0.f, L = 0.f;
-        for (int i = 0; i < n; ++i) {
-          const float f = exp2f(__ldcg(ml + int64_t(2) * G * i) - M);
-          acc = fmaf(f, __ldcg(o0 + int64_t(G) * D * i), acc);
-          L = fmaf(f, __ldcg(ml + int64_t(2) * G * i + 1), L);
-        }
-        a.out[(int64_t(sg.bi) * a.n_q_heads + sg.h * G + g) * D + d] = __float2half_rn(acc / L);
+        float acc = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < n; ++i) acc = fmaf(wts[i * G + g], __ldcg(o0 + int64_t(G) * D * i), acc);
+        a.out[(int64_t(sg.bi) * a.n_q_heads + sg.h * G + g) * D + d] = __float2half_rn(acc * linv[g]);
       }
     }
   }
@@ -488,16 +516,23 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
   const int fmap = rs_map<LPT, GW>(half);
   const int xr = kq2_rot<KB, D>(tl);
   const int bswap = KB == 8 ? (xr >> 1) : xr;          // slot sp holds block 2 half + (sp ^ bswap)
-  uint32_t it = 0, itm = 0, itw = 0;
+  uint32_t it = 0, itm = 0, itw = 0, itc = 0;
   for (int64_t x = x0; x < x1;) {
     const DecodeSeg sg = decode_find_seg(b, x, x1);
     const SeqDesc sd = b.s[sg.bi];
-    // ---- query digits in permuted slots: slot j <-> head hg * GW + (j ^ fmap), this lane's two blocks
-    const __half* qbase = a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + hg * GW) * D + 64 * half;
+    // ---- query digits in permuted slots: slot j <-> head hg * GW + (j ^ fmap), this lane's two blocks.
+    // The warp's GW query rows are staged in shared memory with 16-byte loads, then each lane reads its
+    // elements in its own (bank-rotated) word order from there.
+    __half* qs = sm.qbuf + warp * GW * D;
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + hg * GW) * D);
+      for (int i = lane; i < GW * D / 8; i += 32) reinterpret_cast<uint4*>(qs)[i] = src[i];
+      __syncwarp();
+    }
     float amax[GW];
 #pragma unroll
     for (int j = 0; j < GW; ++j) {
-      const uint4* qr = reinterpret_cast<const uint4*>(qbase + (j ^ fmap) * D);
+      const uint4* qr = reinterpret_cast<const uint4*>(qs + (j ^ fmap) * D + 64 * half);
       float mx = 0.f;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
@@ -506,7 +541,7 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 f = h2_to_f2(ws[i]);
-          mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+          mx = fmax3(mx, fabsf(f.x), fabsf(f.y));
         }
       }
       amax[j] = mx * fabsf(a.scale_log2);
@@ -521,32 +556,36 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
       for (int j = 0; j < GW; ++j) amax[j] = fmaxf(amax[j], t[j]);
     }
+    // n = rint(q / s) with s = max|q| / 32512 (|n| <= 32512), as hi = (n + 128) >> 8 and the low byte
+    // lo = n mod 256 read as int8, so that n = 256 hi + lo
     uint32_t qh[GW][16], ql[GW][16];
     int qcorr[GW][2];
 #pragma unroll
     for (int j = 0; j < GW; ++j) {
-      const __half* qr = qbase + (j ^ fmap) * D;
-      const float inv = amax[j] > 0.f ? 32512.f / amax[j] : 0.f;
+      const __half* qr = qs + (j ^ fmap) * D + 64 * half;
+      const float mul = amax[j] > 0.f ? a.scale_log2 * (32512.f / amax[j]) : 0.f;
 #pragma unroll
       for (int sp = 0; sp < 2; ++sp) {
         const __half* qb = qr + 32 * (sp ^ bswap);
         int corr = 0;
 #pragma unroll
         for (int w = 0; w < 8; ++w) {
-          uint32_t hw = 0, lw = 0;
+          // the word's 4 elements are consecutive in the row
+          const uint2 h4 = *reinterpret_cast<const uint2*>(qb + kq2_elem<KB>(w, 0, xr));
+          const float2 f01 = h2_to_f2(h4.x), f23 = h2_to_f2(h4.y);
+          int n[4];
+          n[0] = __float_as_int(fmaf(f01.x, mul, 12582912.f)) - 0x4B400000;   // round to nearest
+          n[1] = __float_as_int(fmaf(f01.y, mul, 12582912.f)) - 0x4B400000;
+          n[2] = __float_as_int(fmaf(f23.x, mul, 12582912.f)) - 0x4B400000;
+          n[3] = __float_as_int(fmaf(f23.y, mul, 12582912.f)) - 0x4B400000;
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float qv = __half2float(qb[kq2_elem<KB>(w, e, xr)]) * a.scale_log2;
-            int n = __float2int_rn(qv * inv);
-            n = max(-32512, min(32512, n));
-            const int lo = ((n + 128) & 255) - 128;
-            const int hi = (n - lo) >> 8;
-            hw |= uint32_t(hi & 255) << (8 * e);
-            lw |= uint32_t(lo & 255) << (8 * e);
-            corr += n;
+            n[e] = max(-32512, min(32512, n[e]));
+            corr += n[e];
           }
-          qh[j][8 * sp + w] = hw;
-          ql[j][8 * sp + w] = lw;
+          ql[j][8 * sp + w] = __byte_perm(__byte_perm(n[0], n[1], 0x0040), __byte_perm(n[2], n[3], 0x0040), 0x5410);
+          const int h0 = (n[0] + 128) >> 8, h1 = (n[1] + 128) >> 8, h2 = (n[2] + 128) >> 8, h3 = (n[3] + 128) >> 8;
+          qh[j][8 * sp + w] = __byte_perm(__byte_perm(h0, h1, 0x0040), __byte_perm(h2, h3, 0x0040), 0x5410);
         }
         qcorr[j][sp] = KB == 4 ? -8 * corr : 0;          // 4-bit codes are read as u = c + 8
       }
@@ -700,7 +739,7 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
         sm.mrg_ml[(part * G + g) * 2 + 1] = l_own[j];
       }
     }
-    if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw)) return;
+    if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw, itc)) return;
     x += sg.n;
   }
 }
@@ -716,7 +755,7 @@ __device__ __forceinline__ void value_role(const DecodeQArgs& a, const Batch& b,
   const int vw_ = warp - T::NS;
   const int part = vw_ / T::NPP, pw = vw_ % T::NPP;
   const int tv = lane / T::LPV, sl = lane % T::LPV;    // lane = tv * LPV + sl
-  uint32_t it = 0, itm = 0, itw = 0;
+  uint32_t it = 0, itm = 0, itw = 0, itc = 0;
   for (int64_t x = x0; x < x1;) {
     const DecodeSeg sg = decode_find_seg(b, x, x1);
     const SeqDesc sd = b.s[sg.bi];
@@ -832,7 +871,7 @@ __device__ __forceinline__ void value_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
         for (int i = 0; i < E; ++i) mo[g * D + v_elem_of<VB, E>(sl, i)] = O[g][i];
     }
-    if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw)) return;
+    if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw, itc)) return;
     x += sg.n;
   }
 }
@@ -856,6 +895,7 @@ __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
     mbar_init(sm.mfree, T::NCW);
     mbar_init(sm.mws, T::NCW);
     mbar_init(sm.mlast, 1);
+    mbar_init(sm.mcomb, T::NCW);
     *sm.abort_flag = 0;
     fence_mbar_init();
   }

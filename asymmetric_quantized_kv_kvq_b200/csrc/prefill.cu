@@ -705,9 +705,10 @@ PrefillBatch plan(const Batch& in, const std::vector<int>& order, const Wave& v,
   return b;
 }
 
-int64_t max_wave_tiles(const std::vector<Wave>& w) {
+// Tiles of the largest wave among those that alternate into workspace half k (waves k, k + 2, ...).
+int64_t half_tiles(const std::vector<Wave>& w, int k) {
   int64_t m = 0;
-  for (const Wave& v : w) m = std::max(m, v.tiles);
+  for (size_t i = k; i < w.size(); i += 2) m = std::max(m, w[i].tiles);
   return m;
 }
 
@@ -772,7 +773,7 @@ cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  const size_t half_bytes = size_t(max_wave_tiles(waves)) * kKT * D * 3 * sizeof(__half);
+  const size_t half_bytes = size_t(half_tiles(waves, 0)) * kKT * D * 3 * sizeof(__half);   // start of half 1
   if (waves.size() == 1) {
     int64_t nt = 0, nq = 0;
     const PrefillBatch b = plan(in, order, waves[0], H, n_q_heads, &nt, &nq);
@@ -801,9 +802,8 @@ cudaError_t run(const Layout& L, int layer, const Batch& in, int total_q, int n_
 
 size_t prefill_workspace_bytes(const Layout& L, const Batch& b) {
   const std::vector<Wave> waves = make_waves(b, length_order(b), L.n_kv_heads);
-  // K_hi, K_lo, V^T of the largest wave, twice when waves alternate between two halves
-  const size_t half = size_t(max_wave_tiles(waves)) * kKT * L.head_dim * 3 * sizeof(__half);
-  return waves.size() > 1 ? 2 * half : half;
+  // K_hi, K_lo, V^T: half 0 holds the largest even-numbered wave, half 1 the largest odd-numbered one
+  return size_t(half_tiles(waves, 0) + half_tiles(waves, 1)) * kKT * L.head_dim * 3 * sizeof(__half);
 }
 
 cudaError_t launch_prefill(const Layout& L, int layer, const Batch& b, int total_q, int n_q_heads, const void* q,
