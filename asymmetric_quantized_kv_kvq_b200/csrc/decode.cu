@@ -80,7 +80,7 @@ __global__ void lse_combine_kernel(const __grid_constant__ Batch b, int H, int G
 
 }  // namespace
 
-int decode_max_ctas(int num_sms) { return num_sms; }
+int decode_max_ctas(int num_sms) { return num_sms < kMaxDecodeCtas ? num_sms : kMaxDecodeCtas; }
 
 size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D) {
   const size_t slots = size_t(max_ctas) + size_t(n_items);

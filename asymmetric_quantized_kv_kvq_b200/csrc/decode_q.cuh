@@ -16,33 +16,34 @@
 // by the last of those CTAs to finish (a counter per item; no CTA ever waits
 // for another): o = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 //
-// CTA = 4 warpgroups: score warps (4), value warps (8), the producer warp (+3
-// idle warps); after launch the producer group gives registers back
-// (setmaxnreg) and the score group, whose query digits live in registers, takes
-// them (208 per thread; value warps 120, producer 64):
+// CTA = 8 consumer warps + 1 producer warp:
 //  - producer: streams each chunk's K codes, K scales, V codes and V scales
 //    (four contiguous ranges of one page's head block) into a ring of shared-
 //    memory stages with 1-D TMA bulk copies; with a fused append it first
 //    quantises the new token's K and V row into the page (same block
 //    quantiser as the append kernel), for the one chunk that holds it;
-//  - a stage's tokens are split into NPART partitions; each partition has its
-//    own running softmax state (m, l per head) kept by its score warp(s) and
-//    its own accumulators O kept by its value warps;
-//  - score warps hold the query as two int8 digits per element (15 bits:
-//    q ~= s (256 hi + lo), s = max|q| / 32512 per head) and take dot products
-//    with dp4a directly on the stored key codes (4-bit codes unpacked to
-//    bytes, their +8 offset folded into the accumulator's start); a lane sums
-//    two 32-element blocks of one token for GW heads (16 independent dp4a
-//    chains), and one exchange with the token's other lane (head_dim 128; none
-//    at 64) leaves each lane the full scores of its own heads (the query's
-//    register slots are permuted per lane so the exchange needs no selects);
-//    online softmax with a lazily moved maximum (moved only when a score passes
-//    it by 2^8); each lane then publishes p' = p d_v for its two value blocks
-//    and all GW heads (16-byte stores);
-//  - value warps convert each value code once (a byte placed in the mantissa
-//    of 2^23, then one subtraction per pair) and accumulate O += p' c with one
-//    scalar FMA per element and head; a lane owns E elements of one token, so
-//    one converted code feeds all G heads.
+//  - a stage's 128 tokens are split into partitions, one per consumer warp (at
+//    8 query heads per KV head two warps share a partition, 4 heads each); a
+//    warp keeps its own running softmax (m, l per head) and accumulators O, so
+//    consumer warps never wait for one another inside an item;
+//  - a warp is software-pipelined by one stage: the score passes of stage k and
+//    the value passes of stage k - 1 form one straight-line block, so the long
+//    dependency chains of the scores (shared-memory loads, dp4a chains,
+//    shuffles) are filled with the independent FMAs of the values;
+//  - scores: a lane owns one 32-element key block of one token and holds the
+//    query as two int8 digits per element (15 bits: q ~= s (256 hi + lo),
+//    s = max|q| / 32512 per head) for the warp's heads; dp4a on the stored key
+//    codes (4-bit codes unpacked to bytes, their +8 offset folded into the
+//    accumulator's start) gives exact integer dot products, then one int->float
+//    conversion and one multiply by d_k per (token, block, head); a
+//    reduce-scatter over the token's lanes (query register slots permuted per
+//    lane, so that it needs no selects) leaves each lane its own heads' scores;
+//  - online softmax with a lazily moved maximum (moved only when a score passes
+//    it by 2^8); p' = p d_v per (token, value block, head) goes to a
+//    warp-private buffer;
+//  - values: a lane owns E elements of one token; each code is converted to
+//    fp32 exactly once (a byte placed in the mantissa of 2^23, then one
+//    subtraction per pair) and feeds all of the warp's heads, one scalar FMA each.
 // Every wait is bounded: on expiry the kernel records an error code, raises a
 // CTA-wide abort flag, drains its own copies and returns.
 #pragma once
@@ -75,60 +76,51 @@ struct DecodeQArgs {
 
 template <int KB, int VB, int D, int G>
 struct QDec {
-  static constexpr int NB = D / 32;                  // 32-element blocks per row
-  static constexpr int SBL = 2;                      // key blocks per score lane
-  static constexpr int LPT = NB / SBL;               // score lanes per token
-  static constexpr int TPP = 32 / LPT;               // tokens per score pass
-  static constexpr int GW = G > 4 ? 4 : G;           // query heads per score warp
-  static constexpr int NHG = G / GW;                 // score warps per partition (head groups)
-  static constexpr int NF = GW > LPT ? GW / LPT : 1; // heads a score lane owns after the reduce-scatter
-  static constexpr int NS = 4;                       // score warps
-  static constexpr int NP = 8;                       // value warps
-  static constexpr int NPART = NS / NHG;             // token partitions of a stage
-  static constexpr int NPP = NP / NPART;             // value warps per partition (split its tokens)
-  static constexpr int NCW = NS + NP;                // consumer warps
-  static constexpr int NT = 16 * 32;                 // 4 warpgroups: score, value, value, producer (+3 idle)
-  // registers per thread after the split (setmaxnreg; the block launches with 128 each):
-  // 128 * (REG_S + 2 REG_V + REG_P) <= 65536
-  static constexpr int REG_S = 208, REG_V = 120, REG_P = 64;
-  static_assert(REG_S + 2 * REG_V + REG_P <= 512, "register split");
-  static_assert(NS == 4 && NP == 8, "warp roles are whole warpgroups");
   static constexpr int C = 128;                      // tokens per stage
+  static constexpr int NB = D / 32;                  // 32-element blocks per row
+  static constexpr int GW = G > 4 ? 4 : G;           // query heads per consumer warp
+  static constexpr int NHG = G / GW;                 // warps sharing one partition (head groups)
+  static constexpr int NW = 8;                       // consumer warps
+  static constexpr int NPART = NW / NHG;             // token partitions of a stage
   static constexpr int W = C / NPART;                // tokens per partition
+  static constexpr int LPT = NB;                     // score lanes per token: one key block each
+  static constexpr int TPP = 32 / LPT;               // tokens per score pass
   static constexpr int NPASS = W / TPP;              // score passes per stage
-  static constexpr int WP = W / NPP;                 // tokens per value warp per stage
-  static constexpr int E = G >= 4 ? 64 / G : 16;    // value elements per lane (E x G <= 64 accumulators)
+  static constexpr int NF = GW > LPT ? GW / LPT : 1; // heads a score lane owns after the reduce-scatter
+  static constexpr int E = 32 / GW;                  // value elements per lane (E x GW = 32 accumulators)
   static constexpr int LPV = D / E;                  // value lanes per token
   static constexpr int TPV = 32 / LPV;               // tokens per value pass
-  static constexpr int NPV = WP / TPV;               // value passes per stage
+  static constexpr int NPV = W / TPV;                // value passes per stage
+  static constexpr int NT = (NW + 1) * 32;
   static constexpr int K_ROW = KB == 8 ? D : D / 2;
   static constexpr int V_ROW = VB == 8 ? D : D / 2;
+  static constexpr int KBLK = K_ROW / NB;            // code bytes of one key block
   static constexpr int S_ROW = NB * 2;               // fp16 scales per row
   static constexpr int TOK_BYTES = K_ROW + S_ROW + V_ROW + S_ROW;
   static constexpr int BPL = VB == 8 ? E : E / 2;    // value code bytes per lane
   static constexpr int VBLK = VB == 8 ? 32 : 16;     // code bytes per value block
-  static constexpr int NBL = BPL > VBLK ? BPL / VBLK : 1;   // value blocks per lane
   static constexpr int OFF_KS = C * K_ROW;
   static constexpr int OFF_VC = OFF_KS + C * S_ROW;
   static constexpr int OFF_VS = OFF_VC + C * V_ROW;
   static constexpr int STAGE = OFF_VS + C * S_ROW;
-  static constexpr int PBUF = NPART * 2 * W * NB * G * 4;        // p', two buffers per partition
-  static constexpr int ALPHA = (NPART * 2 * (G + NHG) * 4 + 15) / 16 * 16;   // rescale factors + flags
-  static constexpr int MRG_O = NP * G * D * 4;                   // one partial O per value warp
-  static constexpr int MRG_ML = NPART * G * 2 * 4;
-  static constexpr int QBUF = NS * GW * D * 2;                   // each score warp's query rows (fp16)
-  static constexpr int BARS = 512;
-  static constexpr int FIXED = PBUF + ALPHA + MRG_O + MRG_ML + QBUF + BARS;
+  static constexpr int PBUF = NW * W * NB * GW * 4;  // per warp: p' [W][NB][GW]
+  // partial O per partition; the last CTA of a split item reuses it for one weight per CTA and head
+  static constexpr int MRG_O_F = NPART * G * D > (kMaxDecodeCtas + 1) * G ? NPART * G * D : (kMaxDecodeCtas + 1) * G;
+  static constexpr int MRG_O = (MRG_O_F * 4 + 15) / 16 * 16;
+  static constexpr int MRG_ML = (NPART * G * 2 * 4 + 15) / 16 * 16;
+  static constexpr int QBUF = NW * GW * D * 2;       // each warp's query rows (fp16)
+  static constexpr int BARS = 256;
+  static constexpr int FIXED = PBUF + MRG_O + MRG_ML + QBUF + BARS;
   static constexpr int SMEM_LIMIT = 227 * 1024;
   static constexpr int S_FIT = (SMEM_LIMIT - FIXED) / STAGE;
   static constexpr int S = S_FIT > 8 ? 8 : S_FIT;    // stages in the ring
   static constexpr int SMEM = S * STAGE + FIXED;
   static_assert(S >= 3, "stage ring does not fit");
-  static_assert(W % TPP == 0 && WP % TPV == 0 && NPV >= 1 && NPASS >= 1, "tiling");
-  static_assert(E * G <= 64 && BPL % 4 == 0, "value lane");
+  static_assert(W % TPP == 0 && NPASS >= 1 && W % TPV == 0 && NPV >= 1, "tiling");
+  static_assert(BPL % 4 == 0 && BPL <= VBLK, "a value lane's codes lie in one value block");
   static_assert(STAGE % 16 == 0 && OFF_KS % 16 == 0 && OFF_VC % 16 == 0 && OFF_VS % 16 == 0, "alignment");
-  static_assert(S * STAGE % 16 == 0 && PBUF % 16 == 0 && ALPHA % 16 == 0 && MRG_O % 16 == 0, "alignment");
-  static_assert(MRG_ML % 16 == 0 && QBUF % 16 == 0, "alignment");
+  static_assert(PBUF % 16 == 0 && QBUF % 16 == 0, "alignment");
+  static_assert((2 * S + 5) * 8 + 8 <= BARS, "barrier area");
 };
 
 // ---- the permuted reduce-scatter of the score lanes ------------------------------
@@ -182,45 +174,35 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 // ---- stored codes -------------------------------------------------------------
-// A score lane reads the codes of its token's two key blocks (64 bytes of 8-bit
-// codes in four 16-byte chunks, or 32 bytes of 4-bit codes in two), chunk
-// c ^ x at load step c, x depending on the lane's token, so that the 16-byte
-// loads of a warp spread over all shared-memory banks.  The words land in two
-// slots of 8: slot sp holds the lane's key block sp ^ bswap (bswap = x >> 1 for
-// 8-bit, x for 4-bit), words in this order: 8-bit: element
-// 16 ((w >> 2) ^ (x & 1)) + 4 (w & 3) + e of the block for byte e of word w;
-// 4-bit: words 0..3 the low nibbles (elements 4w + e), 4..7 the high nibbles
-// (elements 16 + 4 (w - 4) + e), unpacked to one byte each (0..15).
+// A score lane reads the codes of its key block: 8-bit codes as two 16-byte
+// chunks, chunk c ^ x at load step c (x depends on the lane's token, so that
+// the 16-byte loads of a warp spread over all shared-memory banks); 4-bit codes
+// as one 16-byte chunk, unpacked to one byte per code (0..15).  Byte e of word w
+// is then element kq_elem(w, e, x) of the block.
 template <int KB>
-__device__ __forceinline__ void load_kq2(const uint8_t* span, int x, uint32_t (&cw)[16]) {
+__device__ __forceinline__ void load_kq(const uint8_t* blk, int x, uint32_t (&cw)[8]) {
   if constexpr (KB == 8) {
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 a = *reinterpret_cast<const uint4*>(span + 16 * (c ^ x));
+    for (int c = 0; c < 2; ++c) {
+      const uint4 a = *reinterpret_cast<const uint4*>(blk + 16 * (c ^ x));
       cw[4 * c] = a.x; cw[4 * c + 1] = a.y; cw[4 * c + 2] = a.z; cw[4 * c + 3] = a.w;
     }
   } else {
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const uint4 a = *reinterpret_cast<const uint4*>(span + 16 * (c ^ x));
-      cw[8 * c] = a.x & 0x0F0F0F0Fu; cw[8 * c + 1] = a.y & 0x0F0F0F0Fu;
-      cw[8 * c + 2] = a.z & 0x0F0F0F0Fu; cw[8 * c + 3] = a.w & 0x0F0F0F0Fu;
-      cw[8 * c + 4] = (a.x >> 4) & 0x0F0F0F0Fu; cw[8 * c + 5] = (a.y >> 4) & 0x0F0F0F0Fu;
-      cw[8 * c + 6] = (a.z >> 4) & 0x0F0F0F0Fu; cw[8 * c + 7] = (a.w >> 4) & 0x0F0F0F0Fu;
-    }
+    const uint4 a = *reinterpret_cast<const uint4*>(blk);
+    cw[0] = a.x & 0x0F0F0F0Fu; cw[1] = a.y & 0x0F0F0F0Fu; cw[2] = a.z & 0x0F0F0F0Fu; cw[3] = a.w & 0x0F0F0F0Fu;
+    cw[4] = (a.x >> 4) & 0x0F0F0F0Fu; cw[5] = (a.y >> 4) & 0x0F0F0F0Fu;
+    cw[6] = (a.z >> 4) & 0x0F0F0F0Fu; cw[7] = (a.w >> 4) & 0x0F0F0F0Fu;
   }
 }
-// Element (within its block) of byte e of word w of a slot, for the load order above.
 template <int KB>
-__host__ __device__ constexpr int kq2_elem(int w, int e, int x) {
-  if (KB == 8) return 16 * ((w >> 2) ^ (x & 1)) + 4 * (w & 3) + e;
-  return w < 4 ? 4 * w + e : 16 + 4 * (w - 4) + e;
+__host__ __device__ constexpr int kq_elem(int w, int e, int x) {
+  if (KB == 8) return 16 * ((w >> 2) ^ x) + 4 * (w & 3) + e;
+  return w < 4 ? 4 * w + e : 16 + 4 * (w - 4) + e;   // byte j of a 4-bit block: elements j (low), j + 16 (high)
 }
-// Chunk rotation x of a score lane of token tl (see load_kq2) and the block swap it implies.
+// Chunk rotation of a score lane of token tl: rows 128 bytes apart share banks.
 template <int KB, int D>
-__device__ __forceinline__ int kq2_rot(int tl) {
-  if (KB == 8) return D == 128 ? (tl & 3) : ((tl >> 1) & 3);
-  return D == 128 ? ((tl >> 1) & 1) : ((tl >> 2) & 1);
+__device__ __forceinline__ int kq_rot(int tl) {
+  return KB == 8 ? ((tl * D) / 128) & 1 : 0;
 }
 
 // Value lane's codes of one 4-byte word -> 8 exact values (u - 8 or c) as fp32,
@@ -256,54 +238,49 @@ template <int KB, int VB, int D, int G>
 struct QDecSmem {
   using T = QDec<KB, VB, D, G>;
   uint8_t* stages;
-  float* pbuf;          // [part][parity][W][NB][G]  p' = p d_v
-  float* palpha;        // [part][parity][G]         O rescale factors
-  int* pflag;           // [part][parity][NHG]       1 when the head group moved its maximum
-  float* mrg_o;         // [value warp][G][D]
+  float* pbuf;          // [warp][W][NB][GW]  p' = p d_v
+  float* mrg_o;         // [part][G][D]
   float* mrg_ml;        // [part][G][2]
-  __half* qbuf;         // [score warp][GW][D]
-  uint32_t full0, empty0, ready0, free0, mfull, mfree, mws, mlast, mcomb;
+  __half* qbuf;         // [warp][GW][D]
+  uint32_t full0, empty0, mfull, mfree, mws, mlast, mcomb;
   volatile int* abort_flag;
   volatile int* last_flag;
 
   __device__ __forceinline__ explicit QDecSmem(uint8_t* smem) {
     stages = smem;
-    pbuf = reinterpret_cast<float*>(smem + T::S * T::STAGE);
-    palpha = reinterpret_cast<float*>(smem + T::S * T::STAGE + T::PBUF);
-    pflag = reinterpret_cast<int*>(palpha + T::NPART * 2 * G);
-    mrg_o = reinterpret_cast<float*>(smem + T::S * T::STAGE + T::PBUF + T::ALPHA);
-    mrg_ml = mrg_o + T::NP * G * D;
-    qbuf = reinterpret_cast<__half*>(mrg_ml + T::NPART * G * 2);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::S * T::STAGE + T::FIXED - T::BARS);
+    uint8_t* p = smem + T::S * T::STAGE;
+    pbuf = reinterpret_cast<float*>(p);
+    mrg_o = reinterpret_cast<float*>(p + T::PBUF);
+    mrg_ml = reinterpret_cast<float*>(p + T::PBUF + T::MRG_O);
+    qbuf = reinterpret_cast<__half*>(p + T::PBUF + T::MRG_O + T::MRG_ML);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(p + T::FIXED - T::BARS);
     full0 = smem_u32(bars);                              // [S]: stage filled (tx bytes)
     empty0 = full0 + 8 * T::S;                           // [S]: stage released by every consumer warp
-    ready0 = empty0 + 8 * T::S;                          // [part][parity]: p' published by the score warps
-    free0 = ready0 + 16 * T::NPART;                      // [part][parity]: p' consumed by the value warps
-    mfull = free0 + 16 * T::NPART;                       // merge data written
+    mfull = empty0 + 8 * T::S;                           // merge data written
     mfree = mfull + 8;                                   // merge data consumed
     mws = mfull + 16;                                    // partial written to the workspace
     mlast = mfull + 24;                                  // "last CTA of the item" decided
     mcomb = mfull + 32;                                  // merge weights of a split item written
-    abort_flag = reinterpret_cast<volatile int*>(bars + 2 * T::S + 4 * T::NPART + 5);
+    abort_flag = reinterpret_cast<volatile int*>(bars + 2 * T::S + 5);
     last_flag = abort_flag + 1;
   }
 };
 
 // End of an item segment, run by every consumer warp after it published its
-// part (m, l or O) into the merge area: combine the partitions, write the
-// output (item inside this CTA) or this CTA's partial, and let the last CTA of
-// a split item merge all partials.  Returns false when a wait gave up.
+// (m, l) and O into the merge area: combine the partitions, write the output
+// (item inside this CTA) or this CTA's partial, and let the last CTA of a
+// split item merge all partials.  Returns false when a wait gave up.
 template <int KB, int VB, int D, int G>
 __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<KB, VB, D, G>& sm,
                                            const DecodeSeg& sg, const SeqDesc& sd, uint32_t& itm,
                                            uint32_t& itw, uint32_t& itc) {
   using T = QDec<KB, VB, D, G>;
-  constexpr int NPART = T::NPART, NPP = T::NPP, NCW = T::NCW;
+  constexpr int NPART = T::NPART, NW = T::NW;
   const int lane = threadIdx.x & 31;
   const int H = a.L.n_kv_heads;
   const int item = sg.bi * H + sg.h;
   __syncwarp();
-  if (lane == 0) mbar_arrive(sm.mfull);
+  mbar_arrive_if(sm.mfull, lane == 0);
   if (!mbar_wait(sm.mfull, itm & 1, sm.abort_flag, a.L.wait_ns)) {
     if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 6);
     *sm.abort_flag = 1;
@@ -312,8 +289,8 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
   const int nch = sd.c;
   const int64_t off = int64_t(sd.b) + int64_t(sg.h) * nch;
   const int64_t c0 = off / a.cpc, c1 = (off + nch - 1) / a.cpc;
-  const int ct = threadIdx.x;                          // consumer threads are 0 .. NCW * 32 - 1
-  for (int e = ct; e < G * D; e += NCW * 32) {
+  const int ct = threadIdx.x;                          // consumer threads are 0 .. NW * 32 - 1
+  for (int e = ct; e < G * D; e += NW * 32) {
     const int g = e / D, d = e % D;
     float M = -INFINITY;
 #pragma unroll
@@ -322,10 +299,7 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
 #pragma unroll
     for (int pt = 0; pt < NPART; ++pt) {
       const float f = exp2f(sm.mrg_ml[(pt * G + g) * 2] - M);   // 0 for a partition without tokens
-      float o = 0.f;
-#pragma unroll
-      for (int q2 = 0; q2 < NPP; ++q2) o += sm.mrg_o[((pt * NPP + q2) * G + g) * D + d];
-      acc = fmaf(f, o, acc);
+      acc = fmaf(f, sm.mrg_o[(pt * G + g) * D + d], acc);
       L = fmaf(f, sm.mrg_ml[(pt * G + g) * 2 + 1], L);
     }
     if (c0 == c1) {
@@ -343,7 +317,7 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
     // the last CTA of the item to finish merges every CTA's partial (fixed slot order)
     __threadfence();
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.mws);
+    mbar_arrive_if(sm.mws, lane == 0);
     if (ct == 0) {
       const bool ok = mbar_wait(sm.mws, itw & 1, sm.abort_flag, a.L.wait_ns);
       int last = 0;
@@ -367,12 +341,12 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
     ++itw;
     if (*sm.last_flag) {
       __threadfence();
-      const int n = int(c1 - c0 + 1);
+      const int n = int(c1 - c0 + 1);                  // <= grid size <= kMaxDecodeCtas
       // weights 2^(m_i - M) of every partial slot i and 1 / L per head, one warp per head (lanes
       // share the slots), into the merge area, which this CTA's own merge no longer reads
       float* wts = sm.mrg_o;                             // [n][G]
       float* linv = sm.mrg_o + n * G;                    // [G]
-      for (int g = ct >> 5; g < G; g += NCW) {
+      for (int g = ct >> 5; g < G; g += NW) {
         const float* ml = a.ws_ml + ((c0 + item) * G + g) * 2;
         float M = -INFINITY;
         for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(ml + int64_t(2) * G * i));
@@ -389,7 +363,7 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
         if (lane == 0) linv[g] = 1.f / L;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(sm.mcomb);
+      mbar_arrive_if(sm.mcomb, lane == 0);
       if (!mbar_wait(sm.mcomb, itc & 1, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 9);
         *sm.abort_flag = 1;
@@ -397,7 +371,7 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
       }
       ++itc;
       // every output element: the weighted sum of its slots, slots in a fixed order (loads unrolled)
-      for (int e = ct; e < G * D; e += NCW * 32) {
+      for (int e = ct; e < G * D; e += NW * 32) {
         const int g = e / D, d = e % D;
         const float* o0 = a.ws_o + ((c0 + item) * G + g) * D + d;
         float acc = 0.f;
@@ -408,7 +382,7 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
     }
   }
   __syncwarp();
-  if (lane == 0) mbar_arrive(sm.mfree);
+  mbar_arrive_if(sm.mfree, lane == 0);
   ++itm;
   return true;
 }
@@ -424,6 +398,8 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
   const int H = a.L.n_kv_heads;
   const uint64_t pol = l2_evict_first_policy();
   uint32_t it = 0;
+  int s = 0;                                           // ring slot of stage `it` and its fill parity
+  uint32_t ph = 0;
   bool ok = true;
   // Page ids of the next 32 chunks, one per lane, loaded together once every 32 chunks: the
   // page-table read (a global load, ~1 us) would otherwise sit in front of every stage's copies.
@@ -432,7 +408,6 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
     const DecodeSeg sg = decode_find_seg(b, x, x1);
     const SeqDesc sd = b.s[sg.bi];
     for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
-      const int s = it % S;
       if ((it & 31) == 0) {
         const int64_t xl = x0 + it + lane;                  // this lane's chunk of the flat list
         my_page = -1;
@@ -444,7 +419,7 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
         }
       }
       const int page = __shfl_sync(0xffffffffu, my_page, it & 31);
-      if (!mbar_wait(sm.empty0 + 8 * s, ((it / S) & 1) ^ 1, sm.abort_flag, a.L.wait_ns)) {
+      if (!mbar_wait(sm.empty0 + 8 * s, ph ^ 1, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 1);
         *sm.abort_flag = 1;
         ok = false;
@@ -494,6 +469,10 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
         bulk_g2s(dst + T::OFF_VS, hb + a.L.v_scales_off + int64_t(r) * T::S_ROW, ncopy * T::S_ROW, bar, pol);
       }
       ++it;
+      if (++s == S) {
+        s = 0;
+        ph ^= 1;
+      }
     }
     x += sg.n;
   }
@@ -502,27 +481,209 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
     for (uint32_t j = it > uint32_t(S) ? it - S : 0; j < it; ++j) mbar_wait(sm.full0 + 8 * (j % S), (j / S) & 1, nullptr, a.L.wait_ns);
 }
 
-// Score warp: q . k over its partition's tokens, online softmax, p' = p d_v.
+// A consumer warp's state for one item segment: the query digits of its heads,
+// its running softmax and its accumulators.
 template <int KB, int VB, int D, int G>
-__device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b, const QDecSmem<KB, VB, D, G>& sm,
-                                           int64_t x0, int64_t x1) {
+struct QWarp {
   using T = QDec<KB, VB, D, G>;
-  constexpr int S = T::S, W = T::W, NB = T::NB, GW = T::GW, NF = T::NF, LPT = T::LPT, NHG = T::NHG;
-  constexpr int KSPAN = 2 * (T::K_ROW / NB);           // code bytes of the lane's two key blocks
+  uint32_t qh[T::GW][8], ql[T::GW][8];   // query digits of the lane's key block, slot j = head j ^ fmap
+  int qcorr[T::GW];                      // 4-bit keys: -8 * sum of the digits (codes are read as c + 8)
+  float qsc[T::NF], m[T::NF], l[T::NF];  // per owned head: digit scale, running max and sum
+  float O[T::GW][T::E];                  // value lane's accumulators, all of the warp's heads
+};
+
+// Score passes of one stage: sc[pass][j] for the lane's token and owned heads (-inf outside
+// the valid rows [rv0, rv1) of the chunk).
+template <int KB, int VB, int D, int G>
+__device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G>& w, const uint8_t* st, int prow0, int tl, int blk,
+                                         int xr, bool masked, int rv0, int rv1,
+                                         float (&sc)[QDec<KB, VB, D, G>::NPASS][QDec<KB, VB, D, G>::NF]) {
+  using T = QDec<KB, VB, D, G>;
+  constexpr int GW = T::GW, NF = T::NF;
+#pragma unroll
+  for (int ps = 0; ps < T::NPASS; ++ps) {
+    const int row = prow0 + ps * T::TPP + tl;
+    uint32_t cw[8];
+    load_kq<KB>(st + row * T::K_ROW + blk * T::KBLK, xr, cw);
+    const float dk = __half2float(*reinterpret_cast<const __half*>(st + T::OFF_KS + row * T::S_ROW + 2 * blk));
+    int hs[GW], ls[GW];
+#pragma unroll
+    for (int j = 0; j < GW; ++j) {
+      hs[j] = 0;
+      ls[j] = w.qcorr[j];
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+#pragma unroll
+      for (int j = 0; j < GW; ++j) {
+        hs[j] = __dp4a(int(cw[k]), int(w.qh[j][k]), hs[j]);
+        ls[j] = __dp4a(int(cw[k]), int(w.ql[j][k]), ls[j]);
+      }
+    float ps_[GW];
+#pragma unroll
+    for (int j = 0; j < GW; ++j) ps_[j] = __int2float_rn(hs[j] * 256 + ls[j]) * dk;
+    reduce_scatter_perm<T::LPT, GW>(ps_);
+#pragma unroll
+    for (int j = 0; j < NF; ++j) {
+      const float v = ps_[j] * w.qsc[j];
+      sc[ps][j] = (!masked || (row >= rv0 && row < rv1)) ? v : -INFINITY;
+    }
+  }
+}
+
+// Value passes of one stage: O += p' c over the lane's tokens of the partition.
+template <int KB, int VB, int D, int G>
+__device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G>& w, const uint8_t* st, const float* pb, int prow0, int tv,
+                                         int sl) {
+  using T = QDec<KB, VB, D, G>;
+  constexpr int GW = T::GW, NB = T::NB;
+  const int vblk = (sl * T::BPL) / T::VBLK;
+#pragma unroll
+  for (int pv = 0; pv < T::NPV; ++pv) {
+    const int t = pv * T::TPV + tv;
+    const uint8_t* vrow = st + T::OFF_VC + (prow0 + t) * T::V_ROW + sl * T::BPL;
+    uint32_t vw[T::BPL / 4];
+    if constexpr (T::BPL == 4) {
+      vw[0] = *reinterpret_cast<const uint32_t*>(vrow);
+    } else if constexpr (T::BPL == 8) {
+      const uint2 u = *reinterpret_cast<const uint2*>(vrow);
+      vw[0] = u.x;
+      vw[1] = u.y;
+    } else {
+#pragma unroll
+      for (int c = 0; c < T::BPL / 16; ++c) {
+        const uint4 u = reinterpret_cast<const uint4*>(vrow)[c];
+        vw[4 * c] = u.x; vw[4 * c + 1] = u.y; vw[4 * c + 2] = u.z; vw[4 * c + 3] = u.w;
+      }
+    }
+    const float* pp = pb + (t * NB + vblk) * GW;
+    float pg[GW];
+    if constexpr (GW == 4) {
+      const float4 f = *reinterpret_cast<const float4*>(pp);
+      pg[0] = f.x; pg[1] = f.y; pg[2] = f.z; pg[3] = f.w;
+    } else if constexpr (GW == 2) {
+      const float2 f = *reinterpret_cast<const float2*>(pp);
+      pg[0] = f.x;
+      pg[1] = f.y;
+    } else {
+      pg[0] = *pp;
+    }
+#pragma unroll
+    for (int wi = 0; wi < T::BPL / 4; ++wi) {
+      if constexpr (VB == 4) {
+        float f[8];
+        cvt_v4_word(vw[wi], f);
+#pragma unroll
+        for (int g = 0; g < GW; ++g)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w.O[g][8 * wi + e] = fmaf(pg[g], f[e], w.O[g][8 * wi + e]);
+      } else {
+        float f[4];
+        cvt_v8_word(vw[wi], f);
+#pragma unroll
+        for (int g = 0; g < GW; ++g)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) w.O[g][4 * wi + e] = fmaf(pg[g], f[e], w.O[g][4 * wi + e]);
+      }
+    }
+  }
+}
+
+// Online softmax of one stage's scores, then p' = p d_v into the warp's buffer (which the
+// warp's value passes of the previous stage have finished reading).
+template <int KB, int VB, int D, int G>
+__device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G>& w,
+                                              const float (&sc)[QDec<KB, VB, D, G>::NPASS][QDec<KB, VB, D, G>::NF],
+                                              const uint8_t* st, float* pb, int prow0, int tl, int blk, bool masked,
+                                              int rv0, int rv1) {
+  using T = QDec<KB, VB, D, G>;
+  constexpr int GW = T::GW, NF = T::NF, LPT = T::LPT, NB = T::NB;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  // lazy maximum: moved only when a score passes it by 2^8
+  bool need = false;
+#pragma unroll
+  for (int ps = 0; ps < T::NPASS; ++ps)
+#pragma unroll
+    for (int j = 0; j < NF; ++j) need |= sc[ps][j] > w.m[j] + 8.f;
+  if (__any_sync(FULL, need)) {
+    float alpha[NF];
+#pragma unroll
+    for (int j = 0; j < NF; ++j) {
+      float mx = sc[0][j];
+#pragma unroll
+      for (int ps = 1; ps < T::NPASS; ++ps) mx = fmaxf(mx, sc[ps][j]);
+#pragma unroll
+      for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+      const float mn = fmaxf(w.m[j], mx);
+      alpha[j] = fast_exp2(w.m[j] - mn);               // 0 while m is -inf
+      w.m[j] = mn;
+      w.l[j] *= alpha[j];
+    }
+    // rescale the accumulators of every head: head g's factor is held by the lane of token 0
+    // that owns g after the reduce-scatter (all tokens hold the same maximum)
+#pragma unroll
+    for (int g = 0; g < GW; ++g) {
+      const float al = __shfl_sync(FULL, alpha[g % NF], rs_lane_of<LPT, GW>(g));
+#pragma unroll
+      for (int i = 0; i < T::E; ++i) w.O[g][i] *= al;
+    }
+  }
+  __syncwarp();                                        // the previous stage's p' has been read
+#pragma unroll
+  for (int ps = 0; ps < T::NPASS; ++ps) {
+    const int t = ps * T::TPP + tl;
+    const bool valid = !masked || (prow0 + t >= rv0 && prow0 + t < rv1);
+    float p[NF];
+#pragma unroll
+    for (int j = 0; j < NF; ++j) {
+      const float e2 = fast_exp2(sc[ps][j] - w.m[j]);
+      p[j] = valid ? e2 : 0.f;
+      w.l[j] += p[j];
+    }
+    float pa[GW];
+#pragma unroll
+    for (int g = 0; g < GW; ++g) pa[g] = __shfl_sync(FULL, p[g % NF], (lane & ~(LPT - 1)) | rs_lane_of<LPT, GW>(g));
+    const float dv =
+        valid ? __half2float(*reinterpret_cast<const __half*>(st + T::OFF_VS + (prow0 + t) * T::S_ROW + 2 * blk)) : 0.f;
+    float* dst = pb + (t * NB + blk) * GW;
+    if constexpr (GW == 4) {
+      *reinterpret_cast<float4*>(dst) = make_float4(pa[0] * dv, pa[1] * dv, pa[2] * dv, pa[3] * dv);
+    } else if constexpr (GW == 2) {
+      *reinterpret_cast<float2*>(dst) = make_float2(pa[0] * dv, pa[1] * dv);
+    } else {
+      *dst = pa[0] * dv;
+    }
+  }
+  __syncwarp();
+}
+
+// Consumer warp: for each item segment of the CTA's range, the query digits, then the
+// stage pipeline (scores of stage k with the values of stage k - 1), then the merge.
+template <int KB, int VB, int D, int G>
+__device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch& b, const QDecSmem<KB, VB, D, G>& sm,
+                                              int64_t x0, int64_t x1) {
+  using T = QDec<KB, VB, D, G>;
+  constexpr int S = T::S, GW = T::GW, NF = T::NF, LPT = T::LPT, NHG = T::NHG, E = T::E;
   constexpr uint32_t FULL = 0xffffffffu;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int part = warp / NHG, hg = warp % NHG;
-  const int tl = lane / LPT, half = lane % LPT;        // lane = tl * LPT + half: blocks 2 half, 2 half + 1
-  const int fmap = rs_map<LPT, GW>(half);
-  const int xr = kq2_rot<KB, D>(tl);
-  const int bswap = KB == 8 ? (xr >> 1) : xr;          // slot sp holds block 2 half + (sp ^ bswap)
-  uint32_t it = 0, itm = 0, itw = 0, itc = 0;
+  const int prow0 = part * T::W;
+  const int tl = lane / LPT, blk = lane % LPT;         // score lane: token tl of a pass, key block blk
+  const int tv = lane / T::LPV, sl = lane % T::LPV;    // value lane: token tv of a pass, element slot sl
+  const int fmap = rs_map<LPT, GW>(blk);
+  const int xr = kq_rot<KB, D>(tl);
+  float* pb = sm.pbuf + warp * (T::W * T::NB * GW);
+  QWarp<KB, VB, D, G> w;
+  uint32_t itm = 0, itw = 0, itc = 0;
+  int s = 0;                                           // ring slot of the next stage and its fill parity
+  uint32_t ph = 0;
   for (int64_t x = x0; x < x1;) {
     const DecodeSeg sg = decode_find_seg(b, x, x1);
     const SeqDesc sd = b.s[sg.bi];
-    // ---- query digits in permuted slots: slot j <-> head hg * GW + (j ^ fmap), this lane's two blocks.
-    // The warp's GW query rows are staged in shared memory with 16-byte loads, then each lane reads its
-    // elements in its own (bank-rotated) word order from there.
+    // ---- query digits in permuted slots: slot j <-> head hg * GW + (j ^ fmap), this lane's block.
+    // The warp's GW query rows are staged in shared memory with 16-byte loads, then each lane reads
+    // its elements in its own (bank-rotated) word order from there.
     __half* qs = sm.qbuf + warp * GW * D;
     {
       const uint4* src = reinterpret_cast<const uint4*>(a.q + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + hg * GW) * D);
@@ -532,10 +693,10 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
     float amax[GW];
 #pragma unroll
     for (int j = 0; j < GW; ++j) {
-      const uint4* qr = reinterpret_cast<const uint4*>(qs + (j ^ fmap) * D + 64 * half);
+      const uint4* qr = reinterpret_cast<const uint4*>(qs + (j ^ fmap) * D + 32 * blk);
       float mx = 0.f;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         const uint4 w4 = qr[c];
         const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
@@ -558,170 +719,80 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
     }
     // n = rint(q / s) with s = max|q| / 32512 (|n| <= 32512), as hi = (n + 128) >> 8 and the low byte
     // lo = n mod 256 read as int8, so that n = 256 hi + lo
-    uint32_t qh[GW][16], ql[GW][16];
-    int qcorr[GW][2];
 #pragma unroll
     for (int j = 0; j < GW; ++j) {
-      const __half* qr = qs + (j ^ fmap) * D + 64 * half;
+      const __half* qb = qs + (j ^ fmap) * D + 32 * blk;
       const float mul = amax[j] > 0.f ? a.scale_log2 * (32512.f / amax[j]) : 0.f;
+      int corr = 0;
 #pragma unroll
-      for (int sp = 0; sp < 2; ++sp) {
-        const __half* qb = qr + 32 * (sp ^ bswap);
-        int corr = 0;
+      for (int k = 0; k < 8; ++k) {
+        // the word's 4 elements are consecutive in the row
+        const uint2 h4 = *reinterpret_cast<const uint2*>(qb + kq_elem<KB>(k, 0, xr));
+        const float2 f01 = h2_to_f2(h4.x), f23 = h2_to_f2(h4.y);
+        int n[4];
+        n[0] = __float_as_int(fmaf(f01.x, mul, 12582912.f)) - 0x4B400000;   // round to nearest
+        n[1] = __float_as_int(fmaf(f01.y, mul, 12582912.f)) - 0x4B400000;
+        n[2] = __float_as_int(fmaf(f23.x, mul, 12582912.f)) - 0x4B400000;
+        n[3] = __float_as_int(fmaf(f23.y, mul, 12582912.f)) - 0x4B400000;
 #pragma unroll
-        for (int w = 0; w < 8; ++w) {
-          // the word's 4 elements are consecutive in the row
-          const uint2 h4 = *reinterpret_cast<const uint2*>(qb + kq2_elem<KB>(w, 0, xr));
-          const float2 f01 = h2_to_f2(h4.x), f23 = h2_to_f2(h4.y);
-          int n[4];
-          n[0] = __float_as_int(fmaf(f01.x, mul, 12582912.f)) - 0x4B400000;   // round to nearest
-          n[1] = __float_as_int(fmaf(f01.y, mul, 12582912.f)) - 0x4B400000;
-          n[2] = __float_as_int(fmaf(f23.x, mul, 12582912.f)) - 0x4B400000;
-          n[3] = __float_as_int(fmaf(f23.y, mul, 12582912.f)) - 0x4B400000;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            n[e] = max(-32512, min(32512, n[e]));
-            corr += n[e];
-          }
-          ql[j][8 * sp + w] = __byte_perm(__byte_perm(n[0], n[1], 0x0040), __byte_perm(n[2], n[3], 0x0040), 0x5410);
-          const int h0 = (n[0] + 128) >> 8, h1 = (n[1] + 128) >> 8, h2 = (n[2] + 128) >> 8, h3 = (n[3] + 128) >> 8;
-          qh[j][8 * sp + w] = __byte_perm(__byte_perm(h0, h1, 0x0040), __byte_perm(h2, h3, 0x0040), 0x5410);
+        for (int e = 0; e < 4; ++e) {
+          n[e] = max(-32512, min(32512, n[e]));
+          corr += n[e];
         }
-        qcorr[j][sp] = KB == 4 ? -8 * corr : 0;          // 4-bit codes are read as u = c + 8
+        w.ql[j][k] = __byte_perm(__byte_perm(n[0], n[1], 0x0040), __byte_perm(n[2], n[3], 0x0040), 0x5410);
+        const int h0 = (n[0] + 128) >> 8, h1 = (n[1] + 128) >> 8, h2 = (n[2] + 128) >> 8, h3 = (n[3] + 128) >> 8;
+        w.qh[j][k] = __byte_perm(__byte_perm(h0, h1, 0x0040), __byte_perm(h2, h3, 0x0040), 0x5410);
       }
+      w.qcorr[j] = KB == 4 ? -8 * corr : 0;
     }
-    float qsc[NF], m_own[NF], l_own[NF];
 #pragma unroll
     for (int j = 0; j < NF; ++j) {                         // slot j < NF ends with head j ^ fmap
-      qsc[j] = amax[j] * (1.f / 32512.f);
-      m_own[j] = -INFINITY;
-      l_own[j] = 0.f;
+      w.qsc[j] = amax[j] * (1.f / 32512.f);
+      w.m[j] = -INFINITY;
+      w.l[j] = 0.f;
     }
+#pragma unroll
+    for (int g = 0; g < GW; ++g)
+#pragma unroll
+      for (int i = 0; i < E; ++i) w.O[g][i] = 0.f;
 
+    // ---- stage pipeline: chunk k's scores together with chunk k - 1's values
+    const int base_tok = sd.lo / a.chunk * a.chunk;        // chunks start at the window's first chunk
+    const uint8_t* st_prev = sm.stages;
+    int s_prev = 0;
     for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
-      const int s = it % S, par = it & 1;
-      const uint32_t pph = (it >> 1) & 1;
-      if (!mbar_wait(sm.full0 + 8 * s, (it / S) & 1, sm.abort_flag, a.L.wait_ns)) {
+      if (!mbar_wait(sm.full0 + 8 * s, ph, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 2);
         *sm.abort_flag = 1;
         return;
       }
       const uint8_t* st = sm.stages + s * T::STAGE;
-      const int tok0 = sd.lo / a.chunk * a.chunk + k * a.chunk;
+      const int tok0 = base_tok + k * a.chunk;
       const int rv0 = max(0, sd.lo - tok0), rv1 = min(a.chunk, sd.a - tok0);   // valid rows [rv0, rv1)
-      const int row0 = part * W;
-      const bool masked = rv0 > row0 || rv1 < row0 + W;
+      const bool masked = rv0 > prow0 || rv1 < prow0 + T::W;
       float sc[T::NPASS][NF];
-#pragma unroll
-      for (int ps = 0; ps < T::NPASS; ++ps) {
-        const int row = row0 + ps * T::TPP + tl;
-        uint32_t cw[16];
-        load_kq2<KB>(st + row * T::K_ROW + half * KSPAN, xr, cw);
-        const float2 dk2 = h2_to_f2(*reinterpret_cast<const uint32_t*>(st + T::OFF_KS + row * T::S_ROW + 4 * half));
-        const float dks0 = bswap ? dk2.y : dk2.x, dks1 = bswap ? dk2.x : dk2.y;
-        int hs[GW][2], ls[GW][2];
-#pragma unroll
-        for (int j = 0; j < GW; ++j) {
-          hs[j][0] = hs[j][1] = 0;
-          ls[j][0] = qcorr[j][0];
-          ls[j][1] = qcorr[j][1];
-        }
-#pragma unroll
-        for (int w = 0; w < 8; ++w)
-#pragma unroll
-          for (int sp = 0; sp < 2; ++sp)
-#pragma unroll
-            for (int j = 0; j < GW; ++j) {
-              hs[j][sp] = __dp4a(int(cw[8 * sp + w]), int(qh[j][8 * sp + w]), hs[j][sp]);
-              ls[j][sp] = __dp4a(int(cw[8 * sp + w]), int(ql[j][8 * sp + w]), ls[j][sp]);
-            }
-        float ps_[GW];
-#pragma unroll
-        for (int j = 0; j < GW; ++j)
-          ps_[j] = fmaf(__int2float_rn(hs[j][1] * 256 + ls[j][1]), dks1,
-                        __int2float_rn(hs[j][0] * 256 + ls[j][0]) * dks0);
-        reduce_scatter_perm<LPT, GW>(ps_);
-#pragma unroll
-        for (int j = 0; j < NF; ++j) {
-          const float v = ps_[j] * qsc[j];
-          sc[ps][j] = (!masked || (row >= rv0 && row < rv1)) ? v : -INFINITY;
-        }
+      if (k == sg.k0) {
+        qk_stage<KB, VB, D, G>(w, st, prow0, tl, blk, xr, masked, rv0, rv1, sc);
+      } else {
+        // one straight-line block: the previous stage's values and this stage's scores
+        pv_stage<KB, VB, D, G>(w, st_prev, pb, prow0, tv, sl);
+        qk_stage<KB, VB, D, G>(w, st, prow0, tl, blk, xr, masked, rv0, rv1, sc);
+        __syncwarp();
+        mbar_arrive_if(sm.empty0 + 8 * s_prev, lane == 0);
       }
-      // lazy maximum: moved only when a score passes it by 2^8
-      bool need = false;
-#pragma unroll
-      for (int ps = 0; ps < T::NPASS; ++ps)
-#pragma unroll
-        for (int j = 0; j < NF; ++j) need |= sc[ps][j] > m_own[j] + 8.f;
-      const bool any = __any_sync(FULL, need);
-      // the value warps must be done with this buffer (two stages back) before it is rewritten
-      if (!mbar_wait(sm.free0 + 8 * (part * 2 + par), pph ^ 1, sm.abort_flag, a.L.wait_ns)) {
-        if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 3);
-        *sm.abort_flag = 1;
-        return;
+      softmax_stage<KB, VB, D, G>(w, sc, st, pb, prow0, tl, blk, masked, rv0, rv1);
+      st_prev = st;
+      s_prev = s;
+      if (++s == S) {
+        s = 0;
+        ph ^= 1;
       }
-      if (any) {
-        float alpha[NF];
-#pragma unroll
-        for (int j = 0; j < NF; ++j) {
-          float mx = sc[0][j];
-#pragma unroll
-          for (int ps = 1; ps < T::NPASS; ++ps) mx = fmaxf(mx, sc[ps][j]);
-#pragma unroll
-          for (int o = LPT; o < 32; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
-          const float mn = fmaxf(m_own[j], mx);
-          alpha[j] = fast_exp2(m_own[j] - mn);           // 0 while m_own is -inf
-          m_own[j] = mn;
-          l_own[j] *= alpha[j];
-        }
-        if (tl == 0) {
-#pragma unroll
-          for (int j = 0; j < NF; ++j) sm.palpha[(part * 2 + par) * G + hg * GW + (j ^ fmap)] = alpha[j];
-        }
-      }
-      if (lane == 0) sm.pflag[(part * 2 + par) * NHG + hg] = any ? 1 : 0;
-      // p, and p' = p d_v of this lane's two value blocks for the group's GW heads
-      float* pb = sm.pbuf + (part * 2 + par) * (W * NB * G);
-#pragma unroll
-      for (int ps = 0; ps < T::NPASS; ++ps) {
-        const int t = ps * T::TPP + tl;
-        const bool valid = !masked || (row0 + t >= rv0 && row0 + t < rv1);
-        float p[NF];
-#pragma unroll
-        for (int j = 0; j < NF; ++j) {
-          const float e2 = fast_exp2(sc[ps][j] - m_own[j]);
-          p[j] = valid ? e2 : 0.f;
-          l_own[j] += p[j];
-        }
-        float pa[GW];
-#pragma unroll
-        for (int g = 0; g < GW; ++g) {
-          if constexpr (LPT == 1) pa[g] = p[g];           // this lane holds every head (slot g = head g)
-          else pa[g] = __shfl_sync(FULL, p[g % NF], (lane & ~(LPT - 1)) | rs_lane_of<LPT, GW>(g));
-        }
-        float2 dv2 = h2_to_f2(*reinterpret_cast<const uint32_t*>(st + T::OFF_VS + (row0 + t) * T::S_ROW + 4 * half));
-        if (!valid) dv2 = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const float dv = bb ? dv2.y : dv2.x;
-          float* dst = pb + (t * NB + 2 * half + bb) * G + hg * GW;
-          if constexpr (GW == 4) {
-            *reinterpret_cast<float4*>(dst) = make_float4(pa[0] * dv, pa[1] * dv, pa[2] * dv, pa[3] * dv);
-          } else if constexpr (GW == 2) {
-            *reinterpret_cast<float2*>(dst) = make_float2(pa[0] * dv, pa[1] * dv);
-          } else {
-            *dst = pa[0] * dv;
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(sm.ready0 + 8 * (part * 2 + par));
-        mbar_arrive(sm.empty0 + 8 * s);
-      }
-      ++it;
     }
-    // ---- publish (m, l) of this partition's heads, then merge
+    pv_stage<KB, VB, D, G>(w, st_prev, pb, prow0, tv, sl);
+    __syncwarp();
+    mbar_arrive_if(sm.empty0 + 8 * s_prev, lane == 0);
+
+    // ---- publish (m, l) of the owned heads and O of all the warp's heads, then merge
     if (!mbar_wait(sm.mfree, (itm & 1) ^ 1, sm.abort_flag, a.L.wait_ns)) {
       if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 5);
       *sm.abort_flag = 1;
@@ -730,146 +801,27 @@ __device__ __forceinline__ void score_role(const DecodeQArgs& a, const Batch& b,
 #pragma unroll
     for (int j = 0; j < NF; ++j)
 #pragma unroll
-      for (int o = LPT; o < 32; o <<= 1) l_own[j] += __shfl_xor_sync(FULL, l_own[j], o);
+      for (int o = LPT; o < 32; o <<= 1) w.l[j] += __shfl_xor_sync(FULL, w.l[j], o);
     if (tl == 0) {
 #pragma unroll
       for (int j = 0; j < NF; ++j) {
         const int g = hg * GW + (j ^ fmap);
-        sm.mrg_ml[(part * G + g) * 2] = m_own[j];
-        sm.mrg_ml[(part * G + g) * 2 + 1] = l_own[j];
+        sm.mrg_ml[(part * G + g) * 2] = w.m[j];
+        sm.mrg_ml[(part * G + g) * 2 + 1] = w.l[j];
       }
-    }
-    if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw, itc)) return;
-    x += sg.n;
-  }
-}
-
-// Value warp: O += p' c over its share of the partition's tokens.
-template <int KB, int VB, int D, int G>
-__device__ __forceinline__ void value_role(const DecodeQArgs& a, const Batch& b, const QDecSmem<KB, VB, D, G>& sm,
-                                           int64_t x0, int64_t x1) {
-  using T = QDec<KB, VB, D, G>;
-  constexpr int S = T::S, W = T::W, NB = T::NB, GW = T::GW, NHG = T::NHG, E = T::E;
-  constexpr uint32_t FULL = 0xffffffffu;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int vw_ = warp - T::NS;
-  const int part = vw_ / T::NPP, pw = vw_ % T::NPP;
-  const int tv = lane / T::LPV, sl = lane % T::LPV;    // lane = tv * LPV + sl
-  uint32_t it = 0, itm = 0, itw = 0, itc = 0;
-  for (int64_t x = x0; x < x1;) {
-    const DecodeSeg sg = decode_find_seg(b, x, x1);
-    const SeqDesc sd = b.s[sg.bi];
-    float O[G][E];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int i = 0; i < E; ++i) O[g][i] = 0.f;
-    for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
-      const int s = it % S, par = it & 1;
-      const uint32_t pph = (it >> 1) & 1;
-      if (!mbar_wait(sm.full0 + 8 * s, (it / S) & 1, sm.abort_flag, a.L.wait_ns) ||
-          !mbar_wait(sm.ready0 + 8 * (part * 2 + par), pph, sm.abort_flag, a.L.wait_ns)) {
-        if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 4);
-        *sm.abort_flag = 1;
-        return;
-      }
-      const uint8_t* st = sm.stages + s * T::STAGE;
-      const float* pb = sm.pbuf + (part * 2 + par) * (W * NB * G);
-#pragma unroll
-      for (int h2 = 0; h2 < NHG; ++h2) {
-        if (sm.pflag[(part * 2 + par) * NHG + h2]) {       // that head group moved its maximum
-#pragma unroll
-          for (int g = 0; g < GW; ++g) {
-            const float al = sm.palpha[(part * 2 + par) * G + h2 * GW + g];
-#pragma unroll
-            for (int i = 0; i < E; ++i) O[h2 * GW + g][i] *= al;
-          }
-        }
-      }
-      const int t0 = pw * T::WP;                            // this warp's first token in the partition
-#pragma unroll 2
-      for (int pv = 0; pv < T::NPV; ++pv) {
-        const int tloc = t0 + pv * T::TPV + tv;
-        const uint8_t* vrow = st + T::OFF_VC + (part * W + tloc) * T::V_ROW + sl * T::BPL;
-        uint32_t vw[T::BPL / 4];
-        if constexpr (T::BPL == 4) {
-          vw[0] = *reinterpret_cast<const uint32_t*>(vrow);
-        } else if constexpr (T::BPL == 8) {
-          const uint2 u = *reinterpret_cast<const uint2*>(vrow);
-          vw[0] = u.x;
-          vw[1] = u.y;
-        } else {
-#pragma unroll
-          for (int c = 0; c < T::BPL / 16; ++c) {
-            const uint4 u = reinterpret_cast<const uint4*>(vrow)[c];
-            vw[4 * c] = u.x; vw[4 * c + 1] = u.y; vw[4 * c + 2] = u.z; vw[4 * c + 3] = u.w;
-          }
-        }
-#pragma unroll
-        for (int bl = 0; bl < T::NBL; ++bl) {
-          const int vblk = (sl * T::BPL) / T::VBLK + bl;
-          const float* pp = pb + (tloc * NB + vblk) * G;
-          float pg[G];
-          if constexpr (G >= 4) {
-#pragma unroll
-            for (int c = 0; c < G / 4; ++c) {
-              const float4 f = reinterpret_cast<const float4*>(pp)[c];
-              pg[4 * c] = f.x; pg[4 * c + 1] = f.y; pg[4 * c + 2] = f.z; pg[4 * c + 3] = f.w;
-            }
-          } else if constexpr (G == 2) {
-            const float2 f = *reinterpret_cast<const float2*>(pp);
-            pg[0] = f.x;
-            pg[1] = f.y;
-          } else {
-            pg[0] = *pp;
-          }
-          constexpr int WPB = (T::BPL / T::NBL) / 4;      // code words of one value block in this lane
-#pragma unroll
-          for (int wq = 0; wq < WPB; ++wq) {
-            const int wi = bl * WPB + wq;
-            if constexpr (VB == 4) {
-              float f[8];
-              cvt_v4_word(vw[wi], f);
-#pragma unroll
-              for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) O[g][8 * wi + e] = fmaf(pg[g], f[e], O[g][8 * wi + e]);
-            } else {
-              float f[4];
-              cvt_v8_word(vw[wi], f);
-#pragma unroll
-              for (int g = 0; g < G; ++g)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) O[g][4 * wi + e] = fmaf(pg[g], f[e], O[g][4 * wi + e]);
-            }
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(sm.free0 + 8 * (part * 2 + par));
-        mbar_arrive(sm.empty0 + 8 * s);
-      }
-      ++it;
-    }
-    // ---- publish this warp's O (summed over its token lanes), then merge
-    if (!mbar_wait(sm.mfree, (itm & 1) ^ 1, sm.abort_flag, a.L.wait_ns)) {
-      if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 5);
-      *sm.abort_flag = 1;
-      return;
     }
 #pragma unroll
     for (int o = T::LPV; o < 32; o <<= 1)
 #pragma unroll
-      for (int g = 0; g < G; ++g)
+      for (int g = 0; g < GW; ++g)
 #pragma unroll
-        for (int i = 0; i < E; ++i) O[g][i] += __shfl_xor_sync(FULL, O[g][i], o);
+        for (int i = 0; i < E; ++i) w.O[g][i] += __shfl_xor_sync(FULL, w.O[g][i], o);
     if (tv == 0) {
-      float* mo = sm.mrg_o + vw_ * G * D;
+      float* mo = sm.mrg_o + (part * G + hg * GW) * D;
 #pragma unroll
-      for (int g = 0; g < G; ++g)
+      for (int g = 0; g < GW; ++g)
 #pragma unroll
-        for (int i = 0; i < E; ++i) mo[g * D + v_elem_of<VB, E>(sl, i)] = O[g][i];
+        for (int i = 0; i < E; ++i) mo[g * D + v_elem_of<VB, E>(sl, i)] = w.O[g][i];
     }
     if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw, itc)) return;
     x += sg.n;
@@ -885,17 +837,13 @@ __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::S; ++s) {
       mbar_init(sm.full0 + 8 * s, 1);
-      mbar_init(sm.empty0 + 8 * s, T::NCW);
+      mbar_init(sm.empty0 + 8 * s, T::NW);
     }
-    for (int i = 0; i < 2 * T::NPART; ++i) {
-      mbar_init(sm.ready0 + 8 * i, T::NHG);
-      mbar_init(sm.free0 + 8 * i, T::NPP);
-    }
-    mbar_init(sm.mfull, T::NCW);
-    mbar_init(sm.mfree, T::NCW);
-    mbar_init(sm.mws, T::NCW);
+    mbar_init(sm.mfull, T::NW);
+    mbar_init(sm.mfree, T::NW);
+    mbar_init(sm.mws, T::NW);
     mbar_init(sm.mlast, 1);
-    mbar_init(sm.mcomb, T::NCW);
+    mbar_init(sm.mcomb, T::NW);
     *sm.abort_flag = 0;
     fence_mbar_init();
   }
@@ -903,20 +851,8 @@ __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
   const int warp = threadIdx.x >> 5;
   const int64_t x0 = int64_t(blockIdx.x) * a.cpc;
   const int64_t x1 = min(a.total_chunks, x0 + a.cpc);
-  // register split by warpgroup: the producer group gives registers back first, then the
-  // score group (query digits in registers) takes more; the value groups keep theirs
-  if (warp >= T::NCW) {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(T::REG_P));
-    if (warp == T::NCW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1);
-    return;                                                 // the group's other 3 warps have no role
-  }
-  if (warp < T::NS) {
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(T::REG_S));
-    score_role<KB, VB, D, G>(a, b, sm, x0, x1);
-  } else {
-    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(T::REG_V));
-    value_role<KB, VB, D, G>(a, b, sm, x0, x1);
-  }
+  if (warp == T::NW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1);
+  else consumer_role<KB, VB, D, G>(a, b, sm, x0, x1);
 }
 
 }  // namespace kvq

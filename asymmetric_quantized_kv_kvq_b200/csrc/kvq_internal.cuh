@@ -146,6 +146,9 @@ struct DecodePlan {
 
 // decode: workspace = partial slots [(max_ctas + n_items)][G][D + 2] fp32
 size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D);
+// Decode grids have at most one CTA per SM and never more than kMaxDecodeCtas (the
+// in-kernel merge of a split item keeps one weight per CTA in shared memory).
+constexpr int kMaxDecodeCtas = 256;
 int decode_max_ctas(int num_sms);
 int decode_chunk_tokens(const Layout& L, int G);
 // k_new / v_new: fp16 [B, Hkv, D] rows of position len - 1 to quantise into the
