@@ -47,6 +47,12 @@ cudaError_t launch_decode_q_one(const Layout& L, int layer, const Batch& b, cons
     cudaError_t e = cudaFuncSetAttribute(decode_q_kernel<KB, VB, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          T::SMEM);
     if (e != cudaSuccess) return e;
+    // the in-kernel register split (setmaxnreg) adds up to the launch allocation; a build that
+    // launched with fewer registers per thread would leave a growing warpgroup waiting
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, decode_q_kernel<KB, VB, D, G>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != T::REG_L) return cudaErrorInvalidDeviceFunction;
     configured = true;
   }
   DecodeQArgs a;

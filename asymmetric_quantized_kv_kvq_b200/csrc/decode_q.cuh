@@ -91,7 +91,8 @@ struct QDec {
   static constexpr int LPV = D / E;                  // value lanes per token
   static constexpr int TPV = 32 / LPV;               // tokens per value pass
   static constexpr int NPV = W / TPV;                // value passes per stage
-  static constexpr int NT = (NW + 1) * 32;
+  static constexpr int NT = (NW + 4) * 32;
+  static constexpr int REG_L = 168, REG_C = 216, REG_P = 72;
   static constexpr int K_ROW = KB == 8 ? D : D / 2;
   static constexpr int V_ROW = VB == 8 ? D : D / 2;
   static constexpr int KBLK = K_ROW / NB;            // code bytes of one key block
@@ -177,23 +178,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // A score lane reads the codes of its key block: 8-bit codes as two 16-byte
 // chunks, chunk c ^ x at load step c (x depends on the lane's token, so that
 // the 16-byte loads of a warp spread over all shared-memory banks); 4-bit codes
-// as one 16-byte chunk, unpacked to one byte per code (0..15).  Byte e of word w
-// is then element kq_elem(w, e, x) of the block.
-template <int KB>
-__device__ __forceinline__ void load_kq(const uint8_t* blk, int x, uint32_t (&cw)[8]) {
-  if constexpr (KB == 8) {
-#pragma unroll
-    for (int c = 0; c < 2; ++c) {
-      const uint4 a = *reinterpret_cast<const uint4*>(blk + 16 * (c ^ x));
-      cw[4 * c] = a.x; cw[4 * c + 1] = a.y; cw[4 * c + 2] = a.z; cw[4 * c + 3] = a.w;
-    }
-  } else {
-    const uint4 a = *reinterpret_cast<const uint4*>(blk);
-    cw[0] = a.x & 0x0F0F0F0Fu; cw[1] = a.y & 0x0F0F0F0Fu; cw[2] = a.z & 0x0F0F0F0Fu; cw[3] = a.w & 0x0F0F0F0Fu;
-    cw[4] = (a.x >> 4) & 0x0F0F0F0Fu; cw[5] = (a.y >> 4) & 0x0F0F0F0Fu;
-    cw[6] = (a.z >> 4) & 0x0F0F0F0Fu; cw[7] = (a.w >> 4) & 0x0F0F0F0Fu;
-  }
-}
+// as one 16-byte chunk, unpacked to one byte per code (0..15: words 0..3 the low
+// nibbles, 4..7 the high nibbles).  Byte e of word w is then element
+// kq_elem(w, e, x) of the block.
 template <int KB>
 __host__ __device__ constexpr int kq_elem(int w, int e, int x) {
   if (KB == 8) return 16 * ((w >> 2) ^ x) + 4 * (w & 3) + e;
@@ -492,20 +479,39 @@ struct QWarp {
   float O[T::GW][T::E];                  // value lane's accumulators, all of the warp's heads
 };
 
+// Per-lane byte offsets (pass 0) inside a stage and inside the warp's p' buffer; the other
+// passes add compile-time constants, so every shared-memory access is one 32-bit register plus
+// an immediate.
+struct QLaneOff {
+  uint32_t kc0, kc1;   // key codes of the lane's block: its first and second 16-byte chunk (8-bit keys)
+  uint32_t ks, vs;     // K and V scale of the lane's block (score-lane layout)
+  uint32_t vc;         // V codes of the value lane
+  uint32_t pst, pld;   // p' store (score-lane layout) and load (value-lane layout)
+};
+
 // Score passes of one stage: sc[pass][j] for the lane's token and owned heads (-inf outside
-// the valid rows [rv0, rv1) of the chunk).
+// the valid rows [rv0, rv1) of the chunk; row0 = the lane's row in pass 0).
 template <int KB, int VB, int D, int G>
-__device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G>& w, const uint8_t* st, int prow0, int tl, int blk,
-                                         int xr, bool masked, int rv0, int rv1,
+__device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G>& w, uint32_t u_st, const QLaneOff& lo, int row0,
+                                         bool masked, int rv0, int rv1,
                                          float (&sc)[QDec<KB, VB, D, G>::NPASS][QDec<KB, VB, D, G>::NF]) {
   using T = QDec<KB, VB, D, G>;
   constexpr int GW = T::GW, NF = T::NF;
 #pragma unroll
   for (int ps = 0; ps < T::NPASS; ++ps) {
-    const int row = prow0 + ps * T::TPP + tl;
     uint32_t cw[8];
-    load_kq<KB>(st + row * T::K_ROW + blk * T::KBLK, xr, cw);
-    const float dk = __half2float(*reinterpret_cast<const __half*>(st + T::OFF_KS + row * T::S_ROW + 2 * blk));
+    if constexpr (KB == 8) {
+      const uint4 c0 = lds_v4(u_st + lo.kc0 + ps * T::TPP * T::K_ROW);
+      const uint4 c1 = lds_v4(u_st + lo.kc1 + ps * T::TPP * T::K_ROW);
+      cw[0] = c0.x; cw[1] = c0.y; cw[2] = c0.z; cw[3] = c0.w;
+      cw[4] = c1.x; cw[5] = c1.y; cw[6] = c1.z; cw[7] = c1.w;
+    } else {
+      const uint4 c = lds_v4(u_st + lo.kc0 + ps * T::TPP * T::K_ROW);
+      cw[0] = c.x & 0x0F0F0F0Fu; cw[1] = c.y & 0x0F0F0F0Fu; cw[2] = c.z & 0x0F0F0F0Fu; cw[3] = c.w & 0x0F0F0F0Fu;
+      cw[4] = (c.x >> 4) & 0x0F0F0F0Fu; cw[5] = (c.y >> 4) & 0x0F0F0F0Fu;
+      cw[6] = (c.z >> 4) & 0x0F0F0F0Fu; cw[7] = (c.w >> 4) & 0x0F0F0F0Fu;
+    }
+    const float dk = h_bits_to_f(lds_u16(u_st + lo.ks + ps * T::TPP * T::S_ROW));
     int hs[GW], ls[GW];
 #pragma unroll
     for (int j = 0; j < GW; ++j) {
@@ -523,6 +529,7 @@ __device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G>& w, const uin
 #pragma unroll
     for (int j = 0; j < GW; ++j) ps_[j] = __int2float_rn(hs[j] * 256 + ls[j]) * dk;
     reduce_scatter_perm<T::LPT, GW>(ps_);
+    const int row = row0 + ps * T::TPP;
 #pragma unroll
     for (int j = 0; j < NF; ++j) {
       const float v = ps_[j] * w.qsc[j];
@@ -533,40 +540,37 @@ __device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G>& w, const uin
 
 // Value passes of one stage: O += p' c over the lane's tokens of the partition.
 template <int KB, int VB, int D, int G>
-__device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G>& w, const uint8_t* st, const float* pb, int prow0, int tv,
-                                         int sl) {
+__device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G>& w, uint32_t u_st, uint32_t u_pb, const QLaneOff& lo) {
   using T = QDec<KB, VB, D, G>;
   constexpr int GW = T::GW, NB = T::NB;
-  const int vblk = (sl * T::BPL) / T::VBLK;
 #pragma unroll
   for (int pv = 0; pv < T::NPV; ++pv) {
-    const int t = pv * T::TPV + tv;
-    const uint8_t* vrow = st + T::OFF_VC + (prow0 + t) * T::V_ROW + sl * T::BPL;
+    const uint32_t va = u_st + lo.vc + pv * T::TPV * T::V_ROW;
     uint32_t vw[T::BPL / 4];
     if constexpr (T::BPL == 4) {
-      vw[0] = *reinterpret_cast<const uint32_t*>(vrow);
+      vw[0] = lds_u32(va);
     } else if constexpr (T::BPL == 8) {
-      const uint2 u = *reinterpret_cast<const uint2*>(vrow);
+      const uint2 u = lds_v2(va);
       vw[0] = u.x;
       vw[1] = u.y;
     } else {
 #pragma unroll
       for (int c = 0; c < T::BPL / 16; ++c) {
-        const uint4 u = reinterpret_cast<const uint4*>(vrow)[c];
+        const uint4 u = lds_v4(va + 16 * c);
         vw[4 * c] = u.x; vw[4 * c + 1] = u.y; vw[4 * c + 2] = u.z; vw[4 * c + 3] = u.w;
       }
     }
-    const float* pp = pb + (t * NB + vblk) * GW;
+    const uint32_t pa = u_pb + lo.pld + pv * T::TPV * NB * GW * 4;
     float pg[GW];
     if constexpr (GW == 4) {
-      const float4 f = *reinterpret_cast<const float4*>(pp);
+      const float4 f = lds_f4(pa);
       pg[0] = f.x; pg[1] = f.y; pg[2] = f.z; pg[3] = f.w;
     } else if constexpr (GW == 2) {
-      const float2 f = *reinterpret_cast<const float2*>(pp);
+      const float2 f = lds_f2(pa);
       pg[0] = f.x;
       pg[1] = f.y;
     } else {
-      pg[0] = *pp;
+      pg[0] = lds_f32(pa);
     }
 #pragma unroll
     for (int wi = 0; wi < T::BPL / 4; ++wi) {
@@ -594,7 +598,7 @@ __device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G>& w, const uint8_t* 
 template <int KB, int VB, int D, int G>
 __device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G>& w,
                                               const float (&sc)[QDec<KB, VB, D, G>::NPASS][QDec<KB, VB, D, G>::NF],
-                                              const uint8_t* st, float* pb, int prow0, int tl, int blk, bool masked,
+                                              uint32_t u_st, uint32_t u_pb, const QLaneOff& lo, int row0, bool masked,
                                               int rv0, int rv1) {
   using T = QDec<KB, VB, D, G>;
   constexpr int GW = T::GW, NF = T::NF, LPT = T::LPT, NB = T::NB;
@@ -632,8 +636,8 @@ __device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G>& w,
   __syncwarp();                                        // the previous stage's p' has been read
 #pragma unroll
   for (int ps = 0; ps < T::NPASS; ++ps) {
-    const int t = ps * T::TPP + tl;
-    const bool valid = !masked || (prow0 + t >= rv0 && prow0 + t < rv1);
+    const int row = row0 + ps * T::TPP;
+    const bool valid = !masked || (row >= rv0 && row < rv1);
     float p[NF];
 #pragma unroll
     for (int j = 0; j < NF; ++j) {
@@ -644,15 +648,15 @@ __device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G>& w,
     float pa[GW];
 #pragma unroll
     for (int g = 0; g < GW; ++g) pa[g] = __shfl_sync(FULL, p[g % NF], (lane & ~(LPT - 1)) | rs_lane_of<LPT, GW>(g));
-    const float dv =
-        valid ? __half2float(*reinterpret_cast<const __half*>(st + T::OFF_VS + (prow0 + t) * T::S_ROW + 2 * blk)) : 0.f;
-    float* dst = pb + (t * NB + blk) * GW;
+    const float dv0 = h_bits_to_f(lds_u16(u_st + lo.vs + ps * T::TPP * T::S_ROW));
+    const float dv = valid ? dv0 : 0.f;
+    const uint32_t dst = u_pb + lo.pst + ps * T::TPP * NB * GW * 4;
     if constexpr (GW == 4) {
-      *reinterpret_cast<float4*>(dst) = make_float4(pa[0] * dv, pa[1] * dv, pa[2] * dv, pa[3] * dv);
+      sts_f4(dst, pa[0] * dv, pa[1] * dv, pa[2] * dv, pa[3] * dv);
     } else if constexpr (GW == 2) {
-      *reinterpret_cast<float2*>(dst) = make_float2(pa[0] * dv, pa[1] * dv);
+      sts_f2(dst, pa[0] * dv, pa[1] * dv);
     } else {
-      *dst = pa[0] * dv;
+      sts_f32(dst, pa[0] * dv);
     }
   }
   __syncwarp();
@@ -673,7 +677,21 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
   const int tv = lane / T::LPV, sl = lane % T::LPV;    // value lane: token tv of a pass, element slot sl
   const int fmap = rs_map<LPT, GW>(blk);
   const int xr = kq_rot<KB, D>(tl);
-  float* pb = sm.pbuf + warp * (T::W * T::NB * GW);
+  const uint32_t u_stages = smem_u32(sm.stages);
+  const uint32_t u_pb = smem_u32(sm.pbuf + warp * (T::W * T::NB * GW));
+  QLaneOff lo;
+  {
+    const int row = prow0 + tl;                        // score lane's row in pass 0
+    const int vrow = prow0 + tv;                       // value lane's row in pass 0
+    lo.kc0 = uint32_t(row * T::K_ROW + blk * T::KBLK + 16 * xr);
+    lo.kc1 = uint32_t(row * T::K_ROW + blk * T::KBLK + 16 * (xr ^ 1));
+    lo.ks = uint32_t(T::OFF_KS + row * T::S_ROW + 2 * blk);
+    lo.vs = uint32_t(T::OFF_VS + row * T::S_ROW + 2 * blk);
+    lo.vc = uint32_t(T::OFF_VC + vrow * T::V_ROW + sl * T::BPL);
+    lo.pst = uint32_t((tl * T::NB + blk) * GW * 4);
+    lo.pld = uint32_t((tv * T::NB + (sl * T::BPL) / T::VBLK) * GW * 4);
+  }
+  const int row0 = prow0 + tl;
   QWarp<KB, VB, D, G> w;
   uint32_t itm = 0, itw = 0, itc = 0;
   int s = 0;                                           // ring slot of the next stage and its fill parity
@@ -758,7 +776,7 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
 
     // ---- stage pipeline: chunk k's scores together with chunk k - 1's values
     const int base_tok = sd.lo / a.chunk * a.chunk;        // chunks start at the window's first chunk
-    const uint8_t* st_prev = sm.stages;
+    uint32_t u_prev = u_stages;
     int s_prev = 0;
     for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
       if (!mbar_wait(sm.full0 + 8 * s, ph, sm.abort_flag, a.L.wait_ns)) {
@@ -766,29 +784,29 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
         *sm.abort_flag = 1;
         return;
       }
-      const uint8_t* st = sm.stages + s * T::STAGE;
+      const uint32_t u_st = u_stages + s * T::STAGE;
       const int tok0 = base_tok + k * a.chunk;
       const int rv0 = max(0, sd.lo - tok0), rv1 = min(a.chunk, sd.a - tok0);   // valid rows [rv0, rv1)
       const bool masked = rv0 > prow0 || rv1 < prow0 + T::W;
       float sc[T::NPASS][NF];
       if (k == sg.k0) {
-        qk_stage<KB, VB, D, G>(w, st, prow0, tl, blk, xr, masked, rv0, rv1, sc);
+        qk_stage<KB, VB, D, G>(w, u_st, lo, row0, masked, rv0, rv1, sc);
       } else {
         // one straight-line block: the previous stage's values and this stage's scores
-        pv_stage<KB, VB, D, G>(w, st_prev, pb, prow0, tv, sl);
-        qk_stage<KB, VB, D, G>(w, st, prow0, tl, blk, xr, masked, rv0, rv1, sc);
+        qk_stage<KB, VB, D, G>(w, u_st, lo, row0, masked, rv0, rv1, sc);
+        pv_stage<KB, VB, D, G>(w, u_prev, u_pb, lo);
         __syncwarp();
         mbar_arrive_if(sm.empty0 + 8 * s_prev, lane == 0);
       }
-      softmax_stage<KB, VB, D, G>(w, sc, st, pb, prow0, tl, blk, masked, rv0, rv1);
-      st_prev = st;
+      softmax_stage<KB, VB, D, G>(w, sc, u_st, u_pb, lo, row0, masked, rv0, rv1);
+      u_prev = u_st;
       s_prev = s;
       if (++s == S) {
         s = 0;
         ph ^= 1;
       }
     }
-    pv_stage<KB, VB, D, G>(w, st_prev, pb, prow0, tv, sl);
+    pv_stage<KB, VB, D, G>(w, u_prev, u_pb, lo);
     __syncwarp();
     mbar_arrive_if(sm.empty0 + 8 * s_prev, lane == 0);
 
@@ -828,6 +846,15 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
   }
 }
 
+// Per-warpgroup register count after launch: setmaxnreg.inc to grow, .dec to shrink (the
+// direction must match, and every warp of the warpgroup executes it).
+template <int R, int R_LAUNCH>
+__device__ __forceinline__ void set_max_regs() {
+  static_assert(R % 8 == 0 && R >= 24 && R <= 256, "setmaxnreg range");
+  if constexpr (R > R_LAUNCH) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(R));
+  else if constexpr (R < R_LAUNCH) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
+}
+
 template <int KB, int VB, int D, int G>
 __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
     decode_q_kernel(const DecodeQArgs a, const __grid_constant__ Batch b) {
@@ -851,8 +878,13 @@ __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
   const int warp = threadIdx.x >> 5;
   const int64_t x0 = int64_t(blockIdx.x) * a.cpc;
   const int64_t x1 = min(a.total_chunks, x0 + a.cpc);
-  if (warp == T::NW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1);
-  else consumer_role<KB, VB, D, G>(a, b, sm, x0, x1);
+  if (warp >= T::NW) {
+    set_max_regs<T::REG_P, T::REG_L>();
+    if (warp == T::NW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1);
+    return;                                                 // the group's other 3 warps have no role
+  }
+  set_max_regs<T::REG_C, T::REG_L>();
+  consumer_role<KB, VB, D, G>(a, b, sm, x0, x1);
 }
 
 }  // namespace kvq
