@@ -43,7 +43,8 @@
 //    warp-private buffer;
 //  - values: a lane owns E elements of one token; each code is converted to
 //    fp32 exactly once (a byte placed in the mantissa of 2^23, then one
-//    subtraction per pair) and feeds all of the warp's heads, one scalar FMA each.
+//    subtraction per pair) and feeds all of the warp's heads; the FMAs are
+//    packed two elements at a time (fma.rn.f32x2).
 // Every wait is bounded: on expiry the kernel records an error code, raises a
 // CTA-wide abort flag, drains its own copies and returns.
 #pragma once
@@ -538,6 +539,14 @@ __device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G>& w, uint32_t 
   }
 }
 
+// (o0, o1) += p (x0, x1) as one packed fp32 FMA (two correctly rounded FMAs: the same result as
+// two scalar ones, in half the issue slots).
+__device__ __forceinline__ void fma_pair(float& o0, float& o1, float p, float x0, float x1) {
+  const float2 r = ffma2(make_float2(p, p), make_float2(x0, x1), make_float2(o0, o1));
+  o0 = r.x;
+  o1 = r.y;
+}
+
 // Value passes of one stage: O += p' c over the lane's tokens of the partition.
 template <int KB, int VB, int D, int G>
 __device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G>& w, uint32_t u_st, uint32_t u_pb, const QLaneOff& lo) {
@@ -580,14 +589,14 @@ __device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G>& w, uint32_t u_st, 
 #pragma unroll
         for (int g = 0; g < GW; ++g)
 #pragma unroll
-          for (int e = 0; e < 8; ++e) w.O[g][8 * wi + e] = fmaf(pg[g], f[e], w.O[g][8 * wi + e]);
+          for (int e = 0; e < 8; e += 2) fma_pair(w.O[g][8 * wi + e], w.O[g][8 * wi + e + 1], pg[g], f[e], f[e + 1]);
       } else {
         float f[4];
         cvt_v8_word(vw[wi], f);
 #pragma unroll
         for (int g = 0; g < GW; ++g)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) w.O[g][4 * wi + e] = fmaf(pg[g], f[e], w.O[g][4 * wi + e]);
+          for (int e = 0; e < 4; e += 2) fma_pair(w.O[g][4 * wi + e], w.O[g][4 * wi + e + 1], pg[g], f[e], f[e + 1]);
       }
     }
   }
