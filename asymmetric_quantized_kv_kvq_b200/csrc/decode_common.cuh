@@ -26,10 +26,13 @@ struct DecodeArgs {
 };
 
 struct DecodeSeg {
-  int bi, h, k0, n;
+  int bi, h, k0, n;   // n: chunks holding tokens to process (0 inside an item's padding)
+  int adv;            // flat positions the segment covers (n plus the padding after it)
 };
 
-// Segment of the flat chunk list starting at x: (sequence, head, first chunk, count).
+// Segment of the flat chunk list starting at x: (sequence, head, first chunk, count).  An
+// item may be padded to a whole number of CTA ranges, so that no range crosses an item; the
+// padded chunks hold no tokens and are skipped (n counts only the real ones, adv all).
 __device__ __forceinline__ DecodeSeg decode_find_seg(const Batch& b, int64_t x, int64_t x1) {
   int lo = 0, hi = b.n - 1;
   while (lo < hi) {
@@ -41,7 +44,10 @@ __device__ __forceinline__ DecodeSeg decode_find_seg(const Batch& b, int64_t x, 
   const int h = int(rel / nch);
   const int k0 = int(rel - int64_t(h) * nch);
   const int64_t item_end = b.s[lo].b + int64_t(h + 1) * nch;
-  return {lo, h, k0, int((x1 < item_end ? x1 : item_end) - x)};
+  const int adv = int((x1 < item_end ? x1 : item_end) - x);
+  const int real = b.s[lo].cr > 0 ? b.s[lo].cr : nch;
+  const int n = real - k0 < adv ? (real - k0 > 0 ? real - k0 : 0) : adv;
+  return {lo, h, k0, n, adv};
 }
 
 // ---- value codes on CUDA cores ------------------------------------------------

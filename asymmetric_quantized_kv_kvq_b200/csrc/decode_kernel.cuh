@@ -255,8 +255,8 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         if ((it & 31) == 0) {
           const int64_t xl = x0 + it + lane;
           my_page = -1;
-          if (xl < x1) {
-            const DecodeSeg gl = decode_find_seg(b, xl, x1);
+          const DecodeSeg gl = xl < x1 ? decode_find_seg(b, xl, x1) : DecodeSeg{0, 0, 0, 0, 0};
+          if (gl.n > 0) {                                   // a chunk that holds tokens
             const SeqDesc dl = b.s[gl.bi];
             const int t0 = dl.lo / a.chunk * a.chunk + gl.k0 * a.chunk;
             my_page = a.L.page_table[int64_t(dl.seq_id) * a.L.max_pages_per_seq + page_slot(t0 / a.L.page_tokens, dl.ring)];
@@ -291,7 +291,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         }
         ++it;
       }
-      x += sg.n;
+      x += sg.adv;
     }
     // no copy may outlive the CTA: wait (bounded) for the last fills to land
     if (lane == 0)
@@ -601,7 +601,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(mfree);
     ++itm;
-    x += sg.n;
+    x += sg.adv;
   }
 }
 

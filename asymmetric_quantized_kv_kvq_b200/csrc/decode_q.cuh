@@ -399,8 +399,8 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
       if ((it & 31) == 0) {
         const int64_t xl = x0 + it + lane;                  // this lane's chunk of the flat list
         my_page = -1;
-        if (xl < x1) {
-          const DecodeSeg gl = decode_find_seg(b, xl, x1);
+        const DecodeSeg gl = xl < x1 ? decode_find_seg(b, xl, x1) : DecodeSeg{0, 0, 0, 0, 0};
+        if (gl.n > 0) {                                     // a chunk that holds tokens
           const SeqDesc dl = b.s[gl.bi];
           const int t0 = dl.lo / a.chunk * a.chunk + gl.k0 * a.chunk;
           my_page = a.L.page_table[int64_t(dl.seq_id) * a.L.max_pages_per_seq + page_slot(t0 / a.L.page_tokens, dl.ring)];
@@ -462,7 +462,7 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
         ph ^= 1;
       }
     }
-    x += sg.n;
+    x += sg.adv;
   }
   // no copy may outlive the CTA: wait (bounded) for the last fills to land
   if (lane == 0)
@@ -851,7 +851,7 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
         for (int i = 0; i < E; ++i) mo[g * D + v_elem_of<VB, E>(sl, i)] = w.O[g][i];
     }
     if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw, itc)) return;
-    x += sg.n;
+    x += sg.adv;
   }
 }
 

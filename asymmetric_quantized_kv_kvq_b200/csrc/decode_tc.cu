@@ -282,7 +282,7 @@ __global__ void __launch_bounds__(352, 1)
           bulk_g2s(st + T::OFF_VS, hb + a.L.v_scales_off + int64_t(r) * T::VS_ROW, ncopy * T::VS_ROW, full, pol);
           ++it;
         }
-        x += sg.n;
+        x += sg.adv;
       }
       // no copy may outlive the CTA
       for (uint32_t j = it > uint32_t(NS) ? it - NS : 0; j < it; ++j) mbar_wait(bar(B_FULL + j % NS), (j / NS) & 1, nullptr);
@@ -312,7 +312,7 @@ __global__ void __launch_bounds__(352, 1)
           umma_commit(bar(B_SFULL + (j & 1)));
           umma_commit(bar(B_EMPTY + s));
         }
-        x += sg.n;
+        x += sg.adv;
       }
       if (!ok) {
         record_error(a.L.err, kErrWaitTimeout | 0x22);
@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(352, 1)
           umma_commit(bar(B_PVDONE + (j & 1)));
         }
         if (ok) umma_commit(bar(B_OFULL + ip));
-        x += sg.n;
+        x += sg.adv;
       }
       if (!ok) {
         record_error(a.L.err, kErrWaitTimeout | 0x25);
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(352, 1)
       write_q(sg, 0, qsc);
     }
     while (x < x1) {
-      const int64_t nx = x + sg.n;
+      const int64_t nx = x + sg.adv;
       DecodeSeg nsg{0, 0, 0, 0};
       if (nx < x1) {
         // the next item's digits go to the buffer of the item before this one, whose
@@ -591,7 +591,7 @@ __global__ void __launch_bounds__(352, 1)
           mbar_arrive(bar(B_EMPTY + s));
         }
       }
-      x += sg.n;
+      x += sg.adv;
     }
     if (!ok) {
       if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 0x24);

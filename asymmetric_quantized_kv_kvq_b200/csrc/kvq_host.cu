@@ -782,21 +782,43 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   kvq::Batch b;
   b.n = n;
   int64_t flat = 0;
+  int32_t max_nch = 0;
   for (int i = 0; i < n; ++i) {
     const int64_t len = c->len[ids[i]];
     if (len < 1) return fail(KVQ_ERR_INVALID_ARG, "sequence %d is empty", ids[i]);
     const int64_t lo = first_attended(c, ids[i]), base = lo / C * C;
     const int32_t nch = int32_t((len - base + C - 1) / C);
-    b.s[i] = {ids[i], int32_t(len), int32_t(flat), nch, int32_t(lo), ring_pages(c, ids[i])};
+    b.s[i] = {ids[i], int32_t(len), 0, nch, int32_t(lo), ring_pages(c, ids[i]), nch};
     flat += int64_t(H) * nch;
+    max_nch = std::max(max_nch, nch);
+  }
+  if (flat >= (int64_t(1) << 31)) return fail(KVQ_ERR_INVALID_ARG, "batch too large");
+  const int max_ctas = kvq::decode_max_ctas(c->num_sms);
+  // Every CTA takes cpc consecutive chunks of the flat (sequence, head, chunk) list.  When the
+  // grid still fits in max_ctas, each item is padded to a whole number of CTA ranges, so that no
+  // range crosses an item (such a CTA runs two items back to back, each with its own merge), and
+  // items of at most kWholeItemChunks chunks go to one CTA whole (nothing to merge across CTAs).
+  constexpr int kWholeItemChunks = 4;
+  int64_t cpc = (flat + max_ctas - 1) / max_ctas;
+  if (!kvq::decode_tc_supported(LV, G)) {
+    const int64_t cp = max_nch <= kWholeItemChunks ? std::max<int64_t>(cpc, max_nch) : cpc;
+    int64_t pf = 0;
+    for (int i = 0; i < n; ++i) pf += int64_t(H) * ((b.s[i].c + cp - 1) / cp) * cp;
+    if (pf / cp <= max_ctas) {
+      cpc = cp;
+      for (int i = 0; i < n; ++i) b.s[i].c = int32_t((b.s[i].c + cp - 1) / cp * cp);
+    }
+  }
+  int64_t off = 0;
+  for (int i = 0; i < n; ++i) {
+    b.s[i].b = int32_t(off);
+    off += int64_t(H) * b.s[i].c;
   }
   plan.n_items = n * H;
-  plan.total_chunks = flat;
-  const int max_ctas = kvq::decode_max_ctas(c->num_sms);
+  plan.total_chunks = off;
   plan.max_ctas = max_ctas;
-  plan.chunks_per_cta = (flat + max_ctas - 1) / max_ctas;
-  plan.n_cta = int((flat + plan.chunks_per_cta - 1) / plan.chunks_per_cta);
-  if (flat >= (int64_t(1) << 31)) return fail(KVQ_ERR_INVALID_ARG, "batch too large");
+  plan.chunks_per_cta = cpc;
+  plan.n_cta = int((off + cpc - 1) / cpc);
   const float sigma = softmax_scale > 0.f ? softmax_scale : 1.0f / std::sqrt(float(c->L.head_dim));
   const float scale_log2 = sigma * 1.4426950408889634f;
   const bool fused = appending && kvq::decode_fuses_append(LV, G);

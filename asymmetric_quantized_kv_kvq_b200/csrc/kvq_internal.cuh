@@ -70,6 +70,7 @@ struct SeqDesc {
   int32_t seq_id;
   int32_t a, b, c;
   int32_t lo, ring;
+  int32_t cr;   // decode: chunks per head that hold tokens (c may be padded past them; 0 = c)
 };
 
 // Page-table slot of logical page p of a sequence.
@@ -151,6 +152,7 @@ size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D);
 constexpr int kMaxDecodeCtas = 256;
 int decode_max_ctas(int num_sms);
 int decode_chunk_tokens(const Layout& L, int G);
+bool decode_tc_supported(const Layout& L, int G);
 // k_new / v_new: fp16 [B, Hkv, D] rows of position len - 1 to quantise into the
 // cache first (nullptr: plain decode); only when decode_fuses_append(L, G).
 cudaError_t launch_decode(const Layout& L, int layer, const Batch& b, const DecodePlan& plan,
