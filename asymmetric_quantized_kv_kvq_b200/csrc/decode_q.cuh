@@ -105,7 +105,11 @@ struct QDec {
   static constexpr int OFF_VC = OFF_KS + C * S_ROW;
   static constexpr int OFF_VS = OFF_VC + C * V_ROW;
   static constexpr int STAGE = OFF_VS + C * S_ROW;
-  static constexpr int PBUF = NW * W * NB * GW * 4;  // per warp: p' [W][NB][GW]
+  // per warp: p' [W][NB][GW] during the stages; at an item's start the query digits of the
+  // warp's heads (hi and lo words [GW][D / 4] each, 4-bit-key corrections [GW][NB], max|q| [GW])
+  static constexpr int QD_BYTES = GW * D * 2 + GW * NB * 4 + GW * 4;
+  static constexpr int PB_WARP = ((W * NB * GW * 4 > QD_BYTES ? W * NB * GW * 4 : QD_BYTES) + 15) / 16 * 16;
+  static constexpr int PBUF = NW * PB_WARP;
   // partial O per partition; the last CTA of a split item reuses it for one weight per CTA and head
   static constexpr int MRG_O_F = NPART * G * D > (kMaxDecodeCtas + 1) * G ? NPART * G * D : (kMaxDecodeCtas + 1) * G;
   static constexpr int MRG_O = (MRG_O_F * 4 + 15) / 16 * 16;
@@ -122,7 +126,7 @@ struct QDec {
   static_assert(BPL % 4 == 0 && BPL <= VBLK, "a value lane's codes lie in one value block");
   static_assert(STAGE % 16 == 0 && OFF_KS % 16 == 0 && OFF_VC % 16 == 0 && OFF_VS % 16 == 0, "alignment");
   static_assert(PBUF % 16 == 0 && QBUF % 16 == 0, "alignment");
-  static_assert((2 * S + 5) * 8 + 8 <= BARS, "barrier area");
+  static_assert((2 * S + 6) * 8 + 8 <= BARS, "barrier area");
 };
 
 // ---- the permuted reduce-scatter of the score lanes ------------------------------
@@ -226,11 +230,11 @@ template <int KB, int VB, int D, int G>
 struct QDecSmem {
   using T = QDec<KB, VB, D, G>;
   uint8_t* stages;
-  float* pbuf;          // [warp][W][NB][GW]  p' = p d_v
+  float* pbuf;          // [warp][PB_WARP bytes]  p' = p d_v [W][NB][GW], or the query digits
   float* mrg_o;         // [part][G][D]
   float* mrg_ml;        // [part][G][2]
   __half* qbuf;         // [warp][GW][D]
-  uint32_t full0, empty0, mfull, mfree, mws, mlast, mcomb;
+  uint32_t full0, empty0, mfull, mfree, mws, mlast, mcomb, abar;
   volatile int* abort_flag;
   volatile int* last_flag;
 
@@ -249,7 +253,8 @@ struct QDecSmem {
     mws = mfull + 16;                                    // partial written to the workspace
     mlast = mfull + 24;                                  // "last CTA of the item" decided
     mcomb = mfull + 32;                                  // merge weights of a split item written
-    abort_flag = reinterpret_cast<volatile int*>(bars + 2 * T::S + 5);
+    abar = mfull + 40;                                   // fused append: the chunk's copies landed
+    abort_flag = reinterpret_cast<volatile int*>(bars + 2 * T::S + 6);
     last_flag = abort_flag + 1;
   }
 };
@@ -330,21 +335,33 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
     if (*sm.last_flag) {
       __threadfence();
       const int n = int(c1 - c0 + 1);                  // <= grid size <= kMaxDecodeCtas
-      // weights 2^(m_i - M) of every partial slot i and 1 / L per head, one warp per head (lanes
-      // share the slots), into the merge area, which this CTA's own merge no longer reads
+      // weights 2^(m_i - M) of every partial slot i and 1 / L per head, one warp per head: the
+      // (m, l) pairs of all slots are loaded at once (a lane holds slots lane + 32 q), into the
+      // merge area, which this CTA's own merge no longer reads
       float* wts = sm.mrg_o;                             // [n][G]
       float* linv = sm.mrg_o + n * G;                    // [G]
+      constexpr int QS = kMaxDecodeCtas / 32;
       for (int g = ct >> 5; g < G; g += NW) {
-        const float* ml = a.ws_ml + ((c0 + item) * G + g) * 2;
+        const float2* ml = reinterpret_cast<const float2*>(a.ws_ml) + (c0 + item) * G + g;   // slot i: ml[G i]
+        float2 v[QS];
         float M = -INFINITY;
-        for (int i = lane; i < n; i += 32) M = fmaxf(M, __ldcg(ml + int64_t(2) * G * i));
+#pragma unroll
+        for (int q = 0; q < QS; ++q) {
+          const int i = lane + 32 * q;
+          v[q] = i < n ? __ldcg(ml + int64_t(G) * i) : make_float2(-INFINITY, 0.f);
+          M = fmaxf(M, v[q].x);
+        }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float L = 0.f;
-        for (int i = lane; i < n; i += 32) {
-          const float w = exp2f(__ldcg(ml + int64_t(2) * G * i) - M);   // 0 for a slot without tokens
-          wts[i * G + g] = w;
-          L = fmaf(w, __ldcg(ml + int64_t(2) * G * i + 1), L);
+#pragma unroll
+        for (int q = 0; q < QS; ++q) {
+          const int i = lane + 32 * q;
+          if (i < n) {
+            const float w = exp2f(v[q].x - M);         // 0 for a slot without tokens
+            wts[i * G + g] = w;
+            L = fmaf(w, v[q].y, L);
+          }
         }
 #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
@@ -358,14 +375,47 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
         return false;
       }
       ++itc;
-      // every output element: the weighted sum of its slots, slots in a fixed order (loads unrolled)
-      for (int e = ct; e < G * D; e += NW * 32) {
-        const int g = e / D, d = e % D;
-        const float* o0 = a.ws_o + ((c0 + item) * G + g) * D + d;
-        float acc = 0.f;
-#pragma unroll 8
-        for (int i = 0; i < n; ++i) acc = fmaf(wts[i * G + g], __ldcg(o0 + int64_t(G) * D * i), acc);
-        a.out[(int64_t(sg.bi) * a.n_q_heads + sg.h * G + g) * D + d] = __float2half_rn(acc * linv[g]);
+      // every output element: the weighted sum of its slots.  A thread takes 4 consecutive
+      // elements (16-byte loads) and every SG-th slot, loads up to 16 slots at once, and the SG
+      // threads of a column (adjacent lanes) add their sums in a fixed order
+      constexpr int NCOL = G * D / 4;
+      constexpr int SG = NCOL >= NW * 32 ? 1 : NW * 32 / NCOL;
+      static_assert(NCOL * SG == NW * 32 || SG == 1, "one column per thread");
+      for (int cb = ct / SG; cb < NCOL; cb += NW * 32 / SG) {
+        const int sgi = ct % SG;
+        const int g = (cb * 4) / D, d0 = (cb * 4) % D;
+        const float4* o0 = reinterpret_cast<const float4*>(a.ws_o + ((c0 + item) * G + g) * D + d0);   // slot i: o0[NCOL i]
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i0 = sgi; i0 < n; i0 += 16 * SG) {
+          float4 t[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int i = i0 + q * SG;
+            t[q] = i < n ? __ldcg(o0 + int64_t(NCOL) * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const int i = i0 + q * SG;
+            const float wgt = i < n ? wts[i * G + g] : 0.f;
+            acc.x = fmaf(wgt, t[q].x, acc.x);
+            acc.y = fmaf(wgt, t[q].y, acc.y);
+            acc.z = fmaf(wgt, t[q].z, acc.z);
+            acc.w = fmaf(wgt, t[q].w, acc.w);
+          }
+        }
+#pragma unroll
+        for (int o = 1; o < SG; o <<= 1) {
+          acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+          acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+          acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+          acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+        }
+        if (sgi == 0) {
+          const float li = linv[g];
+          __half2* dst = reinterpret_cast<__half2*>(a.out + (int64_t(sg.bi) * a.n_q_heads + sg.h * G + g) * D + d0);
+          dst[0] = __floats2half2_rn(acc.x * li, acc.y * li);
+          dst[1] = __floats2half2_rn(acc.z * li, acc.w * li);
+        }
       }
     }
   }
@@ -375,11 +425,129 @@ __device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<
   return true;
 }
 
+// Page of the chunk at flat position xl of a CTA range ending at x1 (-1 outside it or for a chunk
+// that holds no tokens).
+__device__ __forceinline__ int chunk_page(const DecodeQArgs& a, const Batch& b, int64_t xl, int64_t x1) {
+  if (xl >= x1) return -1;
+  const DecodeSeg gl = decode_find_seg(b, xl, x1);
+  if (gl.n <= 0) return -1;
+  const SeqDesc dl = b.s[gl.bi];
+  const int t0 = dl.lo / a.chunk * a.chunk + gl.k0 * a.chunk;
+  return a.L.page_table[int64_t(dl.seq_id) * a.L.max_pages_per_seq + page_slot(t0 / a.L.page_tokens, dl.ring)];
+}
+
+// Fused append, quantised by the whole producer warp: the row's 2 NB blocks (K blocks, then V
+// blocks), LB lanes per block, EQ consecutive elements per lane.  Same arithmetic as the block
+// quantiser of the append kernel, element for element, so the bytes are the same.
+template <int D>
+struct NewRow {
+  static constexpr int NB = D / 32, LB = 32 / (2 * NB), EQ = 32 / LB;   // D 128: 4 lanes x 8; D 64: 8 x 4
+  uint32_t raw[EQ / 2];                                                 // the lane's EQ fp16 values
+};
+template <int D>
+__device__ __forceinline__ void new_row_load(NewRow<D>& nr, const DecodeQArgs& a, int bi, int h, int lane) {
+  using R = NewRow<D>;
+  const int blk = lane / R::LB, l = lane % R::LB;
+  const bool is_v = blk >= R::NB;
+  const __half* src = (is_v ? a.v_new : a.k_new) + (int64_t(bi) * a.L.n_kv_heads + h) * D + 32 * (blk % R::NB) + R::EQ * l;
+  if constexpr (R::EQ == 8) {
+    const uint4 v = *reinterpret_cast<const uint4*>(src);
+    nr.raw[0] = v.x; nr.raw[1] = v.y; nr.raw[2] = v.z; nr.raw[3] = v.w;
+  } else {
+    const uint2 v = *reinterpret_cast<const uint2*>(src);
+    nr.raw[0] = v.x; nr.raw[1] = v.y;
+  }
+}
+// Codes of the lane's part (cw: its EQ bytes for 8 bits; for 4 bits the lanes of the block's
+// first 16 elements hold the EQ packed bytes j | j + 16 << 4, the others nothing) and the
+// block's scale.  The warp's blocks mix 8- and 4-bit codes (K8V4, K4V8), so every shuffle sits
+// on the path that all 32 lanes take: both reductions run in every lane, and each lane picks
+// its own afterwards.
+template <int D>
+__device__ __forceinline__ __half new_row_quant(const NewRow<D>& nr, bool q8, int lane, uint32_t (&cw)[2]) {
+  using R = NewRow<D>;
+  constexpr int LB = R::LB, EQ = R::EQ;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int l = lane % LB;
+  float x[EQ];
+#pragma unroll
+  for (int i = 0; i < EQ / 2; ++i) {
+    const float2 f = h2_to_f2(nr.raw[i]);
+    x[2 * i] = f.x;
+    x[2 * i + 1] = f.y;
+  }
+  // 8 bits: amax over the block; 4 bits: m = the element of largest |x|, the lowest index on ties
+  float am = fabsf(x[0]), m = x[0];
+  int mi = EQ * l;
+#pragma unroll
+  for (int i = 1; i < EQ; ++i)
+    if (fabsf(x[i]) > am) {
+      am = fabsf(x[i]);
+      m = x[i];
+      mi = EQ * l + i;
+    }
+#pragma unroll
+  for (int o = 1; o < LB; o <<= 1) {
+    const float am2 = __shfl_xor_sync(FULL, am, o), m2 = __shfl_xor_sync(FULL, m, o);
+    const int mi2 = __shfl_xor_sync(FULL, mi, o);
+    if (am2 > am || (am2 == am && mi2 < mi)) {
+      am = am2;
+      m = m2;
+      mi = mi2;
+    }
+  }
+  const __half d = q8 ? __float2half_rn(__fdiv_rn(am, 127.0f)) : __float2half_rn(m * -0.125f);   // m / -8 exact
+  const float df = __half2float(d);
+  float c[EQ];                                           // 4-bit codes (unused by 8-bit lanes)
+  cw[0] = cw[1] = 0u;
+  if (df != 0.f) {
+    const RoundCtx r = round_ctx(df);
+    if (q8) {
+#pragma unroll
+      for (int k = 0; k < EQ / 4; ++k)
+        cw[k] = pack_low_bytes(float_int_bits(round_code8(x[4 * k], r)), float_int_bits(round_code8(x[4 * k + 1], r)),
+                               float_int_bits(round_code8(x[4 * k + 2], r)), float_int_bits(round_code8(x[4 * k + 3], r)));
+    }
+    const uint32_t dbits = __float_as_uint(df);
+#pragma unroll
+    for (int i = 0; i < EQ; ++i) c[i] = q8 ? 0.f : round_code4(x[i], r, dbits);
+  } else {
+#pragma unroll
+    for (int i = 0; i < EQ; ++i) c[i] = 0.f;
+  }
+  // element j + 16 lies LB / 2 lanes further on (all lanes shuffle)
+  float ch[EQ];
+#pragma unroll
+  for (int i = 0; i < EQ; ++i) ch[i] = __shfl_xor_sync(FULL, c[i], LB / 2);
+  if (!q8) {
+    uint32_t by[EQ];
+#pragma unroll
+    for (int i = 0; i < EQ; ++i) by[i] = float_int_bits(__fmaf_rn(ch[i], 16.f, c[i]) + 136.f);   // u_j + 16 u_{j+16}
+#pragma unroll
+    for (int k = 0; k < EQ / 4; ++k) cw[k] = pack_low_bytes(by[4 * k], by[4 * k + 1], by[4 * k + 2], by[4 * k + 3]);
+  }
+  return d;
+}
+// Store the lane's part of the row: codes at `codes` (the block's first byte), the scale at `scale`.
+template <int D>
+__device__ __forceinline__ void new_row_store(uint8_t* codes, __half* scale, bool q8, int lane, const uint32_t (&cw)[2],
+                                              __half d) {
+  using R = NewRow<D>;
+  constexpr int LB = R::LB, EQ = R::EQ;
+  const int l = lane % LB;
+  if (q8 || l < LB / 2) {
+    uint8_t* dst = codes + EQ * l;
+    if constexpr (EQ == 8) *reinterpret_cast<uint2*>(dst) = make_uint2(cw[0], cw[1]);
+    else *reinterpret_cast<uint32_t*>(dst) = cw[0];
+  }
+  if (l == 0) *scale = d;
+}
+
 // Producer warp: streams the CTA's chunks into the stage ring (and, with a fused
-// append, quantises each item's new token into its page first).
+// append, quantises each item's new token into its page and the stage).
 template <int KB, int VB, int D, int G>
 __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch& b,
-                                              const QDecSmem<KB, VB, D, G>& sm, int64_t x0, int64_t x1) {
+                                              const QDecSmem<KB, VB, D, G>& sm, int64_t x0, int64_t x1, int page0) {
   using T = QDec<KB, VB, D, G>;
   constexpr int S = T::S, NB = T::NB;
   const int lane = threadIdx.x & 31;
@@ -387,25 +555,21 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
   const uint64_t pol = l2_evict_first_policy();
   uint32_t it = 0;
   int s = 0;                                           // ring slot of stage `it` and its fill parity
-  uint32_t ph = 0;
+  uint32_t ph = 0, aph = 0;                            // aph: phase of abar
   bool ok = true;
   // Page ids of the next 32 chunks, one per lane, loaded together once every 32 chunks: the
-  // page-table read (a global load, ~1 us) would otherwise sit in front of every stage's copies.
-  int my_page = -1;
+  // page-table read (a global load, ~1 us) would otherwise sit in front of every stage's copies
+  // (the first 32 were loaded at the kernel's start: page0).
+  int my_page = page0;
+  NewRow<D> nr;
   for (int64_t x = x0; x < x1 && ok;) {
     const DecodeSeg sg = decode_find_seg(b, x, x1);
     const SeqDesc sd = b.s[sg.bi];
+    // fused append: the new token's K and V, loaded as soon as the segment's last chunk is the
+    // item's last (the one that holds the token)
+    if (a.k_new != nullptr && sg.n > 0 && sg.k0 + sg.n == (sd.cr > 0 ? sd.cr : sd.c)) new_row_load<D>(nr, a, sg.bi, sg.h, lane);
     for (int k = sg.k0; k < sg.k0 + sg.n; ++k) {
-      if ((it & 31) == 0) {
-        const int64_t xl = x0 + it + lane;                  // this lane's chunk of the flat list
-        my_page = -1;
-        const DecodeSeg gl = xl < x1 ? decode_find_seg(b, xl, x1) : DecodeSeg{0, 0, 0, 0, 0};
-        if (gl.n > 0) {                                     // a chunk that holds tokens
-          const SeqDesc dl = b.s[gl.bi];
-          const int t0 = dl.lo / a.chunk * a.chunk + gl.k0 * a.chunk;
-          my_page = a.L.page_table[int64_t(dl.seq_id) * a.L.max_pages_per_seq + page_slot(t0 / a.L.page_tokens, dl.ring)];
-        }
-      }
+      if ((it & 31) == 0 && it > 0) my_page = chunk_page(a, b, x0 + it + lane, x1);
       const int page = __shfl_sync(0xffffffffu, my_page, it & 31);
       if (!mbar_wait(sm.empty0 + 8 * s, ph ^ 1, sm.abort_flag, a.L.wait_ns)) {
         if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 1);
@@ -424,37 +588,51 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
       }
       const int r = tok0 % a.L.page_tokens;
       uint8_t* hb = a.L.head_ptr(a.layer, page, sg.h);
-      if (a.k_new != nullptr && tok0 + ntok == sd.a) {
-        // fused append: quantise the new token (position len - 1 = page row r + ntok - 1)
-        // before the copy that reads it; lane i < NB takes K block i, NB <= i < 2 NB a V block
-        const int rn = r + ntok - 1;
-        if (lane < 2 * NB) {
-          const bool is_v = lane >= NB;
-          const int blk = lane % NB;
-          const __half* src = (is_v ? a.v_new : a.k_new) + (int64_t(sg.bi) * H + sg.h) * D + 32 * blk;
-          float xv[32];
-          load_block(src, xv);
-          uint8_t* codes = hb + (is_v ? a.L.v_codes_off : 0) + int64_t(rn) * (is_v ? T::V_ROW : T::K_ROW);
-          __half* scales =
-              reinterpret_cast<__half*>(hb + (is_v ? a.L.v_scales_off : a.L.k_scales_off) + int64_t(rn) * T::S_ROW);
-          if ((is_v ? VB : KB) == 8) quant8_block(xv, codes + 32 * blk, scales + blk);
-          else quant4_block(xv, codes + 16 * blk, scales + blk);
-          // the bulk copy below reads these bytes through the async proxy
-          asm volatile("fence.proxy.async.global;" ::: "memory");
-        }
-        __syncwarp();
-      }
+      // fused append: this chunk holds the new token (position len - 1, chunk row ntok - 1)
+      const bool app = a.k_new != nullptr && tok0 + ntok == sd.a;
       // test hook (cache created with KVQ_TEST_WITHHOLD_ARRIVAL set): CTA 0 never fills its
       // first stage, so its consumers' bounded waits run out and report kErrWaitTimeout
       const bool withhold = a.L.test_withhold && blockIdx.x == 0 && it == 0;
       if (lane == 0 && !withhold) {
-        const uint32_t bar = sm.full0 + 8 * s;
+        // an appending chunk's copies complete on abar: the stage is released to the consumers
+        // only after the new row has been written into it
+        const uint32_t bar = app ? sm.abar : sm.full0 + 8 * s;
         const uint32_t dst = smem_u32(sm.stages + s * T::STAGE);
         mbar_arrive_expect_tx(bar, uint32_t(ncopy * T::TOK_BYTES));
         bulk_g2s(dst, hb + int64_t(r) * T::K_ROW, ncopy * T::K_ROW, bar, pol);
         bulk_g2s(dst + T::OFF_KS, hb + a.L.k_scales_off + int64_t(r) * T::S_ROW, ncopy * T::S_ROW, bar, pol);
         bulk_g2s(dst + T::OFF_VC, hb + a.L.v_codes_off + int64_t(r) * T::V_ROW, ncopy * T::V_ROW, bar, pol);
         bulk_g2s(dst + T::OFF_VS, hb + a.L.v_scales_off + int64_t(r) * T::S_ROW, ncopy * T::S_ROW, bar, pol);
+      }
+      if (app) {
+        // quantise the new K and V row into registers while the copies are in flight; once they
+        // landed, write it over the copied (stale) row and release the stage, and only then store
+        // it into the page (so that the release does not wait for those global stores)
+        const int rl = ntok - 1;
+        const int blk = lane / NewRow<D>::LB;
+        const bool is_v = blk >= NB;
+        const bool q8 = (is_v ? VB : KB) == 8;
+        const int cb = q8 ? 32 : 16;                       // code bytes of one block
+        const int row_b = is_v ? T::V_ROW : T::K_ROW;
+        uint32_t cw[2];
+        const __half d = new_row_quant<D>(nr, q8, lane, cw);
+        if (!mbar_wait(sm.abar, aph, sm.abort_flag, a.L.wait_ns)) {
+          if (lane == 0) record_error(a.L.err, kErrWaitTimeout | 10);
+          *sm.abort_flag = 1;
+          ok = false;
+          break;
+        }
+        aph ^= 1;
+        uint8_t* st = sm.stages + s * T::STAGE;
+        new_row_store<D>(st + (is_v ? T::OFF_VC : 0) + rl * row_b + cb * (blk % NB),
+                         reinterpret_cast<__half*>(st + (is_v ? T::OFF_VS : T::OFF_KS) + rl * T::S_ROW) + blk % NB, q8,
+                         lane, cw, d);
+        __syncwarp();
+        mbar_arrive_if(sm.full0 + 8 * s, lane == 0);       // release: the row is visible to the consumers
+        new_row_store<D>(hb + (is_v ? a.L.v_codes_off : 0) + int64_t(r + rl) * row_b + cb * (blk % NB),
+                         reinterpret_cast<__half*>(hb + (is_v ? a.L.v_scales_off : a.L.k_scales_off) +
+                                                   int64_t(r + rl) * T::S_ROW) + blk % NB,
+                         q8, lane, cw, d);
       }
       ++it;
       if (++s == S) {
@@ -687,7 +865,7 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
   const int fmap = rs_map<LPT, GW>(blk);
   const int xr = kq_rot<KB, D>(tl);
   const uint32_t u_stages = smem_u32(sm.stages);
-  const uint32_t u_pb = smem_u32(sm.pbuf + warp * (T::W * T::NB * GW));
+  const uint32_t u_pb = smem_u32(sm.pbuf) + warp * T::PB_WARP;
   QLaneOff lo;
   {
     const int row = prow0 + tl;                        // score lane's row in pass 0
@@ -717,45 +895,47 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
       for (int i = lane; i < GW * D / 8; i += 32) reinterpret_cast<uint4*>(qs)[i] = src[i];
       __syncwarp();
     }
-    float amax[GW];
-#pragma unroll
-    for (int j = 0; j < GW; ++j) {
-      const uint4* qr = reinterpret_cast<const uint4*>(qs + (j ^ fmap) * D + 32 * blk);
+    // The digits are computed once per warp: lane (head j, slice u) takes EPL consecutive elements
+    // of head row j, finds max|q| with its head's other lanes, and writes the packed hi and lo
+    // words of its elements (and, for 4-bit keys, the sum of the digits of each key block) into
+    // the warp's p' buffer, which is idle at an item's start.  Each lane then loads the words of
+    // its own key block in its own word order.
+    {
+      constexpr int LH = 32 / GW < D / 4 ? 32 / GW : D / 4;   // lanes per head
+      constexpr int EPL = D / LH;                              // elements per lane (4, 8 or 16)
+      constexpr int WPL = EPL / 4;                             // digit words per lane
+      const uint32_t qd_hi = u_pb, qd_lo = u_pb + GW * D;      // [GW][D / 4] words each
+      const uint32_t qd_corr = u_pb + 2 * GW * D, qd_amax = qd_corr + GW * T::NB * 4;
+      const int j = lane / LH, u = lane % LH;
+      const bool act = j < GW;
+      const __half* qe = qs + (act ? j : 0) * D + u * EPL;
+      uint32_t hw[EPL / 2];
+      if constexpr (EPL == 16) {
+        const uint4 a0 = reinterpret_cast<const uint4*>(qe)[0], a1 = reinterpret_cast<const uint4*>(qe)[1];
+        hw[0] = a0.x; hw[1] = a0.y; hw[2] = a0.z; hw[3] = a0.w; hw[4] = a1.x; hw[5] = a1.y; hw[6] = a1.z; hw[7] = a1.w;
+      } else if constexpr (EPL == 8) {
+        const uint4 a0 = reinterpret_cast<const uint4*>(qe)[0];
+        hw[0] = a0.x; hw[1] = a0.y; hw[2] = a0.z; hw[3] = a0.w;
+      } else {
+        const uint2 a0 = reinterpret_cast<const uint2*>(qe)[0];
+        hw[0] = a0.x; hw[1] = a0.y;
+      }
       float mx = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const uint4 w4 = qr[c];
-        const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 f = h2_to_f2(ws[i]);
-          mx = fmax3(mx, fabsf(f.x), fabsf(f.y));
-        }
+      for (int i = 0; i < EPL / 2; ++i) {
+        const float2 f = h2_to_f2(hw[i]);
+        mx = fmax3(mx, fabsf(f.x), fabsf(f.y));
       }
-      amax[j] = mx * fabsf(a.scale_log2);
-    }
-    // per-head max over the token's lanes: the lane at lane ^ o holds this lane's slot-j head in
-    // its slot j ^ rs_map(o)
 #pragma unroll
-    for (int o = 1; o < LPT; o <<= 1) {
-      float t[GW];
-#pragma unroll
-      for (int j = 0; j < GW; ++j) t[j] = __shfl_xor_sync(FULL, amax[j ^ rs_map<LPT, GW>(o)], o);
-#pragma unroll
-      for (int j = 0; j < GW; ++j) amax[j] = fmaxf(amax[j], t[j]);
-    }
-    // n = rint(q / s) with s = max|q| / 32512 (|n| <= 32512), as hi = (n + 128) >> 8 and the low byte
-    // lo = n mod 256 read as int8, so that n = 256 hi + lo
-#pragma unroll
-    for (int j = 0; j < GW; ++j) {
-      const __half* qb = qs + (j ^ fmap) * D + 32 * blk;
-      const float mul = amax[j] > 0.f ? a.scale_log2 * (32512.f / amax[j]) : 0.f;
+      for (int o = 1; o < LH; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+      const float amax = mx * fabsf(a.scale_log2);
+      // n = rint(q / s) with s = max|q| / 32512 (|n| <= 32512), as hi = (n + 128) >> 8 and the low byte
+      // lo = n mod 256 read as int8, so that n = 256 hi + lo
+      const float mul = amax > 0.f ? a.scale_log2 * (32512.f / amax) : 0.f;
       int corr = 0;
 #pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        // the word's 4 elements are consecutive in the row
-        const uint2 h4 = *reinterpret_cast<const uint2*>(qb + kq_elem<KB>(k, 0, xr));
-        const float2 f01 = h2_to_f2(h4.x), f23 = h2_to_f2(h4.y);
+      for (int k = 0; k < WPL; ++k) {
+        const float2 f01 = h2_to_f2(hw[2 * k]), f23 = h2_to_f2(hw[2 * k + 1]);
         int n[4];
         n[0] = __float_as_int(fmaf(f01.x, mul, 12582912.f)) - 0x4B400000;   // round to nearest
         n[1] = __float_as_int(fmaf(f01.y, mul, 12582912.f)) - 0x4B400000;
@@ -766,17 +946,42 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
           n[e] = max(-32512, min(32512, n[e]));
           corr += n[e];
         }
-        w.ql[j][k] = __byte_perm(__byte_perm(n[0], n[1], 0x0040), __byte_perm(n[2], n[3], 0x0040), 0x5410);
+        const uint32_t lo = __byte_perm(__byte_perm(n[0], n[1], 0x0040), __byte_perm(n[2], n[3], 0x0040), 0x5410);
         const int h0 = (n[0] + 128) >> 8, h1 = (n[1] + 128) >> 8, h2 = (n[2] + 128) >> 8, h3 = (n[3] + 128) >> 8;
-        w.qh[j][k] = __byte_perm(__byte_perm(h0, h1, 0x0040), __byte_perm(h2, h3, 0x0040), 0x5410);
+        const uint32_t hi = __byte_perm(__byte_perm(h0, h1, 0x0040), __byte_perm(h2, h3, 0x0040), 0x5410);
+        if (act) {
+          const uint32_t wo = 4 * uint32_t(j * (D / 4) + u * WPL + k);
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd_hi + wo), "r"(hi) : "memory");
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd_lo + wo), "r"(lo) : "memory");
+        }
       }
-      w.qcorr[j] = KB == 4 ? -8 * corr : 0;
-    }
+      // digit sum of each 32-element block: the block's 32 / EPL lanes are adjacent
 #pragma unroll
-    for (int j = 0; j < NF; ++j) {                         // slot j < NF ends with head j ^ fmap
-      w.qsc[j] = amax[j] * (1.f / 32512.f);
-      w.m[j] = -INFINITY;
-      w.l[j] = 0.f;
+      for (int o = 1; o < 32 / EPL; o <<= 1) corr += __shfl_xor_sync(FULL, corr, o);
+      if (act && u % (32 / EPL) == 0)
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(qd_corr + 4 * uint32_t(j * T::NB + u * EPL / 32)), "r"(corr) : "memory");
+      if (act && u == 0) sts_f32(qd_amax + 4 * j, amax);
+      __syncwarp();
+      // this lane's words: slot j holds head j ^ fmap; word w of its order is natural word
+      // 4 ((w >> 2) ^ xr) + (w & 3) of its block (xr = 0 for 4-bit keys)
+#pragma unroll
+      for (int jj = 0; jj < GW; ++jj) {
+        const uint32_t base = 4 * uint32_t((jj ^ fmap) * (D / 4) + blk * 8);
+        const uint4 h0 = lds_v4(qd_hi + base + 16 * xr), h1 = lds_v4(qd_hi + base + 16 * (xr ^ 1));
+        const uint4 l0 = lds_v4(qd_lo + base + 16 * xr), l1 = lds_v4(qd_lo + base + 16 * (xr ^ 1));
+        w.qh[jj][0] = h0.x; w.qh[jj][1] = h0.y; w.qh[jj][2] = h0.z; w.qh[jj][3] = h0.w;
+        w.qh[jj][4] = h1.x; w.qh[jj][5] = h1.y; w.qh[jj][6] = h1.z; w.qh[jj][7] = h1.w;
+        w.ql[jj][0] = l0.x; w.ql[jj][1] = l0.y; w.ql[jj][2] = l0.z; w.ql[jj][3] = l0.w;
+        w.ql[jj][4] = l1.x; w.ql[jj][5] = l1.y; w.ql[jj][6] = l1.z; w.ql[jj][7] = l1.w;
+        w.qcorr[jj] = KB == 4 ? -8 * int(lds_u32(qd_corr + 4 * uint32_t((jj ^ fmap) * T::NB + blk))) : 0;
+      }
+#pragma unroll
+      for (int jj = 0; jj < NF; ++jj) {                        // slot jj < NF ends with head jj ^ fmap
+        w.qsc[jj] = lds_f32(qd_amax + 4 * (jj ^ fmap)) * (1.f / 32512.f);
+        w.m[jj] = -INFINITY;
+        w.l[jj] = 0.f;
+      }
+      __syncwarp();                                            // the p' stores may now reuse the area
     }
 #pragma unroll
     for (int g = 0; g < GW; ++g)
@@ -870,6 +1075,11 @@ __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
   using T = QDec<KB, VB, D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
   const QDecSmem<KB, VB, D, G> sm(smem);
+  const int warp = threadIdx.x >> 5;
+  const int64_t x0 = int64_t(blockIdx.x) * a.cpc;
+  const int64_t x1 = min(a.total_chunks, x0 + a.cpc);
+  // the producer's first 32 page ids, read while the barriers are set up
+  const int page0 = warp == T::NW ? chunk_page(a, b, x0 + (threadIdx.x & 31), x1) : -1;
   if (threadIdx.x == 0) {
     for (int s = 0; s < T::S; ++s) {
       mbar_init(sm.full0 + 8 * s, 1);
@@ -880,16 +1090,14 @@ __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
     mbar_init(sm.mws, T::NW);
     mbar_init(sm.mlast, 1);
     mbar_init(sm.mcomb, T::NW);
+    mbar_init(sm.abar, 1);
     *sm.abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5;
-  const int64_t x0 = int64_t(blockIdx.x) * a.cpc;
-  const int64_t x1 = min(a.total_chunks, x0 + a.cpc);
   if (warp >= T::NW) {
     set_max_regs<T::REG_P, T::REG_L>();
-    if (warp == T::NW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1);
+    if (warp == T::NW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1, page0);
     return;                                                 // the group's other 3 warps have no role
   }
   set_max_regs<T::REG_C, T::REG_L>();

@@ -89,14 +89,14 @@ __device__ __forceinline__ void load_block(const __half* src, float (&x)[32]) {
   }
 }
 
-// 8-bit: d = fp16(fp32(amax / 127)), c = clamp(roundf(x / d), -127, 127).
-__device__ __forceinline__ void quant8_block(const float (&x)[32], uint8_t* codes, __half* scale) {
+// 8-bit: d = fp16(fp32(amax / 127)), c = clamp(roundf(x / d), -127, 127).  The codes as 8 words
+// (byte i of the block in byte i % 4 of word i / 4); returns d.
+__device__ __forceinline__ __half quant8_words(const float (&x)[32], uint32_t (&w)[8]) {
   float a = 0.f;
 #pragma unroll
   for (int i = 0; i < 32; i += 2) a = fmax3(a, fabsf(x[i]), fabsf(x[i + 1]));
   const __half d = __float2half_rn(__fdiv_rn(a, 127.0f));
   const float df = __half2float(d);
-  uint32_t w[8];
   if (df != 0.f) {
     const RoundCtx r = round_ctx(df);
 #pragma unroll
@@ -107,14 +107,20 @@ __device__ __forceinline__ void quant8_block(const float (&x)[32], uint8_t* code
 #pragma unroll
     for (int k = 0; k < 8; ++k) w[k] = 0u;
   }
+  return d;
+}
+__device__ __forceinline__ void quant8_block(const float (&x)[32], uint8_t* codes, __half* scale) {
+  uint32_t w[8];
+  const __half d = quant8_words(x, w);
   reinterpret_cast<uint4*>(codes)[0] = make_uint4(w[0], w[1], w[2], w[3]);
   reinterpret_cast<uint4*>(codes)[1] = make_uint4(w[4], w[5], w[6], w[7]);
   *scale = d;
 }
 
 // 4-bit: m = the largest-|x| element (lowest index on ties), d = fp16(m / -8),
-// c = clamp(roundf(x / d), -8, 7), u = c + 8, byte i = u_i | u_{i+16} << 4.
-__device__ __forceinline__ void quant4_block(const float (&x)[32], uint8_t* codes, __half* scale) {
+// c = clamp(roundf(x / d), -8, 7), u = c + 8, byte i = u_i | u_{i+16} << 4.  The 16 bytes as 4
+// words; returns d.
+__device__ __forceinline__ __half quant4_words(const float (&x)[32], uint32_t (&w)[4]) {
   // the largest-|x| element is max(x) or min(x); only when max(x) == -min(x) (a +- tie, or a zero
   // block) does the index decide, by a scan in which the lowest index wins
   float mx = x[0], mn = x[0];
@@ -134,7 +140,6 @@ __device__ __forceinline__ void quant4_block(const float (&x)[32], uint8_t* code
   }
   const __half d = __float2half_rn(m * -0.125f);            // m / -8, exact in fp32
   const float df = __half2float(d);
-  uint32_t w[4];
   if (df != 0.f) {
     const RoundCtx r = round_ctx(df);
     const uint32_t dbits = __float_as_uint(df);
@@ -151,6 +156,11 @@ __device__ __forceinline__ void quant4_block(const float (&x)[32], uint8_t* code
 #pragma unroll
     for (int k = 0; k < 4; ++k) w[k] = 0x88888888u;         // all codes 0: u = 8 in both nibbles
   }
+  return d;
+}
+__device__ __forceinline__ void quant4_block(const float (&x)[32], uint8_t* codes, __half* scale) {
+  uint32_t w[4];
+  const __half d = quant4_words(x, w);
   reinterpret_cast<uint4*>(codes)[0] = make_uint4(w[0], w[1], w[2], w[3]);
   *scale = d;
 }
