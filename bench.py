@@ -719,6 +719,8 @@ def parse():
     ap.add_argument("--separate", action="store_true",
                     help="quantized caches: kvq_append + kvq_decode_attn per layer instead of the fused "
                          "kvq_decode_append_attn launch")
+    ap.add_argument("--dedup-probe", action="store_true",
+                    help="time one kvq_cache_dedup pass over the resident cache (on by default for the default run)")
     ap.add_argument("--no-extras", action="store_true",
                     help="default run: skip the 70B-shaped decode and the prefill sub-records")
     ap.add_argument("--decode-tc", action="store_true",
@@ -742,7 +744,7 @@ def main():
     from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS, parse_precision
     default_run = args.workload is None
     args.workload = args.workload or DEFAULT_WORKLOAD
-    args.dedup_probe = default_run and not args.no_extras
+    args.dedup_probe = (default_run and not args.no_extras) or args.dedup_probe
     wl = WORKLOADS[args.workload]
     if args.layers or args.batch or args.cached:
         import dataclasses
