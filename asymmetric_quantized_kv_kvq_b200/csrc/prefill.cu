@@ -31,8 +31,8 @@
 //     tiles (two pass-1 tiles) with 2-D / 3-D TMA tensor loads (128-byte
 //     swizzle): lane 0 fills a ring of K_hi / K_lo slots, lane 1 a separate
 //     ring of V^T slots, so a key slot refills as soon as its scores are done.
-//     Warp 1 owns all 512 TMEM columns (S double buffer, O, P double buffer)
-//     and issues the score MMAs, warp 10 the PV MMAs (fp32 accumulators):
+//     Warp 1 owns all 512 TMEM columns (a ring of three S buffers, O) and
+//     issues the score MMAs, warp 10 the PV MMAs (fp32 accumulators):
 //        S_j = Q K_hi,j^T + Q8 K_lo,j^T  (M 128, N 128: D/16 kind::f16 MMAs and, at
 //                                         head_dim 128, D/32 kind::f8f6f4 MMAs on e5m2
 //                                         operands, Q8 = e5m2(Q 2^-8) converted once
@@ -41,13 +41,19 @@
 //        O  += P_j V_j                   (kind::f16, A = P read from TMEM, 8 MMAs per 128 keys).
 //     A tcgen05.mma costs roughly the same time for N up to 128, so wide key
 //     tiles halve the instruction count of 64-key ones.  Warps 2-9 run the
-//     softmax, two per TMEM lane quadrant (one thread per row, 64 keys each):
-//     one tcgen05.ld of the raw scores, the row max exchanged between the two
-//     halves through shared memory at a named barrier, sigma log2 e and the
-//     causal mask applied, the online softmax (running max moved only when it
-//     grows by more than 2^8; then O is rescaled in TMEM), and P stored as fp16
-//     pairs into TMEM (tcgen05.st), where the PV MMA takes its A operand.  At
-//     the end they normalise O and store it.  Every wait is bounded.
+//     softmax, two per TMEM lane quadrant (one thread per row) taking whole
+//     tiles in turn: tile j goes to the warp of parity j % 2, which reads the
+//     row's 128 raw scores, takes their max, hands the running max on to the
+//     other warp at once (shared memory and a named barrier of the pair), and
+//     then computes the exponentials while the other warp reads and reduces
+//     tile j + 1, so the MUFU unit is kept busy.  sigma log2 e and the causal
+//     mask are applied, the online softmax moves the running max only when it
+//     grows by more than 2^8 (then O is rescaled in TMEM), and P is stored as
+//     fp16 pairs (tcgen05.st) over the first half of its own S buffer, where
+//     the PV MMA takes its A operand; the S buffer returns to the score MMAs
+//     when that PV is done, three tiles later.  Each warp keeps a partial row
+//     sum; at the end the pair joins them, normalises O and stores it.  Every
+//     wait is bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
@@ -102,6 +108,16 @@ __device__ __forceinline__ float ex2_ftz(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Named CTA barrier between a producing and a consuming warp: the producer
+// arrives without waiting once its shared-memory writes are done, the consumer
+// waits; `threads` counts both sides.
+__device__ __forceinline__ void nbar_arrive(int id, int threads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+__device__ __forceinline__ void nbar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
 // The remainder K_lo = k^ - fp16(k^) enters the scores at head_dim 128 as e5m2
@@ -252,14 +268,15 @@ struct PTraits {
   static constexpr int OFF_BAR = OFF_V + NSTAGE * V_BYTES;
   // + alignment slack; never less than ~116 KB so that a second CTA cannot
   // share the SM and wait in tcgen05.alloc
-  static constexpr int SMEM_NEED = OFF_BAR + 256 + 2 * 2 * 128 * 4 + 1024;   // barriers, TMEM slot, row maxima
+  static constexpr int SMEM_NEED = OFF_BAR + 256 + (128 + 4 * 128) * 4 + 1024;   // barriers, TMEM slot, row (m, l)
   static constexpr int SMEM = SMEM_NEED > 118 * 1024 ? SMEM_NEED : 118 * 1024;
   static constexpr int NT = 352;                         // 11 warps: copies, score MMAs, 2 x 4 softmax, PV MMAs
   static constexpr uint32_t TMEM_COLS = 512;
-  // S double buffer [0, 256) (fp32, 128 keys each), O [256, 256 + D), P double buffer [384, 512)
-  // (fp16 pairs, 64 columns = 128 keys each)
-  static constexpr uint32_t S_COL0 = 0, O_COL = 256, P_COL0 = 384;
-  static_assert(O_COL + D <= P_COL0 && P_COL0 + 2 * kKV / 2 <= TMEM_COLS, "TMEM");
+  // S ring of three 128-column buffers [0, 384) (fp32 scores of 128 keys; P_j is written over the first
+  // 64 columns of its own S_j as fp16 pairs once the scores are in registers), O [384, 384 + D)
+  static constexpr int NSB = 3;
+  static constexpr uint32_t S_COL0 = 0, O_COL = NSB * kKV;
+  static_assert(O_COL + D <= TMEM_COLS, "TMEM");
   static_assert(OFF_Q8 % 1024 == 0 && OFF_K % 1024 == 0 && OFF_V % 1024 == 0 && KSLOT % 1024 == 0 &&
                     K_BYTES % 1024 == 0 && V_BYTES % 1024 == 0,
                 "swizzle atoms");
@@ -286,13 +303,16 @@ __global__ void __launch_bounds__(352, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::OFF_BAR);
   const uint32_t bar0 = smem_u32(bars);
   auto bar = [&](int i) { return bar0 + 8u * i; };
-  // barriers: q_full | k_full[NS] | k_empty[NS] | v_full[NS] | v_empty[NS] | s_full[2] | p_full | pv_done | done
+  // barriers: q_full | k_full[NS] | k_empty[NS] | v_full[NS] | v_empty[NS] | s_full[3] | p_full[3] | pv_done[3]
+  // | done | done2 | q8; S, P and PV have one barrier per buffer of the S ring (tile j uses buffer j % 3;
+  // pv_done of a buffer also frees it for the scores three tiles later)
+  constexpr int NSB = T::NSB;
   constexpr int B_Q = 0, B_KFULL = 1, B_KEMPTY = 1 + NS, B_VFULL = 1 + 2 * NS, B_VEMPTY = 1 + 3 * NS,
-                B_S = 1 + 4 * NS, B_SFREE = 3 + 4 * NS, B_P = 5 + 4 * NS, B_PV = 7 + 4 * NS, B_DONE = 9 + 4 * NS,
-                B_DONE2 = 10 + 4 * NS, B_Q8 = 11 + 4 * NS;   // S, SFREE, P, PV: one barrier per buffer parity
-  static_assert(B_Q8 < 24, "barrier area");
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 24);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 25);
+                B_S = 1 + 4 * NS, B_P = B_S + NSB, B_PV = B_P + NSB, B_DONE = B_PV + NSB, B_DONE2 = B_DONE + 1,
+                B_Q8 = B_DONE2 + 1;
+  static_assert(B_Q8 < 28, "barrier area");
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 28);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 29);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int si = find_seq_by(b, blockIdx.x, false);
@@ -309,7 +329,7 @@ __global__ void __launch_bounds__(352, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i <= B_Q8; ++i)
-      mbar_init(bar(i), (i == B_P || i == B_P + 1 || i == B_SFREE || i == B_SFREE + 1 || i == B_Q8) ? 256u : 1u);
+      mbar_init(bar(i), (i >= B_P && i < B_P + NSB) ? 128u : i == B_Q8 ? 256u : 1u);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -380,13 +400,13 @@ __global__ void __launch_bounds__(352, 1)
       const uint64_t q8d0 = sdesc_k_sw128(base + T::OFF_Q8);
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % NS;
-        // S buffer j & 1 was read by the softmax of tile j - 2; the key slot is full
-        if (j >= 2) ok = mbar_wait(bar(B_SFREE + (j & 1)), ((j - 2) >> 1) & 1, abort_flag);
+        // S buffer j % 3 held P_(j-3), read by PV(j - 3); the key slot is full
+        if (j >= NSB) ok = mbar_wait(bar(B_PV + j % NSB), ((j - NSB) / NSB) & 1, abort_flag);
         if (ok) ok = mbar_wait(bar(B_KFULL + s), (j / NS) & 1, abort_flag);
         if (!ok) break;
         tc_fence_after();
         const uint64_t kd0 = sdesc_k_sw128(base + T::OFF_K + s * T::KSLOT);
-        const uint32_t dst = tmem + T::S_COL0 + (j & 1) * kKV;
+        const uint32_t dst = tmem + T::S_COL0 + (j % NSB) * kKV;
         if constexpr (T::LO8) {
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {          // Q K_hi^T (fp16)
@@ -414,7 +434,7 @@ __global__ void __launch_bounds__(352, 1)
             }
           }
         }
-        umma_commit(bar(B_S + (j & 1)));
+        umma_commit(bar(B_S + j % NSB));
         umma_commit(bar(B_KEMPTY + s));                 // the key slot refills once S_j is done
       }
       if (!ok) {
@@ -432,20 +452,20 @@ __global__ void __launch_bounds__(352, 1)
       bool ok = true;
       for (int j = 0; ok && j < n_kv; ++j) {
         const int s = j % NS;
-        if (!mbar_wait(bar(B_P + (j & 1)), (j >> 1) & 1, abort_flag) ||
+        if (!mbar_wait(bar(B_P + j % NSB), (j / NSB) & 1, abort_flag) ||
             !mbar_wait(bar(B_VFULL + s), (j / NS) & 1, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         // O += P V: A = P in TMEM (16 keys = 8 columns per step), B = V^T [D][128 keys] in two 64-key blocks
-        const uint32_t pa = tmem + T::P_COL0 + (j & 1) * (kKV / 2);
+        const uint32_t pa = tmem + T::S_COL0 + (j % NSB) * kKV;   // P_j over S_j
         const uint64_t vd0 = sdesc_k_sw128(base + T::OFF_V + s * T::V_BYTES);
 #pragma unroll
         for (int k = 0; k < kKV / 16; ++k)
           umma_f16_ta(tmem + T::O_COL, pa + 8 * k, vd0 + (((k >> 2) * D * 128 + (k & 3) * 32) >> 4), idO,
                       (j > 0 || k > 0));
-        umma_commit(bar(B_PV + (j & 1)));
+        umma_commit(bar(B_PV + j % NSB));
         umma_commit(bar(B_VEMPTY + s));
       }
       if (!ok) {
@@ -457,18 +477,21 @@ __global__ void __launch_bounds__(352, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax (warps 2..9)
-    // Two warps per TMEM lane quadrant: `half` 0 takes keys [0, 64) of each tile and head_dim
-    // columns [0, D/2) of O, half 1 keys [64, 128) and columns [D/2, D).  The row max is exchanged
-    // through shared memory at a 256-thread named barrier that also makes every exit uniform.
-    constexpr int BAR_MAX = 1, BAR_L = 2, NTH = 256;
-    const int quad = warp & 3, half = (warp - 2) >> 2;
+    // Two warps per TMEM lane quadrant (one thread per row) take turns: the warp of parity `par` runs
+    // the whole 128-key tiles j with j % 2 == par.  The running row max m passes from tile j to tile
+    // j + 1 through shared memory at a named barrier of the quadrant's two warps (arrive after
+    // writing, wait before reading), and is handed on as soon as the tile's max is known, so one
+    // warp's exponentials (the MUFU unit) overlap the other's TMEM read and max of the next tile.
+    // Each warp keeps its own partial row sum l against its own last m; the two are joined at the end.
+    constexpr int BAR_L = 9, NTH = 256;
+    const int quad = warp & 3, par = (warp - 2) >> 2;
     const int row = quad * 32 + lane;
     const uint32_t lane_addr = tmem + (uint32_t(quad * 32) << 16);
     const int qpos = qpos0 + row / G;
-    // [2 tile parities][2 halves][128 rows]: a buffer is rewritten two tiles later, after every thread
-    // has passed the next tile's BAR_MAX, so no second barrier guards the reads
-    float* redmax = reinterpret_cast<float*>(bars + 32);
-    float m_used = -INFINITY, l = 0.f;
+    const int bar_from = 1 + quad + 4 * (par ^ 1), bar_to = 1 + quad + 4 * par;   // named barriers 1..8
+    float* mrow = reinterpret_cast<float*>(bars + 32);   // [128 rows]: m of the latest tile
+    float* fin_ml = mrow + 128;                          // [2 parities][m, l][128 rows]
+    float m_own = -INFINITY, l_own = 0.f;
     bool wok = true;
     if constexpr (T::LO8) {
       // Q8 = e5m2(Q 2^-8): thread (row r, half hf) converts elements [64 hf, 64 hf + 64) of row r from
@@ -494,59 +517,72 @@ __global__ void __launch_bounds__(352, 1)
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // visible to the tensor core
       mbar_arrive(bar(B_Q8));
     }
-    int j = 0;
-    for (; j < n_kv; ++j) {
-      bool w = __all_sync(0xffffffffu, mbar_wait(bar(B_S + (j & 1)), (j >> 1) & 1, abort_flag));
-      const uint32_t sbuf = lane_addr + T::S_COL0 + (j & 1) * kKV + 64 * half;
-      const int kpos0 = j * kKV + 64 * half;
-      // pass 1: this half's 64 raw scores into registers (one TMEM read) and their max (sigma log2 e > 0
-      // keeps the order); only 32-key chunks that reach past the first row's position need the causal mask
-      uint32_t sv[64];
+    for (int j = par; j < n_kv; j += 2) {
+      const int sb = j % NSB;
+      wok = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_S + sb), (j / NSB) & 1, abort_flag));
+      const uint32_t sbuf = lane_addr + T::S_COL0 + sb * kKV;
+      const int kpos0 = j * kKV;
+      // pass 1: the row's 128 raw scores and their max (sigma log2 e > 0 keeps the order); only
+      // 32-key chunks that reach past the first row's position need the causal mask
       float mx = -INFINITY;
-      if (w) {
+      if (wok) {
         tc_fence_after();
-        tmem_ld32(sbuf, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-        tmem_ld32(sbuf + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(bar(B_SFREE + (j & 1)));           // S buffer j & 1 may be overwritten by S_(j+2)
+        float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (kpos0 + 32 * c + 31 > qpos0) {
+        for (int hh = 0; hh < 2; ++hh) {   // two reads of 64 keys
+          uint32_t sv[64];
+          tmem_ld32(sbuf + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+          tmem_ld32(sbuf + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (kpos0 + 32 * c + i <= qpos) mx = fmaxf(mx, __uint_as_float(sv[32 * c + i]));
-          } else {
+          for (int cc = 0; cc < 2; ++cc) {
+            const int c = 2 * hh + cc;
+            if (kpos0 + 32 * c + 31 > qpos0) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 2)
-              mx = fmax3(mx, __uint_as_float(sv[32 * c + i]), __uint_as_float(sv[32 * c + i + 1]));
+              for (int i = 0; i < 32; ++i)
+                if (kpos0 + 32 * c + i <= qpos) mq[i & 3] = fmaxf(mq[i & 3], __uint_as_float(sv[32 * cc + i]));
+            } else {
+              // four independent three-input max chains (a short dependency chain)
+#pragma unroll
+              for (int i = 0; i < 32; i += 8)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  mq[q] = fmax3(mq[q], __uint_as_float(sv[32 * cc + i + 2 * q]),
+                                __uint_as_float(sv[32 * cc + i + 2 * q + 1]));
+            }
           }
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 64; ++i) sv[i] = 0u;
+        mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       }
-      float* rm = redmax + (j & 1) * 256;
-      rm[half * 128 + row] = mx;
-      if (!bar_red_and(BAR_MAX, NTH, w && wok)) break;
-      mx = fmaxf(mx, rm[(half ^ 1) * 128 + row]) * a.scale_log2;
-      // P buffer j & 1 was read by PV(j - 2); PV(j - 1) may still run
-      if (j > 1) wok = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV + (j & 1)), ((j - 2) >> 1) & 1, abort_flag));
-      if (!wok) *abort_flag = 1;
-      const bool need = mx > m_used + 8.f;
-      if (__any_sync(0xffffffffu, need)) {
-        const float mnew = need ? mx : m_used;
-        const float alpha = exp2f(m_used - mnew);   // 0 when m_used = -inf
-        l *= alpha;
-        m_used = mnew;
-        // O is rescaled once every PV issued so far (up to PV(j - 1)) is done
-        if (j > 0) wok = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV + ((j - 1) & 1)), ((j - 1) >> 1) & 1, abort_flag));
-        if (j > 0 && wok) {
+      mx *= a.scale_log2;
+      // the running max after tile j - 1, from the quadrant's other warp
+      float m_prev = -INFINITY;
+      if (j > 0) {
+        nbar_sync(bar_from, 64);
+        m_prev = mrow[row];
+      }
+      // lazy max: m moves only when the tile's max exceeds it by more than 2^8 (p <= 2^8 fits fp16)
+      const bool need = mx > m_prev + 8.f;
+      const float m_used = need ? mx : m_prev;
+      if (j + 1 < n_kv) {
+        mrow[row] = m_used;
+        nbar_arrive(bar_to, 64);
+      }
+      if (m_used != m_own) {   // this warp's partial sum follows the new m (0 while it has none)
+        l_own *= exp2f(m_own - m_used);
+        m_own = m_used;
+      }
+      if (__any_sync(0xffffffffu, need) && j > 0) {
+        // O holds every PV up to PV(j - 1) at m_prev: rescale it once PV(j - 1) is done, before
+        // P_j is released (PV(j) follows in the PV warp's order)
+        const float alpha = exp2f(m_prev - m_used);   // 0 when m_prev = -inf, 1 where m stays
+        wok = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV + (j - 1) % NSB), ((j - 1) / NSB) & 1, abort_flag));
+        if (wok) {
           tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < D / 64; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t r32[32];
-            const uint32_t oc = lane_addr + T::O_COL + (D / 2) * half + 32 * c;
+            const uint32_t oc = lane_addr + T::O_COL + 32 * c;
             tmem_ld32(oc, r32);
             tmem_wait_ld();
 #pragma unroll
@@ -556,19 +592,27 @@ __global__ void __launch_bounds__(352, 1)
           tmem_wait_st();
         }
       }
-      // pass 2: P = 2^(sigma log2 e s - m) as fp16 pairs into P buffer j & 1 (this half's 32 columns)
-      // (pairs: one f32x2 FMA scales and shifts two scores, one f32x2 add sums two p)
+      // pass 2: P = 2^(sigma log2 e s - m) as fp16 pairs over the first 64 columns of S_j: the scores
+      // are read again 32 keys at a time, the next chunk's read in flight while one is processed (P of
+      // chunk c lands in columns [16c, 16c + 16), whose scores are already in registers); pairs: one
+      // f32x2 FMA scales and shifts two scores, one f32x2 add sums two p
+      if (!wok) *abort_flag = 1;
       const float2 sc2 = make_float2(a.scale_log2, a.scale_log2), nm2 = make_float2(-m_used, -m_used);
       float2 l2 = make_float2(0.f, 0.f);
-      const uint32_t pbuf = lane_addr + T::P_COL0 + (j & 1) * (kKV / 2) + 32 * half;
+      uint32_t sv[2][32];
+      if (wok) {
+        tmem_ld32(sbuf, sv[0]);
+        tmem_wait_ld();
+      }
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 4; ++c) {
+        if (wok && c < 3) tmem_ld32(sbuf + 32 * (c + 1), sv[(c + 1) & 1]);
         uint32_t pk[16];
         const bool masked = kpos0 + 32 * c + 31 > qpos0;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float2 x = ffma2(make_float2(__uint_as_float(sv[32 * c + 2 * i]),
-                                             __uint_as_float(sv[32 * c + 2 * i + 1])), sc2, nm2);
+          const float2 x = ffma2(make_float2(__uint_as_float(sv[c & 1][2 * i]),
+                                             __uint_as_float(sv[c & 1][2 * i + 1])), sc2, nm2);
           float p0 = ex2_ftz(x.x);
           float p1 = ex2_ftz(x.y);
           if (masked) {
@@ -580,34 +624,38 @@ __global__ void __launch_bounds__(352, 1)
           __half2 hp = __floats2half2_rn(p0, p1);
           pk[i] = *reinterpret_cast<uint32_t*>(&hp);
         }
-        if (wok) tmem_st16(pbuf + 16 * c, pk);
+        if (wok) {
+          tmem_st16(sbuf + 16 * c, pk);
+          if (c < 3) tmem_wait_ld();
+        }
       }
-      l += l2.x + l2.y;
+      l_own += l2.x + l2.y;
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(B_P + (j & 1)));
+      mbar_arrive(bar(B_P + sb));
     }
-    const bool done = j == n_kv;
-    bool fin = done && wok &&
-               __all_sync(0xffffffffu, mbar_wait(bar(B_PV + ((n_kv - 1) & 1)), ((n_kv - 1) >> 1) & 1, abort_flag));
-    // the l of both halves of each row; every thread takes part so the barrier is uniform
-    if (done) {
-      redmax[(n_kv & 1) * 256 + half * 128 + row] = l;   // the buffer last read two tiles back
-      fin = bar_red_and(BAR_L, NTH, fin);
-    }
-    if (!done || !fin) {
+    // the (m, l) of both warps of each row; every softmax thread takes part, so the exit is uniform
+    fin_ml[(2 * par) * 128 + row] = m_own;
+    fin_ml[(2 * par + 1) * 128 + row] = l_own;
+    bool fin = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_PV + (n_kv - 1) % NSB), ((n_kv - 1) / NSB) & 1,
+                                                      abort_flag));
+    fin = bar_red_and(BAR_L, NTH, fin);
+    if (!fin) {
       record_error(a.err, kErrWaitTimeout | 0x13);
       *abort_flag = 1;
     } else {
-      l += redmax[(n_kv & 1) * 256 + (half ^ 1) * 128 + row];
+      // O is at the last tile's m, the larger of the two warps' m
+      const float mo = fin_ml[(2 * (par ^ 1)) * 128 + row], lo = fin_ml[(2 * (par ^ 1) + 1) * 128 + row];
+      const float mf = fmaxf(m_own, mo);
+      const float l = (m_own == mf ? l_own : l_own * exp2f(m_own - mf)) + (mo == mf ? lo : lo * exp2f(mo - mf));
       tc_fence_after();
       const int t = tok0 + row / G;
       const float inv = 1.f / l;
-      __half* orow = a.out + (int64_t(sq.q_off + t) * b.Hq + h * G + row % G) * D + (D / 2) * half;
+      __half* orow = a.out + (int64_t(sq.q_off + t) * b.Hq + h * G + row % G) * D + (D / 2) * par;
 #pragma unroll 1
       for (int c = 0; c < D / 64; ++c) {
         uint32_t r32[32];
-        tmem_ld32(lane_addr + T::O_COL + (D / 2) * half + 32 * c, r32);
+        tmem_ld32(lane_addr + T::O_COL + (D / 2) * par + 32 * c, r32);
         tmem_wait_ld();
         if (t < sq.q_len) {
 #pragma unroll
