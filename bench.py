@@ -99,11 +99,15 @@ def ncu_traffic(workload: str, precision: str, kernel: str = "decode_split"):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    """nvidia-smi clocks, power and throttle reasons sampled every 100 ms (the four named reasons and
+    the whole active-reason mask, whose other bits are decoded by name)."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+              "clocks_event_reasons.sw_power_cap,clocks_event_reasons.active")
     NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+    MASK_NAMES = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+                  0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+                  0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
     def __init__(self, gpu_id: str):
         self.gpu_id = gpu_id
@@ -114,7 +118,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
         except OSError:
@@ -124,7 +128,7 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) == 7:
+            if len(parts) == 8:
                 self.samples.append(parts)
 
     def __exit__(self, *exc):
@@ -138,9 +142,23 @@ class ClockSampler:
     def summary(self) -> dict:
         sm = [float(s[0]) for s in self.samples if s[0].replace(".", "").isdigit()]
         mx = [float(s[1]) for s in self.samples if s[1].replace(".", "").isdigit()]
-        reasons = sorted({self.NAMES[i] for s in self.samples for i in range(4) if s[3 + i] == "Active"})
+        reasons = {self.NAMES[i] for s in self.samples for i in range(4) if s[3 + i] == "Active"}
+        mask = 0
+        for smp in self.samples:
+            try:
+                mask |= int(smp[7], 16)
+            except ValueError:
+                pass
+        reasons |= {name for bit, name in self.MASK_NAMES.items() if mask & bit and bit != 0x1}
+        pw = []
+        for smp in self.samples:
+            try:
+                pw.append(float(smp[2]))
+            except ValueError:
+                pass
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(self.samples)}
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "power_w": round(statistics.median(pw), 1) if pw else None, "reasons_mask": hex(mask)}
 
 
 # --------------------------------------------------------------------------- decode workload
