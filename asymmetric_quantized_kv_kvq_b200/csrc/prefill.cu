@@ -522,12 +522,15 @@ __global__ void __launch_bounds__(352, 1)
       wok = wok && __all_sync(0xffffffffu, mbar_wait(bar(B_S + sb), (j / NSB) & 1, abort_flag));
       const uint32_t sbuf = lane_addr + T::S_COL0 + sb * kKV;
       const int kpos0 = j * kKV;
-      // pass 1: the row's 128 raw scores and their max (sigma log2 e > 0 keeps the order); only
-      // 32-key chunks that reach past the first row's position need the causal mask
+      // pass 1: the row's 128 raw scores and their max (sigma log2 e > 0 keeps the order).  Only
+      // 32-key chunks that reach past the first row's position need the causal mask: there the
+      // keys past the row's position are set to -inf and the chunk is written back to S, so that
+      // the exponentials (2^-inf = 0) need no mask on any tile
       float mx = -INFINITY;
       if (wok) {
         tc_fence_after();
         float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        bool wrote = false;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {   // two reads of 64 keys
           uint32_t sv[64];
@@ -539,8 +542,13 @@ __global__ void __launch_bounds__(352, 1)
             const int c = 2 * hh + cc;
             if (kpos0 + 32 * c + 31 > qpos0) {
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                if (kpos0 + 32 * c + i <= qpos) mq[i & 3] = fmaxf(mq[i & 3], __uint_as_float(sv[32 * cc + i]));
+              for (int i = 0; i < 32; ++i) {
+                const float v = kpos0 + 32 * c + i <= qpos ? __uint_as_float(sv[32 * cc + i]) : -INFINITY;
+                sv[32 * cc + i] = __float_as_uint(v);
+                mq[i & 3] = fmaxf(mq[i & 3], v);
+              }
+              tmem_st32(sbuf + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&sv[32 * cc]));
+              wrote = true;
             } else {
               // four independent three-input max chains (a short dependency chain)
 #pragma unroll
@@ -553,6 +561,7 @@ __global__ void __launch_bounds__(352, 1)
           }
         }
         mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+        if (wrote) tmem_wait_st();                   // the masked chunks are in S before pass 2 reads them
       }
       mx *= a.scale_log2;
       // the running max after tile j - 1, from the quadrant's other warp
@@ -608,18 +617,12 @@ __global__ void __launch_bounds__(352, 1)
       for (int c = 0; c < 4; ++c) {
         if (wok && c < 3) tmem_ld32(sbuf + 32 * (c + 1), sv[(c + 1) & 1]);
         uint32_t pk[16];
-        const bool masked = kpos0 + 32 * c + 31 > qpos0;
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 x = ffma2(make_float2(__uint_as_float(sv[c & 1][2 * i]),
                                              __uint_as_float(sv[c & 1][2 * i + 1])), sc2, nm2);
-          float p0 = ex2_ftz(x.x);
-          float p1 = ex2_ftz(x.y);
-          if (masked) {
-            const int k0 = kpos0 + 32 * c + 2 * i;
-            p0 = k0 > qpos ? 0.f : p0;
-            p1 = k0 + 1 > qpos ? 0.f : p1;
-          }
+          const float p0 = ex2_ftz(x.x);   // 0 for a masked key (-inf)
+          const float p1 = ex2_ftz(x.y);
           l2 = fadd2(l2, make_float2(p0, p1));
           __half2 hp = __floats2half2_rn(p0, p1);
           pk[i] = *reinterpret_cast<uint32_t*>(&hp);
