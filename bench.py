@@ -905,7 +905,8 @@ def run_extras(args) -> list:
     from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS, parse_precision
     out = []
     sub = _ap.Namespace(**vars(args))
-    sub.steps, sub.warmup, sub.no_e2e, sub.decode_tc, sub.separate = 5, 3, True, False, False
+    # timed regions of a few hundred ms each, so that the clock sampler (100 ms) sees several samples
+    sub.steps, sub.warmup, sub.no_e2e, sub.decode_tc, sub.separate = 20, 3, True, False, False
     sub.dedup_probe = False
     for name, prec in (("llama70b-b1-128k", "K8V4"), ("llama70b-b1-128k", "FP16")):
         wl = WORKLOADS[name]
@@ -922,6 +923,7 @@ def run_extras(args) -> list:
     wl = WORKLOADS["prefill-16x4096"]
     kb, vb = parse_precision("K8V4")
     torch.cuda.empty_cache()
+    sub.steps = 10
     r = run_prefill_bench(sub, wl, kb, vb, 0, 1)
     peak = measured_tensor_peak()
     out.append({"workload": wl.name, "precision": "K8V4", "metric": PREFILL_METRIC, "value": r["value"],
