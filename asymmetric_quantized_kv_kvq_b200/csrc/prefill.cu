@@ -46,8 +46,11 @@
 //     row's 128 raw scores, takes their max, hands the running max on to the
 //     other warp at once (shared memory and a named barrier of the pair), and
 //     then computes the exponentials while the other warp reads and reduces
-//     tile j + 1, so the MUFU unit is kept busy.  sigma log2 e and the causal
-//     mask are applied, the online softmax moves the running max only when it
+//     tile j + 1, so the MUFU unit is kept busy.  The causal mask is applied in
+//     the read: on the chunks that reach past the tile's first row the keys
+//     beyond the row's position become -inf and are written back to S, so the
+//     exponentials carry no mask.  sigma log2 e is applied with the max
+//     subtracted, the online softmax moves the running max only when it
 //     grows by more than 2^8 (then O is rescaled in TMEM), and P is stored as
 //     fp16 pairs (tcgen05.st) over the first half of its own S buffer, where
 //     the PV MMA takes its A operand; the S buffer returns to the score MMAs
