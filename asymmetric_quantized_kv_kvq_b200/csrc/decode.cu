@@ -12,7 +12,7 @@ template <int KB, int VB>
 cudaError_t launch_decode_kv(const Layout&, int, const Batch&, const DecodePlan&, int, const void*, void*, const void*,
                              const void*, float, void*, cudaStream_t, bool*);
 template <int KB, int VB>
-int decode_chunk_tokens_kv(int D, int G);
+int decode_chunk_tokens_kv(int D, int G, int page_tokens);
 
 bool decode_tc_supported(const Layout& L, int G);
 int decode_tc_tile_tokens();
@@ -90,11 +90,11 @@ size_t decode_workspace_bytes(int n_items, int max_ctas, int G, int D) {
 static int stage_tokens(const Layout& L, int G) {
   const int kb = L.k_bits, vb = L.v_bits, D = L.head_dim;
   if (decode_tc_supported(L, G)) return decode_tc_tile_tokens();
-  if (kb == 16) return decode_chunk_tokens_kv<16, 16>(D, G);
-  if (kb == 8 && vb == 8) return decode_chunk_tokens_kv<8, 8>(D, G);
-  if (kb == 8 && vb == 4) return decode_chunk_tokens_kv<8, 4>(D, G);
-  if (kb == 4 && vb == 4) return decode_chunk_tokens_kv<4, 4>(D, G);
-  return decode_chunk_tokens_kv<4, 8>(D, G);
+  if (kb == 16) return decode_chunk_tokens_kv<16, 16>(D, G, L.page_tokens);
+  if (kb == 8 && vb == 8) return decode_chunk_tokens_kv<8, 8>(D, G, L.page_tokens);
+  if (kb == 8 && vb == 4) return decode_chunk_tokens_kv<8, 4>(D, G, L.page_tokens);
+  if (kb == 4 && vb == 4) return decode_chunk_tokens_kv<4, 4>(D, G, L.page_tokens);
+  return decode_chunk_tokens_kv<4, 8>(D, G, L.page_tokens);
 }
 
 // Work chunk = gcd(stage capacity, page_tokens): both are multiples of 64, the

@@ -4,5 +4,5 @@
 namespace kvq {
 template cudaError_t launch_decode_kv<16, 16>(const Layout&, int, const Batch&, const DecodePlan&, int, const void*,
                                               void*, const void*, const void*, float, void*, cudaStream_t, bool*);
-template int decode_chunk_tokens_kv<16, 16>(int, int);
+template int decode_chunk_tokens_kv<16, 16>(int, int, int);
 }  // namespace kvq

@@ -37,20 +37,20 @@ cudaError_t launch_decode_one(const Layout& L, int layer, const Batch& b, const 
   return cudaGetLastError();
 }
 
-template <int KB, int VB, int D, int G>
+template <int KB, int VB, int D, int G, int CT>
 cudaError_t launch_decode_q_one(const Layout& L, int layer, const Batch& b, const DecodePlan& plan, int n_q_heads,
                                 const void* q, void* out, const void* k_new, const void* v_new, float scale_log2,
                                 void* ws, cudaStream_t s) {
-  using T = QDec<KB, VB, D, G>;
+  using T = QDec<KB, VB, D, G, CT>;
   static bool configured = false;   // per instantiation; set once per process
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_q_kernel<KB, VB, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_q_kernel<KB, VB, D, G, CT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          T::SMEM);
     if (e != cudaSuccess) return e;
     // the in-kernel register split (setmaxnreg) adds up to the launch allocation; a build that
     // launched with fewer registers per thread would leave a growing warpgroup waiting
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, decode_q_kernel<KB, VB, D, G>);
+    e = cudaFuncGetAttributes(&fa, decode_q_kernel<KB, VB, D, G, CT>);
     if (e != cudaSuccess) return e;
     if (fa.numRegs != T::REG_L) return cudaErrorInvalidDeviceFunction;
     configured = true;
@@ -71,7 +71,7 @@ cudaError_t launch_decode_q_one(const Layout& L, int layer, const Batch& b, cons
   a.total_chunks = plan.total_chunks;
   a.cpc = plan.chunks_per_cta;
   a.chunk = plan.chunk_tokens;
-  decode_q_kernel<KB, VB, D, G><<<plan.n_cta, T::NT, T::SMEM, s>>>(a, b);
+  decode_q_kernel<KB, VB, D, G, CT><<<plan.n_cta, T::NT, T::SMEM, s>>>(a, b);
   return cudaGetLastError();
 }
 
@@ -85,10 +85,17 @@ cudaError_t launch_decode_kv(const Layout& L, int layer, const Batch& b, const D
   const int G = n_q_heads / L.n_kv_heads;
   if constexpr (KB != 16 && VB != 16) {
     *combined = true;
-#define KVQ_DECQ(D_, G_)                                                                                        \
-  if (L.head_dim == D_ && G == G_)                                                                              \
-    return launch_decode_q_one<KB, VB, D_, G_>(L, layer, b, plan, n_q_heads, q, out, k_new, v_new, scale_log2, \
-                                               ws, s);
+    // 256-token stages when the chunk is a whole 256 tokens (pages of 256k tokens) and three of them
+    // fit in shared memory; 128-token stages otherwise
+#define KVQ_DECQ(D_, G_)                                                                                         \
+  if (L.head_dim == D_ && G == G_) {                                                                             \
+    if constexpr (QDec<KB, VB, D_, G_, 256>::FITS)                                                               \
+      if (plan.chunk_tokens == 256)                                                                              \
+        return launch_decode_q_one<KB, VB, D_, G_, 256>(L, layer, b, plan, n_q_heads, q, out, k_new, v_new,      \
+                                                        scale_log2, ws, s);                                      \
+    return launch_decode_q_one<KB, VB, D_, G_, 128>(L, layer, b, plan, n_q_heads, q, out, k_new, v_new,          \
+                                                    scale_log2, ws, s);                                          \
+  }
     KVQ_DECQ(128, 1) KVQ_DECQ(128, 2) KVQ_DECQ(128, 4) KVQ_DECQ(128, 8)
     KVQ_DECQ(64, 1) KVQ_DECQ(64, 2) KVQ_DECQ(64, 4) KVQ_DECQ(64, 8)
 #undef KVQ_DECQ
@@ -105,14 +112,19 @@ cudaError_t launch_decode_kv(const Layout& L, int layer, const Batch& b, const D
   return cudaErrorInvalidValue;
 }
 
-// Tokens per work chunk of the kernel that runs for (D, G).
+// Stage capacity (tokens) of the kernel that runs for (D, G) on pages of page_tokens tokens.
 template <int KB, int VB>
-int decode_chunk_tokens_kv(int D, int G) {
+int decode_chunk_tokens_kv(int D, int G, int page_tokens) {
   if constexpr (KB != 16 && VB != 16) {
-    (void)D;
-    (void)G;
-    return QDec<KB, VB, 128, 4>::C;
+    const bool p256 = page_tokens % 256 == 0;
+#define KVQ_CQ(D_, G_) \
+  if (D == D_ && G == G_) return p256 && QDec<KB, VB, D_, G_, 256>::FITS ? 256 : 128;
+    KVQ_CQ(128, 1) KVQ_CQ(128, 2) KVQ_CQ(128, 4) KVQ_CQ(128, 8)
+    KVQ_CQ(64, 1) KVQ_CQ(64, 2) KVQ_CQ(64, 4) KVQ_CQ(64, 8)
+#undef KVQ_CQ
+    return 128;
   } else {
+    (void)page_tokens;
 #define KVQ_C(D_, G_) \
   if (D == D_ && G == G_) return DecodeTraits<KB, VB, D_, G_>::C;
     KVQ_C(128, 1) KVQ_C(128, 2) KVQ_C(128, 4) KVQ_C(128, 8)

@@ -75,9 +75,9 @@ struct DecodeQArgs {
   int chunk;             // tokens per work chunk (divides page_tokens, <= C)
 };
 
-template <int KB, int VB, int D, int G>
+template <int KB, int VB, int D, int G, int CT>
 struct QDec {
-  static constexpr int C = 128;                      // tokens per stage
+  static constexpr int C = CT;                       // tokens per stage (128, or 256 on 256-token pages)
   static constexpr int NB = D / 32;                  // 32-element blocks per row
   static constexpr int GW = G > 4 ? 4 : G;           // query heads per consumer warp
   static constexpr int NHG = G / GW;                 // warps sharing one partition (head groups)
@@ -121,7 +121,7 @@ struct QDec {
   static constexpr int S_FIT = (SMEM_LIMIT - FIXED) / STAGE;
   static constexpr int S = S_FIT > 8 ? 8 : S_FIT;    // stages in the ring
   static constexpr int SMEM = S * STAGE + FIXED;
-  static_assert(S >= 3, "stage ring does not fit");
+  static constexpr bool FITS = S_FIT >= 3;           // three stages of C tokens fit (checked by the kernel)
   static_assert(W % TPP == 0 && NPASS >= 1 && W % TPV == 0 && NPV >= 1, "tiling");
   static_assert(BPL % 4 == 0 && BPL <= VBLK, "a value lane's codes lie in one value block");
   static_assert(STAGE % 16 == 0 && OFF_KS % 16 == 0 && OFF_VC % 16 == 0 && OFF_VS % 16 == 0, "alignment");
@@ -226,9 +226,9 @@ __host__ __device__ constexpr int v_elem_of(int sl, int i) {
 }
 
 // Shared-memory carve-up and barriers of one CTA.
-template <int KB, int VB, int D, int G>
+template <int KB, int VB, int D, int G, int CT>
 struct QDecSmem {
-  using T = QDec<KB, VB, D, G>;
+  using T = QDec<KB, VB, D, G, CT>;
   uint8_t* stages;
   float* pbuf;          // [warp][PB_WARP bytes]  p' = p d_v [W][NB][GW], or the query digits
   float* mrg_o;         // [part][G][D]
@@ -263,11 +263,11 @@ struct QDecSmem {
 // (m, l) and O into the merge area: combine the partitions, write the output
 // (item inside this CTA) or this CTA's partial, and let the last CTA of a
 // split item merge all partials.  Returns false when a wait gave up.
-template <int KB, int VB, int D, int G>
-__device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<KB, VB, D, G>& sm,
+template <int KB, int VB, int D, int G, int CT>
+__device__ __forceinline__ bool merge_item(const DecodeQArgs& a, const QDecSmem<KB, VB, D, G, CT>& sm,
                                            const DecodeSeg& sg, const SeqDesc& sd, uint32_t& itm,
                                            uint32_t& itw, uint32_t& itc) {
-  using T = QDec<KB, VB, D, G>;
+  using T = QDec<KB, VB, D, G, CT>;
   constexpr int NPART = T::NPART, NW = T::NW;
   const int lane = threadIdx.x & 31;
   const int H = a.L.n_kv_heads;
@@ -545,10 +545,10 @@ __device__ __forceinline__ void new_row_store(uint8_t* codes, __half* scale, boo
 
 // Producer warp: streams the CTA's chunks into the stage ring (and, with a fused
 // append, quantises each item's new token into its page and the stage).
-template <int KB, int VB, int D, int G>
+template <int KB, int VB, int D, int G, int CT>
 __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch& b,
-                                              const QDecSmem<KB, VB, D, G>& sm, int64_t x0, int64_t x1, int page0) {
-  using T = QDec<KB, VB, D, G>;
+                                              const QDecSmem<KB, VB, D, G, CT>& sm, int64_t x0, int64_t x1, int page0) {
+  using T = QDec<KB, VB, D, G, CT>;
   constexpr int S = T::S, NB = T::NB;
   const int lane = threadIdx.x & 31;
   const int H = a.L.n_kv_heads;
@@ -649,9 +649,9 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
 
 // A consumer warp's state for one item segment: the query digits of its heads,
 // its running softmax and its accumulators.
-template <int KB, int VB, int D, int G>
+template <int KB, int VB, int D, int G, int CT>
 struct QWarp {
-  using T = QDec<KB, VB, D, G>;
+  using T = QDec<KB, VB, D, G, CT>;
   uint32_t qh[T::GW][8], ql[T::GW][8];   // query digits of the lane's key block, slot j = head j ^ fmap
   int qcorr[T::GW];                      // 4-bit keys: -8 * sum of the digits (codes are read as c + 8)
   float qsc[T::NF], m[T::NF], l[T::NF];  // per owned head: digit scale, running max and sum
@@ -670,11 +670,11 @@ struct QLaneOff {
 
 // Score passes of one stage: sc[pass][j] for the lane's token and owned heads (-inf outside
 // the valid rows [rv0, rv1) of the chunk; row0 = the lane's row in pass 0).
-template <int KB, int VB, int D, int G>
-__device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G>& w, uint32_t u_st, const QLaneOff& lo, int row0,
+template <int KB, int VB, int D, int G, int CT>
+__device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G, CT>& w, uint32_t u_st, const QLaneOff& lo, int row0,
                                          bool masked, int rv0, int rv1,
-                                         float (&sc)[QDec<KB, VB, D, G>::NPASS][QDec<KB, VB, D, G>::NF]) {
-  using T = QDec<KB, VB, D, G>;
+                                         float (&sc)[QDec<KB, VB, D, G, CT>::NPASS][QDec<KB, VB, D, G, CT>::NF]) {
+  using T = QDec<KB, VB, D, G, CT>;
   constexpr int GW = T::GW, NF = T::NF;
 #pragma unroll
   for (int ps = 0; ps < T::NPASS; ++ps) {
@@ -726,9 +726,9 @@ __device__ __forceinline__ void fma_pair(float& o0, float& o1, float p, float x0
 }
 
 // Value passes of one stage: O += p' c over the lane's tokens of the partition.
-template <int KB, int VB, int D, int G>
-__device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G>& w, uint32_t u_st, uint32_t u_pb, const QLaneOff& lo) {
-  using T = QDec<KB, VB, D, G>;
+template <int KB, int VB, int D, int G, int CT>
+__device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G, CT>& w, uint32_t u_st, uint32_t u_pb, const QLaneOff& lo) {
+  using T = QDec<KB, VB, D, G, CT>;
   constexpr int GW = T::GW, NB = T::NB;
 #pragma unroll
   for (int pv = 0; pv < T::NPV; ++pv) {
@@ -782,12 +782,12 @@ __device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G>& w, uint32_t u_st, 
 
 // Online softmax of one stage's scores, then p' = p d_v into the warp's buffer (which the
 // warp's value passes of the previous stage have finished reading).
-template <int KB, int VB, int D, int G>
-__device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G>& w,
-                                              const float (&sc)[QDec<KB, VB, D, G>::NPASS][QDec<KB, VB, D, G>::NF],
+template <int KB, int VB, int D, int G, int CT>
+__device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G, CT>& w,
+                                              const float (&sc)[QDec<KB, VB, D, G, CT>::NPASS][QDec<KB, VB, D, G, CT>::NF],
                                               uint32_t u_st, uint32_t u_pb, const QLaneOff& lo, int row0, bool masked,
                                               int rv0, int rv1) {
-  using T = QDec<KB, VB, D, G>;
+  using T = QDec<KB, VB, D, G, CT>;
   constexpr int GW = T::GW, NF = T::NF, LPT = T::LPT, NB = T::NB;
   constexpr uint32_t FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
@@ -851,10 +851,10 @@ __device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G>& w,
 
 // Consumer warp: for each item segment of the CTA's range, the query digits, then the
 // stage pipeline (scores of stage k with the values of stage k - 1), then the merge.
-template <int KB, int VB, int D, int G>
-__device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch& b, const QDecSmem<KB, VB, D, G>& sm,
+template <int KB, int VB, int D, int G, int CT>
+__device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch& b, const QDecSmem<KB, VB, D, G, CT>& sm,
                                               int64_t x0, int64_t x1) {
-  using T = QDec<KB, VB, D, G>;
+  using T = QDec<KB, VB, D, G, CT>;
   constexpr int S = T::S, GW = T::GW, NF = T::NF, LPT = T::LPT, NHG = T::NHG, E = T::E;
   constexpr uint32_t FULL = 0xffffffffu;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -879,7 +879,7 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
     lo.pld = uint32_t((tv * T::NB + (sl * T::BPL) / T::VBLK) * GW * 4);
   }
   const int row0 = prow0 + tl;
-  QWarp<KB, VB, D, G> w;
+  QWarp<KB, VB, D, G, CT> w;
   uint32_t itm = 0, itw = 0, itc = 0;
   int s = 0;                                           // ring slot of the next stage and its fill parity
   uint32_t ph = 0;
@@ -1004,15 +1004,15 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
       const bool masked = rv0 > prow0 || rv1 < prow0 + T::W;
       float sc[T::NPASS][NF];
       if (k == sg.k0) {
-        qk_stage<KB, VB, D, G>(w, u_st, lo, row0, masked, rv0, rv1, sc);
+        qk_stage<KB, VB, D, G, CT>(w, u_st, lo, row0, masked, rv0, rv1, sc);
       } else {
         // one straight-line block: the previous stage's values and this stage's scores
-        qk_stage<KB, VB, D, G>(w, u_st, lo, row0, masked, rv0, rv1, sc);
-        pv_stage<KB, VB, D, G>(w, u_prev, u_pb, lo);
+        qk_stage<KB, VB, D, G, CT>(w, u_st, lo, row0, masked, rv0, rv1, sc);
+        pv_stage<KB, VB, D, G, CT>(w, u_prev, u_pb, lo);
         __syncwarp();
         mbar_arrive_if(sm.empty0 + 8 * s_prev, lane == 0);
       }
-      softmax_stage<KB, VB, D, G>(w, sc, u_st, u_pb, lo, row0, masked, rv0, rv1);
+      softmax_stage<KB, VB, D, G, CT>(w, sc, u_st, u_pb, lo, row0, masked, rv0, rv1);
       u_prev = u_st;
       s_prev = s;
       if (++s == S) {
@@ -1020,7 +1020,7 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
         ph ^= 1;
       }
     }
-    pv_stage<KB, VB, D, G>(w, u_prev, u_pb, lo);
+    pv_stage<KB, VB, D, G, CT>(w, u_prev, u_pb, lo);
     __syncwarp();
     mbar_arrive_if(sm.empty0 + 8 * s_prev, lane == 0);
 
@@ -1055,7 +1055,7 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
 #pragma unroll
         for (int i = 0; i < E; ++i) mo[g * D + v_elem_of<VB, E>(sl, i)] = w.O[g][i];
     }
-    if (!merge_item<KB, VB, D, G>(a, sm, sg, sd, itm, itw, itc)) return;
+    if (!merge_item<KB, VB, D, G, CT>(a, sm, sg, sd, itm, itw, itc)) return;
     x += sg.adv;
   }
 }
@@ -1069,12 +1069,13 @@ __device__ __forceinline__ void set_max_regs() {
   else if constexpr (R < R_LAUNCH) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
 }
 
-template <int KB, int VB, int D, int G>
-__global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
+template <int KB, int VB, int D, int G, int CT>
+__global__ void __launch_bounds__(QDec<KB, VB, D, G, CT>::NT, 1)
     decode_q_kernel(const DecodeQArgs a, const __grid_constant__ Batch b) {
-  using T = QDec<KB, VB, D, G>;
+  using T = QDec<KB, VB, D, G, CT>;
+  static_assert(T::FITS, "stage ring does not fit");
   extern __shared__ __align__(128) uint8_t smem[];
-  const QDecSmem<KB, VB, D, G> sm(smem);
+  const QDecSmem<KB, VB, D, G, CT> sm(smem);
   const int warp = threadIdx.x >> 5;
   const int64_t x0 = int64_t(blockIdx.x) * a.cpc;
   const int64_t x1 = min(a.total_chunks, x0 + a.cpc);
@@ -1097,11 +1098,11 @@ __global__ void __launch_bounds__(QDec<KB, VB, D, G>::NT, 1)
   __syncthreads();
   if (warp >= T::NW) {
     set_max_regs<T::REG_P, T::REG_L>();
-    if (warp == T::NW) producer_role<KB, VB, D, G>(a, b, sm, x0, x1, page0);
+    if (warp == T::NW) producer_role<KB, VB, D, G, CT>(a, b, sm, x0, x1, page0);
     return;                                                 // the group's other 3 warps have no role
   }
   set_max_regs<T::REG_C, T::REG_L>();
-  consumer_role<KB, VB, D, G>(a, b, sm, x0, x1);
+  consumer_role<KB, VB, D, G, CT>(a, b, sm, x0, x1);
 }
 
 }  // namespace kvq

@@ -778,7 +778,19 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   for (int i = 0; i < n; ++i) windowed |= c->window[ids[i]] != 0;
   if (windowed) LV.decode_tc = 0;       // rotating windows run on the CUDA-core kernels
   plan.chunk_tokens = kvq::decode_chunk_tokens(LV, G);
-  const int C = plan.chunk_tokens, H = c->L.n_kv_heads;
+  const int H = c->L.n_kv_heads;
+  const int max_ctas = kvq::decode_max_ctas(c->num_sms);
+  if (plan.chunk_tokens == 256) {
+    // 256-token stages pay off when every CTA gets at least two of them (the consumer overlaps one
+    // stage's scores with the previous stage's values); a smaller step keeps 128-token stages
+    int64_t n256 = 0;
+    for (int i = 0; i < n; ++i) {
+      const int64_t len = c->len[ids[i]], lo = first_attended(c, ids[i]);
+      n256 += int64_t(H) * ((len - lo / 256 * 256 + 255) / 256);
+    }
+    if (n256 < 2 * int64_t(max_ctas)) plan.chunk_tokens = 128;
+  }
+  const int C = plan.chunk_tokens;
   kvq::Batch b;
   b.n = n;
   int64_t flat = 0;
@@ -793,7 +805,6 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
     max_nch = std::max(max_nch, nch);
   }
   if (flat >= (int64_t(1) << 31)) return fail(KVQ_ERR_INVALID_ARG, "batch too large");
-  const int max_ctas = kvq::decode_max_ctas(c->num_sms);
   // Every CTA takes cpc consecutive chunks of the flat (sequence, head, chunk) list.  When the
   // grid still fits in max_ctas, each item is padded to a whole number of CTA ranges, so that no
   // range crosses an item (such a CTA runs two items back to back, each with its own merge), and

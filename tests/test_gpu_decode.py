@@ -44,6 +44,25 @@ def test_decode_matches_oracle(kb, vb, D, H, G):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("kb,vb", [(8, 4), (8, 8), (4, 4), (4, 8)])
+@pytest.mark.parametrize("D,G", [(128, 4), (128, 8), (64, 8), (64, 1)])
+def test_decode_256_token_stages(kb, vb, D, G):
+    """A step with at least two 256-token chunks per CTA on 256-token pages runs the kernel with
+    256-token stages (128-token ones where three of them do not fit, K8V8 at head_dim 128); the
+    second sequence ends in a ragged chunk."""
+    m = kvq()
+    H = 8
+    lens = [10000, 300]
+    cache, ids, hat = _build(m, kb, vb, D, H, lens)
+    q = random_fp16((len(lens), H * G, D), 11 + G)
+    out = cache.decode(0, ids, q.cuda())
+    cache.check()
+    ref = oracle.attention_decode_batch(q.numpy(), [hat[(0, s)] for s in ids])
+    assert_close_attention(out, ref, f"K{kb}V{vb} D{D} G{G}")
+    cache.close()
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("kb,vb", [(8, 4), (16, 16)])
 def test_decode_long_sequence_spans_many_ctas(kb, vb):
     """One long sequence: every item is split over many CTAs and merged by the combine kernel."""

@@ -76,6 +76,41 @@ def test_decode_append_matches_oracle_and_the_separate_calls(kb, vb, D, H, G):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("kb,vb", [(8, 4), (4, 4), (4, 8), (8, 8)])
+@pytest.mark.parametrize("D,G", [(128, 4), (64, 8)])
+def test_decode_append_256_token_stages(kb, vb, D, G):
+    """A step large enough for 256-token stages (at least two 256-token chunks per CTA): the new token
+    lands at the start, inside and at the end of a 256-token chunk; the fused step equals the separate
+    calls bit for bit and the oracle within tolerance, and the appended row is bit-exact."""
+    m = kvq()
+    H = 8
+    lens = [10000, 255, 256, 511]
+    cache, ids, raw = _fill(m, kb, vb, D, H, lens)
+    twin, _, _ = _fill(m, kb, vb, D, H, lens)
+    B = len(lens)
+    k_new = decode_kv(B, H, D, 5252)
+    v_new = random_fp16((B, H, D), 5353)
+    q = random_fp16((B, H * G, D), 5454)
+    cache.extend(ids, [1] * B)
+    out = cache.decode_append(0, ids, q.cuda(), k_new.cuda(), v_new.cuda())
+    cache.check()
+    twin.extend(ids, [1] * B)
+    twin.append(0, ids, [1] * B, k_new.cuda(), v_new.cuda())
+    sep = twin.decode(0, ids, q.cuda())
+    twin.check()
+    assert torch.equal(out, sep), "fused step differs from append + decode"
+    kv = []
+    for s in ids:
+        _check_row(cache, 0, s, lens[s], k_new[s:s + 1], v_new[s:s + 1], kb, vb)
+        k = torch.cat([raw[(0, s)][0], k_new[s:s + 1]])
+        v = torch.cat([raw[(0, s)][1], v_new[s:s + 1]])
+        kv.append((oracle_dequant(k, kb), oracle_dequant(v, vb)))
+    assert_close_attention(out, oracle.attention_decode_batch(q.numpy(), kv), f"K{kb}V{vb} D{D} G{G}")
+    cache.close()
+    twin.close()
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("kb,vb", [(8, 4), (4, 8)])
 def test_decode_append_serving_loop_across_pages(kb, vb):
     """300 one-token steps on two layers with 64-token pages: every step's output against the oracle at a
