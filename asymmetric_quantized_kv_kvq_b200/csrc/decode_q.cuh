@@ -670,7 +670,7 @@ struct QLaneOff {
 
 // Score passes of one stage: sc[pass][j] for the lane's token and owned heads (-inf outside
 // the valid rows [rv0, rv1) of the chunk; row0 = the lane's row in pass 0).
-template <int KB, int VB, int D, int G, int CT>
+template <int KB, int VB, int D, int G, int CT, bool MASK = true>
 __device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G, CT>& w, uint32_t u_st, const QLaneOff& lo, int row0,
                                          bool masked, int rv0, int rv1,
                                          float (&sc)[QDec<KB, VB, D, G, CT>::NPASS][QDec<KB, VB, D, G, CT>::NF]) {
@@ -712,7 +712,10 @@ __device__ __forceinline__ void qk_stage(const QWarp<KB, VB, D, G, CT>& w, uint3
 #pragma unroll
     for (int j = 0; j < NF; ++j) {
       const float v = ps_[j] * w.qsc[j];
-      sc[ps][j] = (!masked || (row >= rv0 && row < rv1)) ? v : -INFINITY;
+      if constexpr (MASK)
+        sc[ps][j] = (!masked || (row >= rv0 && row < rv1)) ? v : -INFINITY;
+      else
+        sc[ps][j] = v;
     }
   }
 }
@@ -782,7 +785,7 @@ __device__ __forceinline__ void pv_stage(QWarp<KB, VB, D, G, CT>& w, uint32_t u_
 
 // Online softmax of one stage's scores, then p' = p d_v into the warp's buffer (which the
 // warp's value passes of the previous stage have finished reading).
-template <int KB, int VB, int D, int G, int CT>
+template <int KB, int VB, int D, int G, int CT, bool MASK = true>
 __device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G, CT>& w,
                                               const float (&sc)[QDec<KB, VB, D, G, CT>::NPASS][QDec<KB, VB, D, G, CT>::NF],
                                               uint32_t u_st, uint32_t u_pb, const QLaneOff& lo, int row0, bool masked,
@@ -824,7 +827,7 @@ __device__ __forceinline__ void softmax_stage(QWarp<KB, VB, D, G, CT>& w,
 #pragma unroll
   for (int ps = 0; ps < T::NPASS; ++ps) {
     const int row = row0 + ps * T::TPP;
-    const bool valid = !masked || (row >= rv0 && row < rv1);
+    const bool valid = !MASK || !masked || (row >= rv0 && row < rv1);
     float p[NF];
 #pragma unroll
     for (int j = 0; j < NF; ++j) {
@@ -1003,16 +1006,28 @@ __device__ __forceinline__ void consumer_role(const DecodeQArgs& a, const Batch&
       const int rv0 = max(0, sd.lo - tok0), rv1 = min(a.chunk, sd.a - tok0);   // valid rows [rv0, rv1)
       const bool masked = rv0 > prow0 || rv1 < prow0 + T::W;
       float sc[T::NPASS][NF];
-      if (k == sg.k0) {
-        qk_stage<KB, VB, D, G, CT>(w, u_st, lo, row0, masked, rv0, rv1, sc);
-      } else {
-        // one straight-line block: the previous stage's values and this stage's scores
-        qk_stage<KB, VB, D, G, CT>(w, u_st, lo, row0, masked, rv0, rv1, sc);
+      // the steady state (a full stage after the first) in a copy without the row mask, whose selects
+      // the compiler would otherwise run on every stage; at G = 8 the doubled block costs more than it saves
+      bool steady = false;
+      if constexpr (T::NHG == 1) steady = k != sg.k0 && !masked;
+      if (steady) {
+        qk_stage<KB, VB, D, G, CT, false>(w, u_st, lo, row0, false, rv0, rv1, sc);
         pv_stage<KB, VB, D, G, CT>(w, u_prev, u_pb, lo);
         __syncwarp();
         mbar_arrive_if(sm.empty0 + 8 * s_prev, lane == 0);
+        softmax_stage<KB, VB, D, G, CT, false>(w, sc, u_st, u_pb, lo, row0, false, rv0, rv1);
+      } else {
+        if (k == sg.k0) {
+          qk_stage<KB, VB, D, G, CT>(w, u_st, lo, row0, masked, rv0, rv1, sc);
+        } else {
+          // one straight-line block: the previous stage's values and this stage's scores
+          qk_stage<KB, VB, D, G, CT>(w, u_st, lo, row0, masked, rv0, rv1, sc);
+          pv_stage<KB, VB, D, G, CT>(w, u_prev, u_pb, lo);
+          __syncwarp();
+          mbar_arrive_if(sm.empty0 + 8 * s_prev, lane == 0);
+        }
+        softmax_stage<KB, VB, D, G, CT>(w, sc, u_st, u_pb, lo, row0, masked, rv0, rv1);
       }
-      softmax_stage<KB, VB, D, G, CT>(w, sc, u_st, u_pb, lo, row0, masked, rv0, rv1);
       u_prev = u_st;
       s_prev = s;
       if (++s == S) {
