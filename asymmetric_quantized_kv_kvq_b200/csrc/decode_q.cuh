@@ -22,8 +22,12 @@
 //    memory stages with 1-D TMA bulk copies; with a fused append it first
 //    quantises the new token's K and V row into the page (same block
 //    quantiser as the append kernel), for the one chunk that holds it;
-//  - a stage's 128 tokens are split into partitions, one per consumer warp (at
-//    8 query heads per KV head two warps share a partition, 4 heads each); a
+//  - a stage holds one chunk: 256 tokens on pages of a multiple of 256 tokens
+//    when three such stages fit and the step gives every CTA at least two of
+//    them (fewer, larger stages halve the per-stage control work per token),
+//    else 128 (the stage size is the template parameter CT); its tokens are
+//    split into partitions, one per consumer warp (at 8 query heads per KV
+//    head two warps share a partition, 4 heads each); a
 //    warp keeps its own running softmax (m, l per head) and accumulators O, so
 //    consumer warps never wait for one another inside an item;
 //  - a warp is software-pipelined by one stage: the score passes of stage k and
