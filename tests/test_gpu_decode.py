@@ -63,6 +63,22 @@ def test_decode_256_token_stages(kb, vb, D, G):
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("page_tokens", [512, 768])
+def test_decode_256_token_stages_in_larger_pages(page_tokens):
+    """256-token chunks at offsets 0, 256 (and 512) inside one page."""
+    m = kvq()
+    D, H, G = 128, 8, 4
+    lens = [10000, 700]
+    cache, ids, hat = _build(m, 8, 4, D, H, lens, page_tokens=page_tokens)
+    q = random_fp16((len(lens), H * G, D), 21)
+    out = cache.decode(0, ids, q.cuda())
+    cache.check()
+    ref = oracle.attention_decode_batch(q.numpy(), [hat[(0, s)] for s in ids])
+    assert_close_attention(out, ref, f"pages of {page_tokens}")
+    cache.close()
+
+
+@pytest.mark.gpu
 @pytest.mark.parametrize("kb,vb", [(8, 4), (16, 16)])
 def test_decode_long_sequence_spans_many_ctas(kb, vb):
     """One long sequence: every item is split over many CTAs and merged by the combine kernel."""
