@@ -66,3 +66,49 @@ def test_windowed_decode_matches_oracle(kb, vb, D, H, G):
     if kb != 16:
         assert (exp["k_codes"].cpu().numpy() == kc).all()
     cache.close()
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("kb,vb", [(8, 4), (4, 8)])
+def test_windowed_decode_256_token_stages(kb, vb):
+    """The pages' 8192-token window on 256-token pages, in a step large enough for 256-token stages:
+    two windowed sequences whose rings have wrapped (the window starts inside a chunk, so its first
+    stage is masked) next to an unwindowed one, decode and the fused step against the oracle."""
+    m = kvq()
+    D, H, G, P, W = 128, 8, 4, 256, 8192
+    cache = m.Cache(n_layers=1, n_kv_heads=H, head_dim=D, k_bits=kb, v_bits=vb, max_seqs=3,
+                    max_tokens=P * 140, page_tokens=P, max_seq_tokens=P * 48)
+    cache.set_window(0, W)
+    cache.set_window(2, W)
+    ids = [0, 1, 2]
+    hist = {s: ([], []) for s in ids}
+    for step, n in enumerate([[4000, 4000, 3000], [4000, 4000, 3000], [3100, 2100, 2950]]):
+        cache.extend(ids, n)
+        ks = [decode_kv(x, H, D, 300 + 10 * step + s) for s, x in enumerate(n)]
+        vs = [random_fp16((x, H, D), 700 + 10 * step + s) for s, x in enumerate(n)]
+        cache.append(0, ids, n, torch.cat(ks).cuda(), torch.cat(vs).cuda())
+        for s in ids:
+            hist[s][0].append(ks[s])
+            hist[s][1].append(vs[s])
+    windows = [W, 0, W]
+    q = random_fp16((3, H * G, D), 901)
+    out = cache.decode(0, ids, q.cuda())
+    cache.check()
+    ref = np.stack([oracle.attention_decode_window(
+        q[s].numpy(), oracle_dequant(torch.cat(hist[s][0]), kb), oracle_dequant(torch.cat(hist[s][1]), vb),
+        windows[s]) for s in ids])
+    assert_close_attention(out, ref, "256-token stages, windows")
+    cache.extend(ids, [1, 1, 1])
+    k1 = decode_kv(3, H, D, 911)
+    v1 = random_fp16((3, H, D), 912)
+    q = random_fp16((3, H * G, D), 913)
+    out = cache.decode_append(0, ids, q.cuda(), k1.cuda(), v1.cuda())
+    cache.check()
+    for s in ids:
+        hist[s][0].append(k1[s:s + 1])
+        hist[s][1].append(v1[s:s + 1])
+    ref = np.stack([oracle.attention_decode_window(
+        q[s].numpy(), oracle_dequant(torch.cat(hist[s][0]), kb), oracle_dequant(torch.cat(hist[s][1]), vb),
+        windows[s]) for s in ids])
+    assert_close_attention(out, ref, "256-token stages, windows, fused step")
+    cache.close()
