@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(256) append_kernel(const Layout L, int layer, 
     return;
   }
   const int r = pos % L.page_tokens;
-  uint8_t* hb = L.head_ptr(layer, page, h);
+  uint8_t* hb = L.head_ptr(layer + sd.l, page, h);
   const int bitsw = kv ? L.v_bits : L.k_bits;
   uint8_t* codes_row = hb + (kv ? L.v_codes_off : 0) + int64_t(r) * (kv ? L.v_row : L.k_row);
   __half* scales_row = reinterpret_cast<__half*>(hb + (kv ? L.v_scales_off : L.k_scales_off) + int64_t(r) * L.s_row);

@@ -280,7 +280,7 @@ __global__ void __launch_bounds__(DecodeTraits<KB, VB, D, G>::NT, 1)
         }
         if (lane == 0) {
           const int r = tok0 % a.L.page_tokens;
-          const uint8_t* hb = a.L.head_ptr(a.layer, page, sg.h);
+          const uint8_t* hb = a.L.head_ptr(a.layer + sd.l, page, sg.h);
           const uint32_t bar = full0 + 8 * s;
           const uint32_t dst = smem_u32(stages + s * T::STAGE_BYTES);
           mbar_arrive_expect_tx(bar, uint32_t(ncopy * T::TOK_BYTES));

@@ -591,7 +591,7 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
         break;
       }
       const int r = tok0 % a.L.page_tokens;
-      uint8_t* hb = a.L.head_ptr(a.layer, page, sg.h);
+      uint8_t* hb = a.L.head_ptr(a.layer + sd.l, page, sg.h);
       // fused append: this chunk holds the new token (position len - 1, chunk row ntok - 1)
       const bool app = a.k_new != nullptr && tok0 + ntok == sd.a;
       // test hook (cache created with KVQ_TEST_WITHHOLD_ARRIVAL set): CTA 0 never fills its

@@ -747,18 +747,13 @@ kvq_status kvq_decode_workspace_size(const kvq_cache* c, int32_t n, int32_t n_q_
 
 namespace {
 
-// kvq_decode_attn, and with k_new / v_new the appending variant: position
-// len - 1 of every named sequence is quantised first (fused into the decode
-// kernel for quantized caches, a separate append launch otherwise).
-kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, int32_t n_q_heads, const void* q,
-                       const void* k_new, const void* v_new, void* out, float softmax_scale, void* ws,
-                       size_t ws_bytes, kvq_stream_t stream) {
-  if (kvq_status s = check_cache(c)) return s;
-  if (kvq_status s = check_layer(c, layer)) return s;
+// Argument checks shared by the decode calls (not the layer or the workspace size); *G = the GQA group.
+kvq_status decode_check(kvq_cache* c, int32_t n, const int32_t* ids, int32_t n_q_heads, const void* q,
+                        const void* k_new, const void* v_new, void* out, float softmax_scale, void* ws, int* G) {
   if (kvq_status s = check_ids(c, n, ids)) return s;
   if (n_q_heads < 1 || n_q_heads % c->L.n_kv_heads) return fail(KVQ_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
-  const int G = n_q_heads / c->L.n_kv_heads;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(KVQ_ERR_UNSUPPORTED, "GQA group %d not built (1, 2, 4, 8)", G);
+  *G = n_q_heads / c->L.n_kv_heads;
+  if (*G != 1 && *G != 2 && *G != 4 && *G != 8) return fail(KVQ_ERR_UNSUPPORTED, "GQA group %d not built (1, 2, 4, 8)", *G);
   if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "q or out is NULL");
   if (!aligned16(q) || !aligned16(out)) return fail(KVQ_ERR_INVALID_ARG, "q and out must be 16-byte aligned");
   const bool appending = k_new || v_new;
@@ -767,16 +762,38 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
     return fail(KVQ_ERR_INVALID_ARG, "k_new and v_new must be 16-byte aligned");
   if (ws && !aligned16(ws)) return fail(KVQ_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   if (!(softmax_scale >= 0.f) || std::isinf(softmax_scale)) return fail(KVQ_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
-  size_t need = 0;
-  if (kvq_status s = kvq_decode_workspace_size(c, n, n_q_heads, &need)) return s;
-  if (!ws || ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
-  if (kvq_status s = need_device(c)) return s;
+  for (int i = 0; i < n; ++i)
+    if (c->len[ids[i]] < 1) return fail(KVQ_ERR_INVALID_ARG, "sequence %d is empty", ids[i]);
+  return KVQ_OK;
+}
 
+// Layers from `layer` (at most n_layers) that one layer-batched launch takes: consecutive layers
+// of the first one's format, whose entries (layers x sequences) fit one batch.
+int32_t decode_run_layers(const kvq_cache* c, int32_t layer, int32_t n_layers, int32_t n) {
+  const int32_t cap = std::max<int32_t>(1, kvq::kMaxBatch / n);
+  int32_t nl = 1;
+  while (nl < n_layers && nl < cap && c->k_bits[layer + nl] == c->k_bits[layer] &&
+         c->v_bits[layer + nl] == c->v_bits[layer])
+    ++nl;
+  return nl;
+}
+
+// One decode launch over the entries (layer + l, ids[i]) for l < nl, i < n, entry e = l n + i
+// (rows of q, out, k_new, v_new in that order); with k_new / v_new, position len - 1 of every
+// entry is quantised first (fused into the decode kernel for quantized caches, a separate
+// append launch otherwise).  The nl layers share a format (their head blocks lie one layer's
+// pool apart), so they are one launch's Layout.  batched: part of a layer-batched call.
+// Arguments are checked by the caller.
+kvq_status decode_run(kvq_cache* c, int32_t layer, int32_t nl, bool batched, int32_t n, const int32_t* ids, int G,
+                      int32_t n_q_heads, const void* q, const void* k_new, const void* v_new, void* out,
+                      float softmax_scale, void* ws, kvq_stream_t stream) {
+  const bool appending = k_new != nullptr;
   kvq::DecodePlan plan;
   kvq::Layout LV = c->layers[layer];
   bool windowed = false;
   for (int i = 0; i < n; ++i) windowed |= c->window[ids[i]] != 0;
-  if (windowed) LV.decode_tc = 0;       // rotating windows run on the CUDA-core kernels
+  // rotating windows and layer-batched calls run on the CUDA-core kernels
+  if (windowed || batched) LV.decode_tc = 0;
   plan.chunk_tokens = kvq::decode_chunk_tokens(LV, G);
   const int H = c->L.n_kv_heads;
   const int max_ctas = kvq::decode_max_ctas(c->num_sms);
@@ -786,26 +803,27 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
     int64_t n256 = 0;
     for (int i = 0; i < n; ++i) {
       const int64_t len = c->len[ids[i]], lo = first_attended(c, ids[i]);
-      n256 += int64_t(H) * ((len - lo / 256 * 256 + 255) / 256);
+      n256 += int64_t(nl) * H * ((len - lo / 256 * 256 + 255) / 256);
     }
     if (n256 < 2 * int64_t(max_ctas)) plan.chunk_tokens = 128;
   }
   const int C = plan.chunk_tokens;
+  const int ne = nl * n;                             // entries, <= kMaxBatch
   kvq::Batch b;
-  b.n = n;
+  b.n = ne;
   int64_t flat = 0;
   int32_t max_nch = 0;
-  for (int i = 0; i < n; ++i) {
-    const int64_t len = c->len[ids[i]];
-    if (len < 1) return fail(KVQ_ERR_INVALID_ARG, "sequence %d is empty", ids[i]);
-    const int64_t lo = first_attended(c, ids[i]), base = lo / C * C;
-    const int32_t nch = int32_t((len - base + C - 1) / C);
-    b.s[i] = {ids[i], int32_t(len), 0, nch, int32_t(lo), ring_pages(c, ids[i]), nch};
-    flat += int64_t(H) * nch;
-    max_nch = std::max(max_nch, nch);
-  }
+  for (int l = 0; l < nl; ++l)
+    for (int i = 0; i < n; ++i) {
+      const int64_t len = c->len[ids[i]];
+      const int64_t lo = first_attended(c, ids[i]), base = lo / C * C;
+      const int32_t nch = int32_t((len - base + C - 1) / C);
+      b.s[l * n + i] = {ids[i], int32_t(len), 0, nch, int32_t(lo), ring_pages(c, ids[i]), nch, l};
+      flat += int64_t(H) * nch;
+      max_nch = std::max(max_nch, nch);
+    }
   if (flat >= (int64_t(1) << 31)) return fail(KVQ_ERR_INVALID_ARG, "batch too large");
-  // Every CTA takes cpc consecutive chunks of the flat (sequence, head, chunk) list.  When the
+  // Every CTA takes cpc consecutive chunks of the flat (entry, head, chunk) list.  When the
   // grid still fits in max_ctas, each item is padded to a whole number of CTA ranges, so that no
   // range crosses an item (such a CTA runs two items back to back, each with its own merge), and
   // items of at most kWholeItemChunks chunks go to one CTA whole (nothing to merge across CTAs).
@@ -814,18 +832,18 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   if (!kvq::decode_tc_supported(LV, G)) {
     const int64_t cp = max_nch <= kWholeItemChunks ? std::max<int64_t>(cpc, max_nch) : cpc;
     int64_t pf = 0;
-    for (int i = 0; i < n; ++i) pf += int64_t(H) * ((b.s[i].c + cp - 1) / cp) * cp;
+    for (int e = 0; e < ne; ++e) pf += int64_t(H) * ((b.s[e].c + cp - 1) / cp) * cp;
     if (pf / cp <= max_ctas) {
       cpc = cp;
-      for (int i = 0; i < n; ++i) b.s[i].c = int32_t((b.s[i].c + cp - 1) / cp * cp);
+      for (int e = 0; e < ne; ++e) b.s[e].c = int32_t((b.s[e].c + cp - 1) / cp * cp);
     }
   }
   int64_t off = 0;
-  for (int i = 0; i < n; ++i) {
-    b.s[i].b = int32_t(off);
-    off += int64_t(H) * b.s[i].c;
+  for (int e = 0; e < ne; ++e) {
+    b.s[e].b = int32_t(off);
+    off += int64_t(H) * b.s[e].c;
   }
-  plan.n_items = n * H;
+  plan.n_items = ne * H;
   plan.total_chunks = off;
   plan.max_ctas = max_ctas;
   plan.chunks_per_cta = cpc;
@@ -835,14 +853,31 @@ kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* id
   const bool fused = appending && kvq::decode_fuses_append(LV, G);
   if (appending && !fused) {
     kvq::Batch ab;
-    ab.n = n;
-    for (int i = 0; i < n; ++i) ab.s[i] = {ids[i], int32_t(c->len[ids[i]] - 1), 1, i, 0, ring_pages(c, ids[i])};
-    if (kvq_status s = launched(kvq::launch_append(LV, 0, ab, n, k_new, v_new, (cudaStream_t)stream), "append"))
+    ab.n = ne;
+    for (int l = 0; l < nl; ++l)
+      for (int i = 0; i < n; ++i)
+        ab.s[l * n + i] = {ids[i], int32_t(c->len[ids[i]] - 1), 1, l * n + i, 0, ring_pages(c, ids[i]), 0, l};
+    if (kvq_status s = launched(kvq::launch_append(LV, 0, ab, ne, k_new, v_new, (cudaStream_t)stream), "append"))
       return s;
   }
   return launched(kvq::launch_decode(LV, 0, b, plan, n_q_heads, q, out, fused ? k_new : nullptr,
                                      fused ? v_new : nullptr, scale_log2, ws, (cudaStream_t)stream),
                   "decode");
+}
+
+// kvq_decode_attn, and with k_new / v_new the appending variant.
+kvq_status decode_impl(kvq_cache* c, int32_t layer, int32_t n, const int32_t* ids, int32_t n_q_heads, const void* q,
+                       const void* k_new, const void* v_new, void* out, float softmax_scale, void* ws,
+                       size_t ws_bytes, kvq_stream_t stream) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (kvq_status s = check_layer(c, layer)) return s;
+  int G = 0;
+  if (kvq_status s = decode_check(c, n, ids, n_q_heads, q, k_new, v_new, out, softmax_scale, ws, &G)) return s;
+  size_t need = 0;
+  if (kvq_status s = kvq_decode_workspace_size(c, n, n_q_heads, &need)) return s;
+  if (!ws || ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
+  if (kvq_status s = need_device(c)) return s;
+  return decode_run(c, layer, 1, false, n, ids, G, n_q_heads, q, k_new, v_new, out, softmax_scale, ws, stream);
 }
 
 }  // namespace
@@ -860,6 +895,45 @@ kvq_status kvq_decode_append_attn(kvq_cache* c, int32_t layer, int32_t n, const 
                                   float softmax_scale, void* ws, size_t ws_bytes, kvq_stream_t stream) {
   if (!k_new || !v_new) return fail(KVQ_ERR_INVALID_ARG, "k_new or v_new is NULL");
   return decode_impl(c, layer, n, ids, n_q_heads, q, k_new, v_new, out, softmax_scale, ws, ws_bytes, stream);
+}
+
+kvq_status kvq_decode_layers_workspace_size(const kvq_cache* c, int32_t n_layers, int32_t n, int32_t n_q_heads,
+                                            size_t* bytes) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (n_layers < 1 || n_layers > c->cfg.n_layers) return fail(KVQ_ERR_INVALID_ARG, "n_layers must be in [1, %d]", c->cfg.n_layers);
+  if (n < 1 || n > kvq::kMaxBatch) return fail(KVQ_ERR_INVALID_ARG, "n_seqs must be in [1, %d]", kvq::kMaxBatch);
+  // the largest launch: min(n_layers, kMaxBatch / n) layers of the n sequences
+  const int32_t nl = std::min<int32_t>(n_layers, std::max<int32_t>(1, kvq::kMaxBatch / n));
+  return kvq_decode_workspace_size(c, nl * n, n_q_heads, bytes);
+}
+
+kvq_status kvq_decode_attn_layers(kvq_cache* c, int32_t layer0, int32_t n_layers, int32_t n, const int32_t* ids,
+                                  int32_t n_q_heads, const void* q, const void* k_new, const void* v_new, void* out,
+                                  float softmax_scale, void* ws, size_t ws_bytes, kvq_stream_t stream) {
+  if (kvq_status s = check_cache(c)) return s;
+  if (layer0 < 0 || n_layers < 1 || int64_t(layer0) + n_layers > c->cfg.n_layers)
+    return fail(KVQ_ERR_INVALID_ARG, "layers [%d, %d + %d) outside [0, %d)", layer0, layer0, n_layers, c->cfg.n_layers);
+  int G = 0;
+  if (kvq_status s = decode_check(c, n, ids, n_q_heads, q, k_new, v_new, out, softmax_scale, ws, &G)) return s;
+  size_t need = 0;
+  if (kvq_status s = kvq_decode_layers_workspace_size(c, n_layers, n, n_q_heads, &need)) return s;
+  if (!ws || ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "decode needs %zu workspace bytes, got %zu", need, ws ? ws_bytes : 0);
+  if (kvq_status s = need_device(c)) return s;
+  // rows of one layer in q / out and in k_new / v_new (fp16)
+  const int64_t q_layer = int64_t(n) * n_q_heads * c->L.head_dim * 2;
+  const int64_t kv_layer = int64_t(n) * c->L.n_kv_heads * c->L.head_dim * 2;
+  auto at = [](const void* p, int64_t bytes) -> const void* {
+    return p ? static_cast<const void*>(static_cast<const uint8_t*>(p) + bytes) : nullptr;
+  };
+  for (int32_t l = 0; l < n_layers;) {
+    const int32_t nl = decode_run_layers(c, layer0 + l, n_layers - l, n);
+    if (kvq_status s = decode_run(c, layer0 + l, nl, true, n, ids, G, n_q_heads, at(q, l * q_layer), at(k_new, l * kv_layer),
+                                  at(v_new, l * kv_layer), static_cast<uint8_t*>(out) + l * q_layer, softmax_scale, ws,
+                                  stream))
+      return s;
+    l += nl;
+  }
+  return KVQ_OK;
 }
 
 kvq_status kvq_prefill_workspace_size(const kvq_cache* c, int32_t n, const int32_t* ids, const int32_t* q_lens,

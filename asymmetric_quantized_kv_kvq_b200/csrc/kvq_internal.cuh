@@ -66,11 +66,16 @@ inline int code_row_bytes(int bits, int D) { return bits == 16 ? 2 * D : bits ==
 //   prefill: a = len, b = q_len, c = row offset in q/out
 // ring: page-table slots of a rotating-window sequence (logical page p lives in
 // slot p % ring), 0 for a linear page table.
+// l: layer of the entry, counted from the launch's layer (append and decode):
+// a layer-batched call lists every (layer, sequence) pair as an entry of one
+// launch; the layers of one launch share a format, so layer l's head blocks lie
+// l * n_pages * n_kv_heads head blocks past the launch layer's.
 struct SeqDesc {
   int32_t seq_id;
   int32_t a, b, c;
   int32_t lo, ring;
   int32_t cr;   // decode: chunks per head that hold tokens (c may be padded past them; 0 = c)
+  int32_t l;
 };
 
 // Page-table slot of logical page p of a sequence.

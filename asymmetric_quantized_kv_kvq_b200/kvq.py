@@ -64,6 +64,8 @@ SIGNATURES = {
     "kvq_decode_attn": (_i32, [_p, _i32, _i32, _pi32, _i32, _p, _p, _f32, _p, _sz, _p]),
     "kvq_decode_attn_noalloc": (_i32, [_p, _i32, _i32, _pi32, _i32, _p, _p, _f32, _p]),
     "kvq_decode_append_attn": (_i32, [_p, _i32, _i32, _pi32, _i32, _p, _p, _p, _p, _f32, _p, _sz, _p]),
+    "kvq_decode_layers_workspace_size": (_i32, [_p, _i32, _i32, _i32, _psz]),
+    "kvq_decode_attn_layers": (_i32, [_p, _i32, _i32, _i32, _pi32, _i32, _p, _p, _p, _p, _f32, _p, _sz, _p]),
     "kvq_prefill_workspace_size": (_i32, [_p, _i32, _pi32, _pi32, _i32, _psz]),
     "kvq_prefill_attn": (_i32, [_p, _i32, _i32, _pi32, _pi32, _i32, _p, _p, _f32, _p, _sz, _p]),
     "kvq_export": (_i32, [_p, _i32, _i32, _i64, _i64, _p, _p, _p, _p, _p]),
@@ -281,6 +283,36 @@ class Cache:
         ws = workspace if workspace is not None else self._workspace(need, q.device)
         _check(self._lib.kvq_decode_append_attn(self._h, layer, B, _i32_array(seq_ids), Hq, q.data_ptr(), kp, vp,
                                                 out.data_ptr(), softmax_scale, ws.data_ptr(),
+                                                ws.numel() * ws.element_size(), _stream(stream)))
+        return out
+
+    def decode_layers_workspace_size(self, n_layers: int, n_seqs: int, n_q_heads: int) -> int:
+        n = ctypes.c_size_t()
+        _check(self._lib.kvq_decode_layers_workspace_size(self._h, n_layers, n_seqs, n_q_heads, ctypes.byref(n)))
+        return n.value
+
+    def decode_layers(self, layer0: int, seq_ids: Sequence[int], q, k_new=None, v_new=None, out=None,
+                      softmax_scale: float = 0.0, workspace=None, stream=None):
+        """kvq_decode_attn_layers: one decode step over layers layer0 .. layer0 + NL - 1.
+        q: fp16 [NL, B, Hq, D]; k_new / v_new: fp16 [NL, B, Hkv, D] (quantised into position
+        len - 1 first) or both None -> out fp16 [NL, B, Hq, D]."""
+        import torch
+        B = len(seq_ids)
+        if q.dim() != 4 or q.shape[1] != B or q.shape[3] != self.head_dim:
+            raise KvqError(1, f"q has shape {tuple(q.shape)}, expected [layers, {B}, Hq, {self.head_dim}]")
+        NL, Hq = q.shape[0], q.shape[2]
+        _dev_fp16(q, "q")
+        if (k_new is None) != (v_new is None):
+            raise KvqError(1, "k_new and v_new must both be given or both be None")
+        kp = _dev_fp16(k_new, "k_new", (NL, B, self.n_kv_heads, self.head_dim)) if k_new is not None else None
+        vp = _dev_fp16(v_new, "v_new", (NL, B, self.n_kv_heads, self.head_dim)) if v_new is not None else None
+        if out is None:
+            out = torch.empty_like(q)
+        _dev_fp16(out, "out", tuple(q.shape))
+        need = self.decode_layers_workspace_size(NL, B, Hq)
+        ws = workspace if workspace is not None else self._workspace(need, q.device)
+        _check(self._lib.kvq_decode_attn_layers(self._h, layer0, NL, B, _i32_array(seq_ids), Hq, q.data_ptr(), kp,
+                                                vp, out.data_ptr(), softmax_scale, ws.data_ptr(),
                                                 ws.numel() * ws.element_size(), _stream(stream)))
         return out
 

@@ -166,7 +166,7 @@ class DecodeRun:
     """A resident cache of the workload plus one decode step's inputs."""
 
     def __init__(self, wl, kb: int, vb: int, capacity_extra: int, device, decode_tc: bool = False,
-                 separate: bool = False):
+                 separate: bool = False, layer_batched: bool = False):
         import torch
         from asymmetric_quantized_kv_kvq_b200 import kvq
         from asymmetric_quantized_kv_kvq_b200.inputs import gen_kv, gen_q, GEN_CHUNK
@@ -190,15 +190,26 @@ class DecodeRun:
                 self.cache.append(layer, self.ids, [n] * B, torch.cat(ks), torch.cat(vs))
                 del ks, vs
         torch.cuda.synchronize()
-        # one decode step's inputs (same values every step)
-        self.k_new, self.v_new, self.q, self.out = [], [], [], []
+        # one decode step's inputs (same values every step), stacked over the layers: q / out
+        # [L, B, Hq, D], new K / V [L, B, H, D]; the per-layer lists are views of them
+        ks, vs, qs = [], [], []
         for layer in range(L):
-            ks, vs = zip(*[gen_kv(wl, layer, b, T, 1, device=device) for b in self.ids])
-            self.k_new.append(torch.cat(ks).contiguous())
-            self.v_new.append(torch.cat(vs).contiguous())
-            self.q.append(gen_q(wl, layer, 0, device=device))
-            self.out.append(torch.empty_like(self.q[-1]))
-        self.ws = torch.empty(self.cache.decode_workspace_size(B, wl.n_q_heads), dtype=torch.uint8, device=device)
+            k1, v1 = zip(*[gen_kv(wl, layer, b, T, 1, device=device) for b in self.ids])
+            ks.append(torch.cat(k1))
+            vs.append(torch.cat(v1))
+            qs.append(gen_q(wl, layer, 0, device=device))
+        self.k_all, self.v_all, self.q_all = torch.stack(ks), torch.stack(vs), torch.stack(qs)
+        self.out_all = torch.empty_like(self.q_all)
+        del ks, vs, qs
+        self.k_new, self.v_new = list(self.k_all.unbind(0)), list(self.v_all.unbind(0))
+        self.q, self.out = list(self.q_all.unbind(0)), list(self.out_all.unbind(0))
+        # layer-batched: one kvq_decode_attn_layers call per step, one launch per run of up to
+        # KVQ_MAX_BATCH // B layers
+        self.batched = layer_batched
+        self.runs = -(-L // max(1, 256 // B)) if layer_batched else L
+        ws = self.cache.decode_layers_workspace_size(L, B, wl.n_q_heads) if layer_batched else \
+            self.cache.decode_workspace_size(B, wl.n_q_heads)
+        self.ws = torch.empty(ws, dtype=torch.uint8, device=device)
         self.ones = [1] * B
         self.ev = None
         # one launch per layer (append fused into the decode kernel) for quantized caches on CUDA cores
@@ -219,9 +230,9 @@ class DecodeRun:
     def launches_per_step(self, lens_before) -> int:
         pt = 1 if any(n % 256 == 0 for n in lens_before) else 0
         if self.fused:
-            return pt + self.wl.n_layers                 # one decode kernel (append + split + combine)
+            return pt + self.runs                        # one decode kernel (append + split + combine)
         combine = 0 if (self.kb != 16 and not self.cache_tc) else 1
-        return pt + self.wl.n_layers * (2 + combine)    # append, decode[, combine]
+        return pt + self.runs * (2 + combine)           # append, decode[, combine]
 
     @property
     def cache_tc(self) -> bool:
@@ -229,6 +240,14 @@ class DecodeRun:
 
     def step(self, record=None):
         self.cache.extend(self.ids, self.ones)
+        if self.batched:
+            if record is not None:
+                record[0][0].record()
+            self.cache.decode_layers(0, self.ids, self.q_all, self.k_all, self.v_all, out=self.out_all,
+                                     workspace=self.ws)
+            if record is not None:
+                record[0][1].record()
+            return
         for layer in range(self.wl.n_layers):
             if self.fused:
                 if record is not None:
@@ -250,7 +269,8 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
     torch.cuda.set_device(dev)
     extra = args.warmup + 2 * args.steps + 8
     t0 = time.time()
-    run = DecodeRun(wl, kb, vb, extra, dev, decode_tc=args.decode_tc, separate=args.separate)
+    run = DecodeRun(wl, kb, vb, extra, dev, decode_tc=args.decode_tc, separate=args.separate,
+                    layer_batched=getattr(args, "layer_batched", False))
     setup_s = time.time() - t0
     L = wl.n_layers
     lens0 = run.lengths()
@@ -270,7 +290,9 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
     # ---- timed region: K steps, CUDA events on the launching stream.  With a captured graph every
     #      step is one replay of the same decode step (append of one token per sequence + decode, all
     #      layers): the token is re-appended at the same position and attended over the same length.
-    ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(L)]
+    # event pairs of an eager step: one per layer's call, or one around the layer-batched call
+    n_ev = 1 if run.batched else L
+    ev = [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(n_ev)]
     dec_ms, step_ms, dec_bytes, app_bytes, launches = [], [], 0, 0, 0
     gpu_id = gpu_uuid(dev)
     with ClockSampler(gpu_id) as clk:
@@ -304,13 +326,13 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         dec_ms.extend(e0.elapsed_time(e1) for e0, e1 in ev)
         d_e, a_e = run.step_bytes([n + 1 for n in lens_e])
         in_step_bytes = d_e + (a_e if run.fused else 0)
-    # ---- kernel duration: every layer's decode call once more, back to back on the
-    #      stream behind a short device-side sleep, so that host work between calls
-    #      (binding, plan) never leaves the GPU idle inside the events
+    # ---- kernel duration: every layer's decode call once more (or the layer-batched call 8 times),
+    #      back to back on the stream behind a short device-side sleep, so that host work between
+    #      calls (binding, plan) never leaves the GPU idle inside the events
     lens_k = run.lengths()
     kd, ka = run.step_bytes(lens_k)
-    kern_bytes = (kd + (ka if run.fused else 0)) / L
-    reps = max(L, 8)
+    kern_bytes = (kd + (ka if run.fused else 0)) / n_ev
+    reps = 8 if run.batched else max(L, 8)
     kern_ms = []
     for _ in range(2):
         torch.cuda.synchronize()
@@ -320,7 +342,10 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         k0.record()
         for i in range(reps):
             lay = i % L
-            if run.fused:        # re-appends the last token at the same position, as a replayed step does
+            if run.batched:      # fused: re-appends the last token at the same position
+                run.cache.decode_layers(0, run.ids, run.q_all, run.k_all if run.fused else None,
+                                        run.v_all if run.fused else None, out=run.out_all, workspace=run.ws)
+            elif run.fused:        # re-appends the last token at the same position, as a replayed step does
                 run.cache.decode_append(lay, run.ids, run.q[lay], run.k_new[lay], run.v_new[lay], out=run.out[lay],
                                         workspace=run.ws)
             else:
@@ -340,7 +365,7 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         "ms_per_step": max_ms / args.steps,
         "value": tot_bytes / (max_ms * 1e-3) / 1e9,
         "decode_tokens_per_s": tot_tokens / (max_ms * 1e-3),
-        "dec_bytes_per_launch": in_step_bytes / L,
+        "dec_bytes_per_launch": in_step_bytes / n_ev,
         "launch_mode": launch_mode,
         "dec_ms_per_launch": statistics.mean(dec_ms),
         "kern_bytes_per_launch": kern_bytes,
@@ -351,6 +376,8 @@ def run_decode_bench(args, wl, kb, vb, rank, world) -> dict:
         "setup_s": setup_s,
         "fused": run.fused,
         "step_only_decode": run.fused and graph is not None,
+        "batched": run.batched,
+        "runs": run.runs,
         "step_bytes": (dec_bytes + app_bytes) / args.steps,
     }
 
@@ -741,6 +768,9 @@ def parse():
                     help="time one kvq_cache_dedup pass over the resident cache (on by default for the default run)")
     ap.add_argument("--no-extras", action="store_true",
                     help="default run: skip the 70B-shaped decode and the prefill sub-records")
+    ap.add_argument("--layer-batched", action="store_true",
+                    help="decode: one kvq_decode_attn_layers call per step (one launch per run of layers) "
+                         "instead of one call per layer")
     ap.add_argument("--decode-tc", action="store_true",
                     help="decode on the tensor-core kernel (cache flag KVQ_CACHE_DECODE_TENSOR_CORES) "
                          "instead of the default CUDA-core kernel")
@@ -853,18 +883,21 @@ def decode_line(args, wl, precision, kb, vb, res, world) -> dict:
     isolated = res["kern_bytes_per_launch"] / (res["kern_ms_per_launch"] * 1e-3) / 1e9
     in_step = res["dec_bytes_per_launch"] / (res["dec_ms_per_launch"] * 1e-3) / 1e9
     tc = args.decode_tc and kb == 8 and vb in (4, 8) and wl.head_dim == 128
+    R = res["runs"]                                   # launches of one step's decode (layers, or layer runs)
+    per = "per run of layers" if res["batched"] else "per layer"
     if res["step_only_decode"]:
         achieved = res["value"]
-        ms_launch = res["ms_per_step"] / L
-        timing = (f"CUDA events around each replayed step = {L} back-to-back decode launches (one per layer, "
-                  f"append and combine fused); ms_per_launch = ms_per_step / {L}")
+        ms_launch = res["ms_per_step"] / R
+        timing = (f"CUDA events around each replayed step = {R} back-to-back decode launches (one {per}, "
+                  f"append and combine fused); ms_per_launch = ms_per_step / {R}")
         kernel = "decode_q_kernel (append + split-KV + combine)"
-        bytes_launch = res["step_bytes"] / L
+        bytes_launch = res["step_bytes"] / R
     else:
         achieved = isolated
         ms_launch = res["kern_ms_per_launch"]
-        timing = (f"CUDA events around {max(L, 8)} back-to-back decode calls (one per layer) queued behind a "
-                  f"device sleep; best of 2")
+        timing = ("CUDA events around 8 back-to-back layer-batched decode calls" if res["batched"] else
+                  f"CUDA events around {max(L, 8)} back-to-back decode calls (one per layer)") + \
+            " queued behind a device sleep; best of 2"
         if tc:
             kernel = "decode_tc_kernel + lse_combine_kernel"
         elif kb == 16:
@@ -879,8 +912,10 @@ def decode_line(args, wl, precision, kb, vb, res, world) -> dict:
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": dict(config_of(wl, precision, world, res["flush"]),
                        decode_kernel="tensor cores (opt-in)" if tc else "CUDA cores",
-                       step_launch=res["launch_mode"] + ("; one fused append+decode launch per layer"
-                                                         if res["fused"] else "")),
+                       step_launch=res["launch_mode"] + ("; one fused append+decode launch " + per
+                                                         if res["fused"] else "") +
+                       (f"; layer-batched (kvq_decode_attn_layers): {R} launch(es) for {L} layers"
+                        if res["batched"] else "")),
         "decode_tokens_per_s": res["decode_tokens_per_s"],
         "roofline": {"bound": "hbm", "kernel": kernel, "achieved": achieved, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
@@ -899,7 +934,8 @@ def decode_line(args, wl, precision, kb, vb, res, world) -> dict:
 
 def run_extras(args) -> list:
     """Compact records of the other gate workloads, measured in the same run: the
-    70B-shaped 128K-token decode in K8V4 and FP16, and the ragged chunked prefill."""
+    70B-shaped 128K-token decode and the 22-layer TinyLlama-shaped 8K decode in K8V4
+    and FP16 (per-layer calls and the layer-batched call), and the ragged chunked prefill."""
     import argparse as _ap
     import torch
     from asymmetric_quantized_kv_kvq_b200.inputs import WORKLOADS, parse_precision
@@ -908,18 +944,25 @@ def run_extras(args) -> list:
     # timed regions of a few hundred ms each, so that the clock sampler (100 ms) sees several samples
     sub.steps, sub.warmup, sub.no_e2e, sub.decode_tc, sub.separate = 20, 3, True, False, False
     sub.dedup_probe = False
-    for name, prec in (("llama70b-b1-128k", "K8V4"), ("llama70b-b1-128k", "FP16")):
+    # per-layer calls (a model's step: each layer's query needs the previous layer's output), then
+    # the layer-batched call (kvq_decode_attn_layers, every layer's query known at once)
+    for name, prec, batched in (("llama70b-b1-128k", "K8V4", False), ("llama70b-b1-128k", "FP16", False),
+                                ("llama70b-b1-128k", "K8V4", True), ("llama70b-b1-128k", "FP16", True),
+                                ("tinyllama-22l-8k", "K8V4", False), ("tinyllama-22l-8k", "FP16", False),
+                                ("tinyllama-22l-8k", "K8V4", True), ("tinyllama-22l-8k", "FP16", True)):
         wl = WORKLOADS[name]
         kb, vb = parse_precision(prec)
+        sub.layer_batched = batched
         torch.cuda.empty_cache()
         r = run_decode_bench(sub, wl, kb, vb, 0, 1)
         line = decode_line(sub, wl, prec, kb, vb, r, 1)
-        out.append({"workload": name, "precision": prec, "metric": "decode KV GB/s", "value": r["value"],
-                    "unit": "GB/s", "ms_per_step": r["ms_per_step"], "steps": sub.steps,
+        out.append({"workload": name, "precision": prec, "layer_batched": batched, "metric": "decode KV GB/s",
+                    "value": r["value"], "unit": "GB/s", "ms_per_step": r["ms_per_step"], "steps": sub.steps,
                     "decode_tokens_per_s": r["decode_tokens_per_s"],
                     "roofline_frac": line["roofline"]["frac"], "kernel": line["roofline"]["kernel"],
                     "step_launch": line["config"]["step_launch"], "gpu_launches": r["launches"],
-                    "clocks": r["clocks"]})
+                    "l2": line["config"]["l2"], "clocks": r["clocks"]})
+    sub.layer_batched = False
     wl = WORKLOADS["prefill-16x4096"]
     kb, vb = parse_precision("K8V4")
     torch.cuda.empty_cache()

@@ -259,6 +259,41 @@ KVQ_API kvq_status kvq_decode_append_attn(kvq_cache* cache, int32_t layer, int32
                                           const void* k_new, const void* v_new, void* out, float softmax_scale,
                                           void* workspace, size_t ws_bytes, kvq_stream_t stream);
 
+/* Workspace bytes kvq_decode_attn_layers needs for n_layers layers of a batch
+ * of n_seqs sequences with n_q_heads query heads (independent of lengths and
+ * of the layers' formats).  Pure host arithmetic. */
+KVQ_API kvq_status kvq_decode_layers_workspace_size(const kvq_cache* cache, int32_t n_layers, int32_t n_seqs,
+                                                    int32_t n_q_heads, size_t* bytes);
+
+/* Layer-batched decode: the same result as calling, for l = 0 .. n_layers - 1,
+ * kvq_decode_append_attn (k_new and v_new given) or kvq_decode_attn (both
+ * NULL) on layer layer0 + l with that layer's rows of q, k_new, v_new and out,
+ * but in one launch for every run of consecutive layers that share a format
+ * and fit one batch (n_layers_in_run * n_seqs <= KVQ_MAX_BATCH): the kernel's
+ * work list holds every (layer, sequence, KV head, slice) of the run, so its
+ * CTAs stream the whole run's cache without a launch, a pipeline fill or a
+ * tail per layer.  For use when every layer's query of the step is known at
+ * once (a replayed or precomputed step); a model whose next layer's query
+ * depends on this layer's output calls the per-layer functions.
+ * Codes and scales written are identical to the per-layer calls'; the
+ * attention outputs match them within rounding (the slices of an item may be
+ * split among CTAs differently, which changes the fp32 summation order).
+ * The step is the pages' small-model workload (KVSplit page, "Principais
+ * resultados de benchmark": one decode step over every layer of a 22-layer
+ * cache) with every layer's decode as in kvq_decode_attn.
+ * q, out: device fp16 [n_layers, n_seqs, n_q_heads, head_dim];
+ * k_new, v_new: device fp16 [n_layers, n_seqs, n_kv_heads, head_dim] or both
+ * NULL; all 16-byte aligned.  workspace: device, ws_bytes >=
+ * kvq_decode_layers_workspace_size (the runs reuse it in stream order).
+ * Runs on the CUDA-core decode kernels (the tensor-core flag applies to the
+ * per-layer calls only).  layer0 < 0, n_layers < 1 or layer0 + n_layers >
+ * n_layers of the cache: KVQ_ERR_INVALID_ARG; other errors as
+ * kvq_decode_append_attn. */
+KVQ_API kvq_status kvq_decode_attn_layers(kvq_cache* cache, int32_t layer0, int32_t n_layers, int32_t n_seqs,
+                                          const int32_t* seq_ids, int32_t n_q_heads, const void* q,
+                                          const void* k_new, const void* v_new, void* out, float softmax_scale,
+                                          void* workspace, size_t ws_bytes, kvq_stream_t stream);
+
 /* Size of the scratch array compiled into the library for
  * kvq_decode_attn_noalloc (8 MiB per GPU that loads the library). */
 #define KVQ_NOALLOC_SCRATCH_BYTES (8u << 20)

@@ -413,3 +413,41 @@ def test_dedup_needs_a_device(kvq):
     assert lib.kvq_cache_dedup(c._h, None, ctypes.byref(n)) == 2     # KVQ_ERR_UNSUPPORTED on a host-only cache
     assert n.value == 0
     c.close()
+
+
+def test_layer_batched_decode_validation_and_workspace(kvq):
+    """kvq_decode_attn_layers checks its layer range before anything else and sizes its workspace
+    for the largest launch: min(n_layers, KVQ_MAX_BATCH // n_seqs) layers of the batch."""
+    c = _host_cache(kvq, n_layers=6, max_seqs=256, max_tokens=256 * 256)
+    c.extend([0], [10])
+    lib = kvq.load_library()
+    ids0 = (ctypes.c_int32 * 1)(0)
+    # one sequence: every layer fits one launch, so the workspace is that of 6 entries
+    assert c.decode_layers_workspace_size(6, 1, 4) == c.decode_workspace_size(6, 4)
+    assert c.decode_layers_workspace_size(1, 1, 4) == c.decode_workspace_size(1, 4)
+    # 64 sequences: 4 layers per launch (256 entries); 256 sequences: one layer per launch
+    assert c.decode_layers_workspace_size(5, 64, 4) == c.decode_workspace_size(256, 4)
+    assert c.decode_layers_workspace_size(3, 64, 4) == c.decode_workspace_size(192, 4)
+    assert c.decode_layers_workspace_size(6, 256, 4) == c.decode_workspace_size(256, 4)
+    for bad in ((0, 1), (7, 1), (2, 0), (2, 257)):
+        with pytest.raises(kvq.KvqError):
+            c.decode_layers_workspace_size(bad[0], bad[1], 4)
+    ws = 1 << 20
+    call = lib.kvq_decode_attn_layers
+    # layer range: negative start, empty, past the last layer
+    assert call(c._h, -1, 1, 1, ids0, 4, 16, None, None, 16, 0.0, 16, ws, None) == 1
+    assert call(c._h, 0, 0, 1, ids0, 4, 16, None, None, 16, 0.0, 16, ws, None) == 1
+    assert call(c._h, 4, 3, 1, ids0, 4, 16, None, None, 16, 0.0, 16, ws, None) == 1
+    # heads, GQA group, one of k_new / v_new, alignment, workspace, host-only
+    assert call(c._h, 0, 6, 1, ids0, 3, 16, None, None, 16, 0.0, 16, ws, None) == 1
+    assert call(c._h, 0, 6, 1, ids0, 6, 16, None, None, 16, 0.0, 16, ws, None) == 2
+    assert call(c._h, 0, 6, 1, ids0, 4, 16, 16, None, 16, 0.0, 16, ws, None) == 1
+    assert call(c._h, 0, 6, 1, ids0, 4, 8, None, None, 16, 0.0, 16, ws, None) == 1
+    assert call(c._h, 0, 6, 1, ids0, 4, 16, None, None, 16, 0.0, None, 0, None) == 7
+    assert call(c._h, 0, 6, 1, ids0, 4, 16, None, None, 16, 0.0, 16, 16, None) == 7
+    assert call(c._h, 0, 6, 1, ids0, 4, 16, 16, 16, 16, 0.0, 16, ws, None) == 2
+    # an empty sequence
+    ids1 = (ctypes.c_int32 * 1)(1)
+    assert call(c._h, 0, 6, 1, ids1, 4, 16, None, None, 16, 0.0, 16, ws, None) == 1
+    assert c.length(0) == 10
+    c.close()
