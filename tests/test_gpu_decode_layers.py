@@ -244,3 +244,46 @@ def test_layer_batched_step_replays_in_a_cuda_graph():
     cache.check()
     del g
     cache.close()
+
+
+@pytest.mark.gpu
+def test_layer_batched_step_on_a_tensor_core_cache():
+    """A cache created with the tensor-core decode flag: the layer-batched call runs the CUDA-core
+    kernels (the flag applies to the per-layer calls) and matches the oracle; the per-layer calls on
+    the twin cache (tensor-core kernel) match it too."""
+    m = kvq()
+    D, H, G, NL = 128, 8, 4, 2
+    lens = [300, 2000]
+    B = len(lens)
+
+    def build():
+        cache = m.Cache(n_layers=NL, n_kv_heads=H, head_dim=D, k_bits=8, v_bits=4, max_seqs=B,
+                        max_tokens=sum(lens) + 512 * B, decode_tc=True)
+        raw = {}
+        cache.extend(list(range(B)), lens)
+        for l in range(NL):
+            ks = [decode_kv(n, H, D, 61 + 100 * s + l) for s, n in enumerate(lens)]
+            vs = [random_fp16((n, H, D), 68 + 100 * s + l) for s, n in enumerate(lens)]
+            cache.append(l, list(range(B)), lens, torch.cat(ks).cuda(), torch.cat(vs).cuda())
+            for s in range(B):
+                raw[(l, s)] = (ks[s], vs[s])
+        return cache, raw
+
+    cache, raw = build()
+    twin, _ = build()
+    ids = list(range(B))
+    q, k_new, v_new = _step_inputs(NL, B, H, G, D, 6900)
+    cache.extend(ids, [1] * B)
+    out = cache.decode_layers(0, ids, q.cuda(), k_new.cuda(), v_new.cuda())
+    cache.check()
+    twin.extend(ids, [1] * B)
+    for l in range(NL):
+        sep = twin.decode_append(l, ids, q[l].cuda(), k_new[l].cuda(), v_new[l].cuda())
+        ref = _reference(q[l], raw, l, ids, 8, 4, k_new[l], v_new[l])
+        assert_close_attention(out[l], ref, f"layer-batched, layer {l}")
+        assert_close_attention(sep, ref, f"per-layer tensor-core call, layer {l}")
+        for s in ids:
+            _check_row(cache, l, s, lens[s], k_new[l, s:s + 1], v_new[l, s:s + 1], 8, 4)
+    twin.check()
+    cache.close()
+    twin.close()
