@@ -526,7 +526,7 @@ __device__ __forceinline__ __half new_row_quant(const NewRow<D>& nr, bool q8, in
   if (!q8) {
     uint32_t by[EQ];
 #pragma unroll
-    for (int i = 0; i < EQ; ++i) by[i] = float_int_bits(__fmaf_rn(ch[i], 16.f, c[i]) + 136.f);   // u_j + 16 u_{j+16}
+    for (int i = 0; i < EQ; ++i) by[i] = __float_as_uint(__fmaf_rn(ch[i], 16.f, c[i]) + (kRoundBias + 136.f));   // u_j + 16 u_{j+16}
 #pragma unroll
     for (int k = 0; k < EQ / 4; ++k) cw[k] = pack_low_bytes(by[4 * k], by[4 * k + 1], by[4 * k + 2], by[4 * k + 3]);
   }
@@ -555,7 +555,6 @@ __device__ __forceinline__ void producer_role(const DecodeQArgs& a, const Batch&
   using T = QDec<KB, VB, D, G, CT>;
   constexpr int S = T::S, NB = T::NB;
   const int lane = threadIdx.x & 31;
-  const int H = a.L.n_kv_heads;
   const uint64_t pol = l2_evict_first_policy();
   uint32_t it = 0;
   int s = 0;                                           // ring slot of stage `it` and its fill parity

@@ -18,33 +18,32 @@ namespace kvq {
 
 // Code rounding without a divide and without integer conversions, for
 // fp16-valued x and d != 0: c = clamp(roundf(fp32(x / d)), -cn, cp) as an exact
-// small integer in a float.  With t = |x| / |d| <= 128.5, n = rint(|x| * fp32(1/|d|))
-// (one FMA against 1.5 * 2^23, ties to even) misses t by less than 2^-16, while a
-// quotient of two fp16 values that is not exactly on a half-integer lies at least
-// 2^-15 from one: n is round(t) except on an exact tie t = k + 1/2 that rint took
-// to an even k.  The remainder e = |x| - n |d| is exact in fp32 (n |d| has at most
-// 18 significant bits) and equals +|d|/2 exactly then, so one upward step gives
-// the tie to the larger magnitude (away from zero); e < -|d|/2 never occurs.  The
-// sign of x / d is applied last, then the clamp.  This is the same integer as
-// roundf of the IEEE fp32 quotient for every fp16 magnitude against every
-// positive fp16 scale with t <= 128.5 (checked exhaustively: 7.0e8 pairs).
+// small integer in a float.  With t = |x| / |d| <= 128.5 and ra = 1 / |d| rounded
+// up to fp32, round(t) (halves away from zero) is floor(|x| ra + 1/2) with that FMA
+// rounded down to fp32.  ra >= 1 / |d| keeps the exact |x| ra + 1/2 at or above
+// t + 1/2, so an exact tie t = k + 1/2 reaches k + 1; |x| ra exceeds t by at most
+// t 2^-23 < 2^-16, and a quotient of two fp16 values that is not a half-integer
+// lies at least 2^-15 from one, so neither that excess nor the downward rounding
+// of the FMA (less than one fp32 ulp, 2^-16 below 256) moves the sum across an
+// integer that t + 1/2 does not reach.  The floor is one more addition, of
+// 1.5 * 2^23 rounded down, which leaves M + n (M = 1.5 * 2^23).  The sign of x / d
+// is applied afterwards, then the clamp.  This is the same integer as roundf of the
+// IEEE fp32 quotient for every fp16 magnitude against every positive fp16 scale
+// with t <= 128.5 (checked exhaustively: 7.0e8 pairs).
+constexpr float kRoundBias = 12582912.0f;   // M = 1.5 * 2^23: M + v holds the integer v in its low bits
 struct RoundCtx {
-  float ad, ra, hd;   // |d|, fp32(1 / |d|), |d| / 2
+  float ra;   // 1 / |d|, rounded up to fp32
 };
 __device__ __forceinline__ RoundCtx round_ctx(float d) {
   RoundCtx r;
-  r.ad = fabsf(d);
-  r.ra = __frcp_rn(r.ad);
-  r.hd = 0.5f * r.ad;
+  r.ra = __frcp_ru(fabsf(d));
   return r;
 }
-__device__ __forceinline__ float round_mag(float x, const RoundCtx& r) {
-  const float ax = fabsf(x);
-  float n = __fadd_rn(__fmaf_rn(ax, r.ra, 12582912.0f), -12582912.0f);
-  const float e = __fmaf_rn(-n, r.ad, ax);
-  if (e >= r.hd) n += 1.f;           // an exact tie rounded to the even k below
-  return n;
+// M + round(|x| / |d|)
+__device__ __forceinline__ float round_mag_biased(float x, const RoundCtx& r) {
+  return __fadd_rd(__fmaf_rd(fabsf(x), r.ra, 0.5f), kRoundBias);
 }
+__device__ __forceinline__ float round_mag(float x, const RoundCtx& r) { return round_mag_biased(x, r) - kRoundBias; }
 // 4-bit (d of either sign): the sign of x / d set on the magnitude with one bit
 // operation, then the asymmetric clamp to [-8, 7].
 __device__ __forceinline__ float round_code4(float x, const RoundCtx& r, uint32_t dbits) {
@@ -52,9 +51,9 @@ __device__ __forceinline__ float round_code4(float x, const RoundCtx& r, uint32_
   const float c = __uint_as_float(__float_as_uint(n) | ((__float_as_uint(x) ^ dbits) & 0x80000000u));
   return fmaxf(fminf(c, 7.f), -8.f);
 }
-// 8-bit: d > 0, symmetric clamp
+// 8-bit: d > 0, symmetric clamp (applied to M + n, which is exact)
 __device__ __forceinline__ float round_code8(float x, const RoundCtx& r) {
-  return copysignf(fminf(round_mag(x, r), 127.f), x);
+  return copysignf(fminf(round_mag_biased(x, r), kRoundBias + 127.f) - kRoundBias, x);
 }
 // max(a, b, c) and min(a, b, c) in one instruction each
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -68,7 +67,7 @@ __device__ __forceinline__ float fmin3(float a, float b, float c) {
   return d;
 }
 // Low byte of an exact integer v in [-128, 255] held in a float (two's complement for v < 0).
-__device__ __forceinline__ uint32_t float_int_bits(float v) { return __float_as_uint(v + 12582912.0f); }
+__device__ __forceinline__ uint32_t float_int_bits(float v) { return __float_as_uint(v + kRoundBias); }
 // Bytes 0 of a, b, c, e -> one word.
 __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t e) {
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, e, 0x0040), 0x5410);
@@ -149,7 +148,7 @@ __device__ __forceinline__ __half quant4_words(const float (&x)[32], uint32_t (&
     for (int j = 0; j < 16; ++j) {
       // u_j + 16 u_{j+16} = c_j + 16 c_{j+16} + 136, an exact integer in [0, 255]
       const float c0 = round_code4(x[j], r, dbits), c1 = round_code4(x[j + 16], r, dbits);
-      by[j] = float_int_bits(__fmaf_rn(c1, 16.f, c0) + 136.f);
+      by[j] = __float_as_uint(__fmaf_rn(c1, 16.f, c0) + (kRoundBias + 136.f));   // exact integers throughout
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) w[k] = pack_low_bytes(by[4 * k], by[4 * k + 1], by[4 * k + 2], by[4 * k + 3]);
