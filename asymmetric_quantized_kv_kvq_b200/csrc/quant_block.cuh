@@ -44,16 +44,25 @@ __device__ __forceinline__ float round_mag_biased(float x, const RoundCtx& r) {
   return __fadd_rd(__fmaf_rd(fabsf(x), r.ra, 0.5f), kRoundBias);
 }
 __device__ __forceinline__ float round_mag(float x, const RoundCtx& r) { return round_mag_biased(x, r) - kRoundBias; }
+// The clamps only matter for subnormal scales.  With a normal fp16 scale (|d| >= 2^-14) the
+// largest |x| / |d| of a block is below 127.06 for 8 bits (d = fp16(amax / 127)) and exactly 8
+// for 4 bits (d = m / -8 is exact), so no 8-bit code passes 127 and no 4-bit code falls below -8;
+// a subnormal scale rounds with a coarser step (up to 190 and 11).  Checked for every fp16 amax
+// and m.
+constexpr float kMinNormalHalf = 6.103515625e-05f;   // 2^-14
 // 4-bit (d of either sign): the sign of x / d set on the magnitude with one bit
-// operation, then the asymmetric clamp to [-8, 7].
+// operation, then the asymmetric clamp to [-8, 7] (LOW: the lower bound too).
+template <bool LOW = true>
 __device__ __forceinline__ float round_code4(float x, const RoundCtx& r, uint32_t dbits) {
   const float n = round_mag(x, r);
   const float c = __uint_as_float(__float_as_uint(n) | ((__float_as_uint(x) ^ dbits) & 0x80000000u));
-  return fmaxf(fminf(c, 7.f), -8.f);
+  return LOW ? fmaxf(fminf(c, 7.f), -8.f) : fminf(c, 7.f);
 }
-// 8-bit: d > 0, symmetric clamp (applied to M + n, which is exact)
+// 8-bit: d > 0, symmetric clamp (applied to M + n, which is exact; CLAMP = false for a normal d)
+template <bool CLAMP = true>
 __device__ __forceinline__ float round_code8(float x, const RoundCtx& r) {
-  return copysignf(fminf(round_mag_biased(x, r), kRoundBias + 127.f) - kRoundBias, x);
+  if constexpr (CLAMP) return copysignf(fminf(round_mag_biased(x, r), kRoundBias + 127.f) - kRoundBias, x);
+  return copysignf(round_mag(x, r), x);
 }
 // max(a, b, c) and min(a, b, c) in one instruction each
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -97,7 +106,15 @@ __device__ __forceinline__ __half quant8_words(const float (&x)[32], uint32_t (&
   for (int i = 0; i < 32; i += 2) a = fmax3(a, fabsf(x[i]), fabsf(x[i + 1]));
   const __half d = __float2half_rn(__fdiv_rn(a, 127.0f));
   const float df = __half2float(d);
-  if (df != 0.f) {
+  if (df >= kMinNormalHalf) {
+    const RoundCtx r = round_ctx(df);
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+      w[k] = pack_low_bytes(float_int_bits(round_code8<false>(x[4 * k], r)),
+                            float_int_bits(round_code8<false>(x[4 * k + 1], r)),
+                            float_int_bits(round_code8<false>(x[4 * k + 2], r)),
+                            float_int_bits(round_code8<false>(x[4 * k + 3], r)));
+  } else if (df != 0.f) {
     const RoundCtx r = round_ctx(df);
 #pragma unroll
     for (int k = 0; k < 8; ++k)
@@ -144,11 +161,19 @@ __device__ __forceinline__ __half quant4_words(const float (&x)[32], uint32_t (&
     const RoundCtx r = round_ctx(df);
     const uint32_t dbits = __float_as_uint(df);
     uint32_t by[16];
+    if (fabsf(df) >= kMinNormalHalf) {
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      // u_j + 16 u_{j+16} = c_j + 16 c_{j+16} + 136, an exact integer in [0, 255]
-      const float c0 = round_code4(x[j], r, dbits), c1 = round_code4(x[j + 16], r, dbits);
-      by[j] = __float_as_uint(__fmaf_rn(c1, 16.f, c0) + (kRoundBias + 136.f));   // exact integers throughout
+      for (int j = 0; j < 16; ++j) {
+        // u_j + 16 u_{j+16} = c_j + 16 c_{j+16} + 136, an exact integer in [0, 255]
+        const float c0 = round_code4<false>(x[j], r, dbits), c1 = round_code4<false>(x[j + 16], r, dbits);
+        by[j] = __float_as_uint(__fmaf_rn(c1, 16.f, c0) + (kRoundBias + 136.f));   // exact integers throughout
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float c0 = round_code4(x[j], r, dbits), c1 = round_code4(x[j + 16], r, dbits);
+        by[j] = __float_as_uint(__fmaf_rn(c1, 16.f, c0) + (kRoundBias + 136.f));
+      }
     }
 #pragma unroll
     for (int k = 0; k < 4; ++k) w[k] = pack_low_bytes(by[4 * k], by[4 * k + 1], by[4 * k + 2], by[4 * k + 3]);

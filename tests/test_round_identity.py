@@ -50,3 +50,20 @@ def test_directed_rounding_is_sensitive_to_the_tie_handling():
     n = np.floor((ax * ra + 0.5).astype(np.float32).astype(np.float64))
     q = (ax.astype(np.float32) / np.broadcast_to(d, ax.shape).astype(np.float32)).astype(np.float64)
     assert np.any(sel & (n != np.floor(q + 0.5)))
+
+
+def test_normal_scales_need_no_clamp():
+    """The append kernel skips the clamps that a normal fp16 scale cannot reach: with |d| >= 2^-14,
+    every 8-bit block has amax / d < 127.5 (d = fp16(fp32(amax / 127))), so no code rounds past 127,
+    and every 4-bit block has |m| / |d| < 8.5 (d = fp16(m / -8)), so no code rounds below -8.  Subnormal
+    scales do need them (their amax / d reaches 190 and |m| / |d| 11)."""
+    h = np.arange(1, 0x7C00, dtype=np.uint16).view(np.float16)       # positive finite fp16
+    a = h.astype(np.float64)
+    d8 = (h.astype(np.float32) / np.float32(127.0)).astype(np.float16).astype(np.float64)
+    n8 = d8 >= 2.0**-14
+    assert np.all(2 * a[n8] < 255 * d8[n8])                          # amax < 127.5 d, exactly
+    assert np.any(2 * a[(d8 > 0) & ~n8] >= 255 * d8[(d8 > 0) & ~n8])
+    d4 = (h.astype(np.float32) * np.float32(0.125)).astype(np.float16).astype(np.float64)
+    n4 = d4 >= 2.0**-14
+    assert np.all(2 * a[n4] < 17 * d4[n4])                           # |m| < 8.5 |d|, exactly
+    assert np.any(2 * a[(d4 > 0) & ~n4] >= 17 * d4[(d4 > 0) & ~n4])
