@@ -434,26 +434,26 @@ def capture_step(run, body):
 
 def run_e2e(run, args, world, dev, eager: bool) -> dict:
     """Same step, but every step copies its inputs (q, new K / V for all layers)
-    from pinned host memory and reads all outputs back to pinned host memory;
+    from pinned host memory and reads all outputs back to pinned host memory
+    (one copy per tensor, all layers at once);
     the step is a replayed graph of the copies + calls, or (eager) the host
     calls themselves, binding and validation included."""
     import torch
-    L = run.wl.n_layers
-    hq = [t.cpu().pin_memory() for t in run.q]
-    hk = [t.cpu().pin_memory() for t in run.k_new]
-    hv = [t.cpu().pin_memory() for t in run.v_new]
-    ho = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in run.out]
-    h2d = sum(t.numel() * t.element_size() for t in hq + hk + hv)
-    d2h = sum(t.numel() * t.element_size() for t in ho)
+    # every layer's inputs and outputs sit in one pinned host buffer each ([L, B, ...], the layout of
+    # the device tensors), so a step moves them with three host-to-device copies and one back
+    hq = run.q_all.cpu().pin_memory()
+    hk = run.k_all.cpu().pin_memory()
+    hv = run.v_all.cpu().pin_memory()
+    ho = torch.empty(run.out_all.shape, dtype=run.out_all.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+    d2h = ho.numel() * ho.element_size()
 
     def body():
-        for layer in range(L):
-            run.q[layer].copy_(hq[layer], non_blocking=True)
-            run.k_new[layer].copy_(hk[layer], non_blocking=True)
-            run.v_new[layer].copy_(hv[layer], non_blocking=True)
+        run.q_all.copy_(hq, non_blocking=True)
+        run.k_all.copy_(hk, non_blocking=True)
+        run.v_all.copy_(hv, non_blocking=True)
         run.step()
-        for layer in range(L):
-            ho[layer].copy_(run.out[layer], non_blocking=True)
+        ho.copy_(run.out_all, non_blocking=True)
 
     for _ in range(2):
         body()
