@@ -98,6 +98,9 @@ struct QDec {
   static constexpr int NPV = W / TPV;                // value passes per stage
   static constexpr int NT = (NW + 4) * 32;
   static constexpr int REG_L = 168, REG_C = 216, REG_P = 72;
+  // setmaxnreg moves registers between warpgroups of this block only: the split must fit in what
+  // the block was launched with, or a warpgroup's increase would never be granted
+  static_assert(NW * 32 * REG_C + 4 * 32 * REG_P <= NT * REG_L, "register split exceeds the launch allocation");
   static constexpr int K_ROW = KB == 8 ? D : D / 2;
   static constexpr int V_ROW = VB == 8 ? D : D / 2;
   static constexpr int KBLK = K_ROW / NB;            // code bytes of one key block
